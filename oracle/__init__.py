@@ -1,0 +1,167 @@
+"""fp64 CPU oracle for the Gated DeltaNet layer (forward and backward).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
+baseline leg are the only callers.  The product package never imports this
+module and this module never imports the product package; the two share only
+the seeded input generator, which holds none of the method's arithmetic.
+
+``gdn_ref.c`` holds the token-by-token recurrence (the definition the pages
+hold every kernel to: jax-linear-attention 0.1.0, "How it works").  This
+module gathers per-(document, head) units out of (B, T, H, D) arrays, runs the
+C code over them in threads and scatters the results back.  ``chunked.py`` is
+an independent fp64 restatement of the chunkwise algebra, used only to pin the
+algebra against the token recurrence.
+
+Parity pins: every function here is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py`` (closed forms, invariants, brute force, finite
+differences).  The pages print no worked numeric example for this method.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_ref.c")
+_SO = os.path.join(_HERE, "libgdn_ref.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile gdn_ref.c into libgdn_ref.so next to it (plain gcc, IEEE fp64)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread",
+                               "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+class _Unit(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int64)] + [
+        (n, ctypes.c_void_p) for n in
+        ("q", "k", "v", "g", "beta", "h0", "o", "hT", "do_", "dhT",
+         "dq", "dk", "dv", "dg", "dbeta", "dh0")]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            for name in ("gdn_ref_fwd", "gdn_ref_bwd"):
+                f = getattr(lib, name)
+                f.restype = ctypes.c_int
+                f.argtypes = [ctypes.POINTER(_Unit), ctypes.c_int, ctypes.c_int64,
+                              ctypes.c_int64, ctypes.c_double, ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _segments(B, T, cu_seqlens):
+    """List of (row b, token start, token end) per sequence; dense rows when cu_seqlens is None."""
+    if cu_seqlens is None:
+        return [(b, 0, T) for b in range(B)]
+    cu = [int(x) for x in np.asarray(cu_seqlens).reshape(-1)]
+    assert B == 1 and cu[0] == 0 and cu[-1] == T
+    assert all(cu[i] <= cu[i + 1] for i in range(len(cu) - 1))
+    return [(0, cu[i], cu[i + 1]) for i in range(len(cu) - 1)]
+
+
+def _f64(x):
+    return None if x is None else np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, units=None, nthreads=None):
+    """Token-by-token forward.  q,k: (B,T,H,K); v: (B,T,H,V); g, beta: (B,T,H);
+    h0: (N,H,K,V) or None.  Returns o (B,T,H,V) and hT (N,H,K,V) in fp64.
+
+    ``units``: optional iterable of (sequence, head) pairs to compute; the
+    other entries of o and hT are left NaN (used for sampled parity)."""
+    q, k, v, g, beta, h0 = map(_f64, (q, k, v, g, beta, h0))
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    segs = _segments(B, T, cu_seqlens)
+    N = len(segs)
+    o = np.full((B, T, H, V), np.nan)
+    hT = np.full((N, H, K, V), np.nan)
+    sel = [(n, h) for n in range(N) for h in range(H)] if units is None else list(units)
+    keep, arr = [], (_Unit * max(1, len(sel)))()
+    for i, (n, h) in enumerate(sel):
+        b, t0, t1 = segs[n]
+        L = t1 - t0
+        bufs = dict(q=np.ascontiguousarray(q[b, t0:t1, h]), k=np.ascontiguousarray(k[b, t0:t1, h]),
+                    v=np.ascontiguousarray(v[b, t0:t1, h]), g=np.ascontiguousarray(g[b, t0:t1, h]),
+                    beta=np.ascontiguousarray(beta[b, t0:t1, h]),
+                    h0=None if h0 is None else np.ascontiguousarray(h0[n, h]),
+                    o=np.zeros((max(L, 1), V)), hT=np.zeros((K, V)))
+        keep.append(bufs)
+        arr[i] = _Unit(L, *[_ptr(bufs.get(f)) for f in
+                            ("q", "k", "v", "g", "beta", "h0", "o", "hT")], *([None] * 8))
+    rc = _load().gdn_ref_fwd(arr, len(sel), K, V, float(scale), nthreads or default_threads())
+    if rc:
+        raise MemoryError("oracle forward failed (%d)" % rc)
+    for (n, h), bufs in zip(sel, keep):
+        b, t0, t1 = segs[n]
+        o[b, t0:t1, h] = bufs["o"][: t1 - t0]
+        hT[n, h] = bufs["hT"]
+    return o, hT
+
+
+def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0, units=None,
+            nthreads=None):
+    """Token-by-token backward of o and hT with upstream gradients do (B,T,H,V)
+    and dhT (N,H,K,V) or None.  Returns dq, dk, dv, dg, dbeta, dh0 in fp64."""
+    q, k, v, g, beta, do, h0, dhT = map(_f64, (q, k, v, g, beta, do, h0, dhT))
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    segs = _segments(B, T, cu_seqlens)
+    N = len(segs)
+    out = dict(dq=np.full((B, T, H, K), np.nan), dk=np.full((B, T, H, K), np.nan),
+               dv=np.full((B, T, H, V), np.nan), dg=np.full((B, T, H), np.nan),
+               dbeta=np.full((B, T, H), np.nan), dh0=np.full((N, H, K, V), np.nan))
+    sel = [(n, h) for n in range(N) for h in range(H)] if units is None else list(units)
+    keep, arr = [], (_Unit * max(1, len(sel)))()
+    for i, (n, h) in enumerate(sel):
+        b, t0, t1 = segs[n]
+        L = max(t1 - t0, 1)
+        c = np.ascontiguousarray
+        bufs = dict(q=c(q[b, t0:t1, h]), k=c(k[b, t0:t1, h]), v=c(v[b, t0:t1, h]),
+                    g=c(g[b, t0:t1, h]), beta=c(beta[b, t0:t1, h]),
+                    h0=None if h0 is None else c(h0[n, h]),
+                    do_=c(do[b, t0:t1, h]), dhT=None if dhT is None else c(dhT[n, h]),
+                    dq=np.zeros((L, K)), dk=np.zeros((L, K)), dv=np.zeros((L, V)),
+                    dg=np.zeros(L), dbeta=np.zeros(L), dh0=np.zeros((K, V)))
+        keep.append(bufs)
+        arr[i] = _Unit(t1 - t0, _ptr(bufs["q"]), _ptr(bufs["k"]), _ptr(bufs["v"]), _ptr(bufs["g"]),
+                       _ptr(bufs["beta"]), _ptr(bufs["h0"]), None, None, _ptr(bufs["do_"]),
+                       _ptr(bufs["dhT"]), _ptr(bufs["dq"]), _ptr(bufs["dk"]), _ptr(bufs["dv"]),
+                       _ptr(bufs["dg"]), _ptr(bufs["dbeta"]), _ptr(bufs["dh0"]))
+    rc = _load().gdn_ref_bwd(arr, len(sel), K, V, float(scale), nthreads or default_threads())
+    if rc:
+        raise MemoryError("oracle backward failed (%d)" % rc)
+    for (n, h), bufs in zip(sel, keep):
+        b, t0, t1 = segs[n]
+        L = t1 - t0
+        for name in ("dq", "dk", "dv"):
+            out[name][b, t0:t1, h] = bufs[name][:L]
+        out["dg"][b, t0:t1, h] = bufs["dg"][:L]
+        out["dbeta"][b, t0:t1, h] = bufs["dbeta"][:L]
+        out["dh0"][n, h] = bufs["dh0"]
+    return out["dq"], out["dk"], out["dv"], out["dg"], out["dbeta"], out["dh0"]
