@@ -1,0 +1,388 @@
+"""Benchmark: Gated DeltaNet forward + backward tokens/s on B200.
+
+One step = gdn_fwd + gdn_bwd (the whole hot path) over one batch of the
+workload B=4, T=4096, H=16, d_k=d_v=128, bf16 inputs, fp32 gates/state, with
+inputs resident in HBM.  Each rank runs its own seeded batch (independent
+problems, no collective on the data path): weak scaling.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
+oracle (the only other implementation of this layer here) on the host cores
+over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN fwd+bwd tokens/s (B=4,T=4K,H=16,d=128 bf16); % of TC/HBM roofline"
+WORKLOAD = dict(B=4, T=4096, H=16, K=128, V=128, dtype="bf16", gate_scale=0.1, h0_std=0.02,
+                seed=2, bwd=True)
+C = 64
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], tc=p["bf16_tflops"], tc_sus=p["bf16_tflops_sustained"],
+                    sm_mhz=p.get("sm_max_mhz", 1965.0), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, tc=1590.0, tc_sus=1400.0, sm_mhz=1965.0, src="fallback")
+
+
+# ------------------------------------------------------------------ roofline
+def kernel_work(name, w, n_chunks):
+    """Algorithmic work of one launch of a kernel on workload w: (bound, amount, unit).
+    Bytes are the tensors the step must move for that kernel; flops the
+    chunkwise products the kernel is defined to compute (per chunk-head unit
+    times chunk-heads)."""
+    K, V, H = w["K"], w["V"], w["H"]
+    ch = n_chunks * H
+    f2 = lambda m, n, k: 2.0 * m * n * k
+    table = {
+        "simt_prep": f2(C, C, K) + C ** 3 / 3 + f2(C, K, C) + f2(C, V, C),
+        "simt_state_fwd": f2(C, V, K) + f2(K, V, C),
+        "simt_out": f2(C, C, K) + f2(C, V, K) + f2(C, V, C),
+        "simt_duloc": f2(C, C, K) + f2(C, V, C),
+        "simt_state_bwd": f2(C, V, K) + 2 * f2(K, V, C),
+        "simt_grads": 8 * f2(C, C, K) + 3 * f2(C, C, V) + 3 * f2(C, K, V) + 2 * f2(C, C, C),
+    }
+    if name in table:
+        return "alu", table[name] * ch, "flop"
+    return None, None, None
+
+
+def alu_peak_tflops(sm_mhz):
+    # 148 SMs x 128 fp32 lanes x 2 flop (FMA) per clock
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def step_roofline(w, pk):
+    """Whole-step binding roofline (method flops and bytes per token-head)."""
+    K, V = w["K"], w["V"]
+    th = w["B"] * w["T"] * w["H"]
+    fwd_f = 2 * C * (3 * K + 2 * V) + 6 * K * V + C * C / 3
+    bwd_f = 9 * 2 * C * K + 5 * 2 * C * V + 8 * 2 * K * V + 4 * C * C
+    flops = (fwd_f + bwd_f) * th
+    bytes_ = (1032 + 1808) * th + 3 * w["B"] * w["H"] * K * V * 4
+    t_tc = flops / (pk["tc_sus"] * 1e12)
+    t_hbm = bytes_ / (pk["hbm"] * 1e9)
+    return dict(flops=flops, bytes=bytes_, t_tc_s=t_tc, t_hbm_s=t_hbm,
+                bound="tensor" if t_tc > t_hbm else "hbm", t_bound_s=max(t_tc, t_hbm))
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, uuid):
+        self.uuid, self.proc, self.lines = uuid, None, []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        cmd = ["nvidia-smi", "--query-gpu=" + q, "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_oracle_sample(units_n):
+    """Time the fp64 oracle (fwd + bwd) on `units_n` (row, head) units of the
+    workload; returns (seconds, units, threads, tokens-equivalent)."""
+    import oracle
+    from gated_delta_rule_99_b200.inputs import make_inputs
+    w = dict(WORKLOAD)
+    inp = make_inputs(**w)
+    allu = [(b, h) for b in range(w["B"]) for h in range(w["H"])]
+    units = allu[:units_n]
+    threads = oracle.default_threads()
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.gdn_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, h0=inp.h0, units=units, nthreads=threads)
+    oracle.gdn_bwd(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.do, h0=inp.h0, dhT=inp.dhT,
+                   units=units, nthreads=threads)
+    dt = time.perf_counter() - t0
+    tokens = len(units) * w["T"] / w["H"]  # one token of the metric spans H heads
+    return dt, len(units), threads, tokens
+
+
+def oracle_units_for_cores():
+    import oracle
+    return max(1, min(64, oracle.default_threads()))
+
+
+# ------------------------------------------------------------------ main arms
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    n_units = oracle_units_for_cores()
+    for _ in range(max(0, args.warmup)):
+        cpu_oracle_sample(n_units)
+    times, tokens, threads = [], 0.0, 1
+    for _ in range(args.steps):
+        dt, nu, threads, tk = cpu_oracle_sample(n_units)
+        times.append(dt)
+        tokens += tk
+    total = sum(times)
+    val = tokens / total
+    sample = ("%d (row, head) units of 4096 tokens, fp64 token-recurrence forward+backward per "
+              "step; tokens/s counts units*T/H" % n_units)
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "gdn_fwdbwd_bf16_B4_T4096_H16_d128", "global_batch": 4,
+                       "seq_len": 4096, "heads": 16, "head_dim": 128, "parallelism": "none"},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_99_b200 as gdn
+    from gated_delta_rule_99_b200.inputs import make_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = dict(WORKLOAD)
+    w["seed"] = WORKLOAD["seed"] + rank
+    inp = make_inputs(device="cpu", **w)
+    d = inp.to(dev)
+    B, T, H, K, V = w["B"], w["T"], w["H"], w["K"], w["V"]
+    desc = gdn.make_desc(B, T, H, K, V)
+    ws = gdn.alloc_workspace(max(gdn.fwd_workspace_size(desc), gdn.bwd_workspace_size(desc)), dev)
+    o = torch.empty(B, T, H, V, dtype=torch.bfloat16, device=dev)
+    hT = torch.empty(B, H, K, V, dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(d.q), torch.empty_like(d.k), torch.empty_like(d.v),
+             torch.empty_like(d.g), torch.empty_like(d.beta), torch.empty_like(d.h0))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, h0=d.h0, o=o, hT=hT, workspace=ws)
+        gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, h0=d.h0, dhT=d.dhT, grads=grads,
+                    workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if gdn.device_status(ws) != 0:
+        raise RuntimeError("device status not ok after warm-up")
+
+    n_chunks = B * ((T + C - 1) // C)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    trace = gdn.LaunchTrace(capacity=64 * args.steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(uuid if rank == 0 else None) as clk:
+        with trace:
+            for i in range(args.steps):
+                flush.zero_()  # L2 flush (256 MiB > 126 MB L2), outside the step events
+                evs[i][0].record(stream)
+                step()
+                evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    my_ms = sum(step_ms)
+    t = torch.tensor([my_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    tot_ms = float(t.item())
+    status = gdn.device_status(ws)
+    if status != 0:
+        raise RuntimeError("device status %d after timed steps" % status)
+    per_kernel = trace.per_kernel()
+    launches = trace.count
+
+    # ---- e2e: host buffers, H2D + fwd + bwd + D2H inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda x: None if x is None else x.cpu().pin_memory()
+        hin = [pin(x) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta, inp.h0, inp.do, inp.dhT)]
+        din = [d.q, d.k, d.v, d.g, d.beta, d.h0, d.do, d.dhT]
+        houts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+                 for x in (o, hT) + grads]
+        h2d = sum(x.numel() * x.element_size() for x in hin)
+        d2h = sum(x.numel() * x.element_size() for x in houts)
+
+        def e2e_step():
+            for hsrc, ddst in zip(hin, din):
+                ddst.copy_(hsrc, non_blocking=True)
+            step()
+            for dsrc, hdst in zip((o, hT) + grads, houts):
+                hdst.copy_(dsrc, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * B * T * args.steps / (float(te.item()) / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank != 0:
+        return
+    pk = peaks()
+    value = world * B * T * args.steps / (tot_ms / 1e3)
+    # dominant kernel roofline
+    dom = max(per_kernel.items(), key=lambda kv: kv[1][1]) if per_kernel else None
+    roof = None
+    if dom:
+        name, (n, ms) = dom
+        per_launch_s = ms / n / 1e3
+        bound, amount, unit = kernel_work(name, w, n_chunks)
+        if bound == "alu":
+            peak = alu_peak_tflops(pk["sm_mhz"])
+            ach = amount / per_launch_s / 1e12
+            roof = {"kernel": name, "bound": "alu", "achieved": ach, "peak": peak,
+                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                    "peak_source": "derived: 148 SM x 128 fp32 lanes x 2 x %.0f MHz" % pk["sm_mhz"],
+                    "ms_per_launch": per_launch_s * 1e3}
+        elif bound in ("hbm", "tensor"):
+            peak = pk["hbm"] if bound == "hbm" else pk["tc_sus"]
+            ach = amount / per_launch_s / (1e9 if bound == "hbm" else 1e12)
+            roof = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak,
+                    "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": ach / peak,
+                    "traffic": None, "peak_source": pk["src"], "ms_per_launch": per_launch_s * 1e3}
+    sr = step_roofline(w, pk)
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        n_units = oracle_units_for_cores()
+        dt, nu, threads, tk = cpu_oracle_sample(n_units)
+        cpu = {"value": tk / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": "%d (row, head) units x 4096 tokens, fp64 fwd+bwd, %.1f s; tokens/s = "
+                         "units*T/H / s" % (nu, dt)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "gdn_fwdbwd_bf16_B4_T4096_H16_d128", "global_batch": B * world,
+                   "seq_len": T, "heads": H, "head_dim": K, "parallelism": "dp%d" % world,
+                   "l2": "256 MiB memset before each step, outside the step events"},
+        "roofline": roof,
+        "step_roofline": {"bound": sr["bound"], "t_bound_us": sr["t_bound_s"] * 1e6,
+                          "frac": sr["t_bound_s"] / (tot_ms / args.steps / 1e3),
+                          "flops": sr["flops"], "bytes": sr["bytes"],
+                          "peaks": "%s (hbm %.0f GB/s, bf16 sustained %.0f TFLOP/s)"
+                                   % (pk["src"], pk["hbm"], pk["tc_sus"])},
+        "kernels_ms_per_step": {k: v[1] / args.steps for k, v in per_kernel.items()},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,277 @@
+// C ABI of the Gated DeltaNet layer: validation, workspace layout and launch
+// sequencing on the caller's stream.  Declared in include/gdn.h.
+#include <cstring>
+#include <vector>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+bool tc_supported(const Problem &p);
+size_t tc_workspace_bytes(const Problem &p, bool bwd);
+cudaError_t launch_tc_fwd(const Params &p, const Problem &pb, cudaStream_t stream);
+cudaError_t launch_tc_bwd(const Params &p, const Problem &pb, cudaStream_t stream);
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Shape checks that need no pointers.  Fills everything but NC.
+gdn_status describe(const gdn_desc *d, Problem *p) {
+    if (!d) return GDN_ERR_INVALID_ARG;
+    if (d->B < 1 || d->T < 0 || d->H < 1 || d->n_seqs < 0) return GDN_ERR_INVALID_ARG;
+    if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return GDN_ERR_UNSUPPORTED;
+    if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN_ERR_UNSUPPORTED;
+    if (d->n_seqs > 0 && d->B != 1) return GDN_ERR_INVALID_ARG;
+    if (d->B * d->T >= (int64_t(1) << 31) || d->H >= (1 << 16)) return GDN_ERR_INVALID_ARG;
+    if (!(d->scale == d->scale)) return GDN_ERR_INVALID_ARG;  // NaN scale
+    p->B = d->B;
+    p->T = d->T;
+    p->H = d->H;
+    p->K = d->dk;
+    p->V = d->dv;
+    p->BT = d->B * d->T;
+    p->N = d->n_seqs > 0 ? d->n_seqs : d->B;
+    if (p->N >= (int64_t(1) << 30)) return GDN_ERR_INVALID_ARG;
+    p->NCmax = d->n_seqs > 0 ? (d->T + kChunk - 1) / kChunk + d->n_seqs
+                             : d->B * ((d->T + kChunk - 1) / kChunk);
+    p->NC = 0;
+    p->dtype = d->dtype;
+    p->scale = d->scale;
+    return GDN_OK;
+}
+
+bool misaligned(const void *ptr, size_t a = 16) {
+    return ptr && (reinterpret_cast<uintptr_t>(ptr) % a) != 0;
+}
+
+// Host-side check of cu_seqlens; fills p->NC.
+gdn_status check_seqlens(const gdn_desc *d, const int32_t *cu_dev, const int32_t *cu_host,
+                         cudaStream_t stream, Problem *p) {
+    if (d->n_seqs == 0) {
+        if (cu_dev || cu_host) return GDN_ERR_INVALID_ARG;
+        p->NC = p->NCmax;
+        return GDN_OK;
+    }
+    if (!cu_dev) return GDN_ERR_INVALID_ARG;
+    if (misaligned(cu_dev, 4)) return GDN_ERR_ALIGNMENT;
+    std::vector<int32_t> copy;
+    if (!cu_host) {
+        copy.resize((size_t)d->n_seqs + 1);
+        if (cudaMemcpyAsync(copy.data(), cu_dev, sizeof(int32_t) * copy.size(),
+                            cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
+        cu_host = copy.data();
+    }
+    if (cu_host[0] != 0 || cu_host[d->n_seqs] != d->T) return GDN_ERR_INVALID_ARG;
+    int64_t nc = 0;
+    for (int64_t n = 0; n < d->n_seqs; ++n) {
+        const int64_t len = (int64_t)cu_host[n + 1] - cu_host[n];
+        if (len < 0) return GDN_ERR_INVALID_ARG;
+        nc += (len + kChunk - 1) / kChunk;
+    }
+    if (nc > p->NCmax) return GDN_ERR_INVALID_ARG;
+    p->NC = nc;
+    return GDN_OK;
+}
+
+Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout &L,
+                   const int32_t *cu_dev) {
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = (int32_t)pb.B;
+    p.T = (int32_t)pb.T;
+    p.H = (int32_t)pb.H;
+    p.K = (int32_t)pb.K;
+    p.V = (int32_t)pb.V;
+    p.N = (int32_t)pb.N;
+    p.NC = (int32_t)pb.NC;
+    p.BT = pb.BT;
+    p.scale = d->scale;
+    p.bf16 = d->dtype == GDN_BF16;
+    p.cu = d->n_seqs > 0 ? cu_dev : nullptr;
+    char *base = static_cast<char *>(ws);
+    p.hdr = reinterpret_cast<WsHeader *>(base);
+    p.chunks = reinterpret_cast<ChunkInfo *>(base + L.chunks);
+    p.seq_first = reinterpret_cast<int32_t *>(base + L.seq_first);
+    auto f = [&](size_t off) { return off ? reinterpret_cast<float *>(base + off) : nullptr; };
+    p.W = f(L.W);
+    p.Ut = f(L.Ut);
+    p.A = f(L.A);
+    p.U = f(L.U);
+    p.Hs = f(L.Hs);
+    p.dUloc = f(L.dUloc);
+    p.dU = f(L.dU);
+    p.dHn = f(L.dHn);
+    p.scratch = f(L.scratch);
+    p.tc = L.tc ? base + L.tc : nullptr;
+    return p;
+}
+
+bool use_tc(const Problem &pb) { return pb.dtype == GDN_BF16 && tc_supported(pb); }
+
+}  // namespace
+
+// Workspace layout.  The SIMT path (fp32) keeps fp32 per-(chunk, head)
+// intermediates; the tensor-core path (bf16) has its own region.
+Layout make_layout(const Problem &pb, bool bwd) {
+    Layout L;
+    std::memset(&L, 0, sizeof(L));
+    size_t off = kAlign;  // WsHeader
+    L.chunks = off;
+    off += up(sizeof(ChunkInfo) * (size_t)(pb.NCmax > 0 ? pb.NCmax : 1));
+    L.seq_first = off;
+    off += up(sizeof(int32_t) * (size_t)(pb.N + 1));
+    if (use_tc(pb)) {
+        L.tc = off;
+        off += up(tc_workspace_bytes(pb, bwd));
+    } else {
+        const size_t nch = (size_t)pb.NCmax * pb.H, f = sizeof(float);
+        auto take = [&](size_t bytes) {
+            size_t o = off;
+            off += up(bytes);
+            return o;
+        };
+        L.W = take(nch * kChunk * pb.K * f);
+        L.Ut = take(nch * kChunk * pb.V * f);
+        L.A = take(nch * kChunk * kChunk * f);
+        L.U = take(nch * kChunk * pb.V * f);
+        L.Hs = take(nch * pb.K * pb.V * f);
+        if (bwd) {
+            L.dUloc = take(nch * kChunk * pb.V * f);
+            L.dU = take(nch * kChunk * pb.V * f);
+            L.dHn = take(nch * pb.K * pb.V * f);
+        }
+        L.scratch = take((size_t)kSimtSlots * kSimtScratchFloats * f);
+    }
+    L.total = off;
+    return L;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+int gdn_version(void) { return 100; }
+
+int gdn_chunk_size(void) { return kChunk; }
+
+size_t gdn_fwd_workspace_size(const gdn_desc *desc) {
+    Problem pb;
+    if (describe(desc, &pb) != GDN_OK) return 0;
+    return make_layout(pb, false).total;
+}
+
+size_t gdn_bwd_workspace_size(const gdn_desc *desc) {
+    Problem pb;
+    if (describe(desc, &pb) != GDN_OK) return 0;
+    return make_layout(pb, true).total;
+}
+
+gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const void *v,
+                   const float *g, const float *beta, const int32_t *cu_seqlens,
+                   const int32_t *cu_seqlens_host, const float *h0, void *o, float *hT,
+                   void *workspace, size_t workspace_bytes, void *stream) {
+    Problem pb;
+    gdn_status st = describe(desc, &pb);
+    if (st != GDN_OK) return st;
+    if (pb.BT > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
+    for (const void *ptr : {q, k, v, (const void *)g, (const void *)beta, (const void *)h0,
+                            (const void *)o, (const void *)hT})
+        if (misaligned(ptr)) return GDN_ERR_ALIGNMENT;
+    if (!workspace) return GDN_ERR_WORKSPACE;
+    if (misaligned(workspace, kAlign)) return GDN_ERR_ALIGNMENT;
+    const Layout L = make_layout(pb, false);
+    if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = check_seqlens(desc, cu_seqlens, cu_seqlens_host, s, &pb)) != GDN_OK) return st;
+
+    Params p = base_params(pb, desc, workspace, L, cu_seqlens);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.g = g;
+    p.beta = beta;
+    p.h0 = h0;
+    p.o = o;
+    p.hT = hT;
+    if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
+    cudaError_t e = use_tc(pb) ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_bwd(const gdn_desc *desc, const void *q, const void *k, const void *v,
+                   const float *g, const float *beta, const int32_t *cu_seqlens,
+                   const int32_t *cu_seqlens_host, const float *h0, const void *do_,
+                   const float *dhT, void *dq, void *dk, void *dv, float *dg, float *dbeta,
+                   float *dh0, void *workspace, size_t workspace_bytes, void *stream) {
+    Problem pb;
+    gdn_status st = describe(desc, &pb);
+    if (st != GDN_OK) return st;
+    if (pb.BT > 0 && (!q || !k || !v || !g || !beta || !do_ || !dq || !dk || !dv || !dg || !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    for (const void *ptr : {q, k, v, (const void *)g, (const void *)beta, (const void *)h0, do_,
+                            (const void *)dhT, (const void *)dq, (const void *)dk, (const void *)dv,
+                            (const void *)dg, (const void *)dbeta, (const void *)dh0})
+        if (misaligned(ptr)) return GDN_ERR_ALIGNMENT;
+    if (!workspace) return GDN_ERR_WORKSPACE;
+    if (misaligned(workspace, kAlign)) return GDN_ERR_ALIGNMENT;
+    const Layout L = make_layout(pb, true);
+    if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = check_seqlens(desc, cu_seqlens, cu_seqlens_host, s, &pb)) != GDN_OK) return st;
+
+    Params p = base_params(pb, desc, workspace, L, cu_seqlens);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.g = g;
+    p.beta = beta;
+    p.h0 = h0;
+    p.do_ = do_;
+    p.dhT = dhT;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dg = dg;
+    p.dbeta = dbeta;
+    p.dh0 = dh0;
+    if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
+    cudaError_t e = use_tc(pb) ? launch_tc_bwd(p, pb, s) : launch_simt_bwd(p, s);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_device_status(void *workspace, void *stream) {
+    if (!workspace) return GDN_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsHeader h;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (h.status != 0) {
+        const int32_t zero = 0;
+        if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    return h.status == 0 ? GDN_OK : static_cast<gdn_status>(h.status);
+}
+
+const char *gdn_status_string(gdn_status status) {
+    switch (status) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_INVALID_ARG: return "invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case GDN_ERR_ALIGNMENT: return "misaligned pointer";
+    case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+    case GDN_ERR_CUDA: return "CUDA runtime error";
+    case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+// Internal declarations shared by the C ABI (gdn_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "gdn.h"
+
+namespace gdn {
+
+constexpr int kChunk = 64;        // tokens per chunk (the chunkwise form's block length)
+constexpr int kSimtSlots = 512;   // CTAs of the SIMT chunk-parallel kernels (each owns a scratch slot)
+constexpr int kSimtVSlice = 32;   // value columns per CTA in the SIMT state passes
+
+// One chunk of one sequence: tokens [tok0, tok0 + len) of the flattened B*T rows.
+struct ChunkInfo {
+    int32_t seq;  // sequence (dense row or packed document) index
+    int32_t tok0; // first token (flattened over rows)
+    int32_t len;  // 1..64
+    int32_t idx;  // chunk index inside its sequence
+};
+
+// First 256 bytes of every workspace.
+struct WsHeader {
+    int32_t status;    // gdn_status recorded on the device (0 = ok)
+    int32_t n_chunks;  // chunk count the device built
+    int32_t where;     // diagnostic: which wait gave up (0 = none)
+    int32_t pad[61];
+};
+
+// Everything a kernel needs; passed by value.
+struct Params {
+    // problem
+    int32_t B, T, H, K, V, N, NC;  // N sequences, NC chunks (exact, from the host)
+    int64_t BT;                    // tokens over all rows
+    float scale;
+    int32_t bf16;                  // 1: q/k/v/o/do/dq/dk/dv are bf16, 0: fp32
+    // inputs
+    const void *q, *k, *v, *do_;
+    const float *g, *beta, *h0, *dhT;
+    const int32_t *cu;             // device cu_seqlens, or nullptr for dense rows
+    // outputs
+    void *o, *dq, *dk, *dv;
+    float *hT, *dg, *dbeta, *dh0;
+    // workspace
+    WsHeader *hdr;
+    ChunkInfo *chunks;
+    int32_t *seq_first;            // N + 1 entries: first chunk of each sequence
+    // fp32 per-(chunk, head) intermediates of the SIMT path
+    float *W, *Ut, *A, *U, *Hs, *dUloc, *dU, *dHn;
+    float *scratch;                // kSimtSlots slots of kSimtScratchFloats
+    // bf16 tensor-core path intermediates
+    void *tc;                      // base of the tensor-core region
+};
+
+// Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).
+constexpr size_t kSimtScratchFloats = 64 * 128 * 14 + 64 * 64 * 10 + 64 * 8;
+
+// Host-side problem summary after validation.
+struct Problem {
+    int64_t B, T, H, K, V, N, BT;
+    int64_t NCmax;  // capacity used for the workspace layout (depends only on the descriptor)
+    int64_t NC;     // exact chunk count of this call
+    int dtype;
+    float scale;
+};
+
+// Workspace layout: offsets in bytes from the workspace base.
+struct Layout {
+    size_t chunks, seq_first;
+    size_t W, Ut, A, U, Hs, dUloc, dU, dHn, scratch;
+    size_t tc;
+    size_t total;
+};
+
+Layout make_layout(const Problem &p, bool bwd);
+
+// Kernel launchers (all asynchronous on `stream`; return the launch error).
+cudaError_t launch_build_chunks(const Params &p, cudaStream_t stream);
+cudaError_t launch_simt_fwd(const Params &p, cudaStream_t stream);
+cudaError_t launch_simt_bwd(const Params &p, cudaStream_t stream);
+
+// Kernel ids recorded by the launch trace (gdn_trace_install).
+enum KernelId : int32_t {
+    kKBuildChunks = 0,
+    kKSimtPrep,
+    kKSimtStateFwd,
+    kKSimtOut,
+    kKSimtDuloc,
+    kKSimtStateBwd,
+    kKSimtGrads,
+    kKTcPrep,
+    kKTcStateFwd,
+    kKTcOut,
+    kKTcStateBwd,
+    kKTcGrads,
+    kKTcLocal,
+    kKernelCount
+};
+
+// Brackets one launch with the installed trace's events (no-op when none).
+void trace_before(int32_t id, cudaStream_t stream);
+void trace_after(cudaStream_t stream);
+
+// Launches `...` (a kernel<<<>>>(...) expression) inside a trace bracket and
+// returns its launch error from the enclosing function.
+#define GDN_LAUNCH(id, stream, ...)                              \
+    do {                                                         \
+        ::gdn::trace_before((id), (stream));                     \
+        __VA_ARGS__;                                             \
+        ::gdn::trace_after((stream));                            \
+        cudaError_t gdn_launch_err_ = cudaGetLastError();        \
+        if (gdn_launch_err_ != cudaSuccess) return gdn_launch_err_; \
+    } while (0)
+
+// Device-side status codes written into WsHeader::status.
+enum : int32_t { kDevOk = 0, kDevBadSeqlens = GDN_ERR_INVALID_ARG, kDevTimeout = GDN_ERR_TIMEOUT };
+
+}  // namespace gdn

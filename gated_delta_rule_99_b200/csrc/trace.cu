@@ -1,0 +1,48 @@
+// Optional per-launch CUDA-event tracing (see gdn_trace_install in gdn.h).
+#include "gdn_internal.cuh"
+
+namespace gdn {
+namespace {
+thread_local gdn_trace *g_trace = nullptr;
+thread_local bool g_open = false;
+
+const char *const kNames[kKernelCount] = {
+    "build_chunks", "simt_prep", "simt_state_fwd", "simt_out", "simt_duloc", "simt_state_bwd",
+    "simt_grads", "tc_prep", "tc_state_fwd", "tc_out", "tc_state_bwd", "tc_grads", "tc_local"};
+}  // namespace
+
+void trace_before(int32_t id, cudaStream_t stream) {
+    gdn_trace *t = g_trace;
+    g_open = false;
+    if (!t) return;
+    if (t->count >= t->capacity) {
+        ++t->dropped;
+        return;
+    }
+    t->kernel_ids[t->count] = id;
+    cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * t->count]), stream);
+    g_open = true;
+}
+
+void trace_after(cudaStream_t stream) {
+    gdn_trace *t = g_trace;
+    if (!t || !g_open) return;
+    cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * t->count + 1]), stream);
+    ++t->count;
+    g_open = false;
+}
+
+}  // namespace gdn
+
+extern "C" {
+
+void gdn_trace_install(gdn_trace *trace) {
+    gdn::g_trace = trace;
+    gdn::g_open = false;
+}
+
+const char *gdn_kernel_name(int32_t id) {
+    return (id >= 0 && id < gdn::kKernelCount) ? gdn::kNames[id] : "?";
+}
+
+}  // extern "C"

@@ -81,7 +81,16 @@ def _segments(B, T, cu_seqlens):
 
 
 def _f64(x):
-    return None if x is None else np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    """Contiguous fp64 numpy copy of a numpy array or a CPU torch tensor (bf16 upcasts exactly)."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _shape(x):
+    return tuple(x.shape)
 
 
 def _ptr(a):
@@ -94,9 +103,8 @@ def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, units=None, n
 
     ``units``: optional iterable of (sequence, head) pairs to compute; the
     other entries of o and hT are left NaN (used for sampled parity)."""
-    q, k, v, g, beta, h0 = map(_f64, (q, k, v, g, beta, h0))
-    B, T, H, K = q.shape
-    V = v.shape[-1]
+    B, T, H, K = _shape(q)
+    V = _shape(v)[-1]
     segs = _segments(B, T, cu_seqlens)
     N = len(segs)
     o = np.full((B, T, H, V), np.nan)
@@ -106,10 +114,9 @@ def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, units=None, n
     for i, (n, h) in enumerate(sel):
         b, t0, t1 = segs[n]
         L = t1 - t0
-        bufs = dict(q=np.ascontiguousarray(q[b, t0:t1, h]), k=np.ascontiguousarray(k[b, t0:t1, h]),
-                    v=np.ascontiguousarray(v[b, t0:t1, h]), g=np.ascontiguousarray(g[b, t0:t1, h]),
-                    beta=np.ascontiguousarray(beta[b, t0:t1, h]),
-                    h0=None if h0 is None else np.ascontiguousarray(h0[n, h]),
+        bufs = dict(q=_f64(q[b, t0:t1, h]), k=_f64(k[b, t0:t1, h]), v=_f64(v[b, t0:t1, h]),
+                    g=_f64(g[b, t0:t1, h]), beta=_f64(beta[b, t0:t1, h]),
+                    h0=None if h0 is None else _f64(h0[n, h]),
                     o=np.zeros((max(L, 1), V)), hT=np.zeros((K, V)))
         keep.append(bufs)
         arr[i] = _Unit(L, *[_ptr(bufs.get(f)) for f in
@@ -128,9 +135,8 @@ def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0,
             nthreads=None):
     """Token-by-token backward of o and hT with upstream gradients do (B,T,H,V)
     and dhT (N,H,K,V) or None.  Returns dq, dk, dv, dg, dbeta, dh0 in fp64."""
-    q, k, v, g, beta, do, h0, dhT = map(_f64, (q, k, v, g, beta, do, h0, dhT))
-    B, T, H, K = q.shape
-    V = v.shape[-1]
+    B, T, H, K = _shape(q)
+    V = _shape(v)[-1]
     segs = _segments(B, T, cu_seqlens)
     N = len(segs)
     out = dict(dq=np.full((B, T, H, K), np.nan), dk=np.full((B, T, H, K), np.nan),
@@ -141,7 +147,7 @@ def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0,
     for i, (n, h) in enumerate(sel):
         b, t0, t1 = segs[n]
         L = max(t1 - t0, 1)
-        c = np.ascontiguousarray
+        c = _f64
         bufs = dict(q=c(q[b, t0:t1, h]), k=c(k[b, t0:t1, h]), v=c(v[b, t0:t1, h]),
                     g=c(g[b, t0:t1, h]), beta=c(beta[b, t0:t1, h]),
                     h0=None if h0 is None else c(h0[n, h]),

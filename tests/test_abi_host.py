@@ -1,0 +1,132 @@
+"""Host-side tests of the C ABI: the library loads, exports what include/gdn.h
+declares, sizes workspaces, and rejects bad arguments before launching
+anything (these calls never touch a GPU: validation fails first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_99_b200 as gdn
+from gated_delta_rule_99_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x7F0000000000  # a 256-byte aligned address that is never dereferenced
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    L = gdn.lib()
+    names = header_functions()
+    assert set(names) == set(B.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_chunk():
+    assert gdn.lib().gdn_version() >= 100
+    assert gdn.lib().gdn_chunk_size() == 64
+
+
+def test_status_strings():
+    L = gdn.lib()
+    for code, s in B.STATUS.items():
+        assert L.gdn_status_string(code).decode() == s
+    assert L.gdn_status_string(99).decode() == "unknown status"
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(dk=96), 2), (dict(dv=32), 2), (dict(dtype=7), 2), (dict(B=0), 1), (dict(H=0), 1),
+    (dict(T=-1), 1), (dict(n_seqs=3, B=2), 1), (dict(B=1 << 20, T=1 << 12), 1)])
+def test_workspace_size_rejects_bad_descriptors(bad, code):
+    args = dict(B=2, T=100, H=3, dk=64, dv=128, n_seqs=0, dtype=0, scale=1.0)
+    args.update(bad)
+    d = gdn.make_desc(**args)
+    assert gdn.fwd_workspace_size(d) == 0 and gdn.bwd_workspace_size(d) == 0
+    rc = _fwd(d, ws_bytes=1 << 40)
+    assert rc == code
+
+
+def test_workspace_sizes_grow():
+    a = gdn.fwd_workspace_size(gdn.make_desc(1, 64, 1, 64, 64))
+    b = gdn.fwd_workspace_size(gdn.make_desc(1, 128, 1, 64, 64))
+    c = gdn.bwd_workspace_size(gdn.make_desc(1, 128, 1, 64, 64))
+    assert 0 < a < b <= c
+    for dt in (0, 1):
+        d = gdn.make_desc(4, 4096, 16, 128, 128, dtype=dt)
+        assert gdn.bwd_workspace_size(d) >= gdn.fwd_workspace_size(d) > 0
+
+
+def _fwd(d, ws_bytes=None, ptrs=None, cu=None, cu_host=None, ws=FAKE):
+    L = gdn.lib()
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, h0=None, o=FAKE, hT=None)
+    p.update(ptrs or {})
+    if ws_bytes is None:
+        ws_bytes = gdn.fwd_workspace_size(d)
+    return L.gdn_fwd(ctypes.byref(d), p["q"], p["k"], p["v"], p["g"], p["beta"], cu, cu_host,
+                     p["h0"], p["o"], p["hT"], ws, ws_bytes, None)
+
+
+def _bwd(d, ptrs=None, ws_bytes=None):
+    L = gdn.lib()
+    names = ("q", "k", "v", "g", "beta", "h0", "do", "dhT", "dq", "dk", "dv", "dg", "dbeta", "dh0")
+    p = {n: FAKE for n in names}
+    p.update(h0=None, dhT=None, dh0=None)
+    p.update(ptrs or {})
+    if ws_bytes is None:
+        ws_bytes = gdn.bwd_workspace_size(d)
+    return L.gdn_bwd(ctypes.byref(d), p["q"], p["k"], p["v"], p["g"], p["beta"], None, None,
+                     p["h0"], p["do"], p["dhT"], p["dq"], p["dk"], p["dv"], p["dg"], p["dbeta"],
+                     p["dh0"], FAKE, ws_bytes, None)
+
+
+def test_null_and_misaligned_pointers():
+    d = gdn.make_desc(2, 100, 3, 64, 128)
+    assert _fwd(d, ptrs=dict(q=None)) == 1
+    assert _fwd(d, ptrs=dict(o=None)) == 1
+    assert _fwd(d, ptrs=dict(v=FAKE + 8)) == 3
+    assert _fwd(d, ptrs=dict(hT=FAKE + 4)) == 3
+    assert _fwd(d, ws=FAKE + 16) == 3
+    assert _fwd(d, ws=None) == 4
+    assert _bwd(d, ptrs=dict(dbeta=None)) == 1
+    assert _bwd(d, ptrs=dict(do=None)) == 1
+    assert _bwd(d, ptrs=dict(dh0=FAKE + 2)) == 3
+
+
+def test_workspace_too_small():
+    d = gdn.make_desc(2, 100, 3, 64, 128)
+    assert _fwd(d, ws_bytes=gdn.fwd_workspace_size(d) - 1) == 4
+    assert _bwd(d, ws_bytes=gdn.bwd_workspace_size(d) - 1) == 4
+
+
+def _cu(vals):
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return arr
+
+
+@pytest.mark.parametrize("cu", [[0, 50, 40, 100], [1, 50, 100], [0, 50, 99], [0, 50, 101]])
+def test_bad_seqlens_rejected_on_host(cu):
+    d = gdn.make_desc(1, 100, 2, 64, 64, n_seqs=len(cu) - 1)
+    host = _cu(cu)
+    assert _fwd(d, cu=FAKE, cu_host=ctypes.cast(host, ctypes.c_void_p)) == 1
+
+
+def test_seqlens_require_single_row_and_device_copy():
+    d = gdn.make_desc(1, 100, 2, 64, 64, n_seqs=2)
+    host = _cu([0, 40, 100])
+    assert _fwd(d, cu=None, cu_host=ctypes.cast(host, ctypes.c_void_p)) == 1
+    dense = gdn.make_desc(1, 100, 2, 64, 64)
+    assert _fwd(dense, cu=FAKE, cu_host=ctypes.cast(host, ctypes.c_void_p)) == 1
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16)
+    g = torch.zeros(1, 8, 1)
+    with pytest.raises(ValueError):
+        gdn.gdn_fwd(x, x, x, g, g)

@@ -1,0 +1,188 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (max-normalised error per tensor, max|x - ref| / max|ref|): 1e-4
+for fp32 inputs and 2e-2 for bf16 inputs with fp32 state and accumulation.
+Small cases compare every element; the full-size workloads compare the
+sampled (sequence, head) units the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_99_b200 as gdn
+from gated_delta_rule_99_b200.inputs import make_inputs, workload
+
+from _util import maxnorm_err, np64, oracle_bwd, oracle_fwd, unit_mask
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-4, "bf16": 2e-2}
+
+
+def run_fwd(inp, **kw):
+    d = inp.to("cuda")
+    cu = None if d.cu_seqlens is None else d.cu_seqlens
+    o, hT = gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=cu, h0=d.h0, scale=d.scale, **kw)
+    torch.cuda.synchronize()
+    return o, hT
+
+
+def run_bwd(inp, **kw):
+    d = inp.to("cuda")
+    cu = None if d.cu_seqlens is None else d.cu_seqlens
+    r = gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, cu_seqlens=cu, h0=d.h0, dhT=d.dhT,
+                    scale=d.scale, **kw)
+    torch.cuda.synchronize()
+    return r
+
+
+def check_all(inp, tol, units=None, bwd=True):
+    o, hT = run_fwd(inp)
+    ro, rh = oracle_fwd(inp, units)
+    errs = {"o": maxnorm_err(o, ro), "hT": maxnorm_err(hT, rh)}
+    if bwd:
+        got = run_bwd(inp)
+        ref = oracle_bwd(inp, units)
+        for name, a, b in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), got, ref):
+            errs[name] = maxnorm_err(a, b)
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (errs, tol)
+    return errs
+
+
+def test_tiny_fp32_forward_config():
+    inp = workload(0)
+    errs = check_all(inp, TOL["fp32"], bwd=False)
+    assert errs["o"] < 1e-5
+
+
+def test_fp32_forward_backward_with_states():
+    inp = make_inputs(B=2, T=200, H=2, K=64, V=64, dtype="fp32", seed=10)
+    check_all(inp, TOL["fp32"])
+
+
+def test_fp32_scale_and_mixed_head_dims():
+    inp = make_inputs(B=1, T=150, H=3, K=64, V=128, dtype="fp32", seed=11, scale=0.125)
+    check_all(inp, TOL["fp32"])
+    inp = make_inputs(B=1, T=90, H=1, K=128, V=64, dtype="fp32", seed=12)
+    check_all(inp, TOL["fp32"])
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_packed_ragged_documents(dtype):
+    lengths = [1, 0, 63, 64, 65, 130, 7, 200]
+    inp = make_inputs(B=1, T=sum(lengths), H=3, K=64, V=128, dtype=dtype, seed=13,
+                      lengths=lengths)
+    check_all(inp, TOL[dtype])
+
+
+def test_bf16_ragged_dense_rows():
+    inp = make_inputs(B=2, T=300, H=2, K=128, V=128, dtype="bf16", seed=14)
+    check_all(inp, TOL["bf16"])
+
+
+def test_fp32_strong_decay_and_unit_strength():
+    inp = make_inputs(B=1, T=256, H=2, K=64, V=64, dtype="fp32", seed=15, gate_scale=3.0)
+    inp.beta.fill_(1.0)
+    check_all(inp, TOL["fp32"])
+
+
+def _sampled(idx, units, bwd):
+    inp = workload(idx, bwd=bwd)
+    errs = check_all(inp, TOL[inp.meta["dtype"]], units=units, bwd=bwd)
+    return errs
+
+
+def test_full_size_forward_bf16_sampled():
+    _sampled(1, [(0, 0), (3, 15), (1, 7)], bwd=False)
+
+
+def test_full_size_forward_backward_bf16_sampled():
+    _sampled(2, [(0, 0), (3, 15), (2, 9)], bwd=True)
+
+
+def test_full_size_packed_forward_backward_sampled():
+    inp = workload(3)
+    n = inp.n_seqs
+    _sampled(3, [(0, 0), (n - 1, 15), (n // 2, 5)], bwd=True)
+
+
+def test_long_context_chained_halves_and_prefix():
+    inp = workload(4, device="cuda")
+    T, Th = inp.q.shape[1], inp.q.shape[1] // 2
+    o, hT = gdn.gdn_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, h0=inp.h0)
+    oa, ha = gdn.gdn_fwd(inp.q[:, :Th].contiguous(), inp.k[:, :Th].contiguous(),
+                         inp.v[:, :Th].contiguous(), inp.g[:, :Th].contiguous(),
+                         inp.beta[:, :Th].contiguous(), h0=inp.h0)
+    ob, hb = gdn.gdn_fwd(inp.q[:, Th:].contiguous(), inp.k[:, Th:].contiguous(),
+                         inp.v[:, Th:].contiguous(), inp.g[:, Th:].contiguous(),
+                         inp.beta[:, Th:].contiguous(), h0=ha)
+    torch.cuda.synchronize()
+    assert torch.equal(o[:, :Th], oa) and torch.equal(o[:, Th:], ob)
+    assert torch.equal(hT, hb)
+    # prefix parity: outputs of the first P tokens depend only on those tokens
+    P = 4096
+    cpu = lambda x: x[:, :P].cpu()
+    import oracle
+    ro, _ = oracle.gdn_fwd(cpu(inp.q), cpu(inp.k), cpu(inp.v), cpu(inp.g), cpu(inp.beta),
+                           h0=inp.h0.cpu(), units=[(0, 0), (0, 7)])
+    got = np64(o[:, :P].cpu())
+    m = np.isfinite(ro)
+    assert maxnorm_err(got[m], ro[m]) < TOL["bf16"]
+    del o, oa, ob
+    torch.cuda.empty_cache()
+
+
+def test_packed_equals_per_document_runs_bitwise():
+    lengths = [70, 1, 128, 0, 33]
+    inp = make_inputs(B=1, T=sum(lengths), H=2, K=128, V=128, dtype="bf16", seed=16,
+                      lengths=lengths)
+    o, hT = run_fwd(inp)
+    got = run_bwd(inp)
+    cu = inp.cu_seqlens.tolist()
+    for n in range(len(lengths)):
+        t0, t1 = cu[n], cu[n + 1]
+        sl = lambda x: x[:, t0:t1].contiguous()
+        sub = inp.to("cpu")
+        sub.q, sub.k, sub.v, sub.g, sub.beta, sub.do = map(sl, (inp.q, inp.k, inp.v, inp.g,
+                                                                 inp.beta, inp.do))
+        sub.h0 = inp.h0[n:n + 1].contiguous()
+        sub.dhT = inp.dhT[n:n + 1].contiguous()
+        sub.cu_seqlens = None
+        on, hn = run_fwd(sub)
+        assert torch.equal(o[:, t0:t1], on)
+        assert torch.equal(hT[n:n + 1], hn)
+        gn = run_bwd(sub)
+        for a, b in zip(got[:5], gn[:5]):
+            assert torch.equal(a[:, t0:t1], b)
+        assert torch.equal(got[5][n:n + 1], gn[5])
+
+
+def test_run_to_run_determinism():
+    inp = make_inputs(B=2, T=500, H=4, K=128, V=128, dtype="bf16", seed=17)
+    a = run_fwd(inp) + run_bwd(inp)
+    b = run_fwd(inp) + run_bwd(inp)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_empty_inputs_pass_state_through():
+    inp = make_inputs(B=2, T=0, H=2, K=64, V=64, dtype="bf16", seed=18)
+    o, hT = run_fwd(inp)
+    assert o.numel() == 0 and torch.equal(hT.cpu(), inp.h0)
+    *_, dh0 = run_bwd(inp)
+    assert torch.equal(dh0.cpu(), inp.dhT)
+
+
+def test_device_side_seqlens_check():
+    lengths = [100, 100]
+    inp = make_inputs(B=1, T=200, H=1, K=64, V=64, dtype="bf16", seed=19, lengths=lengths)
+    d = inp.to("cuda")
+    bad_dev = torch.tensor([0, 201, 200], dtype=torch.int32, device="cuda")
+    ws = gdn.alloc_workspace(gdn.fwd_workspace_size(gdn.make_desc(1, 200, 1, 64, 64, 2)), "cuda")
+    gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=bad_dev,
+                cu_seqlens_host=inp.cu_seqlens, h0=d.h0, workspace=ws)
+    assert gdn.device_status(ws) == 1
+    gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=d.cu_seqlens.cuda(),
+                cu_seqlens_host=inp.cu_seqlens, h0=d.h0, workspace=ws)
+    assert gdn.device_status(ws) == 0
