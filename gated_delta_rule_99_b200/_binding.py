@@ -212,6 +212,9 @@ class LaunchTrace:
         self.capacity = int(capacity)
         self.torch_events = [torch.cuda.Event(enable_timing=True)
                              for _ in range(2 * self.capacity)]
+        for e in self.torch_events:  # torch creates the CUDA event on first record
+            e.record()
+        torch.cuda.current_stream().synchronize()
         self._ev = (ctypes.c_void_p * (2 * self.capacity))(
             *[e.cuda_event for e in self.torch_events])
         self._ids = (ctypes.c_int32 * self.capacity)()

@@ -20,15 +20,24 @@ void trace_before(int32_t id, cudaStream_t stream) {
         return;
     }
     t->kernel_ids[t->count] = id;
-    cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * t->count]), stream);
+    if (cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * t->count]), stream) != cudaSuccess) {
+        cudaGetLastError();  // a bad event must not look like a failed launch
+        ++t->dropped;
+        return;
+    }
     g_open = true;
 }
 
 void trace_after(cudaStream_t stream) {
     gdn_trace *t = g_trace;
     if (!t || !g_open) return;
-    cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * t->count + 1]), stream);
-    ++t->count;
+    if (cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * t->count + 1]), stream) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        ++t->dropped;
+    } else {
+        ++t->count;
+    }
     g_open = false;
 }
 
