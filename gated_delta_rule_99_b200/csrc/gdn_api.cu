@@ -145,7 +145,9 @@ Layout make_layout(const Problem &pb, bool bwd) {
             L.dU = take(nch * kChunk * pb.V * f);
             L.dHn = take(nch * pb.K * pb.V * f);
         }
-        L.scratch = take((size_t)kSimtSlots * kSimtScratchFloats * f);
+        // one scratch slot per CTA of the chunk-parallel kernels (grid = min(NC*H, kSimtSlots))
+        const size_t slots = nch < (size_t)kSimtSlots ? (nch > 0 ? nch : 1) : (size_t)kSimtSlots;
+        L.scratch = take(slots * kSimtScratchFloats * f);
     }
     L.total = off;
     return L;
