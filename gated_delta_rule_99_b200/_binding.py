@@ -20,7 +20,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "mi
           4: "workspace missing or too small", 5: "CUDA runtime error",
           6: "device-side wait timed out"}
 EXPORTS = ("gdn_version", "gdn_chunk_size", "gdn_fwd_workspace_size", "gdn_bwd_workspace_size",
-           "gdn_fwd", "gdn_bwd", "gdn_device_status", "gdn_status_string", "gdn_trace_install",
+           "gdn_fwd", "gdn_fwd_noalloc", "gdn_bwd", "gdn_device_status", "gdn_status_string", "gdn_trace_install",
            "gdn_kernel_name")
 
 
@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
                 getattr(L, n).argtypes = [dp]
             L.gdn_fwd.restype = ctypes.c_int
             L.gdn_fwd.argtypes = [dp, vp, vp, vp, fp, fp, i32p, i32p, fp, vp, fp, vp, sz, vp]
+            L.gdn_fwd_noalloc.restype = ctypes.c_int
+            L.gdn_fwd_noalloc.argtypes = [dp, vp, vp, vp, fp, fp, i32p, i32p, fp, vp, fp, vp]
             L.gdn_bwd.restype = ctypes.c_int
             L.gdn_bwd.argtypes = [dp, vp, vp, vp, fp, fp, i32p, i32p, fp, vp, fp, vp, vp, vp, fp,
                                   fp, fp, vp, sz, vp]

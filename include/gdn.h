@@ -101,6 +101,28 @@ gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const voi
                    const int32_t *cu_seqlens_host, const float *h0, void *o, float *hT,
                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* Forward for callers that cannot allocate device memory (no counterpart in
+ * the pages describing the method: it is a packaging variant of gdn_fwd).
+ * A caller whose device memory is all owned elsewhere -- a serving process
+ * that reserved HBM in a fixed pool at start-up and may not call cudaMalloc
+ * while serving, or a plugin handed only its input and output buffers --
+ * passes the same arguments as gdn_fwd minus the workspace.  The scratch is a
+ * static device array of GDN_NOALLOC_MAX_WORKSPACE bytes inside the library;
+ * every GPU that loads the library keeps it until the process exits.
+ * Problems whose gdn_fwd_workspace_size exceeds that return
+ * GDN_ERR_WORKSPACE (use gdn_fwd with your own workspace instead).  The first
+ * call on each device looks up the array's device address with that device
+ * current, so make the first call before any stream capture.  All calls share
+ * the one array: calls that overlap on the GPU (other streams, other host
+ * threads) race and corrupt each other's results, so serialise them.  Device-
+ * side status is not reported for this entry point.  No allocation of any
+ * kind is made. */
+#define GDN_NOALLOC_MAX_WORKSPACE (64u * 1024u * 1024u)
+gdn_status gdn_fwd_noalloc(const gdn_desc *desc, const void *q, const void *k, const void *v,
+                           const float *g, const float *beta, const int32_t *cu_seqlens,
+                           const int32_t *cu_seqlens_host, const float *h0, void *o, float *hT,
+                           void *stream);
+
 /* Backward of (o, hT) given do_ and dhT (NULL means zero): writes dq, dk, dv,
  * dg, dbeta and dh0 (dh0 may be NULL to skip it).  The per-chunk states are
  * recomputed from the inputs, not read from a forward call. */
