@@ -7,11 +7,6 @@
 
 namespace gdn {
 
-bool tc_supported(const Problem &p);
-size_t tc_workspace_bytes(const Problem &p, bool bwd);
-cudaError_t launch_tc_fwd(const Params &p, const Problem &pb, cudaStream_t stream);
-cudaError_t launch_tc_bwd(const Params &p, const Problem &pb, cudaStream_t stream);
-
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -107,11 +102,24 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.dU = f(L.dU);
     p.dHn = f(L.dHn);
     p.scratch = f(L.scratch);
-    p.tc = L.tc ? base + L.tc : nullptr;
+    auto b = [&](size_t off) { return off ? static_cast<void *>(base + off) : nullptr; };
+    p.tW = b(L.tW);
+    p.tUt = b(L.tUt);
+    p.tKd = b(L.tKd);
+    p.tS = b(L.tS);
+    p.tUT = b(L.tUT);
+    p.tQg = b(L.tQg);
+    p.tdUL = b(L.tdUL);
+    p.tdSn = b(L.tdSn);
+    p.tdUT = b(L.tdUT);
+    p.tG = f(L.tG);
+    p.tA = f(L.tA);
     return p;
 }
 
-bool use_tc(const Problem &pb) { return pb.dtype == GDN_BF16 && tc_supported(pb); }
+bool use_tc(const Problem &pb, bool bwd) {
+    return pb.dtype == GDN_BF16 && tc_supported(pb) && (!bwd || tc_bwd_ready());
+}
 
 }  // namespace
 
@@ -125,16 +133,29 @@ Layout make_layout(const Problem &pb, bool bwd) {
     off += up(sizeof(ChunkInfo) * (size_t)(pb.NCmax > 0 ? pb.NCmax : 1));
     L.seq_first = off;
     off += up(sizeof(int32_t) * (size_t)(pb.N + 1));
-    if (use_tc(pb)) {
-        L.tc = off;
-        off += up(tc_workspace_bytes(pb, bwd));
+    const size_t nch = (size_t)pb.NCmax * pb.H, f = sizeof(float);
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += up(bytes > 0 ? bytes : 1);
+        return o;
+    };
+    if (use_tc(pb, bwd)) {
+        // bf16 tile images per (chunk, head); d_k = d_v = 128
+        const size_t img64 = (size_t)kChunk * 128 * 2, img128 = (size_t)128 * 128 * 2;
+        L.tW = take(nch * img64);
+        L.tUt = take(nch * img64);
+        L.tKd = take(nch * img64);
+        L.tG = take(nch * kChunk * f);
+        L.tS = take(nch * img128);
+        L.tUT = take(nch * img64);
+        if (bwd) {
+            L.tA = take(nch * kChunk * kChunk * f);
+            L.tQg = take(nch * img64);
+            L.tdUL = take(nch * img64);
+            L.tdSn = take(nch * img128);
+            L.tdUT = take(nch * img64);
+        }
     } else {
-        const size_t nch = (size_t)pb.NCmax * pb.H, f = sizeof(float);
-        auto take = [&](size_t bytes) {
-            size_t o = off;
-            off += up(bytes);
-            return o;
-        };
         L.W = take(nch * kChunk * pb.K * f);
         L.Ut = take(nch * kChunk * pb.V * f);
         L.A = take(nch * kChunk * kChunk * f);
@@ -203,7 +224,7 @@ gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.o = o;
     p.hT = hT;
     if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
-    cudaError_t e = use_tc(pb) ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
+    cudaError_t e = use_tc(pb, false) ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -244,7 +265,7 @@ gdn_status gdn_bwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.dbeta = dbeta;
     p.dh0 = dh0;
     if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
-    cudaError_t e = use_tc(pb) ? launch_tc_bwd(p, pb, s) : launch_simt_bwd(p, s);
+    cudaError_t e = use_tc(pb, true) ? launch_tc_bwd(p, pb, s) : launch_simt_bwd(p, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -52,8 +52,12 @@ struct Params {
     // fp32 per-(chunk, head) intermediates of the SIMT path
     float *W, *Ut, *A, *U, *Hs, *dUloc, *dU, *dHn;
     float *scratch;                // kSimtSlots slots of kSimtScratchFloats
-    // bf16 tensor-core path intermediates
-    void *tc;                      // base of the tensor-core region
+    // bf16 tensor-core path intermediates, per (chunk, head): tile images
+    // (128-byte-swizzled, as the MMAs read them) and plain rows
+    void *tW, *tUt, *tKd;          // 64x128 W image, 64x128 Ut rows, 64x128 diag(e)K image
+    void *tS, *tUT;                // 128x128 image of the state entering the chunk, 128x64 U^T image
+    void *tQg, *tdUL, *tdSn, *tdUT;  // backward: scaled-q image, local dU^T, dS image, dU^T image
+    float *tG, *tA;                // 64 cumulative gates; 64x64 fp32 A (backward)
 };
 
 // Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).
@@ -72,7 +76,7 @@ struct Problem {
 struct Layout {
     size_t chunks, seq_first;
     size_t W, Ut, A, U, Hs, dUloc, dU, dHn, scratch;
-    size_t tc;
+    size_t tW, tUt, tKd, tS, tUT, tQg, tdUL, tdSn, tdUT, tG, tA;
     size_t total;
 };
 
@@ -82,6 +86,10 @@ Layout make_layout(const Problem &p, bool bwd);
 cudaError_t launch_build_chunks(const Params &p, cudaStream_t stream);
 cudaError_t launch_simt_fwd(const Params &p, cudaStream_t stream);
 cudaError_t launch_simt_bwd(const Params &p, cudaStream_t stream);
+bool tc_supported(const Problem &p);
+bool tc_bwd_ready();
+cudaError_t launch_tc_fwd(const Params &p, const Problem &pb, cudaStream_t stream);
+cudaError_t launch_tc_bwd(const Params &p, const Problem &pb, cudaStream_t stream);
 
 // Kernel ids recorded by the launch trace (gdn_trace_install).
 enum KernelId : int32_t {

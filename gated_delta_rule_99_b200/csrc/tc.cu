@@ -1,11 +1,545 @@
-// Tensor-core (tcgen05) path of the bf16 layer.  Filled in after the SIMT path is green.
+// Tensor-core (tcgen05) path of the bf16 layer, d_k = d_v = 128.
+//
+// Same chunkwise algebra as the fp32 path (chunk of 64 tokens; H = S^T the
+// state entering a chunk; G the in-chunk cumulative log-decay):
+//
+//   A = (I + strict_lower(diag(b) K K^T . Gam))^-1 ; W = A diag(b gam) K ; Ut = A diag(b) V
+//   U = Ut - W H ;  H' = gam_n H + (diag(e) K)^T U ;  O = diag(gam) Q' H + lower(Q' K^T . Gam) U
+//
+// Every product runs on tcgen05 (bf16 operands in 128-byte-swizzled shared
+// memory, fp32 accumulators in TMEM).  The state chain runs in transposed
+// form so its accumulators use all 128 TMEM lanes: thread v of the state
+// kernel owns row v of S = H^T in fp32 registers, and per chunk
+//
+//   U^T = Ut^T - S W^T        (M = 128 rows v, N = 64 tokens, K = 128)
+//   S  <- gam_n S + U^T Kd    (M = 128 rows v, N = 128 keys,  K = 64 tokens)
+//
+// Kernels: tc_prep (chunk-parallel: gates, K K^T, forward substitution for A
+// in fp32, W, Ut, Kd = diag(e) K), tc_state_fwd (serial over the chunks of a
+// sequence; one CTA per (sequence, head); writes the state entering every
+// chunk and U^T as swizzled tile images), tc_out (chunk-parallel output).
 #include "gdn_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdn {
+namespace {
 
-bool tc_supported(const Problem &) { return false; }
-size_t tc_workspace_bytes(const Problem &, bool) { return 0; }
-cudaError_t launch_tc_fwd(const Params &, const Problem &, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_tc_bwd(const Params &, const Problem &, cudaStream_t) { return cudaErrorNotSupported; }
+using namespace ptx;
+using bf16 = __nv_bfloat16;
+
+constexpr int C = kChunk;      // 64
+constexpr int D = 128;         // d_k = d_v
+constexpr int NT = 128;        // threads per CTA
+constexpr uint32_t kWaitLimit = 1u << 23;
+
+constexpr size_t kImg64 = (size_t)C * D * 2;   // 64 x 128 bf16 tile image (16 KB)
+constexpr size_t kImg128 = (size_t)D * D * 2;  // 128 x 128 (32 KB)
+constexpr size_t kImgUT = (size_t)D * C * 2;   // 128 x 64 (16 KB)
+
+__device__ __forceinline__ uint8_t *align1k(uint8_t *p) {
+    return (uint8_t *)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+__device__ void record_timeout(const Params &p, int where) {
+    atomicExch(&p.hdr->status, kDevTimeout);
+    atomicExch(&p.hdr->where, where);
+}
+
+// Bounded wait on an MMA-completion barrier, decided uniformly by the CTA.
+__device__ __forceinline__ bool cta_wait(uint64_t *mbar, uint32_t parity, const Params &p,
+                                         int where) {
+    const bool ok = mbar_wait(mbar, parity, kWaitLimit);
+    const bool all_ok = __syncthreads_and(ok);
+    if (!all_ok && threadIdx.x == 0) record_timeout(p, where);
+    tc_fence_after();
+    return all_ok;
+}
+
+// Barrier that orders generic smem writes (operands) before MMAs issued after it.
+__device__ __forceinline__ void operands_ready() {
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+// Loads rows [0, 64) of one chunk and head of a [tokens][H][128] bf16 tensor
+// into an SW128 tile with R rows (block stride), starting at row `row0`;
+// rows at or past `len` are zero.  Asynchronous (cp.async).
+__device__ __forceinline__ void load_rows_async(uint8_t *tile, int R, int row0, const bf16 *src,
+                                                int64_t tok0, int len, int h, int H) {
+    const uint32_t base = smem_u32(tile);
+    for (int t = threadIdx.x; t < C * 16; t += NT) {
+        const int r = t >> 4, j = t & 15;
+        const bool valid = r < len;
+        const bf16 *g = valid ? src + ((tok0 + r) * H + h) * D + j * 8 : src;
+        cp_async16_zfill(base + sw128_chunk(R, row0 + r, j), g, valid);
+    }
+}
+
+// Linear copy of a tile image (bytes multiple of 16 * NT).
+__device__ __forceinline__ void load_image_async(uint8_t *tile, const void *img, size_t bytes) {
+    const uint32_t base = smem_u32(tile);
+    const uint8_t *g = static_cast<const uint8_t *>(img);
+    for (size_t off = (size_t)threadIdx.x * 16; off < bytes; off += NT * 16)
+        cp_async16(base + (uint32_t)off, g + off);
+}
+
+// In-chunk cumulative log-decay (zero gates past len), summed in token order by
+// one thread so every kernel gets bit-identical values; also the write strengths.
+__device__ void chunk_gates(float *G, float *bta, const Params &p, const ChunkInfo &ci, int h) {
+    const int r = threadIdx.x;
+    if (r < C) {
+        const int64_t idx = (int64_t)(ci.tok0 + r) * p.H + h;
+        G[r] = r < ci.len ? p.g[idx] : 0.f;
+        if (bta) bta[r] = r < ci.len ? p.beta[idx] : 0.f;
+    }
+    __syncthreads();
+    if (r == 0) {
+        float s = 0.f;
+        for (int i = 0; i < C; ++i) {
+            s += G[i];
+            G[i] = s;
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float *f) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float *f) {
+    uint4 u;
+    u.x = pack_bf16(f[0], f[1]);
+    u.y = pack_bf16(f[2], f[3]);
+    u.z = pack_bf16(f[4], f[5]);
+    u.w = pack_bf16(f[6], f[7]);
+    return u;
+}
+
+// TMEM address of (lane base of this warp, column col).
+__device__ __forceinline__ uint32_t tm(uint32_t tmem, int col) {
+    return tmem + ((uint32_t)((threadIdx.x >> 5) * 32) << 16) + (uint32_t)col;
+}
+
+// Row of a 64-row (M = 64) accumulator held by this thread's lane, or -1.
+__device__ __forceinline__ int m64_row() {
+    const int l = threadIdx.x & 31;
+    return l < 16 ? (int)(threadIdx.x >> 5) * 16 + l : -1;
+}
+
+// ============================================================ tc_prep
+// Per (chunk, head): gates, A (fp32 forward substitution), and the tile
+// images W, Kd and the plain rows of Ut that the state pass consumes.
+struct PrepSmem {
+    static constexpr int kK = 0, kV = kK + 16384, kAb = kV + 16384, kAc = kAb + 8192,
+                         kL = kAc + 8192, kG = kL + C * 65 * 4, kB = kG + 256,
+                         kEnd = kB + 256;
+};
+constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
+constexpr int kPrepSmemRequest = 100 * 1024;  // at most two CTAs per SM (TMEM: 256 columns each)
+
+__global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H;
+    const ChunkInfo ci = p.chunks[c];
+    uint8_t *Kt = sm + PrepSmem::kK, *Vt = sm + PrepSmem::kV;
+    uint8_t *Ab = sm + PrepSmem::kAb, *Ac = sm + PrepSmem::kAc;
+    float *L = reinterpret_cast<float *>(sm + PrepSmem::kL);
+    float *G = reinterpret_cast<float *>(sm + PrepSmem::kG);
+    float *bta = reinterpret_cast<float *>(sm + PrepSmem::kB);
+    const int tid = threadIdx.x;
+
+    load_rows_async(Kt, C, 0, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
+    load_rows_async(Vt, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H);
+    cp_async_commit();
+    if (tid == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (tid < 32) {
+        tmem_alloc(&tslot, 256);
+        tmem_relinquish();
+    }
+    chunk_gates(G, bta, p, ci, h);
+    cp_async_wait<0>();
+    operands_ready();
+    const uint32_t tmem = tslot;
+    uint32_t phase = 0;
+    bool ok = true;
+
+    // K K^T (M = 64 rows i, N = 64 cols j, K = 128)
+    if (tid == 0) {
+        const uint32_t kb = smem_u32(Kt), id = idesc_bf16(64, 64, 0, 0);
+        for (int s = 0; s < D / 16; ++s)
+            mma_bf16(tmem, desc_kmajor(kb, C, s), desc_kmajor(kb, C, s), id, s > 0);
+        mma_commit(&mbar);
+    }
+    // meanwhile: Kd = diag(e) K as a tile image, and G
+    {
+        const float Gn = G[C - 1];
+        uint8_t *dst = static_cast<uint8_t *>(p.tKd) + (size_t)ch * kImg64;
+        for (int t = tid; t < C * 16; t += NT) {
+            const int off = t * 16, r = (off & 8191) >> 7;
+            float f[8];
+            unpack8(*reinterpret_cast<const uint4 *>(Kt + off), f);
+            const float e = expf(Gn - G[r]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] *= e;
+            *reinterpret_cast<uint4 *>(dst + off) = pack8(f);
+        }
+        if (tid < C) p.tG[(size_t)ch * C + tid] = G[tid];
+    }
+    ok = cta_wait(&mbar, phase, p, 1);
+    phase ^= 1;
+    if (ok) {
+        // L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32)
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    L[i * 65 + j] = j < i ? bta[i] * expf(G[i] - G[j]) * d[q] : 0.f;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        // forward substitution: thread j owns column j of A = (I + L)^-1
+        if (tid < C) {
+            const int j = tid;
+            float a[C];
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                float s = 0.f;
+#pragma unroll
+                for (int m = 0; m < r; ++m) s = fmaf(L[r * 65 + m], a[m], s);
+                a[r] = r < j ? 0.f : (r == j ? 1.f : -s);
+            }
+            const float bg = bta[j] * expf(G[j]), b = bta[j];
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                *reinterpret_cast<bf16 *>(Ab + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * bg);
+                *reinterpret_cast<bf16 *>(Ac + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * b);
+            }
+            if (want_A) {
+                float *Ag = p.tA + (size_t)ch * C * C;
+#pragma unroll
+                for (int r = 0; r < C; ++r) Ag[r * C + j] = a[r];
+            }
+        }
+        operands_ready();
+        // W = (A diag(b gam)) K and Ut = (A diag(b)) V: M = 64, N = 128, K = 64 tokens
+        if (tid == 0) {
+            const uint32_t id = idesc_bf16(64, 128, 0, 1);
+            const uint32_t ab = smem_u32(Ab), ac = smem_u32(Ac), kb = smem_u32(Kt),
+                           vb = smem_u32(Vt);
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(ab, C, s), desc_mnmajor(kb, C, s), id, s > 0);
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + 128, desc_kmajor(ac, C, s), desc_mnmajor(vb, C, s), id, s > 0);
+            mma_commit(&mbar);
+        }
+        ok = cta_wait(&mbar, phase, p, 2);
+        phase ^= 1;
+    }
+    if (ok) {
+        const int i = m64_row();
+        uint8_t *Wimg = static_cast<uint8_t *>(p.tW) + (size_t)ch * kImg64;
+        bf16 *Ut = static_cast<bf16 *>(p.tUt) + (size_t)ch * C * D;
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float w[16], u[16];
+            tmem_ld16(tm(tmem, c0), w);
+            tmem_ld16(tm(tmem, 128 + c0), u);
+            tmem_ld_wait();
+            if (i >= 0) {
+                *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8)) = pack8(w);
+                *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(w + 8);
+                *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0) = pack8(u);
+                *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0 + 8) = pack8(u + 8);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 32) tmem_dealloc(tmem, 256);
+}
+
+// ============================================================ tc_state_fwd
+// One CTA per (sequence, head); thread v owns row v of S (fp32 registers).
+struct StateSmem {
+    static constexpr int kS = 0, kUT = kS + 32768, kW0 = kUT + 16384, kKd0 = kW0 + 2 * 16384,
+                         kUt0 = kKd0 + 2 * 16384, kEnd = kUt0 + 2 * 16384;
+};
+constexpr int kStateSmem = StateSmem::kEnd + 1024;
+
+__device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p) {
+    load_image_async(sm + StateSmem::kW0 + buf * 16384,
+                     static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
+    load_image_async(sm + StateSmem::kKd0 + buf * 16384,
+                     static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
+    load_image_async(sm + StateSmem::kUt0 + buf * 16384,
+                     static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64);
+    cp_async_commit();
+}
+
+__global__ void __launch_bounds__(NT, 1) tc_state_fwd_kernel(Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, n = blockIdx.x / H, h = blockIdx.x % H, v = threadIdx.x;
+    float S[D];
+    if (p.h0) {
+        const float *h0 = p.h0 + ((size_t)n * H + h) * D * D;
+#pragma unroll
+        for (int kk = 0; kk < D; ++kk) S[kk] = h0[kk * D + v];
+    } else {
+#pragma unroll
+        for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
+    }
+    if (v == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (v < 32) {
+        tmem_alloc(&tslot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot;
+    const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
+    uint32_t phase = 0;
+    if (c0 < c1) state_prefetch(sm, 0, (size_t)c0 * H + h, p);
+    uint8_t *Ss = sm + StateSmem::kS, *UTs = sm + StateSmem::kUT;
+    const uint32_t id1 = idesc_bf16(128, 64, 0, 0), id2 = idesc_bf16(128, 128, 0, 1);
+    for (int c = c0; c < c1; ++c) {
+        const int buf = (c - c0) & 1;
+        const size_t ch = (size_t)c * H + h;
+        if (c + 1 < c1) {
+            state_prefetch(sm, buf ^ 1, ch + H, p);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        // the state entering this chunk, as bf16 operand rows
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
+        const float gC = expf(p.tG[ch * C + C - 1]);
+        operands_ready();
+        if (v == 0) {
+            const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
+            mma_commit(&mbar);
+            bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128, sb, (uint32_t)kImg128);
+            bulk_commit();
+        }
+        if (!cta_wait(&mbar, phase, p, 3)) break;
+        phase ^= 1;
+        // U^T[v][i] = Ut[i][v] - (S W^T)[v][i]
+        const bf16 *Ut = reinterpret_cast<const bf16 *>(sm + StateSmem::kUt0 + buf * 16384);
+#pragma unroll
+        for (int c16 = 0; c16 < C; c16 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, c16), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) d[q] = __bfloat162float(Ut[(c16 + q) * D + v]) - d[q];
+            *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c16 / 8)) = pack8(d);
+            *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
+        }
+        operands_ready();
+        if (v == 0) {
+            const uint32_t ub = smem_u32(UTs), kb = smem_u32(sm + StateSmem::kKd0 + buf * 16384);
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
+            mma_commit(&mbar);
+            bulk_store(static_cast<uint8_t *>(p.tUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
+            bulk_commit();
+        }
+        if (!cta_wait(&mbar, phase, p, 4)) break;
+        phase ^= 1;
+#pragma unroll
+        for (int c16 = 0; c16 < D; c16 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, 64 + c16), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) S[c16 + q] = fmaf(gC, S[c16 + q], d[q]);
+        }
+        // shared operands are rewritten next chunk: their bulk stores must have read them
+        if (v == 0) bulk_wait_read();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if (v == 0) bulk_wait_all();
+    if (p.hT) {
+        float *hT = p.hT + ((size_t)n * H + h) * D * D;
+#pragma unroll
+        for (int kk = 0; kk < D; ++kk) hT[kk * D + v] = S[kk];
+    }
+    cp_async_wait<0>();
+    tc_fence_before();
+    __syncthreads();
+    if (v < 32) tmem_dealloc(tmem, 256);
+}
+
+// ============================================================ tc_out
+// O^T[v][i] = S[v][:] . (scale gam_i q_i) + sum_j U^T[v][j] P[i][j],
+// P = scale lower(Q K^T . Gam).  One CTA per (chunk, head).
+struct OutSmem {
+    static constexpr int kQK = 0, kS = kQK + 32768, kUT = kS + 32768, kQG = kUT + 16384,
+                         kP = kQG + 16384, kG = kP + 8192, kEnd = kG + 256;
+};
+constexpr int kOutSmem = OutSmem::kEnd + 1024;
+
+__global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
+    const ChunkInfo ci = p.chunks[c];
+    uint8_t *QK = sm + OutSmem::kQK, *Ss = sm + OutSmem::kS, *UTs = sm + OutSmem::kUT;
+    uint8_t *QG = sm + OutSmem::kQG, *Ps = sm + OutSmem::kP;
+    float *G = reinterpret_cast<float *>(sm + OutSmem::kG);
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
+    load_image_async(Ss, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128);
+    load_image_async(UTs, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT);
+    cp_async_commit();
+    if (tid < C) G[tid] = p.tG[(size_t)ch * C + tid];
+    if (tid == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (tid < 32) {
+        tmem_alloc(&tslot, 128);
+        tmem_relinquish();
+    }
+    cp_async_wait<0>();
+    operands_ready();
+    const uint32_t tmem = tslot;
+    if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
+        const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
+        for (int s = 0; s < D / 16; ++s)
+            mma_bf16(tmem, desc_kmajor(qb, D, s), desc_kmajor(kb, D, s), id, s > 0);
+        mma_commit(&mbar);
+    }
+    // scale * gam_i * q_i as a K-major operand (rows i)
+    for (int t = tid; t < C * 16; t += NT) {
+        const int r = t >> 4, j = t & 15;
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4 *>(QK + sw128_chunk(D, r, j)), f);
+        const float s = p.scale * expf(G[r]);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] *= s;
+        *reinterpret_cast<uint4 *>(QG + sw128_chunk(C, r, j)) = pack8(f);
+    }
+    bool ok = cta_wait(&mbar, 0, p, 5);
+    if (ok) {
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    d[q] = j <= i ? p.scale * expf(G[i] - G[j]) * d[q] : 0.f;
+                }
+                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
+            }
+        }
+        operands_ready();
+        if (tid == 0) {
+            const uint32_t id = idesc_bf16(128, 64, 0, 0);
+            const uint32_t sb = smem_u32(Ss), qg = smem_u32(QG), ub = smem_u32(UTs),
+                           pb = smem_u32(Ps);
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tmem + 64, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_kmajor(pb, C, s), id, 1);
+            mma_commit(&mbar);
+        }
+        ok = cta_wait(&mbar, 1, p, 6);
+    }
+    if (ok) {
+        bf16 *o = static_cast<bf16 *>(p.o);
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, 64 + c0), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int i = c0 + q;
+                if (i < ci.len) o[((int64_t)(ci.tok0 + i) * H + h) * D + tid] = __float2bfloat16_rn(d[q]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 32) tmem_dealloc(tmem, 128);
+}
+
+template <typename Kern>
+cudaError_t set_smem(Kern k, int bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+bool tc_supported(const Problem &pb) { return pb.K == 128 && pb.V == 128; }
+
+bool tc_bwd_ready() { return false; }
+
+cudaError_t launch_tc_fwd(const Params &p, const Problem &, cudaStream_t stream) {
+    cudaError_t e;
+    const int nch = p.NC * p.H, nseq = p.N * p.H;
+    if (nch > 0) {
+        if ((e = set_smem(tc_prep_kernel, kPrepSmemRequest))) return e;
+        GDN_LAUNCH(kKTcPrep, stream, tc_prep_kernel<<<nch, NT, kPrepSmemRequest, stream>>>(p, 0));
+    }
+    if (nseq > 0) {
+        if ((e = set_smem(tc_state_fwd_kernel, kStateSmem))) return e;
+        GDN_LAUNCH(kKTcStateFwd, stream,
+                   tc_state_fwd_kernel<<<nseq, NT, kStateSmem, stream>>>(p));
+    }
+    if (nch > 0) {
+        if ((e = set_smem(tc_out_kernel, kOutSmem))) return e;
+        GDN_LAUNCH(kKTcOut, stream, tc_out_kernel<<<nch, NT, kOutSmem, stream>>>(p));
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_tc_bwd(const Params &, const Problem &, cudaStream_t) {
+    return cudaErrorNotSupported;
+}
+
+static_assert(kPrepSmem <= kPrepSmemRequest, "prep shared memory");
 
 }  // namespace gdn
