@@ -1,0 +1,674 @@
+// Tensor-core (tcgen05) backward of the bf16 layer, d_k = d_v = 128.
+//
+// Reverse-mode of the chunkwise forward (see tc.cu).  After the forward
+// pieces are recomputed (tc_prep keeps A in fp32; tc_state_fwd rewrites the
+// state entering every chunk and U^T), three kernels run:
+//
+//   tc_local      chunk-parallel: P = scale lower(Q K^T . Gam), the local
+//                 dU^T = dO^T P, and Qg = scale diag(gam) Q (a tile image)
+//   tc_state_bwd  serial over the chunks of a sequence, in reverse; thread v
+//                 owns row v of dS = dH^T (fp32 registers); per chunk
+//                   dU^T = dS Kd^T + (local dU^T)
+//                   dS  <- gam_n dS + dO^T Qg - dU^T W
+//                 and writes dS (the gradient of the state leaving the chunk)
+//                 and dU^T as tile images
+//   tc_grads      chunk-parallel: every chunk-local gradient (dq, dk, dv, dg,
+//                 dbeta) from the recomputed and propagated pieces.
+//
+// Products run in transposed form wherever that lets the accumulator use all
+// 128 TMEM lanes (M = 128 over the key or value dim); 64 x 64 products use the
+// M = 64 form (row m in lane 32 (m / 16) + m % 16).
+#include "tc_common.cuh"
+
+namespace gdn {
+
+cudaError_t tc_launch_prep(const Params &p, int want_A, cudaStream_t stream);
+cudaError_t tc_launch_state_fwd(const Params &p, cudaStream_t stream);
+
+namespace {
+
+using namespace tc;
+
+// ============================================================ tc_local
+struct LocalSmem {
+    static constexpr int kQK = 0, kDO = kQK + 32768, kP = kDO + 16384,
+                         kG = kP + 8192, kEnd = kG + 256;
+};
+constexpr int kLocalSmem = LocalSmem::kEnd + 1024;
+
+__global__ void __launch_bounds__(NT) tc_local_kernel(Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
+    const ChunkInfo ci = p.chunks[c];
+    uint8_t *QK = sm + LocalSmem::kQK, *DO = sm + LocalSmem::kDO, *Ps = sm + LocalSmem::kP;
+    float *G = reinterpret_cast<float *>(sm + LocalSmem::kG);
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
+    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H);
+    cp_async_commit();
+    if (tid < C) G[tid] = p.tG[(size_t)ch * C + tid];
+    if (tid == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (tid < 32) {
+        tmem_alloc(&tslot, 128);
+        tmem_relinquish();
+    }
+    cp_async_wait<0>();
+    operands_ready();
+    const uint32_t tmem = tslot;
+    if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
+        const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
+        for (int s = 0; s < D / 16; ++s)
+            mma_bf16(tmem, desc_kmajor(qb, D, s), desc_kmajor(kb, D, s), id, s > 0);
+        mma_commit(&mbar);
+    }
+    {  // Qg = scale diag(gam) Q: an operand of the reverse state pass (tile image)
+        uint8_t *img = static_cast<uint8_t *>(p.tQg) + (size_t)ch * kImg64;
+        for (int t = tid; t < C * 16; t += NT) {
+            const int r = t >> 4, j = t & 15;
+            float f[8];
+            unpack8(*reinterpret_cast<const uint4 *>(QK + sw128_chunk(D, r, j)), f);
+            const float s = p.scale * expf(G[r]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) f[q] *= s;
+            *reinterpret_cast<uint4 *>(img + sw128_chunk(C, r, j)) = pack8(f);
+        }
+    }
+    bool ok = cta_wait(&mbar, 0, p, 11);
+    if (ok) {
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    d[q] = j <= i ? p.scale * expf(G[i] - G[j]) * d[q] : 0.f;
+                }
+                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
+            }
+        }
+        operands_ready();
+        if (tid == 0) {  // local dU^T[v][j] = sum_i dO[i][v] P[i][j]: M = 128, N = 64, K = 64
+            const uint32_t db = smem_u32(DO), pb = smem_u32(Ps), id = idesc_bf16(128, 64, 1, 1);
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + 64, desc_mnmajor(db, C, s), desc_mnmajor(pb, C, s), id, s > 0);
+            mma_commit(&mbar);
+        }
+        ok = cta_wait(&mbar, 1, p, 12);
+    }
+    if (ok) {
+        bf16 *dul = static_cast<bf16 *>(p.tdUL) + (size_t)ch * D * C + (size_t)tid * C;
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, 64 + c0), d);
+            tmem_ld_wait();
+            *reinterpret_cast<uint4 *>(dul + c0) = pack8(d);
+            *reinterpret_cast<uint4 *>(dul + c0 + 8) = pack8(d + 8);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 32) tmem_dealloc(tmem, 128);
+}
+
+// ============================================================ tc_state_bwd
+struct SbwdSmem {
+    static constexpr int kdS = 0, kdU = kdS + 32768, kBuf = kdU + 16384;
+    // per buffer: Kd image, W image, Qg image, dO tile, local dU^T rows
+    static constexpr int kKd = 0, kW = 16384, kQg = 32768, kDO = 49152, kDUL = 65536,
+                         kBufBytes = 81920;
+    static constexpr int kEnd = kBuf + 2 * kBufBytes;
+};
+constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
+
+__device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
+                                              const ChunkInfo &ci, int h, const Params &p) {
+    uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
+    load_image_async(b + SbwdSmem::kKd, static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
+    load_image_async(b + SbwdSmem::kW, static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
+    load_image_async(b + SbwdSmem::kQg, static_cast<const uint8_t *>(p.tQg) + ch * kImg64, kImg64);
+    load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H);
+    load_image_async(b + SbwdSmem::kDUL, static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT,
+                     kImgUT);
+    cp_async_commit();
+}
+
+__global__ void __launch_bounds__(NT, 1) tc_state_bwd_kernel(Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, n = blockIdx.x / H, h = blockIdx.x % H, v = threadIdx.x;
+    float S[D];  // dS row v (gradient of the state leaving the current chunk)
+    if (p.dhT) {
+        const float *g0 = p.dhT + ((size_t)n * H + h) * D * D;
+#pragma unroll
+        for (int kk = 0; kk < D; ++kk) S[kk] = g0[kk * D + v];
+    } else {
+#pragma unroll
+        for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
+    }
+    if (v == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (v < 32) {
+        tmem_alloc(&tslot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot;
+    const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
+    uint32_t phase = 0;
+    if (c0 < c1) sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, p.chunks[c1 - 1], h, p);
+    uint8_t *dSs = sm + SbwdSmem::kdS, *dUs = sm + SbwdSmem::kdU;
+    const uint32_t id1 = idesc_bf16(128, 64, 0, 0), idx = idesc_bf16(128, 128, 1, 1),
+                   idy = idesc_bf16(128, 128, 0, 1);
+    for (int c = c1 - 1; c >= c0; --c) {
+        const int buf = (c1 - 1 - c) & 1;
+        const size_t ch = (size_t)c * H + h;
+        if (c - 1 >= c0) {
+            sbwd_prefetch(sm, buf ^ 1, ch - H, p.chunks[c - 1], h, p);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
+        const float gC = expf(p.tG[ch * C + C - 1]);
+        operands_ready();
+        if (v == 0) {
+            const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
+                           qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO);
+            // dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, s > 0);
+            // dO^T Qg: M = 128 (v), N = 128 keys, K = 64 tokens
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + 64, desc_mnmajor(ob, C, s), desc_mnmajor(qb, C, s), idx, s > 0);
+            mma_commit(&mbar);
+            bulk_store(static_cast<uint8_t *>(p.tdSn) + ch * kImg128, sb, (uint32_t)kImg128);
+            bulk_commit();
+        }
+        if (!cta_wait(&mbar, phase, p, 13)) break;
+        phase ^= 1;
+        {  // dU^T = dS Kd^T + local dU^T ; -dU^T is the next operand, +dU^T an image for tc_grads
+            const bf16 *dul = reinterpret_cast<const bf16 *>(b + SbwdSmem::kDUL) + v * C;
+            uint8_t *img = static_cast<uint8_t *>(p.tdUT) + ch * kImgUT;
+#pragma unroll
+            for (int c16 = 0; c16 < C; c16 += 16) {
+                float d[16], l[16];
+                tmem_ld16(tm(tmem, c16), d);
+                tmem_ld_wait();
+                unpack8(*reinterpret_cast<const uint4 *>(dul + c16), l);
+                unpack8(*reinterpret_cast<const uint4 *>(dul + c16 + 8), l + 8);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) d[q] += l[q];
+                *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, c16 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) d[q] = -d[q];
+                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
+            }
+        }
+        operands_ready();
+        if (v == 0) {  // - dU^T W: M = 128 (v), N = 128 keys, K = 64 tokens
+            const uint32_t ub = smem_u32(dUs), wb = smem_u32(b + SbwdSmem::kW);
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(wb, C, s), idy, 1);
+            mma_commit(&mbar);
+        }
+        if (!cta_wait(&mbar, phase, p, 14)) break;
+        phase ^= 1;
+#pragma unroll
+        for (int c16 = 0; c16 < D; c16 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, 64 + c16), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) S[c16 + q] = fmaf(gC, S[c16 + q], d[q]);
+        }
+        if (v == 0) bulk_wait_read();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if (v == 0) bulk_wait_all();
+    if (p.dh0) {
+        float *g0 = p.dh0 + ((size_t)n * H + h) * D * D;
+#pragma unroll
+        for (int kk = 0; kk < D; ++kk) g0[kk * D + v] = S[kk];
+    }
+    cp_async_wait<0>();
+    tc_fence_before();
+    __syncthreads();
+    if (v < 32) tmem_dealloc(tmem, 256);
+}
+
+// ============================================================ tc_grads
+struct GradSmem {
+    static constexpr int kQK = 0, kDO = 32768, kV = 49152, kSC = 65536, kDSN = 98304,
+                         kUT = 131072, kDUT = 147456, kAB = 163840, kX3 = 172032,
+                         kDA = 188416, kT1 = 196608, kDPG = 204800, kDLG = 212992,
+                         kVec = 221184, kEnd = kVec + 10 * 256;
+    // reused after the first products: fp32 64x64 P (then dP.P + dL.L) and Gam.KK^T,
+    // and a [128 threads][64] reduction buffer
+    static constexpr int kPE = kSC, kKKG = kSC + 16384, kRed = kDSN;
+};
+constexpr int kGradSmem = GradSmem::kEnd + 1024;
+
+// Deterministic column sums of red[t][i] over the 128 threads t -> out[i].
+__device__ __forceinline__ void reduce_rows(const float *red, float *out) {
+    __syncthreads();
+    if (threadIdx.x < C) {
+        float s = 0.f;
+        for (int t = 0; t < NT; ++t) s += red[t * C + threadIdx.x];
+        out[threadIdx.x] = s;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ float sw_elem(const uint8_t *tile, int R, int r, int c) {
+    return __bfloat162float(*reinterpret_cast<const bf16 *>(tile + sw128_off(R, r, c)));
+}
+
+__global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    __shared__ float s_hd;
+    if (p.hdr->status) return;
+    const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
+    const ChunkInfo ci = p.chunks[c];
+    using S_ = GradSmem;
+    uint8_t *QK = sm + S_::kQK, *DO = sm + S_::kDO, *VT = sm + S_::kV, *SC = sm + S_::kSC,
+            *DSN = sm + S_::kDSN, *UT = sm + S_::kUT, *DUT = sm + S_::kDUT, *AB = sm + S_::kAB,
+            *X3 = sm + S_::kX3, *DA = sm + S_::kDA, *T1 = sm + S_::kT1, *DPG = sm + S_::kDPG,
+            *DLG = sm + S_::kDLG;
+    float *vec = reinterpret_cast<float *>(sm + S_::kVec);
+    float *G = vec, *bta = vec + 64, *gam = vec + 128, *e = vec + 192, *dB = vec + 256,
+          *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576;
+    float *PE = reinterpret_cast<float *>(sm + S_::kPE);
+    float *KKG = reinterpret_cast<float *>(sm + S_::kKKG);
+    float *RED = reinterpret_cast<float *>(sm + S_::kRed);
+
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
+    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H);
+    load_rows_async(VT, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H);
+    load_image_async(SC, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128);
+    load_image_async(DSN, static_cast<const uint8_t *>(p.tdSn) + (size_t)ch * kImg128, kImg128);
+    load_image_async(UT, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT);
+    load_image_async(DUT, static_cast<const uint8_t *>(p.tdUT) + (size_t)ch * kImgUT, kImgUT);
+    cp_async_commit();
+    if (tid < C) {
+        const int64_t idx = (int64_t)(ci.tok0 + tid) * H + h;
+        G[tid] = p.tG[(size_t)ch * C + tid];
+        bta[tid] = tid < ci.len ? p.beta[idx] : 0.f;
+    }
+    {  // A (fp32, from tc_prep) as a bf16 tile: rows m, columns i
+        const float *Ag = p.tA + (size_t)ch * C * C;
+        for (int t = tid; t < C * C; t += NT) {
+            const int m = t / C, i = t % C;
+            *reinterpret_cast<bf16 *>(AB + sw128_off(C, m, i)) = __float2bfloat16_rn(Ag[t]);
+        }
+    }
+    if (tid == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (tid < 32) {
+        tmem_alloc(&tslot, 512);
+        tmem_relinquish();
+    }
+    __syncthreads();
+    if (tid < C) {
+        gam[tid] = expf(G[tid]);
+        e[tid] = expf(G[C - 1] - G[tid]);
+    }
+    cp_async_wait<0>();
+    operands_ready();
+    const uint32_t tmem = tslot;
+    const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128, dob = smem_u32(DO), vb = smem_u32(VT),
+                   scb = smem_u32(SC), dsb = smem_u32(DSN), utb = smem_u32(UT),
+                   dub = smem_u32(DUT), ab = smem_u32(AB), x3b = smem_u32(X3), dab = smem_u32(DA),
+                   t1b = smem_u32(T1), dpb = smem_u32(DPG), dlb = smem_u32(DLG);
+    // TMEM columns
+    constexpr int cQK = 0, cX1 = 64, cX2 = 128, cX3 = 192, cDP = 256, cAU = 320, cY1 = 384,
+                  cY2 = 0, cZ = 448, cT1 = 192, cDL = 0, cDQ = 256, cDK = 320, cDKA = 384;
+    uint32_t phase = 0;
+    bool ok;
+    if (tid == 0) {
+        const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
+                       i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
+                       i64km = idesc_bf16(64, 64, 0, 1), i64mk = idesc_bf16(64, 64, 1, 0);
+        for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
+            mma_bf16(tmem + cQK, desc_kmajor(qkb, D, s), desc_kmajor(kb, D, s), i128, s > 0);
+        for (int s = 0; s < 8; ++s)  // X1^T = S^T dO^T  (over v)
+            mma_bf16(tmem + cX1, desc_mnmajor(scb, D, s), desc_kmajor(dob, C, s), i128mk, s > 0);
+        for (int s = 0; s < 8; ++s)  // X2^T = dSn^T U^T
+            mma_bf16(tmem + cX2, desc_mnmajor(dsb, D, s), desc_mnmajor(utb, D, s), i128mm, s > 0);
+        for (int s = 0; s < 8; ++s)  // X3^T = S^T dU^T
+            mma_bf16(tmem + cX3, desc_mnmajor(scb, D, s), desc_mnmajor(dub, D, s), i128mm, s > 0);
+        for (int s = 0; s < 8; ++s)  // dP = dO U^T (M = 64)
+            mma_bf16(tmem + cDP, desc_kmajor(dob, C, s), desc_mnmajor(utb, D, s), i64km, s > 0);
+        for (int s = 0; s < 4; ++s)  // (A^T dU)^T = dU^T A
+            mma_bf16(tmem + cAU, desc_kmajor(dub, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
+        for (int s = 0; s < 8; ++s)  // Y1 = dU V^T (M = 64)
+            mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, C, s), i64mk, s > 0);
+        mma_commit(&mbar);
+    }
+    ok = cta_wait(&mbar, phase, p, 21);
+    phase ^= 1;
+    if (!ok) goto done;
+    {  // <S, dSn> (elementwise over identically laid out images)
+        float s = 0.f;
+        for (int t = tid; t < D * D / 8; t += NT) {
+            float a[8], b[8];
+            unpack8(*reinterpret_cast<const uint4 *>(SC + t * 16), a);
+            unpack8(*reinterpret_cast<const uint4 *>(DSN + t * 16), b);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) s = fmaf(a[q], b[q], s);
+        }
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if ((tid & 31) == 0) tmp[tid >> 5] = s;
+        __syncthreads();
+        if (tid == 0) s_hd = tmp[0] + tmp[1] + tmp[2] + tmp[3];
+        __syncthreads();
+    }
+    {  // P (scaled, lower incl. diagonal) and Gam . K K^T (strictly lower), fp32
+        const int i = tid & 63;
+        const bool isP = tid < 64;
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cQK + c0), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int j = c0 + q;
+                const float gij = expf(G[i] - G[j]);
+                if (isP) PE[i * C + j] = j <= i ? p.scale * gij * d[q] : 0.f;
+                else KKG[i * C + j] = j < i ? gij * d[q] : 0.f;
+            }
+        }
+    }
+    {  // dv = diag(b) A^T dU ; partial v . (A^T dU)
+        bf16 *dv = static_cast<bf16 *>(p.dv);
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cAU + c0), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int i = c0 + q;
+                RED[tid * C + i] = sw_elem(VT, C, i, tid) * d[q];
+                if (i < ci.len)
+                    dv[((int64_t)(ci.tok0 + i) * H + h) * D + tid] = __float2bfloat16_rn(bta[i] * d[q]);
+            }
+        }
+        reduce_rows(RED, dB);
+    }
+    {  // partial q' . X1 and k . X2 (thread kk), then X3^T as an operand tile (row kk)
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cX1 + c0), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                RED[tid * C + c0 + q] = p.scale * sw_elem(QK, D, c0 + q, tid) * d[q];
+        }
+        reduce_rows(RED, qx);
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cX2 + c0), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) RED[tid * C + c0 + q] = sw_elem(QK, D, C + c0 + q, tid) * d[q];
+        }
+        reduce_rows(RED, kx);
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cX3 + c0), d);
+            tmem_ld_wait();
+            *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, tid, c0 / 8)) = pack8(d);
+            *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, tid, c0 / 8 + 1)) = pack8(d + 8);
+        }
+    }
+    {  // dP: dPG = dP . Gam as an operand tile; PE <- dP . P
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cDP + c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    const float dp = j <= i ? d[q] : 0.f;
+                    PE[i * C + j] *= dp;
+                    d[q] = dp * (j <= i ? expf(G[i] - G[j]) : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i, c0 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
+            }
+        }
+    }
+    operands_ready();
+    if (tid == 0) {
+        const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1);
+        for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
+            mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
+        for (int s = 0; s < 4; ++s)  // Zp^T = X3^T A   (Z = -Zp)
+            mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
+        mma_commit(&mbar);
+    }
+    ok = cta_wait(&mbar, phase, p, 22);
+    phase ^= 1;
+    if (!ok) goto done;
+    {  // dA = (dU V^T) diag(b) - (X3 K^T) diag(b gam)
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float y1[16], y2[16];
+            tmem_ld16(tm(tmem, cY1 + c0), y1);
+            tmem_ld16(tm(tmem, cY2 + c0), y2);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int m = c0 + q;
+                    y1[q] = bta[m] * y1[q] - bta[m] * gam[m] * y2[q];
+                }
+                *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i, c0 / 8)) = pack8(y1);
+                *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(y1 + 8);
+            }
+        }
+        for (int c0 = 0; c0 < C; c0 += 16) {  // partial k . Z = -k . Zp
+            float d[16];
+            tmem_ld16(tm(tmem, cZ + c0), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) RED[tid * C + c0 + q] = -sw_elem(QK, D, C + c0 + q, tid) * d[q];
+        }
+        reduce_rows(RED, kz);
+    }
+    operands_ready();
+    if (tid == 0) {  // T1 = A^T dA (M = 64)
+        const uint32_t id = idesc_bf16(64, 64, 1, 1);
+        for (int s = 0; s < 4; ++s)
+            mma_bf16(tmem + cT1, desc_mnmajor(ab, C, s), desc_mnmajor(dab, C, s), id, s > 0);
+        mma_commit(&mbar);
+    }
+    ok = cta_wait(&mbar, phase, p, 23);
+    phase ^= 1;
+    if (!ok) goto done;
+    {
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cT1 + c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
+                *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i, c0 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
+            }
+        }
+    }
+    operands_ready();
+    if (tid == 0) {  // T1 A^T = -dL (M = 64)
+        const uint32_t id = idesc_bf16(64, 64, 0, 0);
+        for (int s = 0; s < 4; ++s)
+            mma_bf16(tmem + cDL, desc_kmajor(t1b, C, s), desc_kmajor(ab, C, s), id, s > 0);
+        mma_commit(&mbar);
+    }
+    ok = cta_wait(&mbar, phase, p, 24);
+    phase ^= 1;
+    if (!ok) goto done;
+    {  // dL (strictly lower); diag(b) dL . Gam as an operand tile; PE += dL . L; dbeta terms
+        const int i = m64_row();
+        float dbl = 0.f;
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, cDL + c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    const float dl = j < i ? -d[q] : 0.f;
+                    const float kkg = KKG[i * C + j];
+                    PE[i * C + j] += dl * bta[i] * kkg;
+                    dbl = fmaf(dl, kkg, dbl);
+                    d[q] = bta[i] * dl * (j < i ? expf(G[i] - G[j]) : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i, c0 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
+            }
+        }
+        if (i >= 0) dB[i] += dbl + gam[i] * kz[i];
+    }
+    operands_ready();
+    if (tid == 0) {
+        const uint32_t imk = idesc_bf16(128, 64, 1, 0), imm = idesc_bf16(128, 64, 1, 1);
+        for (int s = 0; s < 4; ++s)  // (dPG K)^T = K^T dPG^T
+            mma_bf16(tmem + cDQ, desc_mnmajor(kb, D, s), desc_kmajor(dpb, C, s), imk, s > 0);
+        for (int s = 0; s < 4; ++s)  // (dPG^T Q)^T = Q^T dPG
+            mma_bf16(tmem + cDKA, desc_mnmajor(qkb, D, s), desc_mnmajor(dpb, C, s), imm, s > 0);
+        for (int s = 0; s < 4; ++s)  // (diag(b) dLG K)^T
+            mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_kmajor(dlb, C, s), imk, s > 0);
+        for (int s = 0; s < 4; ++s)  // ((diag(b) dLG)^T K)^T
+            mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_mnmajor(dlb, C, s), imm, 1);
+        mma_commit(&mbar);
+    }
+    // meanwhile: dG and dbeta (rows), then dg = reverse cumulative sum of dG
+    if (tid < C) {
+        const int i = tid;
+        float rs = 0.f, cs = 0.f;
+        for (int j = 0; j < C; ++j) {
+            rs += PE[i * C + j];
+            cs += PE[j * C + i];
+        }
+        dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + rs - cs + bta[i] * gam[i] * kz[i];
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float s = 0.f;
+        for (int j = 0; j < C; ++j) s += e[j] * kx[j];
+        dG[C - 1] += gam[C - 1] * s_hd + s;
+        float acc = 0.f;
+        for (int j = C - 1; j >= 0; --j) {
+            acc += dG[j];
+            dG[j] = acc;
+        }
+    }
+    __syncthreads();
+    if (tid < ci.len) {
+        const int64_t o = (int64_t)(ci.tok0 + tid) * H + h;
+        p.dg[o] = dG[tid];
+        p.dbeta[o] = dB[tid];
+    }
+    ok = cta_wait(&mbar, phase, p, 25);
+    phase ^= 1;
+    if (!ok) goto done;
+    {  // dq = scale (diag(gam) X1 + dPG K) ; dk = diag(e) X2 + diag(b gam) Z + dPG^T Q' + dL terms
+        bf16 *dq = static_cast<bf16 *>(p.dq), *dk = static_cast<bf16 *>(p.dk);
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float x1[16], a[16];
+            tmem_ld16(tm(tmem, cX1 + c0), x1);
+            tmem_ld16(tm(tmem, cDQ + c0), a);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int i = c0 + q;
+                if (i < ci.len)
+                    dq[((int64_t)(ci.tok0 + i) * H + h) * D + tid] =
+                        __float2bfloat16_rn(p.scale * (gam[i] * x1[q] + a[q]));
+            }
+        }
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float x2[16], z[16], ka[16], kd[16];
+            tmem_ld16(tm(tmem, cX2 + c0), x2);
+            tmem_ld16(tm(tmem, cZ + c0), z);
+            tmem_ld16(tm(tmem, cDKA + c0), ka);
+            tmem_ld16(tm(tmem, cDK + c0), kd);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int i = c0 + q;
+                if (i < ci.len)
+                    dk[((int64_t)(ci.tok0 + i) * H + h) * D + tid] = __float2bfloat16_rn(
+                        e[i] * x2[q] - bta[i] * gam[i] * z[q] + p.scale * ka[q] + kd[q]);
+            }
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 32) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream) {
+    cudaError_t e;
+    const int nch = p.NC * p.H, nseq = p.N * p.H;
+    Params pf = p;
+    pf.hT = nullptr;
+    if ((e = tc_launch_prep(p, 1, stream))) return e;
+    if ((e = tc_launch_state_fwd(pf, stream))) return e;
+    if (nch > 0) {
+        if ((e = set_smem(tc_local_kernel, kLocalSmem))) return e;
+        GDN_LAUNCH(kKTcLocal, stream, tc_local_kernel<<<nch, NT, kLocalSmem, stream>>>(p));
+    }
+    if (nseq > 0) {
+        if ((e = set_smem(tc_state_bwd_kernel, kSbwdSmem))) return e;
+        GDN_LAUNCH(kKTcStateBwd, stream,
+                   tc_state_bwd_kernel<<<nseq, NT, kSbwdSmem, stream>>>(p));
+    }
+    if (nch > 0) {
+        if ((e = set_smem(tc_grads_kernel, kGradSmem))) return e;
+        GDN_LAUNCH(kKTcGrads, stream, tc_grads_kernel<<<nch, NT, kGradSmem, stream>>>(p));
+    }
+    return cudaSuccess;
+}
+
+static_assert(kGradSmem <= 227 * 1024, "grads shared memory");
+static_assert(kSbwdSmem <= 227 * 1024, "reverse state shared memory");
+
+}  // namespace gdn

@@ -1,0 +1,131 @@
+// Shared helpers of the tensor-core kernels (forward in tc.cu, backward in
+// tc_bwd.cu): tile loads into 128-byte-swizzled shared memory, per-chunk
+// gates, bounded MMA waits, bf16 packing, TMEM addressing.
+#pragma once
+
+#include "gdn_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace gdn {
+namespace tc {
+
+using namespace ptx;
+using bf16 = __nv_bfloat16;
+
+
+constexpr int C = kChunk;      // 64
+constexpr int D = 128;         // d_k = d_v
+constexpr int NT = 128;        // threads per CTA
+constexpr uint32_t kWaitLimit = 1u << 23;
+
+constexpr size_t kImg64 = (size_t)C * D * 2;   // 64 x 128 bf16 tile image (16 KB)
+constexpr size_t kImg128 = (size_t)D * D * 2;  // 128 x 128 (32 KB)
+constexpr size_t kImgUT = (size_t)D * C * 2;   // 128 x 64 (16 KB)
+
+__device__ __forceinline__ uint8_t *align1k(uint8_t *p) {
+    return (uint8_t *)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+__device__ __forceinline__ void record_timeout(const Params &p, int where) {
+    atomicExch(&p.hdr->status, kDevTimeout);
+    atomicExch(&p.hdr->where, where);
+}
+
+// Bounded wait on an MMA-completion barrier, decided uniformly by the CTA.
+__device__ __forceinline__ bool cta_wait(uint64_t *mbar, uint32_t parity, const Params &p,
+                                         int where) {
+    const bool ok = mbar_wait(mbar, parity, kWaitLimit);
+    const bool all_ok = __syncthreads_and(ok);
+    if (!all_ok && threadIdx.x == 0) record_timeout(p, where);
+    tc_fence_after();
+    return all_ok;
+}
+
+// Barrier that orders generic smem writes (operands) before MMAs issued after it.
+__device__ __forceinline__ void operands_ready() {
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+// Loads rows [0, 64) of one chunk and head of a [tokens][H][128] bf16 tensor
+// into an SW128 tile with R rows (block stride), starting at row `row0`;
+// rows at or past `len` are zero.  Asynchronous (cp.async).
+__device__ __forceinline__ void load_rows_async(uint8_t *tile, int R, int row0, const bf16 *src,
+                                                int64_t tok0, int len, int h, int H) {
+    const uint32_t base = smem_u32(tile);
+    for (int t = threadIdx.x; t < C * 16; t += NT) {
+        const int r = t >> 4, j = t & 15;
+        const bool valid = r < len;
+        const bf16 *g = valid ? src + ((tok0 + r) * H + h) * D + j * 8 : src;
+        cp_async16_zfill(base + sw128_chunk(R, row0 + r, j), g, valid);
+    }
+}
+
+// Linear copy of a tile image (bytes multiple of 16 * NT).
+__device__ __forceinline__ void load_image_async(uint8_t *tile, const void *img, size_t bytes) {
+    const uint32_t base = smem_u32(tile);
+    const uint8_t *g = static_cast<const uint8_t *>(img);
+    for (size_t off = (size_t)threadIdx.x * 16; off < bytes; off += NT * 16)
+        cp_async16(base + (uint32_t)off, g + off);
+}
+
+// In-chunk cumulative log-decay (zero gates past len), summed in token order by
+// one thread so every kernel gets bit-identical values; also the write strengths.
+__device__ __forceinline__ void chunk_gates(float *G, float *bta, const Params &p, const ChunkInfo &ci, int h) {
+    const int r = threadIdx.x;
+    if (r < C) {
+        const int64_t idx = (int64_t)(ci.tok0 + r) * p.H + h;
+        G[r] = r < ci.len ? p.g[idx] : 0.f;
+        if (bta) bta[r] = r < ci.len ? p.beta[idx] : 0.f;
+    }
+    __syncthreads();
+    if (r == 0) {
+        float s = 0.f;
+        for (int i = 0; i < C; ++i) {
+            s += G[i];
+            G[i] = s;
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float *f) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float *f) {
+    uint4 u;
+    u.x = pack_bf16(f[0], f[1]);
+    u.y = pack_bf16(f[2], f[3]);
+    u.z = pack_bf16(f[4], f[5]);
+    u.w = pack_bf16(f[6], f[7]);
+    return u;
+}
+
+// TMEM address of (lane base of this warp, column col).
+__device__ __forceinline__ uint32_t tm(uint32_t tmem, int col) {
+    return tmem + ((uint32_t)((threadIdx.x >> 5) * 32) << 16) + (uint32_t)col;
+}
+
+// Row of a 64-row (M = 64) accumulator held by this thread's lane, or -1.
+__device__ __forceinline__ int m64_row() {
+    const int l = threadIdx.x & 31;
+    return l < 16 ? (int)(threadIdx.x >> 5) * 16 + l : -1;
+}
+
+
+template <typename Kern>
+inline cudaError_t set_smem(Kern k, int bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace tc
+}  // namespace gdn

@@ -45,6 +45,8 @@ def check_all(inp, tol, units=None, bwd=True):
         ref = oracle_bwd(inp, units)
         for name, a, b in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), got, ref):
             errs[name] = maxnorm_err(a, b)
+    print("parity %s: %s" % (inp.meta.get("name", inp.meta.get("dtype")),
+                             " ".join("%s=%.2e" % kv for kv in errs.items())))
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, (errs, tol)
     return errs
