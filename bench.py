@@ -71,6 +71,18 @@ def kernel_work(name, w, n_chunks):
     }
     if name in table:
         return "alu", table[name] * ch, "flop"
+    th = w["B"] * w["T"] * w["H"]  # token-heads
+    # tensor-core path: HBM-facing kernels report the tensors the method must
+    # move through them (bytes per token-head), chain kernels their MMA flops
+    hbm = {"tc_grads": 4 * 2 * K + 8 + 3 * 2 * K + 8,   # q,k,v,do + g,b in; dq,dk,dv + dg,db out
+           "tc_prep": 2 * (K + V) + 8,                  # k, v, g, b
+           "tc_out": 2 * (2 * K + V) + 4 + 2 * V,       # q, k, v-side U via the state; o out
+           "tc_local": 2 * (2 * K + V) + 4}             # q, k, do
+    if name in hbm:
+        return "hbm", float(hbm[name]) * th, "B"
+    chain = {"tc_state_fwd": 2 * f2(C, V, K), "tc_state_bwd": 3 * f2(C, V, K)}
+    if name in chain:
+        return "tensor", chain[name] * ch, "flop"
     return None, None, None
 
 
