@@ -39,6 +39,8 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shape", default=None,
+                    help="B,T,H override of the workload (profiling and size sweeps only)")
     return ap.parse_args()
 
 
@@ -76,7 +78,7 @@ def kernel_work(name, w, n_chunks):
     # move through them (bytes per token-head), chain kernels their MMA flops
     hbm = {"tc_grads": 4 * 2 * K + 8 + 3 * 2 * K + 8,   # q,k,v,do + g,b in; dq,dk,dv + dg,db out
            "tc_prep": 2 * (K + V) + 8,                  # k, v, g, b
-           "tc_out": 2 * (2 * K + V) + 4 + 2 * V,       # q, k, v-side U via the state; o out
+           "tc_out": 2 * (2 * K) + 4 + 2 * V,           # q, k, g in; o out
            "tc_local": 2 * (2 * K + V) + 4}             # q, k, do
     if name in hbm:
         return "hbm", float(hbm[name]) * th, "B"
@@ -226,6 +228,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = dict(WORKLOAD)
+    if args.shape:
+        w["B"], w["T"], w["H"] = (int(x) for x in args.shape.split(","))
     w["seed"] = WORKLOAD["seed"] + rank
     inp = make_inputs(device="cpu", **w)
     d = inp.to(dev)
@@ -356,7 +360,9 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "gdn_fwdbwd_bf16_B4_T4096_H16_d128", "global_batch": B * world,
+        "config": {"workload": ("gdn_fwdbwd_bf16_B4_T4096_H16_d128" if not args.shape else
+                                "gdn_fwdbwd_bf16_B%d_T%d_H%d_d128" % (B, T, H)),
+                   "global_batch": B * world,
                    "seq_len": T, "heads": H, "head_dim": K, "parallelism": "dp%d" % world,
                    "l2": "256 MiB memset before each step, outside the step events"},
         "roofline": roof,
