@@ -82,7 +82,7 @@ def kernel_work(name, w, n_chunks):
            "tc_local": 2 * (2 * K + V) + 4}             # q, k, do
     if name in hbm:
         return "hbm", float(hbm[name]) * th, "B"
-    chain = {"tc_state_fwd": 2 * f2(C, V, K), "tc_state_bwd": 3 * f2(C, V, K)}
+    chain = {"tc_state_fwd": 2 * f2(C, V, K), "tc_chains": 5 * f2(C, V, K)}
     if name in chain:
         return "tensor", chain[name] * ch, "flop"
     return None, None, None

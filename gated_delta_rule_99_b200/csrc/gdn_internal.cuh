@@ -103,7 +103,7 @@ enum KernelId : int32_t {
     kKTcPrep,
     kKTcStateFwd,
     kKTcOut,
-    kKTcStateBwd,
+    kKTcStateBwd,  // backward chains (forward recompute + reverse pass)
     kKTcGrads,
     kKTcLocal,
     kKernelCount

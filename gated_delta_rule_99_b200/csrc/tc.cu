@@ -19,6 +19,7 @@
 // sequence; one CTA per (sequence, head); writes the state entering every
 // chunk and U^T as swizzled tile images), tc_out (chunk-parallel output).
 #include "tc_common.cuh"
+#include "tc_state.cuh"
 
 namespace gdn {
 namespace {
@@ -171,128 +172,8 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
 }
 
 // ============================================================ tc_state_fwd
-// One CTA per (sequence, head); thread v owns row v of S (fp32 registers).
-struct StateSmem {
-    static constexpr int kS = 0, kUT = kS + 32768, kW0 = kUT + 16384, kKd0 = kW0 + 2 * 16384,
-                         kUt0 = kKd0 + 2 * 16384, kEnd = kUt0 + 2 * 16384;
-};
-constexpr int kStateSmem = StateSmem::kEnd + 1024;
-
-__device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p) {
-    load_image_async(sm + StateSmem::kW0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
-    load_image_async(sm + StateSmem::kKd0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
-    load_image_async(sm + StateSmem::kUt0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64);
-    cp_async_commit();
-}
-
 __global__ void __launch_bounds__(NT, 1) tc_state_fwd_kernel(Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
-    __shared__ uint32_t tslot;
-    if (p.hdr->status) return;
-    const int H = p.H, n = blockIdx.x / H, h = blockIdx.x % H, v = threadIdx.x;
-    float S[D];
-    if (p.h0) {
-        const float *h0 = p.h0 + ((size_t)n * H + h) * D * D;
-#pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = h0[kk * D + v];
-    } else {
-#pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
-    }
-    if (v == 0) {
-        mbar_init(&mbar, 1);
-        fence_mbar_init();
-    }
-    if (v < 32) {
-        tmem_alloc(&tslot, 256);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tslot;
-    const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
-    uint32_t phase = 0;
-    if (c0 < c1) state_prefetch(sm, 0, (size_t)c0 * H + h, p);
-    uint8_t *Ss = sm + StateSmem::kS, *UTs = sm + StateSmem::kUT;
-    const uint32_t id1 = idesc_bf16(128, 64, 0, 0), id2 = idesc_bf16(128, 128, 0, 1);
-    for (int c = c0; c < c1; ++c) {
-        const int buf = (c - c0) & 1;
-        const size_t ch = (size_t)c * H + h;
-        if (c + 1 < c1) {
-            state_prefetch(sm, buf ^ 1, ch + H, p);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        // the state entering this chunk, as bf16 operand rows
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        const float gC = expf(p.tG[ch * C + C - 1]);
-        operands_ready();
-        if (v == 0) {
-            const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
-            for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
-            mma_commit(&mbar);
-            bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128, sb, (uint32_t)kImg128);
-            bulk_commit();
-        }
-        if (!cta_wait(&mbar, phase, p, 3)) break;
-        phase ^= 1;
-        // U^T[v][i] = Ut[i][v] - (S W^T)[v][i]
-        const bf16 *Ut = reinterpret_cast<const bf16 *>(sm + StateSmem::kUt0 + buf * 16384);
-#pragma unroll
-        for (int c16 = 0; c16 < C; c16 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, c16), d);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 16; ++q) d[q] = __bfloat162float(Ut[(c16 + q) * D + v]) - d[q];
-            *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c16 / 8)) = pack8(d);
-            *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
-        }
-        operands_ready();
-        if (v == 0) {
-            const uint32_t ub = smem_u32(UTs), kb = smem_u32(sm + StateSmem::kKd0 + buf * 16384);
-            for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
-            mma_commit(&mbar);
-            bulk_store(static_cast<uint8_t *>(p.tUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
-            bulk_commit();
-        }
-        if (!cta_wait(&mbar, phase, p, 4)) break;
-        phase ^= 1;
-#pragma unroll
-        for (int c16 = 0; c16 < D; c16 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, 64 + c16), d);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 16; ++q) S[c16 + q] = fmaf(gC, S[c16 + q], d[q]);
-        }
-        // shared operands are rewritten next chunk: their bulk stores must have read them
-        if (v == 0) bulk_wait_read();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    }
-    if (v == 0) bulk_wait_all();
-    if (p.hT) {
-        float *hT = p.hT + ((size_t)n * H + h) * D * D;
-#pragma unroll
-        for (int kk = 0; kk < D; ++kk) hT[kk * D + v] = S[kk];
-    }
-    cp_async_wait<0>();
-    tc_fence_before();
-    __syncthreads();
-    if (v < 32) tmem_dealloc(tmem, 256);
+    state_fwd_body(p, blockIdx.x);
 }
 
 // ============================================================ tc_out

@@ -19,11 +19,11 @@
 // 128 TMEM lanes (M = 128 over the key or value dim); 64 x 64 products use the
 // M = 64 form (row m in lane 32 (m / 16) + m % 16).
 #include "tc_common.cuh"
+#include "tc_state.cuh"
 
 namespace gdn {
 
 cudaError_t tc_launch_prep(const Params &p, int want_A, cudaStream_t stream);
-cudaError_t tc_launch_state_fwd(const Params &p, cudaStream_t stream);
 
 namespace {
 
@@ -107,13 +107,13 @@ __global__ void __launch_bounds__(NT) tc_local_kernel(Params p) {
         ok = cta_wait(&mbar, 1, p, 12);
     }
     if (ok) {
-        bf16 *dul = static_cast<bf16 *>(p.tdUL) + (size_t)ch * D * C + (size_t)tid * C;
+        uint8_t *dul = static_cast<uint8_t *>(p.tdUL) + (size_t)ch * kImgUT;
         for (int c0 = 0; c0 < C; c0 += 16) {
             float d[16];
             tmem_ld16(tm(tmem, 64 + c0), d);
             tmem_ld_wait();
-            *reinterpret_cast<uint4 *>(dul + c0) = pack8(d);
-            *reinterpret_cast<uint4 *>(dul + c0 + 8) = pack8(d + 8);
+            *reinterpret_cast<uint4 *>(dul + sw128_chunk(D, tid, c0 / 8)) = pack8(d);
+            *reinterpret_cast<uint4 *>(dul + sw128_chunk(D, tid, c0 / 8 + 1)) = pack8(d + 8);
         }
     }
     tc_fence_before();
@@ -143,13 +143,14 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
     cp_async_commit();
 }
 
-__global__ void __launch_bounds__(NT, 1) tc_state_bwd_kernel(Params p) {
+// Body of the reverse state pass for CTA `blk` (sequence blk / H, head blk % H).
+__device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
-    const int H = p.H, n = blockIdx.x / H, h = blockIdx.x % H, v = threadIdx.x;
+    const int H = p.H, n = blk / H, h = blk % H, v = threadIdx.x;
     float S[D];  // dS row v (gradient of the state leaving the current chunk)
     if (p.dhT) {
         const float *g0 = p.dhT + ((size_t)n * H + h) * D * D;
@@ -208,15 +209,16 @@ __global__ void __launch_bounds__(NT, 1) tc_state_bwd_kernel(Params p) {
         if (!cta_wait(&mbar, phase, p, 13)) break;
         phase ^= 1;
         {  // dU^T = dS Kd^T + local dU^T ; -dU^T is the next operand, +dU^T an image for tc_grads
-            const bf16 *dul = reinterpret_cast<const bf16 *>(b + SbwdSmem::kDUL) + v * C;
+            const uint8_t *dul = b + SbwdSmem::kDUL;  // local dU^T, swizzled rows
             uint8_t *img = static_cast<uint8_t *>(p.tdUT) + ch * kImgUT;
 #pragma unroll
             for (int c16 = 0; c16 < C; c16 += 16) {
                 float d[16], l[16];
                 tmem_ld16(tm(tmem, c16), d);
                 tmem_ld_wait();
-                unpack8(*reinterpret_cast<const uint4 *>(dul + c16), l);
-                unpack8(*reinterpret_cast<const uint4 *>(dul + c16 + 8), l + 8);
+                unpack8(*reinterpret_cast<const uint4 *>(dul + sw128_chunk(D, v, c16 / 8)), l);
+                unpack8(*reinterpret_cast<const uint4 *>(dul + sw128_chunk(D, v, c16 / 8 + 1)),
+                        l + 8);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) d[q] += l[q];
                 *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, c16 / 8)) = pack8(d);
@@ -261,16 +263,28 @@ __global__ void __launch_bounds__(NT, 1) tc_state_bwd_kernel(Params p) {
     if (v < 32) tmem_dealloc(tmem, 256);
 }
 
+// Both chains of the backward in one launch: CTAs [0, N*H) recompute the
+// forward states (pf has no final-state output), CTAs [N*H, 2*N*H) run the
+// reverse pass.  They are independent, so each gets its own SMs.
+__global__ void __launch_bounds__(NT, 1) tc_chains_kernel(Params pf, Params pb) {
+    const int nh = pb.N * pb.H;
+    if ((int)blockIdx.x < nh) state_fwd_body(pf, blockIdx.x);
+    else state_bwd_body(pb, blockIdx.x - nh);
+}
+
 // ============================================================ tc_grads
 struct GradSmem {
     static constexpr int kQK = 0, kDO = 32768, kV = 49152, kSC = 65536, kDSN = 98304,
                          kUT = 131072, kDUT = 147456, kAB = 163840, kX3 = 172032,
                          kDA = 188416, kT1 = 196608, kDPG = 204800, kDLG = 212992,
                          kVec = 221184, kEnd = kVec + 10 * 256;
-    // reused after the first products: fp32 64x64 P (then dP.P + dL.L) and Gam.KK^T,
-    // and a [128 threads][64] reduction buffer
-    static constexpr int kPE = kSC, kKKG = kSC + 16384, kRed = kDSN;
+    // reused after the first products (the images there are consumed): fp32
+    // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, and a [128 threads][65]
+    // reduction buffer; rows padded to 65 floats so row-strided access is
+    // free of bank conflicts
+    static constexpr int kPE = kSC, kKKG = kSC + 64 * 65 * 4, kRed = kDSN + 1024;
 };
+constexpr int LP = 65;  // padded row stride (floats) of the fp32 scratch
 constexpr int kGradSmem = GradSmem::kEnd + 1024;
 
 // Deterministic column sums of red[t][i] over the 128 threads t -> out[i].
@@ -278,7 +292,7 @@ __device__ __forceinline__ void reduce_rows(const float *red, float *out) {
     __syncthreads();
     if (threadIdx.x < C) {
         float s = 0.f;
-        for (int t = 0; t < NT; ++t) s += red[t * C + threadIdx.x];
+        for (int t = 0; t < NT; ++t) s += red[t * LP + threadIdx.x];
         out[threadIdx.x] = s;
     }
     __syncthreads();
@@ -404,8 +418,8 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             for (int q = 0; q < 16; ++q) {
                 const int j = c0 + q;
                 const float gij = expf(G[i] - G[j]);
-                if (isP) PE[i * C + j] = j <= i ? p.scale * gij * d[q] : 0.f;
-                else KKG[i * C + j] = j < i ? gij * d[q] : 0.f;
+                if (isP) PE[i * LP + j] = j <= i ? p.scale * gij * d[q] : 0.f;
+                else KKG[i * LP + j] = j < i ? gij * d[q] : 0.f;
             }
         }
     }
@@ -418,7 +432,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
                 const int i = c0 + q;
-                RED[tid * C + i] = sw_elem(VT, C, i, tid) * d[q];
+                RED[tid * LP + i] = sw_elem(VT, C, i, tid) * d[q];
                 if (i < ci.len)
                     dv[((int64_t)(ci.tok0 + i) * H + h) * D + tid] = __float2bfloat16_rn(bta[i] * d[q]);
             }
@@ -432,7 +446,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 16; ++q)
-                RED[tid * C + c0 + q] = p.scale * sw_elem(QK, D, c0 + q, tid) * d[q];
+                RED[tid * LP + c0 + q] = p.scale * sw_elem(QK, D, c0 + q, tid) * d[q];
         }
         reduce_rows(RED, qx);
         for (int c0 = 0; c0 < C; c0 += 16) {
@@ -440,7 +454,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             tmem_ld16(tm(tmem, cX2 + c0), d);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) RED[tid * C + c0 + q] = sw_elem(QK, D, C + c0 + q, tid) * d[q];
+            for (int q = 0; q < 16; ++q) RED[tid * LP + c0 + q] = sw_elem(QK, D, C + c0 + q, tid) * d[q];
         }
         reduce_rows(RED, kx);
         for (int c0 = 0; c0 < C; c0 += 16) {
@@ -462,7 +476,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
                 for (int q = 0; q < 16; ++q) {
                     const int j = c0 + q;
                     const float dp = j <= i ? d[q] : 0.f;
-                    PE[i * C + j] *= dp;
+                    PE[i * LP + j] *= dp;
                     d[q] = dp * (j <= i ? expf(G[i] - G[j]) : 0.f);
                 }
                 *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i, c0 / 8)) = pack8(d);
@@ -504,7 +518,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             tmem_ld16(tm(tmem, cZ + c0), d);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) RED[tid * C + c0 + q] = -sw_elem(QK, D, C + c0 + q, tid) * d[q];
+            for (int q = 0; q < 16; ++q) RED[tid * LP + c0 + q] = -sw_elem(QK, D, C + c0 + q, tid) * d[q];
         }
         reduce_rows(RED, kz);
     }
@@ -552,8 +566,8 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
                 for (int q = 0; q < 16; ++q) {
                     const int j = c0 + q;
                     const float dl = j < i ? -d[q] : 0.f;
-                    const float kkg = KKG[i * C + j];
-                    PE[i * C + j] += dl * bta[i] * kkg;
+                    const float kkg = KKG[i * LP + j];
+                    PE[i * LP + j] += dl * bta[i] * kkg;
                     dbl = fmaf(dl, kkg, dbl);
                     d[q] = bta[i] * dl * (j < i ? expf(G[i] - G[j]) : 0.f);
                 }
@@ -581,8 +595,8 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
         const int i = tid;
         float rs = 0.f, cs = 0.f;
         for (int j = 0; j < C; ++j) {
-            rs += PE[i * C + j];
-            cs += PE[j * C + i];
+            rs += PE[i * LP + j];
+            cs += PE[j * LP + i];
         }
         dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + rs - cs + bta[i] * gam[i] * kz[i];
     }
@@ -651,15 +665,14 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
     Params pf = p;
     pf.hT = nullptr;
     if ((e = tc_launch_prep(p, 1, stream))) return e;
-    if ((e = tc_launch_state_fwd(pf, stream))) return e;
     if (nch > 0) {
         if ((e = set_smem(tc_local_kernel, kLocalSmem))) return e;
         GDN_LAUNCH(kKTcLocal, stream, tc_local_kernel<<<nch, NT, kLocalSmem, stream>>>(p));
     }
     if (nseq > 0) {
-        if ((e = set_smem(tc_state_bwd_kernel, kSbwdSmem))) return e;
-        GDN_LAUNCH(kKTcStateBwd, stream,
-                   tc_state_bwd_kernel<<<nseq, NT, kSbwdSmem, stream>>>(p));
+        const int sm = kSbwdSmem > kStateSmem ? kSbwdSmem : kStateSmem;
+        if ((e = set_smem(tc_chains_kernel, sm))) return e;
+        GDN_LAUNCH(kKTcStateBwd, stream, tc_chains_kernel<<<2 * nseq, NT, sm, stream>>>(pf, p));
     }
     if (nch > 0) {
         if ((e = set_smem(tc_grads_kernel, kGradSmem))) return e;
