@@ -273,27 +273,36 @@ __global__ void __launch_bounds__(NT, 1) tc_chains_kernel(Params pf, Params pb) 
 }
 
 // ============================================================ tc_grads
+// Two warpgroups (256 threads): warp w reaches TMEM lane quadrant w % 4, so
+// for every accumulator warpgroup g handles columns [32 g, 32 g + 32).
+constexpr int NG = 256;
+
 struct GradSmem {
     static constexpr int kQK = 0, kDO = 32768, kV = 49152, kSC = 65536, kDSN = 98304,
                          kUT = 131072, kDUT = 147456, kAB = 163840, kX3 = 172032,
                          kDA = 188416, kT1 = 196608, kDPG = 204800, kDLG = 212992,
-                         kVec = 221184, kEnd = kVec + 10 * 256;
-    // reused after the first products (the images there are consumed): fp32
-    // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, and a [128 threads][65]
-    // reduction buffer; rows padded to 65 floats so row-strided access is
-    // free of bank conflicts
-    static constexpr int kPE = kSC, kKKG = kSC + 64 * 65 * 4, kRed = kDSN + 1024;
+                         kVec = 221184, kEnd = kVec + 12 * 256;
+    // reused once the first products have consumed the images there: fp32
+    // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, a [128][65] reduction
+    // buffer, and the 64 x 64 decay matrix Gam (columns xor-swizzled by row)
+    static constexpr int kPE = kSC, kKKG = kSC + 64 * 65 * 4, kRed = kDSN + 1024,
+                         kGam = kDUT;
 };
-constexpr int LP = 65;  // padded row stride (floats) of the fp32 scratch
 constexpr int kGradSmem = GradSmem::kEnd + 1024;
+constexpr int LP = 65;  // padded row stride (floats) of the fp32 scratch
 
-// Deterministic column sums of red[t][i] over the 128 threads t -> out[i].
+__device__ __forceinline__ int gidx(int i, int j) { return i * 64 + (j ^ (i & 31)); }
+
+// Deterministic column sums of red[t][i] over the 128 rows t -> out[i].
 __device__ __forceinline__ void reduce_rows(const float *red, float *out) {
     __syncthreads();
     if (threadIdx.x < C) {
-        float s = 0.f;
-        for (int t = 0; t < NT; ++t) s += red[t * LP + threadIdx.x];
-        out[threadIdx.x] = s;
+        float s0 = 0.f, s1 = 0.f;
+        for (int t = 0; t < 128; t += 2) {
+            s0 += red[t * LP + threadIdx.x];
+            s1 += red[(t + 1) * LP + threadIdx.x];
+        }
+        out[threadIdx.x] = s0 + s1;
     }
     __syncthreads();
 }
@@ -302,7 +311,14 @@ __device__ __forceinline__ float sw_elem(const uint8_t *tile, int R, int r, int 
     return __bfloat162float(*reinterpret_cast<const bf16 *>(tile + sw128_off(R, r, c)));
 }
 
-__global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
+// 32 consecutive fp32 columns of this thread's TMEM lane (quadrant w % 4).
+__device__ __forceinline__ void ld32(uint32_t tmem, int col, float *d) {
+    tmem_ld16(tmq(tmem, col), d);
+    tmem_ld16(tmq(tmem, col + 16), d + 16);
+    tmem_ld_wait();
+}
+
+__global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar;
@@ -310,6 +326,8 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
     __shared__ float s_hd;
     if (p.hdr->status) return;
     const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
+    const int wg = tid >> 7, r = tid & 127, cb = 32 * wg;
+    const int l = tid & 31, i64 = l < 16 ? ((tid >> 5) & 3) * 16 + l : -1;  // M = 64 row
     const ChunkInfo ci = p.chunks[c];
     using S_ = GradSmem;
     uint8_t *QK = sm + S_::kQK, *DO = sm + S_::kDO, *VT = sm + S_::kV, *SC = sm + S_::kSC,
@@ -318,19 +336,22 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             *DLG = sm + S_::kDLG;
     float *vec = reinterpret_cast<float *>(sm + S_::kVec);
     float *G = vec, *bta = vec + 64, *gam = vec + 128, *e = vec + 192, *dB = vec + 256,
-          *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576;
+          *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576,
+          *dbl2 = vec + 640;
     float *PE = reinterpret_cast<float *>(sm + S_::kPE);
     float *KKG = reinterpret_cast<float *>(sm + S_::kKKG);
     float *RED = reinterpret_cast<float *>(sm + S_::kRed);
+    float *Gam = reinterpret_cast<float *>(sm + S_::kGam);
 
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
-    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H);
-    load_rows_async(VT, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H);
-    load_image_async(SC, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128);
-    load_image_async(DSN, static_cast<const uint8_t *>(p.tdSn) + (size_t)ch * kImg128, kImg128);
-    load_image_async(UT, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT);
-    load_image_async(DUT, static_cast<const uint8_t *>(p.tdUT) + (size_t)ch * kImgUT, kImgUT);
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, NG);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, NG);
+    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H, NG);
+    load_rows_async(VT, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H, NG);
+    load_image_async(SC, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128, NG);
+    load_image_async(DSN, static_cast<const uint8_t *>(p.tdSn) + (size_t)ch * kImg128, kImg128,
+                     NG);
+    load_image_async(UT, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT, NG);
+    load_image_async(DUT, static_cast<const uint8_t *>(p.tdUT) + (size_t)ch * kImgUT, kImgUT, NG);
     cp_async_commit();
     if (tid < C) {
         const int64_t idx = (int64_t)(ci.tok0 + tid) * H + h;
@@ -339,8 +360,8 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
     }
     {  // A (fp32, from tc_prep) as a bf16 tile: rows m, columns i
         const float *Ag = p.tA + (size_t)ch * C * C;
-        for (int t = tid; t < C * C; t += NT) {
-            const int m = t / C, i = t % C;
+        for (int t = tid; t < C * C; t += NG) {
+            const int m = t >> 6, i = t & 63;
             *reinterpret_cast<bf16 *>(AB + sw128_off(C, m, i)) = __float2bfloat16_rn(Ag[t]);
         }
     }
@@ -369,6 +390,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
                   cY2 = 0, cZ = 448, cT1 = 192, cDL = 0, cDQ = 256, cDK = 320, cDKA = 384;
     uint32_t phase = 0;
     bool ok;
+    float d[32];
     if (tid == 0) {
         const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
                        i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
@@ -392,9 +414,14 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
     ok = cta_wait(&mbar, phase, p, 21);
     phase ^= 1;
     if (!ok) goto done;
+    // the decay matrix, once (the dU^T image there is consumed)
+    for (int t = tid; t < C * C; t += NG) {
+        const int i = t >> 6, j = t & 63;
+        Gam[gidx(i, j)] = j <= i ? expf(G[i] - G[j]) : 0.f;
+    }
     {  // <S, dSn> (elementwise over identically laid out images)
         float s = 0.f;
-        for (int t = tid; t < D * D / 8; t += NT) {
+        for (int t = tid; t < D * D / 8; t += NG) {
             float a[8], b[8];
             unpack8(*reinterpret_cast<const uint4 *>(SC + t * 16), a);
             unpack8(*reinterpret_cast<const uint4 *>(DSN + t * 16), b);
@@ -402,87 +429,67 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             for (int q = 0; q < 8; ++q) s = fmaf(a[q], b[q], s);
         }
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if ((tid & 31) == 0) tmp[tid >> 5] = s;
+        if (l == 0) tmp[tid >> 5] = s;
         __syncthreads();
-        if (tid == 0) s_hd = tmp[0] + tmp[1] + tmp[2] + tmp[3];
+        if (tid == 0) {
+            float a = 0.f;
+            for (int w = 0; w < NG / 32; ++w) a += tmp[w];
+            s_hd = a;
+        }
         __syncthreads();
     }
-    {  // P (scaled, lower incl. diagonal) and Gam . K K^T (strictly lower), fp32
-        const int i = tid & 63;
-        const bool isP = tid < 64;
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cQK + c0), d);
-            tmem_ld_wait();
+    // P (scaled, lower incl. diagonal) and Gam . K K^T (strictly lower), fp32
+    ld32(tmem, cQK + cb, d);
+    if (r < 64) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int j = c0 + q;
-                const float gij = expf(G[i] - G[j]);
-                if (isP) PE[i * LP + j] = j <= i ? p.scale * gij * d[q] : 0.f;
-                else KKG[i * LP + j] = j < i ? gij * d[q] : 0.f;
-            }
+        for (int q = 0; q < 32; ++q) {
+            const int j = cb + q;
+            PE[r * LP + j] = j <= r ? p.scale * Gam[gidx(r, j)] * d[q] : 0.f;
+        }
+    } else {
+        const int i = r - 64;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int j = cb + q;
+            KKG[i * LP + j] = j < i ? Gam[gidx(i, j)] * d[q] : 0.f;
         }
     }
     {  // dv = diag(b) A^T dU ; partial v . (A^T dU)
         bf16 *dv = static_cast<bf16 *>(p.dv);
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cAU + c0), d);
-            tmem_ld_wait();
+        ld32(tmem, cAU + cb, d);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int i = c0 + q;
-                RED[tid * LP + i] = sw_elem(VT, C, i, tid) * d[q];
-                if (i < ci.len)
-                    dv[((int64_t)(ci.tok0 + i) * H + h) * D + tid] = __float2bfloat16_rn(bta[i] * d[q]);
-            }
+        for (int q = 0; q < 32; ++q) {
+            const int i = cb + q;
+            RED[r * LP + i] = sw_elem(VT, C, i, r) * d[q];
+            if (i < ci.len)
+                dv[((int64_t)(ci.tok0 + i) * H + h) * D + r] = __float2bfloat16_rn(bta[i] * d[q]);
         }
         reduce_rows(RED, dB);
     }
-    {  // partial q' . X1 and k . X2 (thread kk), then X3^T as an operand tile (row kk)
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cX1 + c0), d);
-            tmem_ld_wait();
+    ld32(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-                RED[tid * LP + c0 + q] = p.scale * sw_elem(QK, D, c0 + q, tid) * d[q];
-        }
-        reduce_rows(RED, qx);
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cX2 + c0), d);
-            tmem_ld_wait();
+    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = p.scale * sw_elem(QK, D, cb + q, r) * d[q];
+    reduce_rows(RED, qx);
+    ld32(tmem, cX2 + cb, d);  // partial k . X2
 #pragma unroll
-            for (int q = 0; q < 16; ++q) RED[tid * LP + c0 + q] = sw_elem(QK, D, C + c0 + q, tid) * d[q];
-        }
-        reduce_rows(RED, kx);
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cX3 + c0), d);
-            tmem_ld_wait();
-            *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, tid, c0 / 8)) = pack8(d);
-            *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, tid, c0 / 8 + 1)) = pack8(d + 8);
-        }
-    }
-    {  // dP: dPG = dP . Gam as an operand tile; PE <- dP . P
-        const int i = m64_row();
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cDP + c0), d);
-            tmem_ld_wait();
-            if (i >= 0) {
+    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = sw_elem(QK, D, C + cb + q, r) * d[q];
+    reduce_rows(RED, kx);
+    ld32(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int j = c0 + q;
-                    const float dp = j <= i ? d[q] : 0.f;
-                    PE[i * LP + j] *= dp;
-                    d[q] = dp * (j <= i ? expf(G[i] - G[j]) : 0.f);
-                }
-                *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i, c0 / 8)) = pack8(d);
-                *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
-            }
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
+    ld32(tmem, cDP + cb, d);  // dP: dPG = dP . Gam as an operand tile; PE <- dP . P
+    if (i64 >= 0) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int j = cb + q;
+            const float dp = j <= i64 ? d[q] : 0.f;
+            PE[i64 * LP + j] *= dp;
+            d[q] = dp * Gam[gidx(i64, j)];
         }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
     }
     operands_ready();
     if (tid == 0) {
@@ -497,31 +504,24 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
     phase ^= 1;
     if (!ok) goto done;
     {  // dA = (dU V^T) diag(b) - (X3 K^T) diag(b gam)
-        const int i = m64_row();
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float y1[16], y2[16];
-            tmem_ld16(tm(tmem, cY1 + c0), y1);
-            tmem_ld16(tm(tmem, cY2 + c0), y2);
-            tmem_ld_wait();
-            if (i >= 0) {
+        float y2[32];
+        ld32(tmem, cY1 + cb, d);
+        ld32(tmem, cY2 + cb, y2);
+        if (i64 >= 0) {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int m = c0 + q;
-                    y1[q] = bta[m] * y1[q] - bta[m] * gam[m] * y2[q];
-                }
-                *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i, c0 / 8)) = pack8(y1);
-                *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(y1 + 8);
+            for (int q = 0; q < 32; ++q) {
+                const int m = cb + q;
+                d[q] = bta[m] * d[q] - bta[m] * gam[m] * y2[q];
             }
-        }
-        for (int c0 = 0; c0 < C; c0 += 16) {  // partial k . Z = -k . Zp
-            float d[16];
-            tmem_ld16(tm(tmem, cZ + c0), d);
-            tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) RED[tid * LP + c0 + q] = -sw_elem(QK, D, C + c0 + q, tid) * d[q];
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
         }
-        reduce_rows(RED, kz);
     }
+    ld32(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
+#pragma unroll
+    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = -sw_elem(QK, D, C + cb + q, r) * d[q];
+    reduce_rows(RED, kz);
     operands_ready();
     if (tid == 0) {  // T1 = A^T dA (M = 64)
         const uint32_t id = idesc_bf16(64, 64, 1, 1);
@@ -532,17 +532,11 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
     ok = cta_wait(&mbar, phase, p, 23);
     phase ^= 1;
     if (!ok) goto done;
-    {
-        const int i = m64_row();
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cT1 + c0), d);
-            tmem_ld_wait();
-            if (i >= 0) {
-                *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i, c0 / 8)) = pack8(d);
-                *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
-            }
-        }
+    ld32(tmem, cT1 + cb, d);
+    if (i64 >= 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
     }
     operands_ready();
     if (tid == 0) {  // T1 A^T = -dL (M = 64)
@@ -554,28 +548,23 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
     ok = cta_wait(&mbar, phase, p, 24);
     phase ^= 1;
     if (!ok) goto done;
-    {  // dL (strictly lower); diag(b) dL . Gam as an operand tile; PE += dL . L; dbeta terms
-        const int i = m64_row();
+    ld32(tmem, cDL + cb, d);  // dL (strictly lower); diag(b) dL . Gam tile; PE += dL . L
+    if (i64 >= 0) {
         float dbl = 0.f;
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, cDL + c0), d);
-            tmem_ld_wait();
-            if (i >= 0) {
+        const float bi = bta[i64];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int j = c0 + q;
-                    const float dl = j < i ? -d[q] : 0.f;
-                    const float kkg = KKG[i * LP + j];
-                    PE[i * LP + j] += dl * bta[i] * kkg;
-                    dbl = fmaf(dl, kkg, dbl);
-                    d[q] = bta[i] * dl * (j < i ? expf(G[i] - G[j]) : 0.f);
-                }
-                *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i, c0 / 8)) = pack8(d);
-                *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
-            }
+        for (int q = 0; q < 32; ++q) {
+            const int j = cb + q;
+            const float dl = j < i64 ? -d[q] : 0.f;
+            const float kkg = KKG[i64 * LP + j];
+            PE[i64 * LP + j] += dl * bi * kkg;
+            dbl = fmaf(dl, kkg, dbl);
+            d[q] = bi * dl * Gam[gidx(i64, j)];
         }
-        if (i >= 0) dB[i] += dbl + gam[i] * kz[i];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
+        dbl2[wg * 64 + i64] = dbl;
     }
     operands_ready();
     if (tid == 0) {
@@ -590,7 +579,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_mnmajor(dlb, C, s), imm, 1);
         mma_commit(&mbar);
     }
-    // meanwhile: dG and dbeta (rows), then dg = reverse cumulative sum of dG
+    // meanwhile: dbeta and dG (rows), then dg = reverse cumulative sum of dG
     if (tid < C) {
         const int i = tid;
         float rs = 0.f, cs = 0.f;
@@ -599,6 +588,7 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
             cs += PE[j * LP + i];
         }
         dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + rs - cs + bta[i] * gam[i] * kz[i];
+        dB[i] += dbl2[i] + dbl2[64 + i] + gam[i] * kz[i];
     }
     __syncthreads();
     if (tid == 0) {
@@ -622,33 +612,29 @@ __global__ void __launch_bounds__(NT, 1) tc_grads_kernel(Params p) {
     if (!ok) goto done;
     {  // dq = scale (diag(gam) X1 + dPG K) ; dk = diag(e) X2 + diag(b gam) Z + dPG^T Q' + dL terms
         bf16 *dq = static_cast<bf16 *>(p.dq), *dk = static_cast<bf16 *>(p.dk);
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float x1[16], a[16];
-            tmem_ld16(tm(tmem, cX1 + c0), x1);
-            tmem_ld16(tm(tmem, cDQ + c0), a);
-            tmem_ld_wait();
+        float a[32];
+        ld32(tmem, cX1 + cb, d);
+        ld32(tmem, cDQ + cb, a);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int i = c0 + q;
-                if (i < ci.len)
-                    dq[((int64_t)(ci.tok0 + i) * H + h) * D + tid] =
-                        __float2bfloat16_rn(p.scale * (gam[i] * x1[q] + a[q]));
-            }
+        for (int q = 0; q < 32; ++q) {
+            const int i = cb + q;
+            if (i < ci.len)
+                dq[((int64_t)(ci.tok0 + i) * H + h) * D + r] =
+                    __float2bfloat16_rn(p.scale * (gam[i] * d[q] + a[q]));
         }
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float x2[16], z[16], ka[16], kd[16];
-            tmem_ld16(tm(tmem, cX2 + c0), x2);
-            tmem_ld16(tm(tmem, cZ + c0), z);
-            tmem_ld16(tm(tmem, cDKA + c0), ka);
-            tmem_ld16(tm(tmem, cDK + c0), kd);
-            tmem_ld_wait();
+        ld32(tmem, cX2 + cb, d);
+        ld32(tmem, cZ + cb, a);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int i = c0 + q;
-                if (i < ci.len)
-                    dk[((int64_t)(ci.tok0 + i) * H + h) * D + tid] = __float2bfloat16_rn(
-                        e[i] * x2[q] - bta[i] * gam[i] * z[q] + p.scale * ka[q] + kd[q]);
-            }
+        for (int q = 0; q < 32; ++q) d[q] = e[cb + q] * d[q] - bta[cb + q] * gam[cb + q] * a[q];
+        ld32(tmem, cDKA + cb, a);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) d[q] += p.scale * a[q];
+        ld32(tmem, cDK + cb, a);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int i = cb + q;
+            if (i < ci.len)
+                dk[((int64_t)(ci.tok0 + i) * H + h) * D + r] = __float2bfloat16_rn(d[q] + a[q]);
         }
     }
 done:
@@ -676,7 +662,7 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
     }
     if (nch > 0) {
         if ((e = set_smem(tc_grads_kernel, kGradSmem))) return e;
-        GDN_LAUNCH(kKTcGrads, stream, tc_grads_kernel<<<nch, NT, kGradSmem, stream>>>(p));
+        GDN_LAUNCH(kKTcGrads, stream, tc_grads_kernel<<<nch, NG, kGradSmem, stream>>>(p));
     }
     return cudaSuccess;
 }

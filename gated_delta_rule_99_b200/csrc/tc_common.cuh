@@ -53,9 +53,10 @@ __device__ __forceinline__ void operands_ready() {
 // into an SW128 tile with R rows (block stride), starting at row `row0`;
 // rows at or past `len` are zero.  Asynchronous (cp.async).
 __device__ __forceinline__ void load_rows_async(uint8_t *tile, int R, int row0, const bf16 *src,
-                                                int64_t tok0, int len, int h, int H) {
+                                                int64_t tok0, int len, int h, int H,
+                                                int nthreads = NT) {
     const uint32_t base = smem_u32(tile);
-    for (int t = threadIdx.x; t < C * 16; t += NT) {
+    for (int t = threadIdx.x; t < C * 16; t += nthreads) {
         const int r = t >> 4, j = t & 15;
         const bool valid = r < len;
         const bf16 *g = valid ? src + ((tok0 + r) * H + h) * D + j * 8 : src;
@@ -64,10 +65,11 @@ __device__ __forceinline__ void load_rows_async(uint8_t *tile, int R, int row0, 
 }
 
 // Linear copy of a tile image (bytes multiple of 16 * NT).
-__device__ __forceinline__ void load_image_async(uint8_t *tile, const void *img, size_t bytes) {
+__device__ __forceinline__ void load_image_async(uint8_t *tile, const void *img, size_t bytes,
+                                                 int nthreads = NT) {
     const uint32_t base = smem_u32(tile);
     const uint8_t *g = static_cast<const uint8_t *>(img);
-    for (size_t off = (size_t)threadIdx.x * 16; off < bytes; off += NT * 16)
+    for (size_t off = (size_t)threadIdx.x * 16; off < bytes; off += (size_t)nthreads * 16)
         cp_async16(base + (uint32_t)off, g + off);
 }
 
@@ -113,6 +115,12 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
 // TMEM address of (lane base of this warp, column col).
 __device__ __forceinline__ uint32_t tm(uint32_t tmem, int col) {
     return tmem + ((uint32_t)((threadIdx.x >> 5) * 32) << 16) + (uint32_t)col;
+}
+
+// TMEM address for CTAs of more than four warps: warp w reaches the lane
+// quadrant w % 4 only.
+__device__ __forceinline__ uint32_t tmq(uint32_t tmem, int col) {
+    return tmem + ((uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16) + (uint32_t)col;
 }
 
 // Row of a 64-row (M = 64) accumulator held by this thread's lane, or -1.
