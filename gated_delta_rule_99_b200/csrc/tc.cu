@@ -35,7 +35,7 @@ struct PrepSmem {
                          kEnd = kB + 256;
 };
 constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
-constexpr int kPrepSmemRequest = 100 * 1024;  // at most two CTAs per SM (TMEM: 256 columns each)
+constexpr int kPrepSmemRequest = 72 * 1024;  // at most three CTAs per SM (TMEM: 128 columns each)
 
 __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
     extern __shared__ uint8_t smem_raw[];
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
         fence_mbar_init();
     }
     if (tid < 32) {
-        tmem_alloc(&tslot, 256);
+        tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
     chunk_gates(G, bta, p, ci, h);
@@ -117,9 +117,16 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
             float a[C];
 #pragma unroll
             for (int r = 0; r < C; ++r) {
-                float s = 0.f;
+                // four independent partial sums shorten the dependent chain
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                for (int m = 0; m < r; ++m) s = fmaf(L[r * 65 + m], a[m], s);
+                for (int m = 0; m < r; m += 4) {
+                    s0 = fmaf(L[r * 65 + m], a[m], s0);
+                    if (m + 1 < r) s1 = fmaf(L[r * 65 + m + 1], a[m + 1], s1);
+                    if (m + 2 < r) s2 = fmaf(L[r * 65 + m + 2], a[m + 2], s2);
+                    if (m + 3 < r) s3 = fmaf(L[r * 65 + m + 3], a[m + 3], s3);
+                }
+                const float s = (s0 + s1) + (s2 + s3);
                 a[r] = r < j ? 0.f : (r == j ? 1.f : -s);
             }
             const float bg = bta[j] * expf(G[j]), b = bta[j];
@@ -135,32 +142,50 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
             }
         }
         operands_ready();
-        // W = (A diag(b gam)) K and Ut = (A diag(b)) V: M = 64, N = 128, K = 64 tokens
+        // W = (A diag(b gam)) K, then Ut = (A diag(b)) V: M = 64, N = 128, K = 64 tokens,
+        // one after the other in the same 128 TMEM columns
+        const uint32_t id = idesc_bf16(64, 128, 0, 1);
         if (tid == 0) {
-            const uint32_t id = idesc_bf16(64, 128, 0, 1);
-            const uint32_t ab = smem_u32(Ab), ac = smem_u32(Ac), kb = smem_u32(Kt),
-                           vb = smem_u32(Vt);
+            const uint32_t ab = smem_u32(Ab), kb = smem_u32(Kt);
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem, desc_kmajor(ab, C, s), desc_mnmajor(kb, C, s), id, s > 0);
-            for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 128, desc_kmajor(ac, C, s), desc_mnmajor(vb, C, s), id, s > 0);
             mma_commit(&mbar);
         }
         ok = cta_wait(&mbar, phase, p, 2);
         phase ^= 1;
+        if (ok) {
+            const int i = m64_row();
+            uint8_t *Wimg = static_cast<uint8_t *>(p.tW) + (size_t)ch * kImg64;
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float w[16];
+                tmem_ld16(tm(tmem, c0), w);
+                tmem_ld_wait();
+                if (i >= 0) {
+                    *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8)) = pack8(w);
+                    *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(w + 8);
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+                const uint32_t ac = smem_u32(Ac), vb = smem_u32(Vt);
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tmem, desc_kmajor(ac, C, s), desc_mnmajor(vb, C, s), id, s > 0);
+                mma_commit(&mbar);
+            }
+            ok = cta_wait(&mbar, phase, p, 2);
+            phase ^= 1;
+        }
     }
     if (ok) {
         const int i = m64_row();
-        uint8_t *Wimg = static_cast<uint8_t *>(p.tW) + (size_t)ch * kImg64;
         bf16 *Ut = static_cast<bf16 *>(p.tUt) + (size_t)ch * C * D;
         for (int c0 = 0; c0 < D; c0 += 16) {
-            float w[16], u[16];
-            tmem_ld16(tm(tmem, c0), w);
-            tmem_ld16(tm(tmem, 128 + c0), u);
+            float u[16];
+            tmem_ld16(tm(tmem, c0), u);
             tmem_ld_wait();
             if (i >= 0) {
-                *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8)) = pack8(w);
-                *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(w + 8);
                 *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0) = pack8(u);
                 *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0 + 8) = pack8(u + 8);
             }
@@ -168,7 +193,7 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
     }
     tc_fence_before();
     __syncthreads();
-    if (tid < 32) tmem_dealloc(tmem, 256);
+    if (tid < 32) tmem_dealloc(tmem, 128);
 }
 
 // ============================================================ tc_state_fwd

@@ -281,7 +281,7 @@ struct GradSmem {
     static constexpr int kQK = 0, kDO = 32768, kV = 49152, kSC = 65536, kDSN = 98304,
                          kUT = 131072, kDUT = 147456, kAB = 163840, kX3 = 172032,
                          kDA = 188416, kT1 = 196608, kDPG = 204800, kDLG = 212992,
-                         kVec = 221184, kEnd = kVec + 12 * 256;
+                         kVec = 221184, kEnd = kVec + 16 * 256;
     // reused once the first products have consumed the images there: fp32
     // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, a [128][65] reduction
     // buffer, and the 64 x 64 decay matrix Gam (columns xor-swizzled by row)
@@ -293,23 +293,58 @@ constexpr int LP = 65;  // padded row stride (floats) of the fp32 scratch
 
 __device__ __forceinline__ int gidx(int i, int j) { return i * 64 + (j ^ (i & 31)); }
 
-// Deterministic column sums of red[t][i] over the 128 rows t -> out[i].
-__device__ __forceinline__ void reduce_rows(const float *red, float *out) {
+// Deterministic column sums of red[t][i] over the 128 rows t -> out[i]:
+// four threads per column each sum 32 rows, then one thread adds the four.
+__device__ __forceinline__ void reduce_rows(const float *red, float *out, float *part) {
     __syncthreads();
-    if (threadIdx.x < C) {
+    {
+        const int i = threadIdx.x & 63, k = threadIdx.x >> 6;
+        const float *src = red + k * 32 * LP + i;
         float s0 = 0.f, s1 = 0.f;
-        for (int t = 0; t < 128; t += 2) {
-            s0 += red[t * LP + threadIdx.x];
-            s1 += red[(t + 1) * LP + threadIdx.x];
+#pragma unroll
+        for (int t = 0; t < 32; t += 2) {
+            s0 += src[t * LP];
+            s1 += src[(t + 1) * LP];
         }
-        out[threadIdx.x] = s0 + s1;
+        part[k * 64 + i] = s0 + s1;
     }
+    __syncthreads();
+    if (threadIdx.x < C)
+        out[threadIdx.x] = (part[threadIdx.x] + part[64 + threadIdx.x]) +
+                           (part[128 + threadIdx.x] + part[192 + threadIdx.x]);
     __syncthreads();
 }
 
-__device__ __forceinline__ float sw_elem(const uint8_t *tile, int R, int r, int c) {
-    return __bfloat162float(*reinterpret_cast<const bf16 *>(tile + sw128_off(R, r, c)));
+// Column c of an SW128 tile with R rows, read row by row: the swizzle term
+// depends on the row only through row % 8, so it is computed once.
+struct ColSw {
+    const uint8_t *col;
+    uint32_t x[8];
+    __device__ __forceinline__ ColSw(const uint8_t *tile, int R, int c) {
+        col = tile + (c >> 6) * R * 128 + (c & 7) * 2;
+        const int cp = (c & 63) >> 3;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) x[b] = (uint32_t)((cp ^ b) << 4);
+    }
+    // row i = i0 + q with i0 a multiple of 8 and q a compile-time constant
+    __device__ __forceinline__ float at(int i0, int q) const {
+        return __bfloat162float(
+            *reinterpret_cast<const bf16 *>(col + (i0 + q) * 128 + x[q & 7]));
+    }
+};
+
+// Copies rows [0, len) of a 64 x 128 bf16 staging tile (plain rows) to one
+// chunk and head of a [tokens][H][128] tensor with 16-byte stores.
+__device__ __forceinline__ void store_rows(bf16 *dst, const uint8_t *stage, int64_t tok0, int len,
+                                           int h, int H) {
+    for (int t = threadIdx.x; t < C * 16; t += NG) {
+        const int i = t >> 4, j = t & 15;
+        if (i < len)
+            *reinterpret_cast<uint4 *>(dst + ((tok0 + i) * H + h) * D + j * 8) =
+                *reinterpret_cast<const uint4 *>(stage + i * 256 + j * 16);
+    }
 }
+
 
 // 32 consecutive fp32 columns of this thread's TMEM lane (quadrant w % 4).
 __device__ __forceinline__ void ld32(uint32_t tmem, int col, float *d) {
@@ -337,7 +372,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     float *vec = reinterpret_cast<float *>(sm + S_::kVec);
     float *G = vec, *bta = vec + 64, *gam = vec + 128, *e = vec + 192, *dB = vec + 256,
           *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576,
-          *dbl2 = vec + 640;
+          *dbl2 = vec + 640, *part = vec + 768;
     float *PE = reinterpret_cast<float *>(sm + S_::kPE);
     float *KKG = reinterpret_cast<float *>(sm + S_::kKKG);
     float *RED = reinterpret_cast<float *>(sm + S_::kRed);
@@ -359,10 +394,14 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         bta[tid] = tid < ci.len ? p.beta[idx] : 0.f;
     }
     {  // A (fp32, from tc_prep) as a bf16 tile: rows m, columns i
-        const float *Ag = p.tA + (size_t)ch * C * C;
-        for (int t = tid; t < C * C; t += NG) {
-            const int m = t >> 6, i = t & 63;
-            *reinterpret_cast<bf16 *>(AB + sw128_off(C, m, i)) = __float2bfloat16_rn(Ag[t]);
+        const float4 *Ag = reinterpret_cast<const float4 *>(p.tA + (size_t)ch * C * C);
+        for (int t = tid; t < C * C / 4; t += NG) {
+            const float4 a = Ag[t];
+            const int m = t >> 4, i = (t & 15) * 4;
+            uint2 u;
+            u.x = pack_bf16(a.x, a.y);
+            u.y = pack_bf16(a.z, a.w);
+            *reinterpret_cast<uint2 *>(AB + sw128_off(C, m, i)) = u;
         }
     }
     if (tid == 0) {
@@ -391,6 +430,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     uint32_t phase = 0;
     bool ok;
     float d[32];
+    const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
     if (tid == 0) {
         const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
                        i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
@@ -454,26 +494,27 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
             KKG[i * LP + j] = j < i ? Gam[gidx(i, j)] * d[q] : 0.f;
         }
     }
-    {  // dv = diag(b) A^T dU ; partial v . (A^T dU)
-        bf16 *dv = static_cast<bf16 *>(p.dv);
+    {  // dv = diag(b) A^T dU (staged as rows in the consumed dO tile); partial v . (A^T dU)
+        bf16 *stage = reinterpret_cast<bf16 *>(DO);
+        const ColSw vcol(VT, C, r);
         ld32(tmem, cAU + cb, d);
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
             const int i = cb + q;
-            RED[r * LP + i] = sw_elem(VT, C, i, r) * d[q];
-            if (i < ci.len)
-                dv[((int64_t)(ci.tok0 + i) * H + h) * D + r] = __float2bfloat16_rn(bta[i] * d[q]);
+            RED[r * LP + i] = vcol.at(cb, q) * d[q];
+            stage[i * D + r] = __float2bfloat16_rn(bta[i] * d[q]);
         }
-        reduce_rows(RED, dB);
+        reduce_rows(RED, dB, part);
+        store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H);
     }
     ld32(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
 #pragma unroll
-    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = p.scale * sw_elem(QK, D, cb + q, r) * d[q];
-    reduce_rows(RED, qx);
+    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = p.scale * qcol.at(cb, q) * d[q];
+    reduce_rows(RED, qx, part);
     ld32(tmem, cX2 + cb, d);  // partial k . X2
 #pragma unroll
-    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = sw_elem(QK, D, C + cb + q, r) * d[q];
-    reduce_rows(RED, kx);
+    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = kcol.at(cb, q) * d[q];
+    reduce_rows(RED, kx, part);
     ld32(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
 #pragma unroll
     for (int q = 0; q < 4; ++q)
@@ -520,8 +561,8 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     }
     ld32(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
 #pragma unroll
-    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = -sw_elem(QK, D, C + cb + q, r) * d[q];
-    reduce_rows(RED, kz);
+    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = -kcol.at(cb, q) * d[q];
+    reduce_rows(RED, kz, part);
     operands_ready();
     if (tid == 0) {  // T1 = A^T dA (M = 64)
         const uint32_t id = idesc_bf16(64, 64, 1, 1);
@@ -611,16 +652,15 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     phase ^= 1;
     if (!ok) goto done;
     {  // dq = scale (diag(gam) X1 + dPG K) ; dk = diag(e) X2 + diag(b gam) Z + dPG^T Q' + dL terms
-        bf16 *dq = static_cast<bf16 *>(p.dq), *dk = static_cast<bf16 *>(p.dk);
+        // staged as rows in the consumed dO and V tiles, then 16-byte stores
+        bf16 *sq = reinterpret_cast<bf16 *>(DO), *sk = reinterpret_cast<bf16 *>(VT);
         float a[32];
         ld32(tmem, cX1 + cb, d);
         ld32(tmem, cDQ + cb, a);
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
             const int i = cb + q;
-            if (i < ci.len)
-                dq[((int64_t)(ci.tok0 + i) * H + h) * D + r] =
-                    __float2bfloat16_rn(p.scale * (gam[i] * d[q] + a[q]));
+            sq[i * D + r] = __float2bfloat16_rn(p.scale * (gam[i] * d[q] + a[q]));
         }
         ld32(tmem, cX2 + cb, d);
         ld32(tmem, cZ + cb, a);
@@ -631,11 +671,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         for (int q = 0; q < 32; ++q) d[q] += p.scale * a[q];
         ld32(tmem, cDK + cb, a);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const int i = cb + q;
-            if (i < ci.len)
-                dk[((int64_t)(ci.tok0 + i) * H + h) * D + r] = __float2bfloat16_rn(d[q] + a[q]);
-        }
+        for (int q = 0; q < 32; ++q) sk[(cb + q) * D + r] = __float2bfloat16_rn(d[q] + a[q]);
+        __syncthreads();
+        store_rows(static_cast<bf16 *>(p.dq), DO, ci.tok0, ci.len, h, H);
+        store_rows(static_cast<bf16 *>(p.dk), VT, ci.tok0, ci.len, h, H);
     }
 done:
     tc_fence_before();
