@@ -175,12 +175,15 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
     uint32_t phase = 0;
     if (c0 < c1) sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, p.chunks[c1 - 1], h, p);
+    float gn_next = c0 < c1 ? p.tG[((size_t)(c1 - 1) * H + h) * C + C - 1] : 0.f;
     uint8_t *dSs = sm + SbwdSmem::kdS, *dUs = sm + SbwdSmem::kdU;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), idx = idesc_bf16(128, 128, 1, 1),
                    idy = idesc_bf16(128, 128, 0, 1);
     for (int c = c1 - 1; c >= c0; --c) {
         const int buf = (c1 - 1 - c) & 1;
         const size_t ch = (size_t)c * H + h;
+        const float gn_cur = gn_next;
+        if (c - 1 >= c0) gn_next = p.tG[(ch - H) * C + C - 1];
         if (c - 1 >= c0) {
             sbwd_prefetch(sm, buf ^ 1, ch - H, p.chunks[c - 1], h, p);
             cp_async_wait<1>();
@@ -191,7 +194,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        const float gC = expf(p.tG[ch * C + C - 1]);
+        const float gC = expf(gn_cur);
         operands_ready();
         if (v == 0) {
             const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),

@@ -58,11 +58,15 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
     const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
     uint32_t phase = 0;
     if (c0 < c1) state_prefetch(sm, 0, (size_t)c0 * H + h, p);
+    // cumulative gate of the next chunk, loaded one chunk ahead (off the chain)
+    float gn_next = c0 < c1 ? p.tG[((size_t)c0 * H + h) * C + C - 1] : 0.f;
     uint8_t *Ss = sm + StateSmem::kS, *UTs = sm + StateSmem::kUT;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), id2 = idesc_bf16(128, 128, 0, 1);
     for (int c = c0; c < c1; ++c) {
         const int buf = (c - c0) & 1;
         const size_t ch = (size_t)c * H + h;
+        const float gn_cur = gn_next;
+        if (c + 1 < c1) gn_next = p.tG[(ch + H) * C + C - 1];
         if (c + 1 < c1) {
             state_prefetch(sm, buf ^ 1, ch + H, p);
             cp_async_wait<1>();
@@ -73,7 +77,7 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        const float gC = expf(p.tG[ch * C + C - 1]);
+        const float gC = expf(gn_cur);
         operands_ready();
         if (v == 0) {
             const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
