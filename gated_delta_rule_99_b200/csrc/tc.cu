@@ -33,61 +33,10 @@ struct PrepSmem {
     // L (fp32 64 x 65) is dead once A is formed; its bytes then hold the two
     // bf16 operand tiles A diag(b gam) and A diag(b).
     static constexpr int kK = 0, kV = kK + 16384, kL = kV + 16384, kAb = kL, kAc = kL + 8192,
-                         kAm = kL + C * 65 * 4, kT = kAm + C * 65 * 4, kG = kT + 3 * 256 * 4,
-                         kB = kG + 256, kEnd = kB + 256;
+                         kG = kL + C * 65 * 4, kB = kG + 256, kEnd = kB + 256;
 };
 constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
-constexpr int kPrepSmemRequest = 72 * 1024;  // three CTAs per SM (TMEM: 128 columns each)
-
-// A = (I + L)^-1 for a strictly lower 64 x 64 L (fp32, row stride 65), by
-// blocks of 16: the four diagonal blocks by forward substitution (one thread
-// per column), then the off-diagonal blocks level by level,
-//   A_ij = -A_ii sum_{m=j}^{i-1} L_im A_mj   (i - j = 1, 2, 3).
-// Am (row stride 65) must be zero on entry; T holds 3 x 16 x 16 temporaries.
-__device__ void invert_blocked(const float *L, float *Am, float *T) {
-    const int t = threadIdx.x;
-    if (t < C) {
-        const int k = t >> 4, jj = t & 15, o = 16 * k;
-        float a[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int m = 0; m < r; m += 2) {
-                s0 = fmaf(L[(o + r) * 65 + o + m], a[m], s0);
-                if (m + 1 < r) s1 = fmaf(L[(o + r) * 65 + o + m + 1], a[m + 1], s1);
-            }
-            a[r] = r < jj ? 0.f : (r == jj ? 1.f : -(s0 + s1));
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Am[(o + r) * 65 + o + jj] = a[r];
-    }
-    __syncthreads();
-    for (int lev = 1; lev < 4; ++lev) {
-        const int nout = (4 - lev) * 256;
-        for (int x = t; x < nout; x += NT) {
-            const int blk = x >> 8, rr = (x >> 4) & 15, cc = x & 15;
-            const int i = lev + blk, j = blk;
-            const float *Lrow = L + (16 * i + rr) * 65;
-            float s0 = 0.f, s1 = 0.f;
-            for (int m = 16 * j; m < 16 * i; m += 2) {
-                s0 = fmaf(Lrow[m], Am[m * 65 + 16 * j + cc], s0);
-                s1 = fmaf(Lrow[m + 1], Am[(m + 1) * 65 + 16 * j + cc], s1);
-            }
-            T[x] = s0 + s1;
-        }
-        __syncthreads();
-        for (int x = t; x < nout; x += NT) {
-            const int blk = x >> 8, rr = (x >> 4) & 15, cc = x & 15;
-            const int i = lev + blk, j = blk;
-            const float *Arow = Am + (16 * i + rr) * 65 + 16 * i;
-            float s = 0.f;
-            for (int m = 0; m <= rr; ++m) s = fmaf(Arow[m], T[(blk << 8) + m * 16 + cc], s);
-            Am[(16 * i + rr) * 65 + 16 * j + cc] = -s;
-        }
-        __syncthreads();
-    }
-}
+constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 columns each)
 
 __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
     extern __shared__ uint8_t smem_raw[];
@@ -114,10 +63,6 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
     if (tid < 32) {
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
-    }
-    {
-        float *Am = reinterpret_cast<float *>(sm + PrepSmem::kAm);
-        for (int x = tid; x < C * 65; x += NT) Am[x] = 0.f;
     }
     chunk_gates(G, bta, p, ci, h);
     cp_async_wait<0>();
@@ -167,24 +112,38 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
         }
         tc_fence_before();
         __syncthreads();
-        // A = (I + L)^-1 (blocked, fp32), then the operand tiles A diag(b gam) and
-        // A diag(b) over the dead L, and A itself for the backward
-        float *Am = reinterpret_cast<float *>(sm + PrepSmem::kAm);
-        invert_blocked(L, Am, reinterpret_cast<float *>(sm + PrepSmem::kT));
-        {
-            float *Ag = want_A ? p.tA + (size_t)ch * C * C : nullptr;
-            for (int x = tid; x < C * C / 8; x += NT) {
-                const int r = x >> 3, j0 = (x & 7) * 8;
-                float f[8], g8[8];
+        // forward substitution: thread j owns column j of A = (I + L)^-1 (fp32)
+        float a[C];
+        if (tid < C) {
+            const int j = tid;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float a = j0 + q <= r ? Am[r * 65 + j0 + q] : 0.f;
-                    f[q] = a * bta[j0 + q] * expf(G[j0 + q]);
-                    g8[q] = a * bta[j0 + q];
-                    if (Ag) Ag[r * C + j0 + q] = a;
+            for (int r = 0; r < C; ++r) {
+                // four independent partial sums shorten the dependent chain
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                for (int m = 0; m < r; m += 4) {
+                    s0 = fmaf(L[r * 65 + m], a[m], s0);
+                    if (m + 1 < r) s1 = fmaf(L[r * 65 + m + 1], a[m + 1], s1);
+                    if (m + 2 < r) s2 = fmaf(L[r * 65 + m + 2], a[m + 2], s2);
+                    if (m + 3 < r) s3 = fmaf(L[r * 65 + m + 3], a[m + 3], s3);
                 }
-                *reinterpret_cast<uint4 *>(Ab + sw128_chunk(C, r, j0 / 8)) = pack8(f);
-                *reinterpret_cast<uint4 *>(Ac + sw128_chunk(C, r, j0 / 8)) = pack8(g8);
+                const float s = (s0 + s1) + (s2 + s3);
+                a[r] = r < j ? 0.f : (r == j ? 1.f : -s);
+            }
+        }
+        __syncthreads();  // L is dead from here: the operand tiles overwrite it
+        if (tid < C) {
+            const int j = tid;
+            const float bg = bta[j] * expf(G[j]), b = bta[j];
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                *reinterpret_cast<bf16 *>(Ab + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * bg);
+                *reinterpret_cast<bf16 *>(Ac + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * b);
+            }
+            if (want_A) {
+                float *Ag = p.tA + (size_t)ch * C * C;
+#pragma unroll
+                for (int r = 0; r < C; ++r) Ag[r * C + j] = a[r];
             }
         }
         operands_ready();

@@ -124,9 +124,9 @@ __global__ void __launch_bounds__(NT) tc_local_kernel(Params p) {
 // ============================================================ tc_state_bwd
 struct SbwdSmem {
     static constexpr int kdS = 0, kdU = kdS + 32768, kBuf = kdU + 16384;
-    // per buffer: Kd image, W image, Qg image, dO tile, local dU^T rows
+    // per buffer: Kd image, W image, Qg image, dO tile, local dU^T rows, gates
     static constexpr int kKd = 0, kW = 16384, kQg = 32768, kDO = 49152, kDUL = 65536,
-                         kBufBytes = 81920;
+                         kG = 81920, kBufBytes = 81920 + 1024;
     static constexpr int kEnd = kBuf + 2 * kBufBytes;
 };
 constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
@@ -140,6 +140,8 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
     load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H);
     load_image_async(b + SbwdSmem::kDUL, static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT,
                      kImgUT);
+    if (threadIdx.x < 16)
+        cp_async16(smem_u32(b + SbwdSmem::kG) + threadIdx.x * 16, p.tG + ch * C + threadIdx.x * 4);
     cp_async_commit();
 }
 
@@ -175,15 +177,12 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
     uint32_t phase = 0;
     if (c0 < c1) sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, p.chunks[c1 - 1], h, p);
-    float gn_next = c0 < c1 ? p.tG[((size_t)(c1 - 1) * H + h) * C + C - 1] : 0.f;
     uint8_t *dSs = sm + SbwdSmem::kdS, *dUs = sm + SbwdSmem::kdU;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), idx = idesc_bf16(128, 128, 1, 1),
                    idy = idesc_bf16(128, 128, 0, 1);
     for (int c = c1 - 1; c >= c0; --c) {
         const int buf = (c1 - 1 - c) & 1;
         const size_t ch = (size_t)c * H + h;
-        const float gn_cur = gn_next;
-        if (c - 1 >= c0) gn_next = p.tG[(ch - H) * C + C - 1];
         if (c - 1 >= c0) {
             sbwd_prefetch(sm, buf ^ 1, ch - H, p.chunks[c - 1], h, p);
             cp_async_wait<1>();
@@ -194,7 +193,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        const float gC = expf(gn_cur);
+        const float gC = expf(reinterpret_cast<const float *>(b + SbwdSmem::kG)[C - 1]);
         operands_ready();
         if (v == 0) {
             const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),

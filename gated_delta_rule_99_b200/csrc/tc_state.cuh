@@ -12,7 +12,7 @@ namespace tc {
 // One CTA per (sequence, head); thread v owns row v of S (fp32 registers).
 struct StateSmem {
     static constexpr int kS = 0, kUT = kS + 32768, kW0 = kUT + 16384, kKd0 = kW0 + 2 * 16384,
-                         kUt0 = kKd0 + 2 * 16384, kEnd = kUt0 + 2 * 16384;
+                         kUt0 = kKd0 + 2 * 16384, kG0 = kUt0 + 2 * 16384, kEnd = kG0 + 2 * 256;
 };
 constexpr int kStateSmem = StateSmem::kEnd + 1024;
 
@@ -23,6 +23,9 @@ __device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, 
                      static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
     load_image_async(sm + StateSmem::kUt0 + buf * 16384,
                      static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64);
+    if (threadIdx.x < 16)
+        cp_async16(smem_u32(sm + StateSmem::kG0 + buf * 256) + threadIdx.x * 16,
+                   p.tG + ch * C + threadIdx.x * 4);
     cp_async_commit();
 }
 
@@ -58,15 +61,11 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
     const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
     uint32_t phase = 0;
     if (c0 < c1) state_prefetch(sm, 0, (size_t)c0 * H + h, p);
-    // cumulative gate of the next chunk, loaded one chunk ahead (off the chain)
-    float gn_next = c0 < c1 ? p.tG[((size_t)c0 * H + h) * C + C - 1] : 0.f;
     uint8_t *Ss = sm + StateSmem::kS, *UTs = sm + StateSmem::kUT;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), id2 = idesc_bf16(128, 128, 0, 1);
     for (int c = c0; c < c1; ++c) {
         const int buf = (c - c0) & 1;
         const size_t ch = (size_t)c * H + h;
-        const float gn_cur = gn_next;
-        if (c + 1 < c1) gn_next = p.tG[(ch + H) * C + C - 1];
         if (c + 1 < c1) {
             state_prefetch(sm, buf ^ 1, ch + H, p);
             cp_async_wait<1>();
@@ -77,7 +76,8 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        const float gC = expf(gn_cur);
+        const float gC =
+            expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
         operands_ready();
         if (v == 0) {
             const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
