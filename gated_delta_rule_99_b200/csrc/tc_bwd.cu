@@ -193,8 +193,9 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        const float gC = expf(reinterpret_cast<const float *>(b + SbwdSmem::kG)[C - 1]);
         operands_ready();
+        // after the barrier: the gate row was copied by other threads' cp.async
+        const float gC = expf(reinterpret_cast<const float *>(b + SbwdSmem::kG)[C - 1]);
         if (v == 0) {
             const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
                            qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO);

@@ -76,9 +76,10 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
+        operands_ready();
+        // after the barrier: the gate row was copied by other threads' cp.async
         const float gC =
             expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
-        operands_ready();
         if (v == 0) {
             const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
             for (int s = 0; s < D / 16; ++s)
