@@ -164,13 +164,18 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle
+_ORACLE_INPUTS = {}
+
+
 def cpu_oracle_sample(units_n):
     """Time the fp64 oracle (fwd + bwd) on `units_n` (row, head) units of the
     workload; returns (seconds, units, threads, tokens-equivalent)."""
     import oracle
     from gated_delta_rule_99_b200.inputs import make_inputs
     w = dict(WORKLOAD)
-    inp = make_inputs(**w)
+    if "inp" not in _ORACLE_INPUTS:  # drawn once, outside every timed call
+        _ORACLE_INPUTS["inp"] = make_inputs(**w)
+    inp = _ORACLE_INPUTS["inp"]
     allu = [(b, h) for b in range(w["B"]) for h in range(w["H"])]
     units = allu[:units_n]
     threads = oracle.default_threads()
@@ -187,6 +192,27 @@ def cpu_oracle_sample(units_n):
 def oracle_units_for_cores():
     import oracle
     return max(1, min(64, oracle.default_threads()))
+
+
+# ------------------------------------------------------------------ ranks
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch: independent problems, no data exchange."""
+    return WORKLOAD["seed"] + rank
+
+
+def max_over_ranks(value_ms: float, world: int, device) -> float:
+    """The job's time is the slowest rank's (a MAX all-reduce; identity at N = 1)."""
+    import torch
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the max-over-ranks time."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
 
 
 # ------------------------------------------------------------------ main arms
@@ -230,7 +256,7 @@ def run_ours(args, rank, world, local_rank):
     w = dict(WORKLOAD)
     if args.shape:
         w["B"], w["T"], w["H"] = (int(x) for x in args.shape.split(","))
-    w["seed"] = WORKLOAD["seed"] + rank
+    w["seed"] = rank_seed(rank)
     inp = make_inputs(device="cpu", **w)
     d = inp.to(dev)
     B, T, H, K, V = w["B"], w["T"], w["H"], w["K"], w["V"]
@@ -277,11 +303,7 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    my_ms = sum(step_ms)
-    t = torch.tensor([my_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    tot_ms = float(t.item())
+    tot_ms = max_over_ranks(sum(step_ms), world, dev)
     status = gdn.device_status(ws)
     if status != 0:
         raise RuntimeError("device status %d after timed steps" % status)
@@ -317,16 +339,14 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * B * T * args.steps / (float(te.item()) / 1e3), "unit": "tokens/s",
+        te = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_tokens_per_s(B * T, world, args.steps, te), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank != 0:
         return
     pk = peaks()
-    value = world * B * T * args.steps / (tot_ms / 1e3)
+    value = job_tokens_per_s(B * T, world, args.steps, tot_ms)
     # dominant kernel roofline
     dom = max(per_kernel.items(), key=lambda kv: kv[1][1]) if per_kernel else None
     roof = None
