@@ -29,11 +29,13 @@ using namespace tc;
 // ============================================================ tc_prep
 // Per (chunk, head): gates, A (fp32 forward substitution), and the tile
 // images W, Kd and the plain rows of Ut that the state pass consumes.
+constexpr int LS = 68;  // row stride (floats) of L: 16-byte aligned rows for vector loads
+
 struct PrepSmem {
-    // L (fp32 64 x 65) is dead once A is formed; its bytes then hold the two
+    // L (fp32 64 x 68) is dead once A is formed; its bytes then hold the two
     // bf16 operand tiles A diag(b gam) and A diag(b).
     static constexpr int kK = 0, kV = kK + 16384, kL = kV + 16384, kAb = kL, kAc = kL + 8192,
-                         kG = kL + C * 65 * 4, kB = kG + 256, kEnd = kB + 256;
+                         kG = kL + C * LS * 4, kB = kG + 256, kEnd = kB + 256;
 };
 constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
 constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 columns each)
@@ -106,26 +108,31 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int j = c0 + q;
-                    L[i * 65 + j] = j < i ? bta[i] * expf(G[i] - G[j]) * d[q] : 0.f;
+                    L[i * LS + j] = j < i ? bta[i] * expf(G[i] - G[j]) * d[q] : 0.f;
                 }
             }
         }
         tc_fence_before();
         __syncthreads();
-        // forward substitution: thread j owns column j of A = (I + L)^-1 (fp32)
+        // forward substitution: thread j owns column j of A = (I + L)^-1 (fp32).
+        // L is zero on and above the diagonal and a[] starts at zero, so whole
+        // 4-blocks of a row can be read with one 16-byte load.
         float a[C];
         if (tid < C) {
             const int j = tid;
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
-                // four independent partial sums shorten the dependent chain
+            for (int r = 0; r < C; ++r) a[r] = 0.f;
+            a[0] = j == 0 ? 1.f : 0.f;
+#pragma unroll
+            for (int r = 1; r < C; ++r) {
                 float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
                 for (int m = 0; m < r; m += 4) {
-                    s0 = fmaf(L[r * 65 + m], a[m], s0);
-                    if (m + 1 < r) s1 = fmaf(L[r * 65 + m + 1], a[m + 1], s1);
-                    if (m + 2 < r) s2 = fmaf(L[r * 65 + m + 2], a[m + 2], s2);
-                    if (m + 3 < r) s3 = fmaf(L[r * 65 + m + 3], a[m + 3], s3);
+                    const float4 l4 = *reinterpret_cast<const float4 *>(L + r * LS + m);
+                    s0 = fmaf(l4.x, a[m], s0);
+                    s1 = fmaf(l4.y, a[m + 1], s1);
+                    s2 = fmaf(l4.z, a[m + 2], s2);
+                    s3 = fmaf(l4.w, a[m + 3], s3);
                 }
                 const float s = (s0 + s1) + (s2 + s3);
                 a[r] = r < j ? 0.f : (r == j ? 1.f : -s);

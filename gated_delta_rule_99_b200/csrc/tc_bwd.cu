@@ -242,12 +242,13 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         if (!cta_wait(&mbar, phase, p, 14)) break;
         phase ^= 1;
 #pragma unroll
-        for (int c16 = 0; c16 < D; c16 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, 64 + c16), d);
+        for (int c32 = 0; c32 < D; c32 += 32) {
+            float d[32];
+            tmem_ld16(tm(tmem, 64 + c32), d);
+            tmem_ld16(tm(tmem, 64 + c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) S[c16 + q] = fmaf(gC, S[c16 + q], d[q]);
+            for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
         }
         if (v == 0) bulk_wait_read();
         tc_fence_before();

@@ -93,14 +93,16 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
         // U^T[v][i] = Ut[i][v] - (S W^T)[v][i]
         const bf16 *Ut = reinterpret_cast<const bf16 *>(sm + StateSmem::kUt0 + buf * 16384);
 #pragma unroll
-        for (int c16 = 0; c16 < C; c16 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, c16), d);
+        for (int c32 = 0; c32 < C; c32 += 32) {
+            float d[32];
+            tmem_ld16(tm(tmem, c32), d);
+            tmem_ld16(tm(tmem, c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) d[q] = __bfloat162float(Ut[(c16 + q) * D + v]) - d[q];
-            *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c16 / 8)) = pack8(d);
-            *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
+            for (int q = 0; q < 32; ++q) d[q] = __bfloat162float(Ut[(c32 + q) * D + v]) - d[q];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
         }
         operands_ready();
         if (v == 0) {
@@ -114,12 +116,13 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
         if (!cta_wait(&mbar, phase, p, 4)) break;
         phase ^= 1;
 #pragma unroll
-        for (int c16 = 0; c16 < D; c16 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, 64 + c16), d);
+        for (int c32 = 0; c32 < D; c32 += 32) {
+            float d[32];
+            tmem_ld16(tm(tmem, 64 + c32), d);
+            tmem_ld16(tm(tmem, 64 + c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) S[c16 + q] = fmaf(gC, S[c16 + q], d[q]);
+            for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
         }
         // shared operands are rewritten next chunk: their bulk stores must have read them
         if (v == 0) bulk_wait_read();
