@@ -88,6 +88,36 @@ def kernel_work(name, w, n_chunks):
     return None, None, None
 
 
+def csrc_hash() -> str:
+    """Hash of the CUDA sources and the ABI header (ties recorded ncu traffic to a build)."""
+    import glob
+    import hashlib
+    h = hashlib.sha1()
+    files = sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_99_b200", "csrc", "*.cu")) +
+                   glob.glob(os.path.join(ROOT, "gated_delta_rule_99_b200", "csrc", "*.cuh")) +
+                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from profiles/traffic.md, or None if the sources changed."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.md")) as f:
+            lines = f.read().splitlines()
+    except OSError:
+        return None
+    cur = csrc_hash()
+    for ln in lines:
+        cells = [c.strip() for c in ln.strip().strip("|").split("|")]
+        if len(cells) == 5 and cells[0] == kernel and cells[3] == cur and cells[4] == workload:
+            return int(cells[1]) + int(cells[2])
+    return None
+
+
 def alu_peak_tflops(sm_mhz):
     # 148 SMs x 128 fp32 lanes x 2 flop (FMA) per clock
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
@@ -364,9 +394,13 @@ def run_ours(args, rank, world, local_rank):
         elif bound in ("hbm", "tensor"):
             peak = pk["hbm"] if bound == "hbm" else pk["tc_sus"]
             ach = amount / per_launch_s / (1e9 if bound == "hbm" else 1e12)
+            wl = ("gdn_fwdbwd_bf16_B4_T4096_H16_d128" if not args.shape else
+                  "gdn_fwdbwd_bf16_B%d_T%d_H%d_d128" % (B, T, H))
             roof = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak,
                     "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": ach / peak,
-                    "traffic": None, "peak_source": pk["src"], "ms_per_launch": per_launch_s * 1e3}
+                    "traffic": recorded_traffic(name, wl),
+                    "algorithmic": amount, "peak_source": pk["src"],
+                    "ms_per_launch": per_launch_s * 1e3}
     sr = step_roofline(w, pk)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
