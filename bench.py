@@ -79,7 +79,8 @@ def kernel_work(name, w, n_chunks):
     hbm = {"tc_grads": 4 * 2 * K + 8 + 3 * 2 * K + 8,   # q,k,v,do + g,b in; dq,dk,dv + dg,db out
            "tc_prep": 2 * (K + V) + 8,                  # k, v, g, b
            "tc_out": 2 * (2 * K) + 4 + 2 * V,           # q, k, g in; o out
-           "tc_local": 2 * (2 * K + V) + 4}             # q, k, do
+           "tc_local": 2 * (2 * K + V) + 4,             # q, k, do
+           "tc_prep_local": 2 * (K + V) + 8 + 2 * (2 * K + V) + 4}  # both of the above
     if name in hbm:
         return "hbm", float(hbm[name]) * th, "B"
     chain = {"tc_state_fwd": 2 * f2(C, V, K), "tc_chains": 5 * f2(C, V, K)}

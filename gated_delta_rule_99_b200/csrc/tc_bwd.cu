@@ -19,11 +19,11 @@
 // 128 TMEM lanes (M = 128 over the key or value dim); 64 x 64 products use the
 // M = 64 form (row m in lane 32 (m / 16) + m % 16).
 #include "tc_common.cuh"
+#include "tc_prep.cuh"
 #include "tc_state.cuh"
 
 namespace gdn {
 
-cudaError_t tc_launch_prep(const Params &p, int want_A, cudaStream_t stream);
 
 namespace {
 
@@ -36,13 +36,16 @@ struct LocalSmem {
 };
 constexpr int kLocalSmem = LocalSmem::kEnd + 1024;
 
-__global__ void __launch_bounds__(NT) tc_local_kernel(Params p) {
+// Body of the local step for CTA `ch` (chunk ch / H, head ch % H).  It forms
+// the chunk gates itself (the same code as tc_prep, so bit-identical), which
+// makes it independent of tc_prep: the two share one launch.
+__device__ __forceinline__ void local_body(const Params &p, int ch) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
-    const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
+    const int H = p.H, c = ch / H, h = ch % H, tid = threadIdx.x;
     const ChunkInfo ci = p.chunks[c];
     uint8_t *QK = sm + LocalSmem::kQK, *DO = sm + LocalSmem::kDO, *Ps = sm + LocalSmem::kP;
     float *G = reinterpret_cast<float *>(sm + LocalSmem::kG);
@@ -50,7 +53,6 @@ __global__ void __launch_bounds__(NT) tc_local_kernel(Params p) {
     load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
     load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H);
     cp_async_commit();
-    if (tid < C) G[tid] = p.tG[(size_t)ch * C + tid];
     if (tid == 0) {
         mbar_init(&mbar, 1);
         fence_mbar_init();
@@ -59,6 +61,7 @@ __global__ void __launch_bounds__(NT) tc_local_kernel(Params p) {
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
+    chunk_gates(G, nullptr, p, ci, h);
     cp_async_wait<0>();
     operands_ready();
     const uint32_t tmem = tslot;
@@ -119,6 +122,14 @@ __global__ void __launch_bounds__(NT) tc_local_kernel(Params p) {
     tc_fence_before();
     __syncthreads();
     if (tid < 32) tmem_dealloc(tmem, 128);
+}
+
+// tc_prep (with A for the backward) on CTAs [0, NC*H) and tc_local on
+// [NC*H, 2*NC*H): independent chunk-parallel steps in one launch.
+__global__ void __launch_bounds__(NT) tc_prep_local_kernel(Params p) {
+    const int nch = p.NC * p.H;
+    if ((int)blockIdx.x < nch) prep_body(p, blockIdx.x, 1);
+    else local_body(p, blockIdx.x - nch);
 }
 
 // ============================================================ tc_state_bwd
@@ -693,10 +704,11 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
     const int nch = p.NC * p.H, nseq = p.N * p.H;
     Params pf = p;
     pf.hT = nullptr;
-    if ((e = tc_launch_prep(p, 1, stream))) return e;
     if (nch > 0) {
-        if ((e = set_smem(tc_local_kernel, kLocalSmem))) return e;
-        GDN_LAUNCH(kKTcLocal, stream, tc_local_kernel<<<nch, NT, kLocalSmem, stream>>>(p));
+        const int sm = kLocalSmem > kPrepSmemRequest ? kLocalSmem : kPrepSmemRequest;
+        if ((e = set_smem(tc_prep_local_kernel, sm))) return e;
+        GDN_LAUNCH(kKTcLocal, stream,
+                   tc_prep_local_kernel<<<2 * nch, NT, sm, stream>>>(p));
     }
     if (nseq > 0) {
         const int sm = kSbwdSmem > kStateSmem ? kSbwdSmem : kStateSmem;

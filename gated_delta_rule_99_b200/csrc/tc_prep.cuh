@@ -1,0 +1,194 @@
+// Per-chunk preparation step of the tensor-core path (shared by the forward
+// launch and by the backward, where it shares a launch with tc_local).
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace tc {
+
+// ============================================================ tc_prep
+// Per (chunk, head): gates, A (fp32 forward substitution), and the tile
+// images W, Kd and the plain rows of Ut that the state pass consumes.
+constexpr int LS = 68;  // row stride (floats) of L: 16-byte aligned rows for vector loads
+
+struct PrepSmem {
+    // L (fp32 64 x 68) is dead once A is formed; its bytes then hold the two
+    // bf16 operand tiles A diag(b gam) and A diag(b).
+    static constexpr int kK = 0, kV = kK + 16384, kL = kV + 16384, kAb = kL, kAc = kL + 8192,
+                         kG = kL + C * LS * 4, kB = kG + 256, kEnd = kB + 256;
+};
+constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
+constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 columns each)
+
+// Body of the prep step for CTA `ch` (chunk ch / H, head ch % H).
+__device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, c = ch / H, h = ch % H;
+    const ChunkInfo ci = p.chunks[c];
+    uint8_t *Kt = sm + PrepSmem::kK, *Vt = sm + PrepSmem::kV;
+    uint8_t *Ab = sm + PrepSmem::kAb, *Ac = sm + PrepSmem::kAc;
+    float *L = reinterpret_cast<float *>(sm + PrepSmem::kL);
+    float *G = reinterpret_cast<float *>(sm + PrepSmem::kG);
+    float *bta = reinterpret_cast<float *>(sm + PrepSmem::kB);
+    const int tid = threadIdx.x;
+
+    load_rows_async(Kt, C, 0, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
+    load_rows_async(Vt, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H);
+    cp_async_commit();
+    if (tid == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (tid < 32) {
+        tmem_alloc(&tslot, 128);
+        tmem_relinquish();
+    }
+    chunk_gates(G, bta, p, ci, h);
+    cp_async_wait<0>();
+    operands_ready();
+    const uint32_t tmem = tslot;
+    uint32_t phase = 0;
+    bool ok = true;
+
+    // K K^T (M = 64 rows i, N = 64 cols j, K = 128)
+    if (tid == 0) {
+        const uint32_t kb = smem_u32(Kt), id = idesc_bf16(64, 64, 0, 0);
+        for (int s = 0; s < D / 16; ++s)
+            mma_bf16(tmem, desc_kmajor(kb, C, s), desc_kmajor(kb, C, s), id, s > 0);
+        mma_commit(&mbar);
+    }
+    // meanwhile: Kd = diag(e) K as a tile image, and G
+    {
+        const float Gn = G[C - 1];
+        uint8_t *dst = static_cast<uint8_t *>(p.tKd) + (size_t)ch * kImg64;
+        for (int t = tid; t < C * 16; t += NT) {
+            const int off = t * 16, r = (off & 8191) >> 7;
+            float f[8];
+            unpack8(*reinterpret_cast<const uint4 *>(Kt + off), f);
+            const float e = expf(Gn - G[r]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] *= e;
+            *reinterpret_cast<uint4 *>(dst + off) = pack8(f);
+        }
+        if (tid < C) p.tG[(size_t)ch * C + tid] = G[tid];
+    }
+    ok = cta_wait(&mbar, phase, p, 1);
+    phase ^= 1;
+    if (ok) {
+        // L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32)
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    L[i * LS + j] = j < i ? bta[i] * expf(G[i] - G[j]) * d[q] : 0.f;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        // forward substitution: thread j owns column j of A = (I + L)^-1 (fp32).
+        // L is zero on and above the diagonal and a[] starts at zero, so whole
+        // 4-blocks of a row can be read with one 16-byte load.
+        float a[C];
+        if (tid < C) {
+            const int j = tid;
+#pragma unroll
+            for (int r = 0; r < C; ++r) a[r] = 0.f;
+            a[0] = j == 0 ? 1.f : 0.f;
+#pragma unroll
+            for (int r = 1; r < C; ++r) {
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                for (int m = 0; m < r; m += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4 *>(L + r * LS + m);
+                    s0 = fmaf(l4.x, a[m], s0);
+                    s1 = fmaf(l4.y, a[m + 1], s1);
+                    s2 = fmaf(l4.z, a[m + 2], s2);
+                    s3 = fmaf(l4.w, a[m + 3], s3);
+                }
+                const float s = (s0 + s1) + (s2 + s3);
+                a[r] = r < j ? 0.f : (r == j ? 1.f : -s);
+            }
+        }
+        __syncthreads();  // L is dead from here: the operand tiles overwrite it
+        if (tid < C) {
+            const int j = tid;
+            const float bg = bta[j] * expf(G[j]), b = bta[j];
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                *reinterpret_cast<bf16 *>(Ab + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * bg);
+                *reinterpret_cast<bf16 *>(Ac + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * b);
+            }
+            if (want_A) {
+                float *Ag = p.tA + (size_t)ch * C * C;
+#pragma unroll
+                for (int r = 0; r < C; ++r) Ag[r * C + j] = a[r];
+            }
+        }
+        operands_ready();
+        // W = (A diag(b gam)) K, then Ut = (A diag(b)) V: M = 64, N = 128, K = 64 tokens,
+        // one after the other in the same 128 TMEM columns
+        const uint32_t id = idesc_bf16(64, 128, 0, 1);
+        if (tid == 0) {
+            const uint32_t ab = smem_u32(Ab), kb = smem_u32(Kt);
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(ab, C, s), desc_mnmajor(kb, C, s), id, s > 0);
+            mma_commit(&mbar);
+        }
+        ok = cta_wait(&mbar, phase, p, 2);
+        phase ^= 1;
+        if (ok) {
+            const int i = m64_row();
+            uint8_t *Wimg = static_cast<uint8_t *>(p.tW) + (size_t)ch * kImg64;
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float w[16];
+                tmem_ld16(tm(tmem, c0), w);
+                tmem_ld_wait();
+                if (i >= 0) {
+                    *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8)) = pack8(w);
+                    *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(w + 8);
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+                const uint32_t ac = smem_u32(Ac), vb = smem_u32(Vt);
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tmem, desc_kmajor(ac, C, s), desc_mnmajor(vb, C, s), id, s > 0);
+                mma_commit(&mbar);
+            }
+            ok = cta_wait(&mbar, phase, p, 2);
+            phase ^= 1;
+        }
+    }
+    if (ok) {
+        const int i = m64_row();
+        bf16 *Ut = static_cast<bf16 *>(p.tUt) + (size_t)ch * C * D;
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float u[16];
+            tmem_ld16(tm(tmem, c0), u);
+            tmem_ld_wait();
+            if (i >= 0) {
+                *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0) = pack8(u);
+                *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0 + 8) = pack8(u + 8);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 32) tmem_dealloc(tmem, 128);
+}
+
+}  // namespace tc
+}  // namespace gdn
