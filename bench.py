@@ -39,6 +39,8 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--mode", choices=("fwdbwd", "decode"), default="fwdbwd",
+                    help="decode: time the recurrent decode step instead (not the headline)")
     ap.add_argument("--shape", default=None,
                     help="B,T,H override of the workload (profiling and size sweeps only)")
     return ap.parse_args()
@@ -433,6 +435,57 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args, rank, world, local_rank):
+    """Recurrent decode step: B sequences x H heads advance one token each; HBM
+    bound by the fp32 state (read and written once per step)."""
+    import torch
+
+    import gated_delta_rule_99_b200 as gdn
+    from gated_delta_rule_99_b200.inputs import make_inputs
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, H, K, V = 256, 16, 128, 128
+    if args.shape:
+        B, _, H = (int(x) for x in args.shape.split(","))
+    inp = make_inputs(B=B, T=1, H=H, K=K, V=V, dtype="bf16", seed=50 + rank, bwd=False)
+    d = inp.to(dev)
+    state = d.h0.clone()
+    o = torch.empty_like(d.v)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        gdn.gdn_decode(d.q, d.k, d.v, d.g, d.beta, state, o=o)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(None) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            gdn.gdn_decode(d.q, d.k, d.v, d.g, d.beta, state, o=o)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+    tot_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
+    if rank != 0:
+        return
+    pk = peaks()
+    per = tot_ms / args.steps / 1e3
+    bytes_ = B * H * (2 * K * V * 4 + 2 * (2 * K + 2 * V) + 8)
+    ach = bytes_ / per / 1e9
+    print(json.dumps({
+        "metric": "GDN recurrent decode tokens/s (B=%d sequences, H=%d, d=128, bf16, fp32 state)"
+                  % (B, H),
+        "value": world * B / per, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "gdn_decode_bf16_B%d_H%d_d128" % (B, H),
+                   "l2": "256 MiB memset before each step, outside the step events"},
+        "roofline": {"kernel": "decode", "bound": "hbm", "achieved": ach, "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": ach / pk["hbm"], "traffic": None,
+                     "algorithmic": bytes_, "peak_source": pk["src"]},
+        "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -450,6 +503,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.mode == "decode":
+            run_decode(args, rank, world, local_rank)
+            return
         run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

@@ -7,9 +7,10 @@ call does, and raises if the library was not built.
 """
 from ._binding import (GDN_BF16, GDN_FP32, EXPORTS, GdnDesc, GdnError, LaunchTrace,  # noqa
                        alloc_workspace,
-                       bwd_workspace_size, device_status, fwd_workspace_size, gdn_bwd, gdn_fwd,
+                       bwd_workspace_size, device_status, fwd_workspace_size, gdn_bwd, gdn_decode,
+                       gdn_fwd,
                        lib, make_desc)
 
-__all__ = ["gdn_fwd", "gdn_bwd", "device_status", "fwd_workspace_size", "bwd_workspace_size",
+__all__ = ["gdn_fwd", "gdn_bwd", "gdn_decode", "device_status", "fwd_workspace_size", "bwd_workspace_size",
            "alloc_workspace", "LaunchTrace", "make_desc", "GdnDesc", "GdnError", "lib", "GDN_BF16", "GDN_FP32",
            "EXPORTS"]

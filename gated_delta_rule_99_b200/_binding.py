@@ -20,7 +20,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "mi
           4: "workspace missing or too small", 5: "CUDA runtime error",
           6: "device-side wait timed out"}
 EXPORTS = ("gdn_version", "gdn_chunk_size", "gdn_fwd_workspace_size", "gdn_bwd_workspace_size",
-           "gdn_fwd", "gdn_fwd_noalloc", "gdn_bwd", "gdn_device_status", "gdn_status_string", "gdn_trace_install",
+           "gdn_fwd", "gdn_fwd_noalloc", "gdn_bwd", "gdn_decode", "gdn_device_status", "gdn_status_string", "gdn_trace_install",
            "gdn_kernel_name")
 
 
@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_bwd.restype = ctypes.c_int
             L.gdn_bwd.argtypes = [dp, vp, vp, vp, fp, fp, i32p, i32p, fp, vp, fp, vp, vp, vp, fp,
                                   fp, fp, vp, sz, vp]
+            L.gdn_decode.restype = ctypes.c_int
+            L.gdn_decode.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, vp]
             L.gdn_device_status.restype = ctypes.c_int
             L.gdn_device_status.argtypes = [vp, vp]
             L.gdn_status_string.restype = ctypes.c_char_p
@@ -192,6 +194,26 @@ def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0,
     if rc:
         raise GdnError(rc, "gdn_bwd")
     return dq, dk, dv, dg, dbeta, dh0
+
+
+def gdn_decode(q, k, v, g, beta, state, scale=1.0, o=None, stream=None):
+    """Recurrent decode through the C ABI: advances ``state`` ([B][H][dk][dv]
+    fp32, updated in place) through the T tokens of q, k, v ([B][T][H][D]) and
+    returns o."""
+    L = lib()
+    desc, (B, T, H, K, V, _) = _desc_from(q, v, None, scale)
+    _check(q, "q", q.dtype, (B, T, H, K)); _check(k, "k", q.dtype, (B, T, H, K))
+    _check(v, "v", q.dtype, (B, T, H, V))
+    _check(g, "g", torch.float32, (B, T, H)); _check(beta, "beta", torch.float32, (B, T, H))
+    _check(state, "state", torch.float32, (B, H, K, V))
+    if o is None:
+        o = torch.empty(B, T, H, V, dtype=q.dtype, device=q.device)
+    _check(o, "o", q.dtype, (B, T, H, V))
+    rc = L.gdn_decode(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                      _ptr(state), _ptr(o), _stream(stream))
+    if rc:
+        raise GdnError(rc, "gdn_decode")
+    return o
 
 
 def device_status(workspace, stream=None) -> int:

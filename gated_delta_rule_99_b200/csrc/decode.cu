@@ -1,0 +1,120 @@
+// Recurrent decode: advance the per-(sequence, head) state token by token.
+//
+// The inference form of the same recurrence (jax-linear-attention 0.1.0,
+// "FAQ": inference decodes with each layer's recurrent state).  For each
+// token t of a short row (T is small, usually 1):
+//
+//   S <- a_t (S - b_t (S k_t) k_t^T) + b_t v_t k_t^T,   a_t = exp(g_t)
+//   o_t = scale S q_t
+//
+// with S = state^T kept in fp32.  One CTA per (sequence, head); thread v owns
+// row v of S in registers (d_k values), so the state is read once and written
+// once per call and every step is thread-local arithmetic.  HBM bound: the
+// state (2 d_k d_v 4 bytes per sequence and head) dominates the traffic.
+#include "gdn_internal.cuh"
+
+namespace gdn {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T *p, int64_t i);
+template <>
+__device__ __forceinline__ float ldf<float>(const float *p, int64_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void stf(float *p, int64_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void stf(__nv_bfloat16 *p, int64_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+template <typename T, int K>
+__global__ void __launch_bounds__(128) decode_kernel(const T *q, const T *k, const T *v,
+                                                     const float *g, const float *beta,
+                                                     float *state, T *o, int Tn, int H, int V,
+                                                     float scale) {
+    __shared__ float qs[K], ks[K];
+    const int bh = blockIdx.x, b = bh / H, h = bh % H, vi = threadIdx.x;
+    const bool active = vi < V;
+    float *st = state + (size_t)bh * K * V;
+    float S[K];
+#pragma unroll
+    for (int kk = 0; kk < K; ++kk) S[kk] = active ? st[(size_t)kk * V + vi] : 0.f;
+    for (int t = 0; t < Tn; ++t) {
+        const int64_t row = ((int64_t)b * Tn + t) * H + h;
+        __syncthreads();  // previous token's q/k no longer read
+        for (int kk = threadIdx.x; kk < K; kk += blockDim.x) {
+            qs[kk] = ldf(q, row * K + kk);
+            ks[kk] = ldf(k, row * K + kk);
+        }
+        __syncthreads();
+        const float a = expf(g[row]), bt = beta[row];
+        const float vv = active ? ldf(v, row * V + vi) : 0.f;
+        float sk0 = 0.f, sk1 = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < K; kk += 2) {
+            sk0 = fmaf(S[kk], ks[kk], sk0);
+            sk1 = fmaf(S[kk + 1], ks[kk + 1], sk1);
+        }
+        const float sk = sk0 + sk1;
+        float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < K; ++kk) {
+            S[kk] = a * (S[kk] - bt * sk * ks[kk]) + bt * vv * ks[kk];
+            if (kk & 1) o1 = fmaf(S[kk], qs[kk], o1);
+            else o0 = fmaf(S[kk], qs[kk], o0);
+        }
+        if (active) stf(o, row * V + vi, scale * (o0 + o1));
+    }
+    if (active) {
+#pragma unroll
+        for (int kk = 0; kk < K; ++kk) st[(size_t)kk * V + vi] = S[kk];
+    }
+}
+
+template <typename T>
+cudaError_t launch_typed(const gdn_desc *d, const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, float *state, void *o,
+                         cudaStream_t s) {
+    const int nbh = (int)(d->B * d->H), Tn = (int)d->T, H = (int)d->H, V = (int)d->dv;
+    if (d->dk == 128) {
+        GDN_LAUNCH(kKDecode, s,
+                   decode_kernel<T, 128><<<nbh, 128, 0, s>>>(
+                       (const T *)q, (const T *)k, (const T *)v, g, beta, state, (T *)o, Tn, H,
+                       V, d->scale));
+    } else {
+        GDN_LAUNCH(kKDecode, s,
+                   decode_kernel<T, 64><<<nbh, 128, 0, s>>>(
+                       (const T *)q, (const T *)k, (const T *)v, g, beta, state, (T *)o, Tn, H,
+                       V, d->scale));
+    }
+    return cudaSuccess;
+}
+
+bool mis(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) % 16) != 0; }
+
+}  // namespace
+}  // namespace gdn
+
+extern "C" gdn_status gdn_decode(const gdn_desc *d, const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta, float *state, void *o,
+                                 void *stream) {
+    using namespace gdn;
+    if (!d) return GDN_ERR_INVALID_ARG;
+    if (d->B < 1 || d->T < 1 || d->H < 1 || d->n_seqs != 0) return GDN_ERR_INVALID_ARG;
+    if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return GDN_ERR_UNSUPPORTED;
+    if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN_ERR_UNSUPPORTED;
+    if (d->B * d->H >= (int64_t(1) << 31) || d->B * d->T >= (int64_t(1) << 31))
+        return GDN_ERR_INVALID_ARG;
+    if (!(d->scale == d->scale)) return GDN_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, state, o};
+    for (const void *p : ptrs)
+        if (mis(p)) return GDN_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = d->dtype == GDN_BF16
+                        ? launch_typed<__nv_bfloat16>(d, q, k, v, g, beta, state, o, s)
+                        : launch_typed<float>(d, q, k, v, g, beta, state, o, s);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}

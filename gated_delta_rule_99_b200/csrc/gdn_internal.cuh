@@ -106,6 +106,7 @@ enum KernelId : int32_t {
     kKTcStateBwd,  // backward chains (forward recompute + reverse pass)
     kKTcGrads,
     kKTcLocal,
+    kKDecode,
     kKernelCount
 };
 

@@ -8,7 +8,7 @@ thread_local bool g_open = false;
 
 const char *const kNames[kKernelCount] = {
     "build_chunks", "simt_prep", "simt_state_fwd", "simt_out", "simt_duloc", "simt_state_bwd",
-    "simt_grads", "tc_prep", "tc_state_fwd", "tc_out", "tc_chains", "tc_grads", "tc_prep_local"};
+    "simt_grads", "tc_prep", "tc_state_fwd", "tc_out", "tc_chains", "tc_grads", "tc_prep_local", "decode"};
 }  // namespace
 
 void trace_before(int32_t id, cudaStream_t stream) {

@@ -132,6 +132,18 @@ gdn_status gdn_bwd(const gdn_desc *desc, const void *q, const void *k, const voi
                    const float *dhT, void *dq, void *dk, void *dv, float *dg, float *dbeta,
                    float *dh0, void *workspace, size_t workspace_bytes, void *stream);
 
+/* Recurrent decode: advance each sequence's state through T tokens (usually
+ * T = 1) with the token-by-token form of the same recurrence, for inference
+ * with a cached per-layer state (jax-linear-attention 0.1.0, "FAQ": decode
+ * runs with each layer's recurrent state).  desc: B sequences of T tokens,
+ * n_seqs must be 0; q, k [B][T][H][dk], v, o [B][T][H][dv] in desc->dtype;
+ * g, beta [B][T][H] fp32; state [B][H][dk][dv] fp32 (= S^T, the layout of
+ * h0/hT), read and overwritten in place with the state after the last token.
+ * Needs no workspace; asynchronous on the stream; argument errors return
+ * before any launch. */
+gdn_status gdn_decode(const gdn_desc *desc, const void *q, const void *k, const void *v,
+                      const float *g, const float *beta, float *state, void *o, void *stream);
+
 /* Synchronises the stream, then returns and clears the device-side status
  * that the last gdn_fwd/gdn_bwd on this workspace recorded (GDN_OK,
  * GDN_ERR_TIMEOUT, or GDN_ERR_INVALID_ARG when the device copy of cu_seqlens

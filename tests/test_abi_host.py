@@ -130,3 +130,16 @@ def test_python_binding_rejects_cpu_tensors():
     g = torch.zeros(1, 8, 1)
     with pytest.raises(ValueError):
         gdn.gdn_fwd(x, x, x, g, g)
+
+
+def test_decode_rejects_bad_arguments():
+    L = gdn.lib()
+    p = [FAKE] * 5
+    ok = gdn.make_desc(4, 1, 2, 128, 128)
+    st = FAKE
+    assert L.gdn_decode(ctypes.byref(gdn.make_desc(4, 1, 2, 96, 128)), *p, st, FAKE, None) == 2
+    assert L.gdn_decode(ctypes.byref(gdn.make_desc(4, 0, 2, 128, 128)), *p, st, FAKE, None) == 1
+    assert L.gdn_decode(ctypes.byref(gdn.make_desc(1, 1, 2, 128, 128, n_seqs=1)), *p, st, FAKE,
+                        None) == 1
+    assert L.gdn_decode(ctypes.byref(ok), *p, None, FAKE, None) == 1
+    assert L.gdn_decode(ctypes.byref(ok), *p, FAKE + 4, FAKE, None) == 3
