@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
     const uint32_t tmem = tslot;
     if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
         const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
+#pragma unroll
         for (int s = 0; s < D / 16; ++s)
             mma_bf16(tmem, desc_kmajor(qb, D, s), desc_kmajor(kb, D, s), id, s > 0);
         mma_commit(&mbar);
@@ -112,8 +113,10 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
             const uint32_t id = idesc_bf16(128, 64, 0, 0);
             const uint32_t sb = smem_u32(Ss), qg = smem_u32(QG), ub = smem_u32(UTs),
                            pb = smem_u32(Ps);
+#pragma unroll
             for (int s = 0; s < D / 16; ++s)
                 mma_bf16(tmem + 64, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
+#pragma unroll
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_kmajor(pb, C, s), id, 1);
             mma_commit(&mbar);

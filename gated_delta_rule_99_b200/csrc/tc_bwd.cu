@@ -67,6 +67,7 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
     const uint32_t tmem = tslot;
     if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
         const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
+#pragma unroll
         for (int s = 0; s < D / 16; ++s)
             mma_bf16(tmem, desc_kmajor(qb, D, s), desc_kmajor(kb, D, s), id, s > 0);
         mma_commit(&mbar);
@@ -103,6 +104,7 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
         operands_ready();
         if (tid == 0) {  // local dU^T[v][j] = sum_i dO[i][v] P[i][j]: M = 128, N = 64, K = 64
             const uint32_t db = smem_u32(DO), pb = smem_u32(Ps), id = idesc_bf16(128, 64, 1, 1);
+#pragma unroll
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_mnmajor(db, C, s), desc_mnmajor(pb, C, s), id, s > 0);
             mma_commit(&mbar);
@@ -211,9 +213,11 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
             const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
                            qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO);
             // dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
+#pragma unroll
             for (int s = 0; s < D / 16; ++s)
                 mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, s > 0);
             // dO^T Qg: M = 128 (v), N = 128 keys, K = 64 tokens
+#pragma unroll
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_mnmajor(ob, C, s), desc_mnmajor(qb, C, s), idx, s > 0);
             mma_commit(&mbar);
@@ -246,6 +250,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         operands_ready();
         if (v == 0) {  // - dU^T W: M = 128 (v), N = 128 keys, K = 64 tokens
             const uint32_t ub = smem_u32(dUs), wb = smem_u32(b + SbwdSmem::kW);
+#pragma unroll
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(wb, C, s), idy, 1);
             mma_commit(&mbar);
@@ -450,18 +455,25 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
                        i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
                        i64km = idesc_bf16(64, 64, 0, 1), i64mk = idesc_bf16(64, 64, 1, 0);
+#pragma unroll
         for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
             mma_bf16(tmem + cQK, desc_kmajor(qkb, D, s), desc_kmajor(kb, D, s), i128, s > 0);
+#pragma unroll
         for (int s = 0; s < 8; ++s)  // X1^T = S^T dO^T  (over v)
             mma_bf16(tmem + cX1, desc_mnmajor(scb, D, s), desc_kmajor(dob, C, s), i128mk, s > 0);
+#pragma unroll
         for (int s = 0; s < 8; ++s)  // X2^T = dSn^T U^T
             mma_bf16(tmem + cX2, desc_mnmajor(dsb, D, s), desc_mnmajor(utb, D, s), i128mm, s > 0);
+#pragma unroll
         for (int s = 0; s < 8; ++s)  // X3^T = S^T dU^T
             mma_bf16(tmem + cX3, desc_mnmajor(scb, D, s), desc_mnmajor(dub, D, s), i128mm, s > 0);
+#pragma unroll
         for (int s = 0; s < 8; ++s)  // dP = dO U^T (M = 64)
             mma_bf16(tmem + cDP, desc_kmajor(dob, C, s), desc_mnmajor(utb, D, s), i64km, s > 0);
+#pragma unroll
         for (int s = 0; s < 4; ++s)  // (A^T dU)^T = dU^T A
             mma_bf16(tmem + cAU, desc_kmajor(dub, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
+#pragma unroll
         for (int s = 0; s < 8; ++s)  // Y1 = dU V^T (M = 64)
             mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, C, s), i64mk, s > 0);
         mma_commit(&mbar);
@@ -550,8 +562,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     operands_ready();
     if (tid == 0) {
         const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
         for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
             mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
+#pragma unroll
         for (int s = 0; s < 4; ++s)  // Zp^T = X3^T A   (Z = -Zp)
             mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
         mma_commit(&mbar);
@@ -581,6 +595,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     operands_ready();
     if (tid == 0) {  // T1 = A^T dA (M = 64)
         const uint32_t id = idesc_bf16(64, 64, 1, 1);
+#pragma unroll
         for (int s = 0; s < 4; ++s)
             mma_bf16(tmem + cT1, desc_mnmajor(ab, C, s), desc_mnmajor(dab, C, s), id, s > 0);
         mma_commit(&mbar);
@@ -597,6 +612,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     operands_ready();
     if (tid == 0) {  // T1 A^T = -dL (M = 64)
         const uint32_t id = idesc_bf16(64, 64, 0, 0);
+#pragma unroll
         for (int s = 0; s < 4; ++s)
             mma_bf16(tmem + cDL, desc_kmajor(t1b, C, s), desc_kmajor(ab, C, s), id, s > 0);
         mma_commit(&mbar);
@@ -625,12 +641,16 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     operands_ready();
     if (tid == 0) {
         const uint32_t imk = idesc_bf16(128, 64, 1, 0), imm = idesc_bf16(128, 64, 1, 1);
+#pragma unroll
         for (int s = 0; s < 4; ++s)  // (dPG K)^T = K^T dPG^T
             mma_bf16(tmem + cDQ, desc_mnmajor(kb, D, s), desc_kmajor(dpb, C, s), imk, s > 0);
+#pragma unroll
         for (int s = 0; s < 4; ++s)  // (dPG^T Q)^T = Q^T dPG
             mma_bf16(tmem + cDKA, desc_mnmajor(qkb, D, s), desc_mnmajor(dpb, C, s), imm, s > 0);
+#pragma unroll
         for (int s = 0; s < 4; ++s)  // (diag(b) dLG K)^T
             mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_kmajor(dlb, C, s), imk, s > 0);
+#pragma unroll
         for (int s = 0; s < 4; ++s)  // ((diag(b) dLG)^T K)^T
             mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_mnmajor(dlb, C, s), imm, 1);
         mma_commit(&mbar);

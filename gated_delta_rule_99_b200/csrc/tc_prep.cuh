@@ -58,6 +58,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     // K K^T (M = 64 rows i, N = 64 cols j, K = 128)
     if (tid == 0) {
         const uint32_t kb = smem_u32(Kt), id = idesc_bf16(64, 64, 0, 0);
+#pragma unroll
         for (int s = 0; s < D / 16; ++s)
             mma_bf16(tmem, desc_kmajor(kb, C, s), desc_kmajor(kb, C, s), id, s > 0);
         mma_commit(&mbar);
@@ -141,6 +142,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         const uint32_t id = idesc_bf16(64, 128, 0, 1);
         if (tid == 0) {
             const uint32_t ab = smem_u32(Ab), kb = smem_u32(Kt);
+#pragma unroll
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem, desc_kmajor(ab, C, s), desc_mnmajor(kb, C, s), id, s > 0);
             mma_commit(&mbar);
@@ -164,6 +166,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             tc_fence_after();
             if (tid == 0) {
                 const uint32_t ac = smem_u32(Ac), vb = smem_u32(Vt);
+#pragma unroll
                 for (int s = 0; s < C / 16; ++s)
                     mma_bf16(tmem, desc_kmajor(ac, C, s), desc_mnmajor(vb, C, s), id, s > 0);
                 mma_commit(&mbar);

@@ -40,13 +40,16 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 }
 
 // Descriptor of k-step s (16 reduction elements) of a K-major SW128 tile of R rows.
+// The step is added to the start-address field of the tile's descriptor (no
+// carry: shared addresses stay below 256 KB), so with s a compile-time
+// constant the tile descriptor is computed once and each step is one add.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int R, int s) {
-    return sdesc(base + (uint32_t)((s >> 2) * R * 128 + (s & 3) * 32), 16, 1024);
+    return sdesc(base, 16, 1024) + (uint64_t)(((s >> 2) * R * 128 + (s & 3) * 32) >> 4);
 }
 
 // Descriptor of k-step s of an MN-major SW128 tile of R rows (rows = reduction).
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int R, int s) {
-    return sdesc(base + (uint32_t)(s * 2048), (uint32_t)(R * 128), 1024);
+    return sdesc(base, (uint32_t)(R * 128), 1024) + (uint64_t)((s * 2048) >> 4);
 }
 
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulate.

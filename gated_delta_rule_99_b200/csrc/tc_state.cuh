@@ -82,6 +82,7 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
             expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
         if (v == 0) {
             const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
+#pragma unroll
             for (int s = 0; s < D / 16; ++s)
                 mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
             mma_commit(&mbar);
@@ -107,6 +108,7 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
         operands_ready();
         if (v == 0) {
             const uint32_t ub = smem_u32(UTs), kb = smem_u32(sm + StateSmem::kKd0 + buf * 16384);
+#pragma unroll
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
             mma_commit(&mbar);
