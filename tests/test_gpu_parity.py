@@ -188,3 +188,24 @@ def test_device_side_seqlens_check():
     gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=d.cu_seqlens.cuda(),
                 cu_seqlens_host=inp.cu_seqlens, h0=d.h0, workspace=ws)
     assert gdn.device_status(ws) == 0
+
+
+# ---- the tensor-core path (bf16, d_k = d_v = 128) on the small edge cases
+def test_tc_packed_ragged_documents_with_scale():
+    lengths = [1, 0, 63, 64, 65, 130, 7, 200]
+    inp = make_inputs(B=1, T=sum(lengths), H=3, K=128, V=128, dtype="bf16", seed=21,
+                      lengths=lengths, scale=0.125)
+    check_all(inp, TOL["bf16"])
+
+
+def test_tc_strong_decay_unit_strength_and_reset_gate():
+    inp = make_inputs(B=2, T=190, H=2, K=128, V=128, dtype="bf16", seed=22, gate_scale=3.0)
+    inp.beta.fill_(1.0)
+    inp.g[:, 77] = -30.0  # decay to ~1e-13 inside a chunk
+    check_all(inp, TOL["bf16"])
+
+
+def test_tc_zero_write_strength_and_no_initial_state():
+    inp = make_inputs(B=1, T=129, H=2, K=128, V=128, dtype="bf16", seed=23, h0_std=0.0)
+    inp.beta[:, 40:90] = 0.0
+    check_all(inp, TOL["bf16"])
