@@ -293,15 +293,16 @@ __global__ void __launch_bounds__(NT, 1) tc_chains_kernel(Params pf, Params pb) 
 }
 
 // ============================================================ tc_grads
-// Two warpgroups (256 threads): warp w reaches TMEM lane quadrant w % 4, so
-// for every accumulator warpgroup g handles columns [32 g, 32 g + 32).
-constexpr int NG = 256;
+// Four warpgroups (512 threads): warp w reaches TMEM lane quadrant w % 4, so
+// for every 64-column accumulator warpgroup g handles columns [16 g, 16 g + 16).
+constexpr int NG = 512;
+constexpr int CW = 16;  // columns per warpgroup
 
 struct GradSmem {
     static constexpr int kQK = 0, kDO = 32768, kV = 49152, kSC = 65536, kDSN = 98304,
                          kUT = 131072, kDUT = 147456, kAB = 163840, kX3 = 172032,
                          kDA = 188416, kT1 = 196608, kDPG = 204800, kDLG = 212992,
-                         kVec = 221184, kEnd = kVec + 16 * 256;
+                         kVec = 221184, kEnd = kVec + 24 * 256;
     // reused once the first products have consumed the images there: fp32
     // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, a [128][65] reduction
     // buffer, and the 64 x 64 decay matrix Gam (columns xor-swizzled by row)
@@ -314,24 +315,27 @@ constexpr int LP = 65;  // padded row stride (floats) of the fp32 scratch
 __device__ __forceinline__ int gidx(int i, int j) { return i * 64 + (j ^ (i & 31)); }
 
 // Deterministic column sums of red[t][i] over the 128 rows t -> out[i]:
-// four threads per column each sum 32 rows, then one thread adds the four.
+// eight threads per column each sum 16 rows, then one thread adds the eight.
 __device__ __forceinline__ void reduce_rows(const float *red, float *out, float *part) {
     __syncthreads();
     {
         const int i = threadIdx.x & 63, k = threadIdx.x >> 6;
-        const float *src = red + k * 32 * LP + i;
+        const float *src = red + k * 16 * LP + i;
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int t = 0; t < 32; t += 2) {
+        for (int t = 0; t < 16; t += 2) {
             s0 += src[t * LP];
             s1 += src[(t + 1) * LP];
         }
         part[k * 64 + i] = s0 + s1;
     }
     __syncthreads();
-    if (threadIdx.x < C)
-        out[threadIdx.x] = (part[threadIdx.x] + part[64 + threadIdx.x]) +
-                           (part[128 + threadIdx.x] + part[192 + threadIdx.x]);
+    if (threadIdx.x < C) {
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s += part[k * 64 + threadIdx.x];
+        out[threadIdx.x] = s;
+    }
     __syncthreads();
 }
 
@@ -366,10 +370,9 @@ __device__ __forceinline__ void store_rows(bf16 *dst, const uint8_t *stage, int6
 }
 
 
-// 32 consecutive fp32 columns of this thread's TMEM lane (quadrant w % 4).
-__device__ __forceinline__ void ld32(uint32_t tmem, int col, float *d) {
+// CW consecutive fp32 columns of this thread's TMEM lane (quadrant w % 4).
+__device__ __forceinline__ void ldcw(uint32_t tmem, int col, float *d) {
     tmem_ld16(tmq(tmem, col), d);
-    tmem_ld16(tmq(tmem, col + 16), d + 16);
     tmem_ld_wait();
 }
 
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     __shared__ float s_hd;
     if (p.hdr->status) return;
     const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
-    const int wg = tid >> 7, r = tid & 127, cb = 32 * wg;
+    const int wg = tid >> 7, r = tid & 127, cb = CW * wg;
     const int l = tid & 31, i64 = l < 16 ? ((tid >> 5) & 3) * 16 + l : -1;  // M = 64 row
     const ChunkInfo ci = p.chunks[c];
     using S_ = GradSmem;
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     float *vec = reinterpret_cast<float *>(sm + S_::kVec);
     float *G = vec, *bta = vec + 64, *gam = vec + 128, *e = vec + 192, *dB = vec + 256,
           *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576,
-          *dbl2 = vec + 640, *part = vec + 768;
+          *dbl2 = vec + 640, *part = vec + 896;
     float *PE = reinterpret_cast<float *>(sm + S_::kPE);
     float *KKG = reinterpret_cast<float *>(sm + S_::kKKG);
     float *RED = reinterpret_cast<float *>(sm + S_::kRed);
@@ -449,7 +452,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
                   cY2 = 0, cZ = 448, cT1 = 192, cDL = 0, cDQ = 256, cDK = 320, cDKA = 384;
     uint32_t phase = 0;
     bool ok;
-    float d[32];
+    float d[CW];
     const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
     if (tid == 0) {
         const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
@@ -506,17 +509,17 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         __syncthreads();
     }
     // P (scaled, lower incl. diagonal) and Gam . K K^T (strictly lower), fp32
-    ld32(tmem, cQK + cb, d);
+    ldcw(tmem, cQK + cb, d);
     if (r < 64) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < CW; ++q) {
             const int j = cb + q;
             PE[r * LP + j] = j <= r ? p.scale * Gam[gidx(r, j)] * d[q] : 0.f;
         }
     } else {
         const int i = r - 64;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < CW; ++q) {
             const int j = cb + q;
             KKG[i * LP + j] = j < i ? Gam[gidx(i, j)] * d[q] : 0.f;
         }
@@ -524,9 +527,9 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     {  // dv = diag(b) A^T dU (staged as rows in the consumed dO tile); partial v . (A^T dU)
         bf16 *stage = reinterpret_cast<bf16 *>(DO);
         const ColSw vcol(VT, C, r);
-        ld32(tmem, cAU + cb, d);
+        ldcw(tmem, cAU + cb, d);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < CW; ++q) {
             const int i = cb + q;
             RED[r * LP + i] = vcol.at(cb, q) * d[q];
             stage[i * D + r] = __float2bfloat16_rn(bta[i] * d[q]);
@@ -534,29 +537,29 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         reduce_rows(RED, dB, part);
         store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H);
     }
-    ld32(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
+    ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
 #pragma unroll
-    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = p.scale * qcol.at(cb, q) * d[q];
+    for (int q = 0; q < CW; ++q) RED[r * LP + cb + q] = p.scale * qcol.at(cb, q) * d[q];
     reduce_rows(RED, qx, part);
-    ld32(tmem, cX2 + cb, d);  // partial k . X2
+    ldcw(tmem, cX2 + cb, d);  // partial k . X2
 #pragma unroll
-    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = kcol.at(cb, q) * d[q];
+    for (int q = 0; q < CW; ++q) RED[r * LP + cb + q] = kcol.at(cb, q) * d[q];
     reduce_rows(RED, kx, part);
-    ld32(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
+    ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < CW / 8; ++q)
         *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
-    ld32(tmem, cDP + cb, d);  // dP: dPG = dP . Gam as an operand tile; PE <- dP . P
+    ldcw(tmem, cDP + cb, d);  // dP: dPG = dP . Gam as an operand tile; PE <- dP . P
     if (i64 >= 0) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < CW; ++q) {
             const int j = cb + q;
             const float dp = j <= i64 ? d[q] : 0.f;
             PE[i64 * LP + j] *= dp;
             d[q] = dp * Gam[gidx(i64, j)];
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < CW / 8; ++q)
             *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
     }
     operands_ready();
@@ -574,23 +577,23 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     phase ^= 1;
     if (!ok) goto done;
     {  // dA = (dU V^T) diag(b) - (X3 K^T) diag(b gam)
-        float y2[32];
-        ld32(tmem, cY1 + cb, d);
-        ld32(tmem, cY2 + cb, y2);
+        float y2[CW];
+        ldcw(tmem, cY1 + cb, d);
+        ldcw(tmem, cY2 + cb, y2);
         if (i64 >= 0) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
+            for (int q = 0; q < CW; ++q) {
                 const int m = cb + q;
                 d[q] = bta[m] * d[q] - bta[m] * gam[m] * y2[q];
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < CW / 8; ++q)
                 *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
         }
     }
-    ld32(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
+    ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
 #pragma unroll
-    for (int q = 0; q < 32; ++q) RED[r * LP + cb + q] = -kcol.at(cb, q) * d[q];
+    for (int q = 0; q < CW; ++q) RED[r * LP + cb + q] = -kcol.at(cb, q) * d[q];
     reduce_rows(RED, kz, part);
     operands_ready();
     if (tid == 0) {  // T1 = A^T dA (M = 64)
@@ -603,10 +606,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     ok = cta_wait(&mbar, phase, p, 23);
     phase ^= 1;
     if (!ok) goto done;
-    ld32(tmem, cT1 + cb, d);
+    ldcw(tmem, cT1 + cb, d);
     if (i64 >= 0) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < CW / 8; ++q)
             *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
     }
     operands_ready();
@@ -620,12 +623,12 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     ok = cta_wait(&mbar, phase, p, 24);
     phase ^= 1;
     if (!ok) goto done;
-    ld32(tmem, cDL + cb, d);  // dL (strictly lower); diag(b) dL . Gam tile; PE += dL . L
+    ldcw(tmem, cDL + cb, d);  // dL (strictly lower); diag(b) dL . Gam tile; PE += dL . L
     if (i64 >= 0) {
         float dbl = 0.f;
         const float bi = bta[i64];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < CW; ++q) {
             const int j = cb + q;
             const float dl = j < i64 ? -d[q] : 0.f;
             const float kkg = KKG[i64 * LP + j];
@@ -634,7 +637,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
             d[q] = bi * dl * Gam[gidx(i64, j)];
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < CW / 8; ++q)
             *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
         dbl2[wg * 64 + i64] = dbl;
     }
@@ -664,7 +667,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
             cs += PE[j * LP + i];
         }
         dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + rs - cs + bta[i] * gam[i] * kz[i];
-        dB[i] += dbl2[i] + dbl2[64 + i] + gam[i] * kz[i];
+        dB[i] += (dbl2[i] + dbl2[64 + i]) + (dbl2[128 + i] + dbl2[192 + i]) + gam[i] * kz[i];
     }
     __syncthreads();
     if (tid == 0) {
@@ -689,24 +692,24 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     {  // dq = scale (diag(gam) X1 + dPG K) ; dk = diag(e) X2 + diag(b gam) Z + dPG^T Q' + dL terms
         // staged as rows in the consumed dO and V tiles, then 16-byte stores
         bf16 *sq = reinterpret_cast<bf16 *>(DO), *sk = reinterpret_cast<bf16 *>(VT);
-        float a[32];
-        ld32(tmem, cX1 + cb, d);
-        ld32(tmem, cDQ + cb, a);
+        float a[CW];
+        ldcw(tmem, cX1 + cb, d);
+        ldcw(tmem, cDQ + cb, a);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < CW; ++q) {
             const int i = cb + q;
             sq[i * D + r] = __float2bfloat16_rn(p.scale * (gam[i] * d[q] + a[q]));
         }
-        ld32(tmem, cX2 + cb, d);
-        ld32(tmem, cZ + cb, a);
+        ldcw(tmem, cX2 + cb, d);
+        ldcw(tmem, cZ + cb, a);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) d[q] = e[cb + q] * d[q] - bta[cb + q] * gam[cb + q] * a[q];
-        ld32(tmem, cDKA + cb, a);
+        for (int q = 0; q < CW; ++q) d[q] = e[cb + q] * d[q] - bta[cb + q] * gam[cb + q] * a[q];
+        ldcw(tmem, cDKA + cb, a);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) d[q] += p.scale * a[q];
-        ld32(tmem, cDK + cb, a);
+        for (int q = 0; q < CW; ++q) d[q] += p.scale * a[q];
+        ldcw(tmem, cDK + cb, a);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) sk[(cb + q) * D + r] = __float2bfloat16_rn(d[q] + a[q]);
+        for (int q = 0; q < CW; ++q) sk[(cb + q) * D + r] = __float2bfloat16_rn(d[q] + a[q]);
         __syncthreads();
         store_rows(static_cast<bf16 *>(p.dq), DO, ci.tok0, ci.len, h, H);
         store_rows(static_cast<bf16 *>(p.dk), VT, ci.tok0, ci.len, h, H);
