@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
 }
 
 // ============================================================ tc_state_fwd
-__global__ void __launch_bounds__(NS, 1) tc_state_fwd_kernel(Params p) {
+__global__ void __launch_bounds__(NT, 1) tc_state_fwd_kernel(Params p) {
     state_fwd_body(p, blockIdx.x);
 }
 
@@ -46,25 +46,21 @@ struct OutSmem {
 };
 constexpr int kOutSmem = OutSmem::kEnd + 1024;
 
-constexpr int NO = 256;  // two warpgroups split every accumulator's columns
-
-__global__ void __launch_bounds__(NO) tc_out_kernel(Params p) {
+__global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
-    const int v = tid & 127, g = tid >> 7, l = tid & 31;
-    const int i64 = l < 16 ? ((tid >> 5) & 3) * 16 + l : -1;  // row of an M = 64 accumulator
     const ChunkInfo ci = p.chunks[c];
     uint8_t *QK = sm + OutSmem::kQK, *Ss = sm + OutSmem::kS, *UTs = sm + OutSmem::kUT;
     uint8_t *QG = sm + OutSmem::kQG, *Ps = sm + OutSmem::kP;
     float *G = reinterpret_cast<float *>(sm + OutSmem::kG);
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, NO);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, NO);
-    load_image_async(Ss, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128, NO);
-    load_image_async(UTs, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT, NO);
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
+    load_image_async(Ss, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128);
+    load_image_async(UTs, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT);
     cp_async_commit();
     if (tid < C) G[tid] = p.tG[(size_t)ch * C + tid];
     if (tid == 0) {
@@ -86,7 +82,7 @@ __global__ void __launch_bounds__(NO) tc_out_kernel(Params p) {
         mma_commit(&mbar);
     }
     // scale * gam_i * q_i as a K-major operand (rows i)
-    for (int t = tid; t < C * 16; t += NO) {
+    for (int t = tid; t < C * 16; t += NT) {
         const int r = t >> 4, j = t & 15;
         float f[8];
         unpack8(*reinterpret_cast<const uint4 *>(QK + sw128_chunk(D, r, j)), f);
@@ -97,20 +93,20 @@ __global__ void __launch_bounds__(NO) tc_out_kernel(Params p) {
     }
     bool ok = cta_wait(&mbar, 0, p, 5);
     if (ok) {
-        const int c0 = 32 * g;  // this warpgroup's columns j
-        float d[32];
-        tmem_ld16(tmq(tmem, c0), d);
-        tmem_ld16(tmq(tmem, c0 + 16), d + 16);
-        tmem_ld_wait();
-        if (i64 >= 0) {
+        const int i = m64_row();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, c0), d);
+            tmem_ld_wait();
+            if (i >= 0) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int j = c0 + q;
-                d[q] = j <= i64 ? p.scale * expf(G[i64] - G[j]) * d[q] : 0.f;
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    d[q] = j <= i ? p.scale * expf(G[i] - G[j]) * d[q] : 0.f;
+                }
+                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
             }
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i64, c0 / 8 + q)) = pack8(d + 8 * q);
         }
         operands_ready();
         if (tid == 0) {
@@ -129,16 +125,16 @@ __global__ void __launch_bounds__(NO) tc_out_kernel(Params p) {
     }
     if (ok) {  // O^T column v -> rows of a staging tile (the consumed Q K tile), 16-byte stores
         bf16 *stage = reinterpret_cast<bf16 *>(QK);
-        const int i0 = 32 * g;
-        float d[32];
-        tmem_ld16(tmq(tmem, 64 + i0), d);
-        tmem_ld16(tmq(tmem, 64 + i0 + 16), d + 16);
-        tmem_ld_wait();
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float d[16];
+            tmem_ld16(tm(tmem, 64 + c0), d);
+            tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 32; ++q) stage[(i0 + q) * D + v] = __float2bfloat16_rn(d[q]);
+            for (int q = 0; q < 16; ++q) stage[(c0 + q) * D + tid] = __float2bfloat16_rn(d[q]);
+        }
         __syncthreads();
         bf16 *o = static_cast<bf16 *>(p.o);
-        for (int t = tid; t < C * 16; t += NO) {
+        for (int t = tid; t < C * 16; t += NT) {
             const int i = t >> 4, j = t & 15;
             if (i < ci.len)
                 *reinterpret_cast<uint4 *>(o + ((int64_t)(ci.tok0 + i) * H + h) * D + j * 8) =
@@ -149,6 +145,7 @@ __global__ void __launch_bounds__(NO) tc_out_kernel(Params p) {
     __syncthreads();
     if (tid < 32) tmem_dealloc(tmem, 128);
 }
+
 
 }  // namespace
 
@@ -171,7 +168,7 @@ cudaError_t tc_launch_state_fwd(const Params &p, cudaStream_t stream) {
     if (nseq == 0) return cudaSuccess;
     cudaError_t e = set_smem(tc_state_fwd_kernel, kStateSmem);
     if (e != cudaSuccess) return e;
-    GDN_LAUNCH(kKTcStateFwd, stream, tc_state_fwd_kernel<<<nseq, NS, kStateSmem, stream>>>(p));
+    GDN_LAUNCH(kKTcStateFwd, stream, tc_state_fwd_kernel<<<nseq, NT, kStateSmem, stream>>>(p));
     return cudaSuccess;
 }
 
@@ -182,7 +179,7 @@ cudaError_t launch_tc_fwd(const Params &p, const Problem &, cudaStream_t stream)
     const int nch = p.NC * p.H;
     if (nch > 0) {
         if ((e = set_smem(tc_out_kernel, kOutSmem))) return e;
-        GDN_LAUNCH(kKTcOut, stream, tc_out_kernel<<<nch, NO, kOutSmem, stream>>>(p));
+        GDN_LAUNCH(kKTcOut, stream, tc_out_kernel<<<nch, NT, kOutSmem, stream>>>(p));
     }
     return cudaSuccess;
 }

@@ -147,46 +147,39 @@ constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
 __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
                                               const ChunkInfo &ci, int h, const Params &p) {
     uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
-    load_image_async(b + SbwdSmem::kKd, static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64,
-                     NS);
-    load_image_async(b + SbwdSmem::kW, static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64,
-                     NS);
-    load_image_async(b + SbwdSmem::kQg, static_cast<const uint8_t *>(p.tQg) + ch * kImg64, kImg64,
-                     NS);
-    load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H, NS);
+    load_image_async(b + SbwdSmem::kKd, static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
+    load_image_async(b + SbwdSmem::kW, static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
+    load_image_async(b + SbwdSmem::kQg, static_cast<const uint8_t *>(p.tQg) + ch * kImg64, kImg64);
+    load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H);
     load_image_async(b + SbwdSmem::kDUL, static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT,
-                     kImgUT, NS);
+                     kImgUT);
     if (threadIdx.x < 16)
         cp_async16(smem_u32(b + SbwdSmem::kG) + threadIdx.x * 16, p.tG + ch * C + threadIdx.x * 4);
     cp_async_commit();
 }
 
 // Body of the reverse state pass for CTA `blk` (sequence blk / H, head blk % H).
-// Two warpgroups: thread (g, v) owns row v of dS = dH^T and its key columns
-// [64 g, 64 g + 64).
 __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
-    const int H = p.H, n = blk / H, h = blk % H, tid = threadIdx.x, v = tid & 127, g = tid >> 7;
-    const int k0 = g * SH;
-    float S[SH];  // dS row v, key columns [k0, k0 + 64): the gradient of the state leaving
-                  // the current chunk
+    const int H = p.H, n = blk / H, h = blk % H, v = threadIdx.x;
+    float S[D];  // dS row v (gradient of the state leaving the current chunk)
     if (p.dhT) {
         const float *g0 = p.dhT + ((size_t)n * H + h) * D * D;
 #pragma unroll
-        for (int kk = 0; kk < SH; ++kk) S[kk] = g0[(k0 + kk) * D + v];
+        for (int kk = 0; kk < D; ++kk) S[kk] = g0[kk * D + v];
     } else {
 #pragma unroll
-        for (int kk = 0; kk < SH; ++kk) S[kk] = 0.f;
+        for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
     }
-    if (tid == 0) {
+    if (v == 0) {
         mbar_init(&mbar, 1);
         fence_mbar_init();
     }
-    if (tid < 32) {
+    if (v < 32) {
         tmem_alloc(&tslot, 256);
         tmem_relinquish();
     }
@@ -211,12 +204,12 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         }
         uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
 #pragma unroll
-        for (int j = 0; j < SH / 8; ++j)
-            *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, k0 / 8 + j)) = pack8(S + 8 * j);
+        for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
         operands_ready();
         // after the barrier: the gate row was copied by other threads' cp.async
         const float gC = expf(reinterpret_cast<const float *>(b + SbwdSmem::kG)[C - 1]);
-        if (tid == 0) {
+        if (v == 0) {
             const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
                            qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO);
             // dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
@@ -233,30 +226,29 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         }
         if (!cta_wait(&mbar, phase, p, 13)) break;
         phase ^= 1;
-        {  // dU^T = dS Kd^T + local dU^T (tokens [32 g, 32 g + 32)); -dU^T is the next
-           // operand, +dU^T an image for tc_grads
+        {  // dU^T = dS Kd^T + local dU^T ; -dU^T is the next operand, +dU^T an image for tc_grads
             const uint8_t *dul = b + SbwdSmem::kDUL;  // local dU^T, swizzled rows
             uint8_t *img = static_cast<uint8_t *>(p.tdUT) + ch * kImgUT;
-            const int i0 = 32 * g;
-            float d[32], l[8];
-            tmem_ld16(tmq(tmem, i0), d);
-            tmem_ld16(tmq(tmem, i0 + 16), d + 16);
-            tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                unpack8(*reinterpret_cast<const uint4 *>(dul + sw128_chunk(D, v, i0 / 8 + q)), l);
+            for (int c16 = 0; c16 < C; c16 += 16) {
+                float d[16], l[16];
+                tmem_ld16(tm(tmem, c16), d);
+                tmem_ld_wait();
+                unpack8(*reinterpret_cast<const uint4 *>(dul + sw128_chunk(D, v, c16 / 8)), l);
+                unpack8(*reinterpret_cast<const uint4 *>(dul + sw128_chunk(D, v, c16 / 8 + 1)),
+                        l + 8);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) d[8 * q + x] += l[x];
-                *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, i0 / 8 + q)) = pack8(d + 8 * q);
+                for (int q = 0; q < 16; ++q) d[q] += l[q];
+                *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, c16 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) d[q] = -d[q];
+                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8)) = pack8(d);
+                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
             }
-#pragma unroll
-            for (int q = 0; q < 32; ++q) d[q] = -d[q];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, i0 / 8 + q)) = pack8(d + 8 * q);
         }
         operands_ready();
-        if (tid == 0) {  // - dU^T W: M = 128 (v), N = 128 keys, K = 64 tokens
+        if (v == 0) {  // - dU^T W: M = 128 (v), N = 128 keys, K = 64 tokens
             const uint32_t ub = smem_u32(dUs), wb = smem_u32(b + SbwdSmem::kW);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
@@ -266,35 +258,35 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         if (!cta_wait(&mbar, phase, p, 14)) break;
         phase ^= 1;
 #pragma unroll
-        for (int c32 = 0; c32 < SH; c32 += 32) {
+        for (int c32 = 0; c32 < D; c32 += 32) {
             float d[32];
-            tmem_ld16(tmq(tmem, 64 + k0 + c32), d);
-            tmem_ld16(tmq(tmem, 64 + k0 + c32 + 16), d + 16);
+            tmem_ld16(tm(tmem, 64 + c32), d);
+            tmem_ld16(tm(tmem, 64 + c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
         }
-        if (tid == 0) bulk_wait_read();
+        if (v == 0) bulk_wait_read();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
-    if (tid == 0) bulk_wait_all();
+    if (v == 0) bulk_wait_all();
     if (p.dh0) {
         float *g0 = p.dh0 + ((size_t)n * H + h) * D * D;
 #pragma unroll
-        for (int kk = 0; kk < SH; ++kk) g0[(k0 + kk) * D + v] = S[kk];
+        for (int kk = 0; kk < D; ++kk) g0[kk * D + v] = S[kk];
     }
     cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
-    if (tid < 32) tmem_dealloc(tmem, 256);
+    if (v < 32) tmem_dealloc(tmem, 256);
 }
 
 // Both chains of the backward in one launch: CTAs [0, N*H) recompute the
 // forward states (pf has no final-state output), CTAs [N*H, 2*N*H) run the
 // reverse pass.  They are independent, so each gets its own SMs.
-__global__ void __launch_bounds__(NS, 1) tc_chains_kernel(Params pf, Params pb) {
+__global__ void __launch_bounds__(NT, 1) tc_chains_kernel(Params pf, Params pb) {
     const int nh = pb.N * pb.H;
     if ((int)blockIdx.x < nh) state_fwd_body(pf, blockIdx.x);
     else state_bwd_body(pb, blockIdx.x - nh);
@@ -744,7 +736,7 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
     if (nseq > 0) {
         const int sm = kSbwdSmem > kStateSmem ? kSbwdSmem : kStateSmem;
         if ((e = set_smem(tc_chains_kernel, sm))) return e;
-        GDN_LAUNCH(kKTcStateBwd, stream, tc_chains_kernel<<<2 * nseq, NS, sm, stream>>>(pf, p));
+        GDN_LAUNCH(kKTcStateBwd, stream, tc_chains_kernel<<<2 * nseq, NT, sm, stream>>>(pf, p));
     }
     if (nch > 0) {
         if ((e = set_smem(tc_grads_kernel, kGradSmem))) return e;

@@ -16,20 +16,13 @@ struct StateSmem {
 };
 constexpr int kStateSmem = StateSmem::kEnd + 1024;
 
-// The chain kernels run two warpgroups (256 threads): thread (g, v) owns row
-// v of the state and its key columns [64 g, 64 g + 64); warp w reaches TMEM
-// lane quadrant w % 4, so both warpgroups read the same lanes (rows v) and
-// split the columns.
-constexpr int NS = 256;
-constexpr int SH = D / 2;  // state columns per thread
-
 __device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p) {
     load_image_async(sm + StateSmem::kW0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64, NS);
+                     static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
     load_image_async(sm + StateSmem::kKd0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64, NS);
+                     static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
     load_image_async(sm + StateSmem::kUt0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64, NS);
+                     static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64);
     if (threadIdx.x < 16)
         cp_async16(smem_u32(sm + StateSmem::kG0 + buf * 256) + threadIdx.x * 16,
                    p.tG + ch * C + threadIdx.x * 4);
@@ -43,22 +36,21 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
     __shared__ uint64_t mbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
-    const int H = p.H, n = blk / H, h = blk % H, tid = threadIdx.x, v = tid & 127, g = tid >> 7;
-    const int k0 = g * SH;  // first key column of this thread
-    float S[SH];
+    const int H = p.H, n = blk / H, h = blk % H, v = threadIdx.x;
+    float S[D];
     if (p.h0) {
         const float *h0 = p.h0 + ((size_t)n * H + h) * D * D;
 #pragma unroll
-        for (int kk = 0; kk < SH; ++kk) S[kk] = h0[(k0 + kk) * D + v];
+        for (int kk = 0; kk < D; ++kk) S[kk] = h0[kk * D + v];
     } else {
 #pragma unroll
-        for (int kk = 0; kk < SH; ++kk) S[kk] = 0.f;
+        for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
     }
-    if (tid == 0) {
+    if (v == 0) {
         mbar_init(&mbar, 1);
         fence_mbar_init();
     }
-    if (tid < 32) {
+    if (v < 32) {
         tmem_alloc(&tslot, 256);
         tmem_relinquish();
     }
@@ -82,13 +74,13 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
         }
         // the state entering this chunk, as bf16 operand rows
 #pragma unroll
-        for (int j = 0; j < SH / 8; ++j)
-            *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, k0 / 8 + j)) = pack8(S + 8 * j);
+        for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
         operands_ready();
         // after the barrier: the gate row was copied by other threads' cp.async
         const float gC =
             expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
-        if (tid == 0) {
+        if (v == 0) {
             const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
@@ -99,21 +91,22 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
         }
         if (!cta_wait(&mbar, phase, p, 3)) break;
         phase ^= 1;
-        {  // U^T[v][i] = Ut[i][v] - (S W^T)[v][i], tokens [32 g, 32 g + 32)
-            const bf16 *Ut = reinterpret_cast<const bf16 *>(sm + StateSmem::kUt0 + buf * 16384);
-            const int i0 = 32 * g;
+        // U^T[v][i] = Ut[i][v] - (S W^T)[v][i]
+        const bf16 *Ut = reinterpret_cast<const bf16 *>(sm + StateSmem::kUt0 + buf * 16384);
+#pragma unroll
+        for (int c32 = 0; c32 < C; c32 += 32) {
             float d[32];
-            tmem_ld16(tmq(tmem, i0), d);
-            tmem_ld16(tmq(tmem, i0 + 16), d + 16);
+            tmem_ld16(tm(tmem, c32), d);
+            tmem_ld16(tm(tmem, c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) d[q] = __bfloat162float(Ut[(i0 + q) * D + v]) - d[q];
+            for (int q = 0; q < 32; ++q) d[q] = __bfloat162float(Ut[(c32 + q) * D + v]) - d[q];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, i0 / 8 + q)) = pack8(d + 8 * q);
+                *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
         }
         operands_ready();
-        if (tid == 0) {
+        if (v == 0) {
             const uint32_t ub = smem_u32(UTs), kb = smem_u32(sm + StateSmem::kKd0 + buf * 16384);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
@@ -125,30 +118,30 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
         if (!cta_wait(&mbar, phase, p, 4)) break;
         phase ^= 1;
 #pragma unroll
-        for (int c32 = 0; c32 < SH; c32 += 32) {
+        for (int c32 = 0; c32 < D; c32 += 32) {
             float d[32];
-            tmem_ld16(tmq(tmem, 64 + k0 + c32), d);
-            tmem_ld16(tmq(tmem, 64 + k0 + c32 + 16), d + 16);
+            tmem_ld16(tm(tmem, 64 + c32), d);
+            tmem_ld16(tm(tmem, 64 + c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
         }
         // shared operands are rewritten next chunk: their bulk stores must have read them
-        if (tid == 0) bulk_wait_read();
+        if (v == 0) bulk_wait_read();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
-    if (tid == 0) bulk_wait_all();
+    if (v == 0) bulk_wait_all();
     if (p.hT) {
         float *hT = p.hT + ((size_t)n * H + h) * D * D;
 #pragma unroll
-        for (int kk = 0; kk < SH; ++kk) hT[(k0 + kk) * D + v] = S[kk];
+        for (int kk = 0; kk < D; ++kk) hT[kk * D + v] = S[kk];
     }
     cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
-    if (tid < 32) tmem_dealloc(tmem, 256);
+    if (v < 32) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace tc
