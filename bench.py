@@ -39,8 +39,9 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--mode", choices=("fwdbwd", "decode"), default="fwdbwd",
-                    help="decode: time the recurrent decode step instead (not the headline)")
+    ap.add_argument("--mode", choices=("fwdbwd", "decode", "report"), default="fwdbwd",
+                    help="decode: the recurrent decode step; report: every workload's "
+                         "throughput (neither is the headline line)")
     ap.add_argument("--shape", default=None,
                     help="B,T,H override of the workload (profiling and size sweeps only)")
     return ap.parse_args()
@@ -486,6 +487,81 @@ def run_decode(args, rank, world, local_rank):
         "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
 
 
+def run_report(args, rank, world, local_rank):
+    """Throughput of every workload on one GPU: forward tokens/s for the forward
+    workloads, forward+backward for the others, each with its whole-call
+    roofline (method flops and bytes against the measured peaks).  One JSON
+    line per workload."""
+    import torch
+
+    import gated_delta_rule_99_b200 as gdn
+    from gated_delta_rule_99_b200.inputs import WORKLOADS, workload
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for idx in sorted(WORKLOADS):
+        w = WORKLOADS[idx]
+        inp = workload(idx, device="cuda" if idx == 4 else "cpu")
+        d = inp.to(dev)
+        cu = inp.cu_seqlens
+        cu_dev = None if cu is None else cu.to(dev)
+        bwd = w["bwd"]
+        B, T, H, K, V = w["B"], w["T"], w["H"], w["K"], w["V"]
+        n = inp.n_seqs
+        desc = gdn.make_desc(B, T, H, K, V, 0 if cu is None else n,
+                             gdn.GDN_BF16 if w["dtype"] == "bf16" else gdn.GDN_FP32)
+        ws = gdn.alloc_workspace(max(gdn.fwd_workspace_size(desc),
+                                     gdn.bwd_workspace_size(desc) if bwd else 0), dev)
+        o = torch.empty_like(d.v)
+        hT = torch.empty(n, H, K, V, dtype=torch.float32, device=dev)
+        grads = None
+        if bwd:
+            grads = (torch.empty_like(d.q), torch.empty_like(d.k), torch.empty_like(d.v),
+                     torch.empty_like(d.g), torch.empty_like(d.beta),
+                     torch.empty(n, H, K, V, dtype=torch.float32, device=dev))
+
+        def step():
+            gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=cu_dev, cu_seqlens_host=cu,
+                        h0=d.h0, o=o, hT=hT, workspace=ws)
+            if bwd:
+                gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, cu_seqlens=cu_dev,
+                            cu_seqlens_host=cu, h0=d.h0, dhT=d.dhT, grads=grads, workspace=ws)
+
+        for _ in range(3):
+            step()
+        steps = 3 if idx == 4 else max(5, args.steps)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        th = B * T * H
+        fwd_f = 2 * C * (3 * K + 2 * V) + 6 * K * V + C * C / 3
+        bwd_f = 9 * 2 * C * K + 5 * 2 * C * V + 8 * 2 * K * V + 4 * C * C
+        flops = (fwd_f + (bwd_f if bwd else 0)) * th
+        el = 2 if w["dtype"] == "bf16" else 4
+        fwd_b = (3 * el * K if K == V else el * (2 * K + V)) + 8 + el * V
+        bwd_b = el * (2 * K + 2 * V) + 8 + el * (2 * K + V) + 8
+        bytes_ = (fwd_b + (bwd_b if bwd else 0)) * th
+        t_bound = max(flops / (pk["tc_sus"] * 1e12), bytes_ / (pk["hbm"] * 1e9))
+        if rank == 0:
+            print(json.dumps({
+                "workload": w["name"], "pass": "fwd+bwd" if bwd else "fwd",
+                "tokens_per_s": B * T / (ms / 1e3), "ms_per_call": ms,
+                "roofline_frac": t_bound * 1e3 / ms, "roofline_us": t_bound * 1e6,
+                "path": "tensor-core" if (w["dtype"] == "bf16" and K == V == 128) else "fp32",
+                "peaks": pk["src"]}), flush=True)
+        del d, ws, o, hT, grads
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -505,6 +581,9 @@ def main():
     try:
         if args.mode == "decode":
             run_decode(args, rank, world, local_rank)
+            return
+        if args.mode == "report":
+            run_report(args, rank, world, local_rank)
             return
         run_ours(args, rank, world, local_rank)
     finally:
