@@ -33,7 +33,10 @@ class GdnError(RuntimeError):
 class GdnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("H", ctypes.c_int64),
                 ("dk", ctypes.c_int64), ("dv", ctypes.c_int64), ("n_seqs", ctypes.c_int64),
-                ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("dtype", ctypes.c_int32), ("scale", ctypes.c_float), ("flags", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+GDN_FLAG_PIECE_SCAN = 1
 
 
 _lock = threading.Lock()
@@ -76,8 +79,9 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def make_desc(B, T, H, dk, dv, n_seqs=0, dtype=GDN_BF16, scale=1.0) -> GdnDesc:
-    return GdnDesc(int(B), int(T), int(H), int(dk), int(dv), int(n_seqs), int(dtype), float(scale))
+def make_desc(B, T, H, dk, dv, n_seqs=0, dtype=GDN_BF16, scale=1.0, flags=0) -> GdnDesc:
+    return GdnDesc(int(B), int(T), int(H), int(dk), int(dv), int(n_seqs), int(dtype), float(scale),
+                   int(flags), 0)
 
 
 def _ptr(t):
@@ -103,14 +107,14 @@ def _check(t, name, dtype=None, shape=None):
         raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
 
 
-def _desc_from(q, v, cu_host, scale):
+def _desc_from(q, v, cu_host, scale, flags=0):
     B, T, H, K = q.shape
     V = v.shape[-1]
     n_seqs = 0 if cu_host is None else cu_host.numel() - 1
     dt = {torch.bfloat16: GDN_BF16, torch.float32: GDN_FP32}.get(q.dtype)
     if dt is None:
         raise ValueError("q must be bf16 or fp32")
-    return make_desc(B, T, H, K, V, n_seqs, dt, scale), (B, T, H, K, V, n_seqs)
+    return make_desc(B, T, H, K, V, n_seqs, dt, scale, flags), (B, T, H, K, V, n_seqs)
 
 
 def _seqlens(cu_seqlens, cu_seqlens_host, device):
@@ -135,12 +139,14 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, output_final_state=True,
-            o=None, hT=None, workspace=None, cu_seqlens_host=None, stream=None):
+            o=None, hT=None, workspace=None, cu_seqlens_host=None, stream=None, piece_scan=False):
     """Forward of the gated delta rule through the C ABI.  Returns (o, hT);
-    hT is None when output_final_state is False."""
+    hT is None when output_final_state is False.  piece_scan sets
+    GDN_FLAG_PIECE_SCAN (parallel pieces of long dense rows, joined exactly)."""
     L = lib()
     cu_dev, cu_host = _seqlens(cu_seqlens, cu_seqlens_host, q.device)
-    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale)
+    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale,
+                                              GDN_FLAG_PIECE_SCAN if piece_scan else 0)
     N = n_seqs if n_seqs else B
     _check(q, "q", q.dtype, (B, T, H, K)); _check(k, "k", q.dtype, (B, T, H, K))
     _check(v, "v", q.dtype, (B, T, H, V))

@@ -35,6 +35,24 @@ gdn_status describe(const gdn_desc *d, Problem *p) {
     p->NC = 0;
     p->dtype = d->dtype;
     p->scale = d->scale;
+    if (d->reserved != 0 || (d->flags & ~GDN_FLAG_PIECE_SCAN)) return GDN_ERR_INVALID_ARG;
+    p->P = 1;
+    p->L = 0;
+    if ((d->flags & GDN_FLAG_PIECE_SCAN) && d->n_seqs == 0 && d->dtype == GDN_BF16 &&
+        p->K == 128 && p->V == 128) {
+        // pieces per row: phase C (one CTA per later piece) fits one wave of the
+        // 148 SMs, phase A (two runs per middle piece) at most two, and every
+        // piece spans at least 16 chunks; fewer than 3 pieces gain nothing
+        const int64_t units = p->B * p->H, npr = (p->T + kChunk - 1) / kChunk;
+        int64_t P = 148 / units + 1;
+        const int64_t pa = (2 * 148 / units + 3) / 2;
+        if (pa < P) P = pa;
+        if (npr / 16 < P) P = npr / 16;
+        if (P >= 3) {
+            p->P = P;
+            p->L = (npr + P - 1) / P;
+        }
+    }
     return GDN_OK;
 }
 
@@ -114,6 +132,11 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.tdUT = b(L.tdUT);
     p.tG = f(L.tG);
     p.tA = f(L.tA);
+    p.P = (int32_t)pb.P;
+    p.L = (int32_t)pb.L;
+    p.tHin = f(L.tHin);
+    p.tMp = f(L.tMp);
+    p.tBp = f(L.tBp);
     return p;
 }
 
@@ -148,6 +171,12 @@ Layout make_layout(const Problem &pb, bool bwd) {
         L.tG = take(nch * kChunk * f);
         L.tS = take(nch * img128);
         L.tUT = take(nch * img64);
+        if (!bwd && pb.P > 1) {
+            const size_t units = (size_t)pb.N * pb.H * pb.P, st = (size_t)128 * 128 * f;
+            L.tHin = take(units * st);
+            L.tMp = take(units * st);
+            L.tBp = take(units * st);
+        }
         if (bwd) {
             L.tA = take(nch * kChunk * kChunk * f);
             L.tQg = take(nch * img64);
@@ -180,7 +209,7 @@ using namespace gdn;
 
 extern "C" {
 
-int gdn_version(void) { return 100; }
+int gdn_version(void) { return 101; }
 
 int gdn_chunk_size(void) { return kChunk; }
 

@@ -58,6 +58,10 @@ struct Params {
     void *tS, *tUT;                // 128x128 image of the state entering the chunk, 128x64 U^T image
     void *tQg, *tdUL, *tdSn, *tdUT;  // backward: scaled-q image, local dU^T, dS image, dU^T image
     float *tG, *tA;                // 64 cumulative gates; 64x64 fp32 A (backward)
+    // piece scan of long rows (forward): pieces per sequence, chunks per piece, and per
+    // (sequence, head, piece) the entering state, the composed transition and offset
+    int32_t P, L;
+    float *tHin, *tMp, *tBp;
 };
 
 // Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).
@@ -70,13 +74,14 @@ struct Problem {
     int64_t NC;     // exact chunk count of this call
     int dtype;
     float scale;
+    int64_t P, L;   // pieces per sequence (1 = no piece scan) and chunks per piece
 };
 
 // Workspace layout: offsets in bytes from the workspace base.
 struct Layout {
     size_t chunks, seq_first;
     size_t W, Ut, A, U, Hs, dUloc, dU, dHn, scratch;
-    size_t tW, tUt, tKd, tS, tUT, tQg, tdUL, tdSn, tdUT, tG, tA;
+    size_t tW, tUt, tKd, tS, tUT, tQg, tdUL, tdSn, tdUT, tG, tA, tHin, tMp, tBp;
     size_t total;
 };
 
@@ -107,6 +112,9 @@ enum KernelId : int32_t {
     kKTcGrads,
     kKTcLocal,
     kKDecode,
+    kKTcPieceA,
+    kKTcPieceScan,
+    kKTcPieceC,
     kKernelCount
 };
 

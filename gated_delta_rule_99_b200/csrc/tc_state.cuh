@@ -16,35 +16,47 @@ struct StateSmem {
 };
 constexpr int kStateSmem = StateSmem::kEnd + 1024;
 
-__device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p) {
+__device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p,
+                                               bool with_ut) {
     load_image_async(sm + StateSmem::kW0 + buf * 16384,
                      static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
     load_image_async(sm + StateSmem::kKd0 + buf * 16384,
                      static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
-    load_image_async(sm + StateSmem::kUt0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64);
+    if (with_ut)
+        load_image_async(sm + StateSmem::kUt0 + buf * 16384,
+                         static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64);
     if (threadIdx.x < 16)
         cp_async16(smem_u32(sm + StateSmem::kG0 + buf * 256) + threadIdx.x * 16,
                    p.tG + ch * C + threadIdx.x * 4);
     cp_async_commit();
 }
 
-// Body of the forward state pass for CTA `blk` (sequence blk / H, head blk % H).
-__device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
+// One run of the forward chain over chunks [c0, c1) of one head.
+struct ChainFwd {
+    int h, c0, c1;
+    const float *init;   // state H entering chunk c0 ([d_k][d_v] fp32), or nullptr for zero
+    int init_identity;   // start from H = I (the transition-matrix run of the piece scan)
+    int zero_ut;         // take Ut as zero (the transition-matrix run)
+    int snapshots;       // write the state entering every chunk and U^T (tile images)
+    float *final_out;    // state leaving chunk c1 - 1 ([d_k][d_v] fp32), or nullptr
+    int where;           // tag recorded if a bounded wait gives up
+};
+
+// The forward state chain: thread v owns row v of S = H^T (fp32 registers).
+__device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
-    const int H = p.H, n = blk / H, h = blk % H, v = threadIdx.x;
+    const int H = p.H, h = a.h, v = threadIdx.x;
     float S[D];
-    if (p.h0) {
-        const float *h0 = p.h0 + ((size_t)n * H + h) * D * D;
+    if (a.init) {
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = h0[kk * D + v];
+        for (int kk = 0; kk < D; ++kk) S[kk] = a.init[kk * D + v];
     } else {
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
+        for (int kk = 0; kk < D; ++kk) S[kk] = (a.init_identity && kk == v) ? 1.f : 0.f;
     }
     if (v == 0) {
         mbar_init(&mbar, 1);
@@ -58,16 +70,17 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
-    const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
+    const int c0 = a.c0, c1 = a.c1;
+    const bool with_ut = !a.zero_ut;
     uint32_t phase = 0;
-    if (c0 < c1) state_prefetch(sm, 0, (size_t)c0 * H + h, p);
+    if (c0 < c1) state_prefetch(sm, 0, (size_t)c0 * H + h, p, with_ut);
     uint8_t *Ss = sm + StateSmem::kS, *UTs = sm + StateSmem::kUT;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), id2 = idesc_bf16(128, 128, 0, 1);
     for (int c = c0; c < c1; ++c) {
         const int buf = (c - c0) & 1;
         const size_t ch = (size_t)c * H + h;
         if (c + 1 < c1) {
-            state_prefetch(sm, buf ^ 1, ch + H, p);
+            state_prefetch(sm, buf ^ 1, ch + H, p, with_ut);
             cp_async_wait<1>();
         } else {
             cp_async_wait<0>();
@@ -86,10 +99,12 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
             for (int s = 0; s < D / 16; ++s)
                 mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
             mma_commit(&mbar);
-            bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128, sb, (uint32_t)kImg128);
-            bulk_commit();
+            if (a.snapshots) {
+                bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128, sb, (uint32_t)kImg128);
+                bulk_commit();
+            }
         }
-        if (!cta_wait(&mbar, phase, p, 3)) break;
+        if (!cta_wait(&mbar, phase, p, a.where)) break;
         phase ^= 1;
         // U^T[v][i] = Ut[i][v] - (S W^T)[v][i]
         const bf16 *Ut = reinterpret_cast<const bf16 *>(sm + StateSmem::kUt0 + buf * 16384);
@@ -100,7 +115,8 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
             tmem_ld16(tm(tmem, c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) d[q] = __bfloat162float(Ut[(c32 + q) * D + v]) - d[q];
+            for (int q = 0; q < 32; ++q)
+                d[q] = (with_ut ? __bfloat162float(Ut[(c32 + q) * D + v]) : 0.f) - d[q];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
@@ -112,10 +128,12 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
             mma_commit(&mbar);
-            bulk_store(static_cast<uint8_t *>(p.tUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
-            bulk_commit();
+            if (a.snapshots) {
+                bulk_store(static_cast<uint8_t *>(p.tUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
+                bulk_commit();
+            }
         }
-        if (!cta_wait(&mbar, phase, p, 4)) break;
+        if (!cta_wait(&mbar, phase, p, a.where + 1)) break;
         phase ^= 1;
 #pragma unroll
         for (int c32 = 0; c32 < D; c32 += 32) {
@@ -127,21 +145,37 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
             for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
         }
         // shared operands are rewritten next chunk: their bulk stores must have read them
-        if (v == 0) bulk_wait_read();
+        if (v == 0 && a.snapshots) bulk_wait_read();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
-    if (v == 0) bulk_wait_all();
-    if (p.hT) {
-        float *hT = p.hT + ((size_t)n * H + h) * D * D;
+    if (v == 0 && a.snapshots) bulk_wait_all();
+    if (a.final_out) {
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) hT[kk * D + v] = S[kk];
+        for (int kk = 0; kk < D; ++kk) a.final_out[kk * D + v] = S[kk];
     }
     cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
     if (v < 32) tmem_dealloc(tmem, 256);
+}
+
+// Body of the forward state pass for CTA `blk` (sequence blk / H, head blk % H):
+// the whole sequence from h0, writing the per-chunk snapshots and hT.
+__device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
+    const int H = p.H, n = blk / H, h = blk % H;
+    ChainFwd a;
+    a.h = h;
+    a.c0 = p.seq_first[n];
+    a.c1 = p.seq_first[n + 1];
+    a.init = p.h0 ? p.h0 + ((size_t)n * H + h) * D * D : nullptr;
+    a.init_identity = 0;
+    a.zero_ut = 0;
+    a.snapshots = 1;
+    a.final_out = p.hT ? p.hT + ((size_t)n * H + h) * D * D : nullptr;
+    a.where = 3;
+    chain_fwd(p, a);
 }
 
 }  // namespace tc

@@ -81,7 +81,23 @@ typedef struct gdn_desc {
     int64_t n_seqs; /* 0: B dense rows; > 0: packed documents given by cu_seqlens */
     int32_t dtype;  /* gdn_dtype */
     float scale;    /* output scale applied to q (1.0 for the plain recurrence) */
+    int32_t flags;  /* GDN_FLAG_* options, 0 for the defaults */
+    int32_t reserved; /* must be 0 */
 } gdn_desc;
+
+/* Forward option: split long dense rows into pieces that run in parallel and
+ * are joined exactly.  Each chunk maps the state affinely, H' = M_c H + B_c
+ * (no history is dropped), so every piece computes its composed (M, B) pair
+ * from a zero and an identity start, a short scan over pieces gives every
+ * piece its entering state, and each piece then reruns its chain from that
+ * state.  It pays off when rows are long and (rows x heads) is small (the
+ * pages' long single rows: jax-linear-attention 0.1.0, "Where we lose", which
+ * splits them exactly; the FlashQLA article, "Skipping the warm-up", whose
+ * split is approximate).  Results equal the default path up to the bf16
+ * rounding of the transition matrices, so the default path's bitwise
+ * one-call-equals-chained-calls property does not carry over.  Applies to the
+ * bf16, d_k = d_v = 128 forward on dense rows; ignored elsewhere. */
+#define GDN_FLAG_PIECE_SCAN 1
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int gdn_version(void);
