@@ -501,7 +501,8 @@ def run_report(args, rank, world, local_rank):
     pk = peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    for idx in sorted(WORKLOADS):
+    runs = [(i, False) for i in sorted(WORKLOADS)] + [(4, True)]  # long row: also piece scan
+    for idx, piece in runs:
         w = WORKLOADS[idx]
         inp = workload(idx, device="cuda" if idx == 4 else "cpu")
         d = inp.to(dev)
@@ -511,7 +512,8 @@ def run_report(args, rank, world, local_rank):
         B, T, H, K, V = w["B"], w["T"], w["H"], w["K"], w["V"]
         n = inp.n_seqs
         desc = gdn.make_desc(B, T, H, K, V, 0 if cu is None else n,
-                             gdn.GDN_BF16 if w["dtype"] == "bf16" else gdn.GDN_FP32)
+                             gdn.GDN_BF16 if w["dtype"] == "bf16" else gdn.GDN_FP32,
+                             flags=gdn.GDN_FLAG_PIECE_SCAN if piece else 0)
         ws = gdn.alloc_workspace(max(gdn.fwd_workspace_size(desc),
                                      gdn.bwd_workspace_size(desc) if bwd else 0), dev)
         o = torch.empty_like(d.v)
@@ -524,7 +526,7 @@ def run_report(args, rank, world, local_rank):
 
         def step():
             gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=cu_dev, cu_seqlens_host=cu,
-                        h0=d.h0, o=o, hT=hT, workspace=ws)
+                        h0=d.h0, o=o, hT=hT, workspace=ws, piece_scan=piece)
             if bwd:
                 gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, cu_seqlens=cu_dev,
                             cu_seqlens_host=cu, h0=d.h0, dhT=d.dhT, grads=grads, workspace=ws)
@@ -553,7 +555,8 @@ def run_report(args, rank, world, local_rank):
         t_bound = max(flops / (pk["tc_sus"] * 1e12), bytes_ / (pk["hbm"] * 1e9))
         if rank == 0:
             print(json.dumps({
-                "workload": w["name"], "pass": "fwd+bwd" if bwd else "fwd",
+                "workload": w["name"] + ("+piece_scan" if piece else ""),
+                "pass": "fwd+bwd" if bwd else "fwd",
                 "tokens_per_s": B * T / (ms / 1e3), "ms_per_call": ms,
                 "roofline_frac": t_bound * 1e3 / ms, "roofline_us": t_bound * 1e6,
                 "path": "tensor-core" if (w["dtype"] == "bf16" and K == V == 128) else "fp32",
