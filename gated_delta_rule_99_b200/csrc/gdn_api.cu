@@ -131,7 +131,7 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.tdSn = b(L.tdSn);
     p.tdUT = b(L.tdUT);
     p.tG = f(L.tG);
-    p.tA = f(L.tA);
+    p.tA = b(L.tA);
     p.P = (int32_t)pb.P;
     p.L = (int32_t)pb.L;
     p.tHin = f(L.tHin);
@@ -178,7 +178,7 @@ Layout make_layout(const Problem &pb, bool bwd) {
             L.tBp = take(units * st);
         }
         if (bwd) {
-            L.tA = take(nch * kChunk * kChunk * f);
+            L.tA = take(nch * kChunk * kChunk * 2);  // bf16 tile image of A
             L.tQg = take(nch * img64);
             L.tdUL = take(nch * img64);
             L.tdSn = take(nch * img128);

@@ -57,7 +57,8 @@ struct Params {
     void *tW, *tUt, *tKd;          // 64x128 W image, 64x128 Ut rows, 64x128 diag(e)K image
     void *tS, *tUT;                // 128x128 image of the state entering the chunk, 128x64 U^T image
     void *tQg, *tdUL, *tdSn, *tdUT;  // backward: scaled-q image, local dU^T, dS image, dU^T image
-    float *tG, *tA;                // 64 cumulative gates; 64x64 fp32 A (backward)
+    float *tG;                     // 64 cumulative gates per (chunk, head)
+    void *tA;                      // 64x64 bf16 tile image of A (backward)
     // piece scan of long rows (forward): pieces per sequence, chunks per piece, and per
     // (sequence, head, piece) the entering state, the composed transition and offset
     int32_t P, L;

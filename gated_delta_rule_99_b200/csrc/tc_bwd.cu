@@ -401,31 +401,33 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     float *RED = reinterpret_cast<float *>(sm + S_::kRed);
     float *Gam = reinterpret_cast<float *>(sm + S_::kGam);
 
+    __shared__ uint64_t lbar;
+    constexpr uint32_t kImgA = C * C * 2;
+    if (tid == 0) {  // the tile images and A by bulk copies (one instruction each)
+        mbar_init(&lbar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&lbar, 2 * kImg128 + 2 * kImgUT + kImgA);
+        bulk_load(smem_u32(SC), static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128,
+                  kImg128, &lbar);
+        bulk_load(smem_u32(DSN), static_cast<const uint8_t *>(p.tdSn) + (size_t)ch * kImg128,
+                  kImg128, &lbar);
+        bulk_load(smem_u32(UT), static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT,
+                  &lbar);
+        bulk_load(smem_u32(DUT), static_cast<const uint8_t *>(p.tdUT) + (size_t)ch * kImgUT,
+                  kImgUT, &lbar);
+        bulk_load(smem_u32(AB), static_cast<const uint8_t *>(p.tA) + (size_t)ch * kImgA, kImgA,
+                  &lbar);
+    }
+    // q, k, v, do rows by cp.async into the swizzled layout
     load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, NG);
     load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, NG);
     load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H, NG);
     load_rows_async(VT, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H, NG);
-    load_image_async(SC, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128, NG);
-    load_image_async(DSN, static_cast<const uint8_t *>(p.tdSn) + (size_t)ch * kImg128, kImg128,
-                     NG);
-    load_image_async(UT, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT, NG);
-    load_image_async(DUT, static_cast<const uint8_t *>(p.tdUT) + (size_t)ch * kImgUT, kImgUT, NG);
     cp_async_commit();
     if (tid < C) {
         const int64_t idx = (int64_t)(ci.tok0 + tid) * H + h;
         G[tid] = p.tG[(size_t)ch * C + tid];
         bta[tid] = tid < ci.len ? p.beta[idx] : 0.f;
-    }
-    {  // A (fp32, from tc_prep) as a bf16 tile: rows m, columns i
-        const float4 *Ag = reinterpret_cast<const float4 *>(p.tA + (size_t)ch * C * C);
-        for (int t = tid; t < C * C / 4; t += NG) {
-            const float4 a = Ag[t];
-            const int m = t >> 4, i = (t & 15) * 4;
-            uint2 u;
-            u.x = pack_bf16(a.x, a.y);
-            u.y = pack_bf16(a.z, a.w);
-            *reinterpret_cast<uint2 *>(AB + sw128_off(C, m, i)) = u;
-        }
     }
     if (tid == 0) {
         mbar_init(&mbar, 1);
@@ -441,6 +443,16 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         e[tid] = expf(G[C - 1] - G[tid]);
     }
     cp_async_wait<0>();
+    {  // the bulk copies (bounded wait, decided by the whole CTA)
+        const bool lok = __syncthreads_and(mbar_wait(&lbar, 0, kWaitLimit));
+        if (!lok) {
+            if (tid == 0) record_timeout(p, 20);
+            tc_fence_before();
+            __syncthreads();
+            if (tid < 32) tmem_dealloc(tslot, 512);
+            return;
+        }
+    }
     operands_ready();
     const uint32_t tmem = tslot;
     const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128, dob = smem_u32(DO), vb = smem_u32(VT),

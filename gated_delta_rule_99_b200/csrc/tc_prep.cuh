@@ -130,10 +130,11 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
                 *reinterpret_cast<bf16 *>(Ab + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * bg);
                 *reinterpret_cast<bf16 *>(Ac + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * b);
             }
-            if (want_A) {
-                float *Ag = p.tA + (size_t)ch * C * C;
+            if (want_A) {  // A as a bf16 tile image (rows m, columns i) for the backward
+                uint8_t *Ag = reinterpret_cast<uint8_t *>(p.tA) + (size_t)ch * C * C * 2;
 #pragma unroll
-                for (int r = 0; r < C; ++r) Ag[r * C + j] = a[r];
+                for (int r = 0; r < C; ++r)
+                    *reinterpret_cast<bf16 *>(Ag + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r]);
             }
         }
         operands_ready();

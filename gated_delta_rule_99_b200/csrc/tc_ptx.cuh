@@ -138,6 +138,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint3
     return false;
 }
 
+// Arrive on an mbarrier and add `bytes` to the transaction count it waits for.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(smem_u32(mbar)), "r"(bytes) : "memory");
+}
+
+// Bulk (async-proxy) copy global -> this CTA's shared memory of `bytes` (multiple
+// of 16, both addresses 16-byte aligned), completing `bytes` of transactions on
+// the mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_load(uint32_t sdst, const void *gsrc, uint32_t bytes,
+                                          uint64_t *mbar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(sdst), "l"(gsrc), "r"(bytes), "r"(smem_u32(mbar)) : "memory");
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (MMA reads).
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
