@@ -304,8 +304,8 @@ struct GradSmem {
                          kDA = 188416, kT1 = 196608, kDPG = 204800, kDLG = 212992,
                          kVec = 221184, kEnd = kVec + 24 * 256;
     // reused once the first products have consumed the images there: fp32
-    // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, a [128][65] reduction
-    // buffer, and the 64 x 64 decay matrix Gam (columns xor-swizzled by row)
+    // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, per-warp partial column sums
+    // [3][4][64], and the 64 x 64 decay matrix Gam (columns xor-swizzled by row)
     static constexpr int kPE = kSC, kKKG = kSC + 64 * 65 * 4, kRed = kDSN + 1024,
                          kGam = kDUT;
 };
@@ -313,31 +313,6 @@ constexpr int kGradSmem = GradSmem::kEnd + 1024;
 constexpr int LP = 65;  // padded row stride (floats) of the fp32 scratch
 
 __device__ __forceinline__ int gidx(int i, int j) { return i * 64 + (j ^ (i & 31)); }
-
-// Deterministic column sums of red[t][i] over the 128 rows t -> out[i]:
-// eight threads per column each sum 16 rows, then one thread adds the eight.
-__device__ __forceinline__ void reduce_rows(const float *red, float *out, float *part) {
-    __syncthreads();
-    {
-        const int i = threadIdx.x & 63, k = threadIdx.x >> 6;
-        const float *src = red + k * 16 * LP + i;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int t = 0; t < 16; t += 2) {
-            s0 += src[t * LP];
-            s1 += src[(t + 1) * LP];
-        }
-        part[k * 64 + i] = s0 + s1;
-    }
-    __syncthreads();
-    if (threadIdx.x < C) {
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) s += part[k * 64 + threadIdx.x];
-        out[threadIdx.x] = s;
-    }
-    __syncthreads();
-}
 
 // Column c of an SW128 tile with R rows, read row by row: the swizzle term
 // depends on the row only through row % 8, so it is computed once.
@@ -370,6 +345,40 @@ __device__ __forceinline__ void store_rows(bf16 *dst, const uint8_t *stage, int6
 }
 
 
+// Column sums over the 32 lanes of a warp of the CW = 16 values v[q] that each
+// thread holds (lane l of the warp is row l of a 32-row slice; v[q] belongs to
+// column cb + q): a butterfly that halves the values at every step leaves the
+// sum of column cb + q(l) in lane l, q(l) = 8 b4 + 4 b3 + 2 b2 + b1 with b the
+// lane's bits, written by the even lanes to wsum[w4][cb + q].
+__device__ __forceinline__ void warp_colsum(float *v, float *wsum, int w4, int cb, int l) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const bool up = l & 16;
+        const float send = up ? v[k] : v[k + 8], keep = up ? v[k + 8] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const bool up = l & 8;
+        const float send = up ? v[k] : v[k + 4], keep = up ? v[k + 4] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const bool up = l & 4;
+        const float send = up ? v[k] : v[k + 2], keep = up ? v[k + 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    {
+        const bool up = l & 2;
+        const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+    const int q = ((l >> 4) & 1) * 8 + ((l >> 3) & 1) * 4 + ((l >> 2) & 1) * 2 + ((l >> 1) & 1);
+    if (!(l & 1)) wsum[w4 * 64 + cb + q] = v[0];
+}
+
 // CW consecutive fp32 columns of this thread's TMEM lane (quadrant w % 4).
 __device__ __forceinline__ void ldcw(uint32_t tmem, int col, float *d) {
     tmem_ld16(tmq(tmem, col), d);
@@ -395,10 +404,11 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     float *vec = reinterpret_cast<float *>(sm + S_::kVec);
     float *G = vec, *bta = vec + 64, *gam = vec + 128, *e = vec + 192, *dB = vec + 256,
           *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576,
-          *dbl2 = vec + 640, *part = vec + 896;
+          *dbl2 = vec + 640;
+    float *wsum = reinterpret_cast<float *>(sm + S_::kRed);  // [3][4 warps][64 columns]
+    const int w4 = (tid >> 5) & 3;
     float *PE = reinterpret_cast<float *>(sm + S_::kPE);
     float *KKG = reinterpret_cast<float *>(sm + S_::kKKG);
-    float *RED = reinterpret_cast<float *>(sm + S_::kRed);
     float *Gam = reinterpret_cast<float *>(sm + S_::kGam);
 
     __shared__ uint64_t lbar;
@@ -493,15 +503,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
             mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, C, s), i64mk, s > 0);
         mma_commit(&mbar);
     }
-    ok = cta_wait(&mbar, phase, p, 21);
-    phase ^= 1;
-    if (!ok) goto done;
-    // the decay matrix, once (the dU^T image there is consumed)
-    for (int t = tid; t < C * C; t += NG) {
-        const int i = t >> 6, j = t & 63;
-        Gam[gidx(i, j)] = j <= i ? expf(G[i] - G[j]) : 0.f;
-    }
-    {  // <S, dSn> (elementwise over identically laid out images)
+    {  // <S, dSn> (elementwise over identically laid out images) while the products run
         float s = 0.f;
         for (int t = tid; t < D * D / 8; t += NG) {
             float a[8], b[8];
@@ -516,10 +518,18 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         if (tid == 0) {
             float a = 0.f;
             for (int w = 0; w < NG / 32; ++w) a += tmp[w];
-            s_hd = a;
+            s_hd = a;  // read after the barrier of the wait below
         }
-        __syncthreads();
     }
+    ok = cta_wait(&mbar, phase, p, 21);
+    phase ^= 1;
+    if (!ok) goto done;
+    // the decay matrix, once (the dU^T image there is consumed)
+    for (int t = tid; t < C * C; t += NG) {
+        const int i = t >> 6, j = t & 63;
+        Gam[gidx(i, j)] = j <= i ? expf(G[i] - G[j]) : 0.f;
+    }
+    __syncthreads();
     // P (scaled, lower incl. diagonal) and Gam . K K^T (strictly lower), fp32
     ldcw(tmem, cQK + cb, d);
     if (r < 64) {
@@ -543,20 +553,27 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
 #pragma unroll
         for (int q = 0; q < CW; ++q) {
             const int i = cb + q;
-            RED[r * LP + i] = vcol.at(cb, q) * d[q];
             stage[i * D + r] = __float2bfloat16_rn(bta[i] * d[q]);
+            d[q] *= vcol.at(cb, q);
         }
-        reduce_rows(RED, dB, part);
-        store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H);
+        warp_colsum(d, wsum, w4, cb, l);
     }
     ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
 #pragma unroll
-    for (int q = 0; q < CW; ++q) RED[r * LP + cb + q] = p.scale * qcol.at(cb, q) * d[q];
-    reduce_rows(RED, qx, part);
+    for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
+    warp_colsum(d, wsum + 256, w4, cb, l);
     ldcw(tmem, cX2 + cb, d);  // partial k . X2
 #pragma unroll
-    for (int q = 0; q < CW; ++q) RED[r * LP + cb + q] = kcol.at(cb, q) * d[q];
-    reduce_rows(RED, kx, part);
+    for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
+    warp_colsum(d, wsum + 512, w4, cb, l);
+    __syncthreads();
+    if (tid < 3 * C) {
+        const int k = tid >> 6, i = tid & 63;
+        const float *w = wsum + k * 256 + i;
+        (k == 0 ? dB : k == 1 ? qx : kx)[i] = (w[0] + w[64]) + (w[128] + w[192]);
+    }
+    __syncthreads();
+    store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H);
     ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
 #pragma unroll
     for (int q = 0; q < CW / 8; ++q)
@@ -590,8 +607,9 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     if (!ok) goto done;
     {  // dA = (dU V^T) diag(b) - (X3 K^T) diag(b gam)
         float y2[CW];
-        ldcw(tmem, cY1 + cb, d);
-        ldcw(tmem, cY2 + cb, y2);
+        tmem_ld16(tmq(tmem, cY1 + cb), d);
+        tmem_ld16(tmq(tmem, cY2 + cb), y2);
+        tmem_ld_wait();
         if (i64 >= 0) {
 #pragma unroll
             for (int q = 0; q < CW; ++q) {
@@ -605,8 +623,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     }
     ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
 #pragma unroll
-    for (int q = 0; q < CW; ++q) RED[r * LP + cb + q] = -kcol.at(cb, q) * d[q];
-    reduce_rows(RED, kz, part);
+    for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
+    warp_colsum(d, wsum, w4, cb, l);
+    __syncthreads();
+    if (tid < C) kz[tid] = (wsum[tid] + wsum[64 + tid]) + (wsum[128 + tid] + wsum[192 + tid]);
     operands_ready();
     if (tid == 0) {  // T1 = A^T dA (M = 64)
         const uint32_t id = idesc_bf16(64, 64, 1, 1);
@@ -671,32 +691,46 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         mma_commit(&mbar);
     }
     // meanwhile: dbeta and dG (rows), then dg = reverse cumulative sum of dG
-    if (tid < C) {
-        const int i = tid;
+    {  // row and column sums of PE: eight threads per token, eight entries each
+        const int i = tid >> 3, part = tid & 7;
         float rs = 0.f, cs = 0.f;
-        for (int j = 0; j < C; ++j) {
-            rs += PE[i * LP + j];
-            cs += PE[j * LP + i];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            rs += PE[i * LP + part * 8 + t];
+            cs += PE[(part * 8 + t) * LP + i];
         }
-        dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + rs - cs + bta[i] * gam[i] * kz[i];
-        dB[i] += (dbl2[i] + dbl2[64 + i]) + (dbl2[128 + i] + dbl2[192 + i]) + gam[i] * kz[i];
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float s = 0.f;
-        for (int j = 0; j < C; ++j) s += e[j] * kx[j];
-        dG[C - 1] += gam[C - 1] * s_hd + s;
-        float acc = 0.f;
-        for (int j = C - 1; j >= 0; --j) {
-            acc += dG[j];
-            dG[j] = acc;
+        float x = rs - cs;
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if (part == 0) {
+            dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + x + bta[i] * gam[i] * kz[i];
+            dB[i] += (dbl2[i] + dbl2[64 + i]) + (dbl2[128 + i] + dbl2[192 + i]) + gam[i] * kz[i];
         }
     }
     __syncthreads();
-    if (tid < ci.len) {
-        const int64_t o = (int64_t)(ci.tok0 + tid) * H + h;
-        p.dg[o] = dG[tid];
-        p.dbeta[o] = dB[tid];
+    if (tid < 32) {  // dg = reverse cumulative sum of dG (+ the terms of the last token)
+        const float a = dG[2 * l], b = dG[2 * l + 1];
+        float s = e[2 * l] * kx[2 * l] + e[2 * l + 1] * kx[2 * l + 1];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        const float extra = gam[C - 1] * s_hd + s;
+        float x = a + b;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float t = __shfl_down_sync(0xffffffffu, x, off);
+            if (l + off < 32) x += t;
+        }
+        const int i0 = 2 * l;
+        if (i0 < ci.len) {
+            const int64_t o = (int64_t)(ci.tok0 + i0) * H + h;
+            p.dg[o] = x + extra;
+            p.dbeta[o] = dB[i0];
+        }
+        if (i0 + 1 < ci.len) {
+            const int64_t o = (int64_t)(ci.tok0 + i0 + 1) * H + h;
+            p.dg[o] = (x - a) + extra;
+            p.dbeta[o] = dB[i0 + 1];
+        }
     }
     ok = cta_wait(&mbar, phase, p, 25);
     phase ^= 1;
@@ -705,15 +739,17 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         // staged as rows in the consumed dO and V tiles, then 16-byte stores
         bf16 *sq = reinterpret_cast<bf16 *>(DO), *sk = reinterpret_cast<bf16 *>(VT);
         float a[CW];
-        ldcw(tmem, cX1 + cb, d);
-        ldcw(tmem, cDQ + cb, a);
+        tmem_ld16(tmq(tmem, cX1 + cb), d);
+        tmem_ld16(tmq(tmem, cDQ + cb), a);
+        tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < CW; ++q) {
             const int i = cb + q;
             sq[i * D + r] = __float2bfloat16_rn(p.scale * (gam[i] * d[q] + a[q]));
         }
-        ldcw(tmem, cX2 + cb, d);
-        ldcw(tmem, cZ + cb, a);
+        tmem_ld16(tmq(tmem, cX2 + cb), d);
+        tmem_ld16(tmq(tmem, cZ + cb), a);
+        tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < CW; ++q) d[q] = e[cb + q] * d[q] - bta[cb + q] * gam[cb + q] * a[q];
         ldcw(tmem, cDKA + cb, a);
