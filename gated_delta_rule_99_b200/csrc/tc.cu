@@ -14,8 +14,8 @@
 //   U^T = Ut^T - S W^T        (M = 128 rows v, N = 64 tokens, K = 128)
 //   S  <- gam_n S + U^T Kd    (M = 128 rows v, N = 128 keys,  K = 64 tokens)
 //
-// Kernels: tc_prep (chunk-parallel: gates, K K^T, forward substitution for A
-// in fp32, W, Ut, Kd = diag(e) K), tc_state_fwd (serial over the chunks of a
+// Kernels: tc_prep (chunk-parallel: gates, K K^T, the blocked inverse A in
+// fp32, W, Ut, Kd = diag(e) K), tc_state_fwd (serial over the chunks of a
 // sequence; one CTA per (sequence, head); writes the state entering every
 // chunk and U^T as swizzled tile images), tc_out (chunk-parallel output).
 #include "tc_common.cuh"

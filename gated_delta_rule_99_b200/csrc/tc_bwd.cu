@@ -31,8 +31,8 @@ using namespace tc;
 
 // ============================================================ tc_local
 struct LocalSmem {
-    static constexpr int kQK = 0, kDO = kQK + 32768, kP = kDO + 16384,
-                         kG = kP + 8192, kEnd = kG + 256;
+    // P overwrites the Q half of the [Q; K] tile once Q K^T and Qg have consumed it
+    static constexpr int kQK = 0, kDO = kQK + 32768, kP = kQK, kG = kDO + 16384, kEnd = kG + 256;
 };
 constexpr int kLocalSmem = LocalSmem::kEnd + 1024;
 
@@ -128,7 +128,7 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
 
 // tc_prep (with A for the backward) on CTAs [0, NC*H) and tc_local on
 // [NC*H, 2*NC*H): independent chunk-parallel steps in one launch.
-__global__ void __launch_bounds__(NT) tc_prep_local_kernel(Params p) {
+__global__ void __launch_bounds__(NT, 4) tc_prep_local_kernel(Params p) {
     const int nch = p.NC * p.H;
     if ((int)blockIdx.x < nch) prep_body(p, blockIdx.x, 1);
     else local_body(p, blockIdx.x - nch);

@@ -8,15 +8,16 @@ namespace gdn {
 namespace tc {
 
 // ============================================================ tc_prep
-// Per (chunk, head): gates, A (fp32 forward substitution), and the tile
-// images W, Kd and the plain rows of Ut that the state pass consumes.
+// Per (chunk, head): gates, A = (I + L)^-1 (fp32, by 16 x 16 blocks), and the
+// tile images W, Kd and the plain rows of Ut that the state pass consumes.
 constexpr int LS = 68;  // row stride (floats) of L: 16-byte aligned rows for vector loads
 
 struct PrepSmem {
-    // L (fp32 64 x 68) is dead once A is formed; its bytes then hold the two
-    // bf16 operand tiles A diag(b gam) and A diag(b).
+    // L (fp32 64 x 68) becomes A in place; once A is read out, its bytes hold
+    // the two bf16 operand tiles A diag(b gam) and A diag(b).  F: per-column
+    // decay factors exp(G_e - G_j) to the end e of column j's 16-block.
     static constexpr int kK = 0, kV = kK + 16384, kL = kV + 16384, kAb = kL, kAc = kL + 8192,
-                         kG = kL + C * LS * 4, kB = kG + 256, kEnd = kB + 256;
+                         kG = kL + C * LS * 4, kB = kG + 256, kF = kB + 256, kEnd = kF + 256;
 };
 constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
 constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 columns each)
@@ -35,6 +36,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     float *L = reinterpret_cast<float *>(sm + PrepSmem::kL);
     float *G = reinterpret_cast<float *>(sm + PrepSmem::kG);
     float *bta = reinterpret_cast<float *>(sm + PrepSmem::kB);
+    float *F = reinterpret_cast<float *>(sm + PrepSmem::kF);
     const int tid = threadIdx.x;
 
     load_rows_async(Kt, C, 0, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
@@ -76,7 +78,10 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             for (int i = 0; i < 8; ++i) f[i] *= e;
             *reinterpret_cast<uint4 *>(dst + off) = pack8(f);
         }
-        if (tid < C) p.tG[(size_t)ch * C + tid] = G[tid];
+        if (tid < C) {
+            p.tG[(size_t)ch * C + tid] = G[tid];
+            F[tid] = expf(G[tid | 15] - G[tid]);
+        }
     }
     ok = cta_wait(&mbar, phase, p, 1);
     phase ^= 1;
@@ -88,53 +93,137 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             tmem_ld16(tm(tmem, c0), d);
             tmem_ld_wait();
             if (i >= 0) {
+                // Gam_ij = exp(G_i - G_e) exp(G_e - G_j), e = c0 + 15, for blocks left of the
+                // diagonal block (both factors <= 1); the diagonal block directly
+                if (c0 + 15 < i) {
+                    const float ri = bta[i] * expf(G[i] - G[c0 + 15]);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int j = c0 + q;
-                    L[i * LS + j] = j < i ? bta[i] * expf(G[i] - G[j]) * d[q] : 0.f;
+                    for (int q = 0; q < 16; ++q) L[i * LS + c0 + q] = ri * F[c0 + q] * d[q];
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int j = c0 + q;
+                        L[i * LS + j] = j < i ? bta[i] * expf(G[i] - G[j]) * d[q] : 0.f;
+                    }
                 }
             }
         }
         tc_fence_before();
         __syncthreads();
-        // forward substitution: thread j owns column j of A = (I + L)^-1 (fp32).
-        // L is zero on and above the diagonal and a[] starts at zero, so whole
-        // 4-blocks of a row can be read with one 16-byte load.
-        float a[C];
-        if (tid < C) {
-            const int j = tid;
+        // A = (I + L)^-1 in fp32 by 16 x 16 blocks, in place over L (stride LS):
+        // the diagonal blocks by forward substitution (one thread per column), then
+        // row block by row block  A_ij = -A_ii sum_{k=j}^{i-1} L_ik A_kj  (j < i),
+        // each row block's products formed in registers before any of its L blocks
+        // is overwritten.  Blocks above the diagonal stay zero.
+        {
+            float a[16];
+            const int b = tid >> 4, jj = tid & 15;
+            if (tid < C) {
+                const float *Lb = L + 16 * b * LS + 16 * b;
 #pragma unroll
-            for (int r = 0; r < C; ++r) a[r] = 0.f;
-            a[0] = j == 0 ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) {
+                    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int r = 1; r < C; ++r) {
-                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-                for (int m = 0; m < r; m += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4 *>(L + r * LS + m);
-                    s0 = fmaf(l4.x, a[m], s0);
-                    s1 = fmaf(l4.y, a[m + 1], s1);
-                    s2 = fmaf(l4.z, a[m + 2], s2);
-                    s3 = fmaf(l4.w, a[m + 3], s3);
+                    for (int m = 0; m < r; m += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(Lb + r * LS + m);
+                        s0 = fmaf(l4.x, a[m], s0);
+                        if (m + 1 < r) s1 = fmaf(l4.y, a[m + 1], s1);
+                        if (m + 2 < r) s0 = fmaf(l4.z, a[m + 2], s0);
+                        if (m + 3 < r) s1 = fmaf(l4.w, a[m + 3], s1);
+                    }
+                    a[r] = r < jj ? 0.f : (r == jj ? 1.f : -(s0 + s1));
                 }
-                const float s = (s0 + s1) + (s2 + s3);
-                a[r] = r < j ? 0.f : (r == j ? 1.f : -s);
             }
+            __syncthreads();
+            if (tid < C) {
+                float *Lb = L + 16 * b * LS + 16 * b;
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Lb[r * LS + jj] = a[r];
+            }
+            __syncthreads();
         }
-        __syncthreads();  // L is dead from here: the operand tiles overwrite it
-        if (tid < C) {
-            const int j = tid;
-            const float bg = bta[j] * expf(G[j]), b = bta[j];
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
-                *reinterpret_cast<bf16 *>(Ab + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * bg);
-                *reinterpret_cast<bf16 *>(Ac + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r] * b);
+        for (int ib = 1; ib < 4; ++ib) {
+            // elements e = tid + 128 n of the ib blocks (j, r, c) left of the diagonal
+            float t[6];
+#pragma unroll
+            for (int n = 0; n < 2 * ib; ++n) {
+                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                const float *Lr = L + (16 * ib + r) * LS;
+                float s0 = 0.f, s1 = 0.f;
+                for (int k = j; k < ib; ++k) {
+                    const float *Ak = L + (16 * k) * LS + 16 * j + c;
+#pragma unroll
+                    for (int m = 0; m < 16; m += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(Lr + 16 * k + m);
+                        s0 = fmaf(l4.x, Ak[m * LS], s0);
+                        s1 = fmaf(l4.y, Ak[(m + 1) * LS], s1);
+                        s0 = fmaf(l4.z, Ak[(m + 2) * LS], s0);
+                        s1 = fmaf(l4.w, Ak[(m + 3) * LS], s1);
+                    }
+                }
+                t[n] = s0 + s1;
             }
-            if (want_A) {  // A as a bf16 tile image (rows m, columns i) for the backward
-                uint8_t *Ag = reinterpret_cast<uint8_t *>(p.tA) + (size_t)ch * C * C * 2;
+            __syncthreads();  // every product of this row block has read its L blocks
 #pragma unroll
-                for (int r = 0; r < C; ++r)
-                    *reinterpret_cast<bf16 *>(Ag + sw128_off(C, r, j)) = __float2bfloat16_rn(a[r]);
+            for (int n = 0; n < 2 * ib; ++n) {
+                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                L[(16 * ib + r) * LS + 16 * j + c] = t[n];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int n = 0; n < 2 * ib; ++n) {
+                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                const float *Ai = L + (16 * ib + r) * LS + 16 * ib;       // row r of A_ii
+                const float *Tc = L + (16 * ib) * LS + 16 * j + c;        // column c of T_ij
+                float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; m += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(Ai + m);
+                    s0 = fmaf(a4.x, Tc[m * LS], s0);
+                    s1 = fmaf(a4.y, Tc[(m + 1) * LS], s1);
+                    s0 = fmaf(a4.z, Tc[(m + 2) * LS], s0);
+                    s1 = fmaf(a4.w, Tc[(m + 3) * LS], s1);
+                }
+                t[n] = -(s0 + s1);
+            }
+            __syncthreads();
+#pragma unroll
+            for (int n = 0; n < 2 * ib; ++n) {
+                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                L[(16 * ib + r) * LS + 16 * j + c] = t[n];
+            }
+            __syncthreads();
+        }
+        // the bf16 operand tiles A diag(b gam), A diag(b) (and A itself for the backward):
+        // every thread reads its four 8-column pieces of A before the tiles overwrite L
+        {
+            float av[4][8];
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int e = tid + NT * n, r = e >> 3, cc = e & 7;
+                const float4 x0 = *reinterpret_cast<const float4 *>(L + r * LS + 8 * cc);
+                const float4 x1 = *reinterpret_cast<const float4 *>(L + r * LS + 8 * cc + 4);
+                av[n][0] = x0.x; av[n][1] = x0.y; av[n][2] = x0.z; av[n][3] = x0.w;
+                av[n][4] = x1.x; av[n][5] = x1.y; av[n][6] = x1.z; av[n][7] = x1.w;
+            }
+            __syncthreads();  // L is dead from here: the operand tiles overwrite it
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int e = tid + NT * n, r = e >> 3, cc = e & 7;
+                float fb[8], fc[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int c = 8 * cc + q;
+                    fc[q] = av[n][q] * bta[c];
+                    fb[q] = fc[q] * expf(G[c]);
+                }
+                *reinterpret_cast<uint4 *>(Ab + sw128_chunk(C, r, cc)) = pack8(fb);
+                *reinterpret_cast<uint4 *>(Ac + sw128_chunk(C, r, cc)) = pack8(fc);
+                if (want_A) {
+                    uint8_t *Ag = reinterpret_cast<uint8_t *>(p.tA) + (size_t)ch * C * C * 2;
+                    *reinterpret_cast<uint4 *>(Ag + sw128_chunk(C, r, cc)) = pack8(av[n]);
+                }
             }
         }
         operands_ready();
