@@ -144,17 +144,25 @@ struct SbwdSmem {
 };
 constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
 
+// Chunk ch's Kd, W and Qg images, local dU^T image and gate row by bulk copies
+// (thread 0, completing on `bar`); its dO rows by cp.async (one commit group).
 __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
-                                              const ChunkInfo &ci, int h, const Params &p) {
+                                              const ChunkInfo &ci, int h, const Params &p,
+                                              uint64_t *bar) {
     uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
-    load_image_async(b + SbwdSmem::kKd, static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
-    load_image_async(b + SbwdSmem::kW, static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
-    load_image_async(b + SbwdSmem::kQg, static_cast<const uint8_t *>(p.tQg) + ch * kImg64, kImg64);
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, 3u * (uint32_t)kImg64 + (uint32_t)kImgUT + C * 4u);
+        bulk_load(smem_u32(b + SbwdSmem::kKd), static_cast<const uint8_t *>(p.tKd) + ch * kImg64,
+                  kImg64, bar);
+        bulk_load(smem_u32(b + SbwdSmem::kW), static_cast<const uint8_t *>(p.tW) + ch * kImg64,
+                  kImg64, bar);
+        bulk_load(smem_u32(b + SbwdSmem::kQg), static_cast<const uint8_t *>(p.tQg) + ch * kImg64,
+                  kImg64, bar);
+        bulk_load(smem_u32(b + SbwdSmem::kDUL),
+                  static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT, kImgUT, bar);
+        bulk_load(smem_u32(b + SbwdSmem::kG), p.tG + ch * C, C * 4, bar);
+    }
     load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H);
-    load_image_async(b + SbwdSmem::kDUL, static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT,
-                     kImgUT);
-    if (threadIdx.x < 16)
-        cp_async16(smem_u32(b + SbwdSmem::kG) + threadIdx.x * 16, p.tG + ch * C + threadIdx.x * 4);
     cp_async_commit();
 }
 
@@ -162,7 +170,7 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
 __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
+    __shared__ uint64_t mbar, lbar[2];
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, n = blk / H, h = blk % H, v = threadIdx.x;
@@ -177,6 +185,8 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     }
     if (v == 0) {
         mbar_init(&mbar, 1);
+        mbar_init(&lbar[0], 1);
+        mbar_init(&lbar[1], 1);
         fence_mbar_init();
     }
     if (v < 32) {
@@ -189,7 +199,12 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     const uint32_t tmem = tslot;
     const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
     uint32_t phase = 0;
-    if (c0 < c1) sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, p.chunks[c1 - 1], h, p);
+    // per buffer b (bit b): bulk copies in flight, and the parity of their next completion
+    uint32_t pend = 0, lpar = 0;
+    if (c0 < c1) {
+        sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, p.chunks[c1 - 1], h, p, &lbar[0]);
+        pend = 1;
+    }
     uint8_t *dSs = sm + SbwdSmem::kdS, *dUs = sm + SbwdSmem::kdU;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), idx = idesc_bf16(128, 128, 1, 1),
                    idy = idesc_bf16(128, 128, 0, 1);
@@ -197,17 +212,27 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         const int buf = (c1 - 1 - c) & 1;
         const size_t ch = (size_t)c * H + h;
         if (c - 1 >= c0) {
-            sbwd_prefetch(sm, buf ^ 1, ch - H, p.chunks[c - 1], h, p);
+            sbwd_prefetch(sm, buf ^ 1, ch - H, p.chunks[c - 1], h, p, &lbar[buf ^ 1]);
+            pend |= 2u >> buf;
             cp_async_wait<1>();
         } else {
             cp_async_wait<0>();
         }
+        const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, kWaitLimit);
         uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        operands_ready();
-        // after the barrier: the gate row was copied by other threads' cp.async
+        fence_async_smem();
+        tc_fence_before();
+        const bool all = __syncthreads_and(lok);
+        tc_fence_after();
+        if (!all) {
+            if (v == 0) record_timeout(p, 45);
+            break;
+        }
+        pend &= ~(1u << buf);
+        lpar ^= 1u << buf;
         const float gC = expf(reinterpret_cast<const float *>(b + SbwdSmem::kG)[C - 1]);
         if (v == 0) {
             const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
@@ -271,7 +296,11 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         __syncthreads();
         tc_fence_after();
     }
-    if (v == 0) bulk_wait_all();
+    if (v == 0) {  // copies still in flight after an early exit
+        for (int q = 0; q < 2; ++q)
+            if ((pend >> q) & 1u) mbar_wait(&lbar[q], (lpar >> q) & 1u, kWaitLimit);
+        bulk_wait_all();
+    }
     if (p.dh0) {
         float *g0 = p.dh0 + ((size_t)n * H + h) * D * D;
 #pragma unroll

@@ -16,19 +16,21 @@ struct StateSmem {
 };
 constexpr int kStateSmem = StateSmem::kEnd + 1024;
 
+// Bulk copies (thread 0) of chunk ch's W and Kd images, its Ut rows (unless
+// the run takes Ut as zero) and its gate row into buffer `buf`, completing
+// on `bar`.
 __device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p,
-                                               bool with_ut) {
-    load_image_async(sm + StateSmem::kW0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64);
-    load_image_async(sm + StateSmem::kKd0 + buf * 16384,
-                     static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64);
+                                               bool with_ut, uint64_t *bar) {
+    if (threadIdx.x != 0) return;
+    mbar_arrive_expect_tx(bar, (with_ut ? 3u : 2u) * (uint32_t)kImg64 + C * 4u);
+    bulk_load(smem_u32(sm + StateSmem::kW0 + buf * 16384),
+              static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64, bar);
+    bulk_load(smem_u32(sm + StateSmem::kKd0 + buf * 16384),
+              static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64, bar);
     if (with_ut)
-        load_image_async(sm + StateSmem::kUt0 + buf * 16384,
-                         static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64);
-    if (threadIdx.x < 16)
-        cp_async16(smem_u32(sm + StateSmem::kG0 + buf * 256) + threadIdx.x * 16,
-                   p.tG + ch * C + threadIdx.x * 4);
-    cp_async_commit();
+        bulk_load(smem_u32(sm + StateSmem::kUt0 + buf * 16384),
+                  static_cast<const uint8_t *>(p.tUt) + ch * kImg64, kImg64, bar);
+    bulk_load(smem_u32(sm + StateSmem::kG0 + buf * 256), p.tG + ch * C, C * 4, bar);
 }
 
 // One run of the forward chain over chunks [c0, c1) of one head.
@@ -46,7 +48,7 @@ struct ChainFwd {
 __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
+    __shared__ uint64_t mbar, lbar[2];
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, h = a.h, v = threadIdx.x;
@@ -60,6 +62,8 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     }
     if (v == 0) {
         mbar_init(&mbar, 1);
+        mbar_init(&lbar[0], 1);
+        mbar_init(&lbar[1], 1);
         fence_mbar_init();
     }
     if (v < 32) {
@@ -73,24 +77,36 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     const int c0 = a.c0, c1 = a.c1;
     const bool with_ut = !a.zero_ut;
     uint32_t phase = 0;
-    if (c0 < c1) state_prefetch(sm, 0, (size_t)c0 * H + h, p, with_ut);
+    // per buffer b (bit b): a copy in flight, and the parity of its next completion
+    uint32_t pend = 0, lpar = 0;
+    if (c0 < c1) {
+        state_prefetch(sm, 0, (size_t)c0 * H + h, p, with_ut, &lbar[0]);
+        pend = 1;
+    }
     uint8_t *Ss = sm + StateSmem::kS, *UTs = sm + StateSmem::kUT;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), id2 = idesc_bf16(128, 128, 0, 1);
     for (int c = c0; c < c1; ++c) {
         const int buf = (c - c0) & 1;
         const size_t ch = (size_t)c * H + h;
         if (c + 1 < c1) {
-            state_prefetch(sm, buf ^ 1, ch + H, p, with_ut);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+            state_prefetch(sm, buf ^ 1, ch + H, p, with_ut, &lbar[buf ^ 1]);
+            pend |= 2u >> buf;
         }
+        const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, kWaitLimit);
         // the state entering this chunk, as bf16 operand rows
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        operands_ready();
-        // after the barrier: the gate row was copied by other threads' cp.async
+        fence_async_smem();
+        tc_fence_before();
+        const bool all = __syncthreads_and(lok);
+        tc_fence_after();
+        if (!all) {
+            if (v == 0) record_timeout(p, 40 + a.where);
+            break;
+        }
+        pend &= ~(1u << buf);
+        lpar ^= 1u << buf;
         const float gC =
             expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
         if (v == 0) {
@@ -150,12 +166,15 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         __syncthreads();
         tc_fence_after();
     }
-    if (v == 0 && a.snapshots) bulk_wait_all();
+    if (v == 0) {  // copies still in flight after an early exit
+        for (int b = 0; b < 2; ++b)
+            if ((pend >> b) & 1u) mbar_wait(&lbar[b], (lpar >> b) & 1u, kWaitLimit);
+        if (a.snapshots) bulk_wait_all();
+    }
     if (a.final_out) {
 #pragma unroll
         for (int kk = 0; kk < D; ++kk) a.final_out[kk * D + v] = S[kk];
     }
-    cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
     if (v < 32) tmem_dealloc(tmem, 256);
