@@ -97,12 +97,32 @@ def _ptr(a):
     return None if a is None else a.ctypes.data
 
 
-def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, units=None, nthreads=None):
+def _l2norm_rows(x):
+    """Rows of x divided by their Euclidean norm (a zero row stays zero), and the norms.
+
+    The optional normalisation of q and k per token and head that the layer
+    applies itself when asked (jax-linear-attention 0.1.0, "Quick start":
+    ``use_qk_l2norm=True``); the pages give no formula, so this is the plain
+    x / sqrt(sum x^2)."""
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return np.where(n > 0, x / np.where(n > 0, n, 1.0), 0.0), n
+
+
+def _l2norm_back(xh, n, dxh):
+    """Gradient w.r.t. the raw rows from the gradient w.r.t. the normalised rows
+    xh = x / |x|:  dx = (dxh - xh (xh . dxh)) / |x|  (zero for a zero row)."""
+    proj = dxh - xh * np.sum(xh * dxh, axis=-1, keepdims=True)
+    return np.where(n > 0, proj / np.where(n > 0, n, 1.0), 0.0)
+
+
+def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, units=None, nthreads=None,
+            qk_l2norm=False):
     """Token-by-token forward.  q,k: (B,T,H,K); v: (B,T,H,V); g, beta: (B,T,H);
     h0: (N,H,K,V) or None.  Returns o (B,T,H,V) and hT (N,H,K,V) in fp64.
 
     ``units``: optional iterable of (sequence, head) pairs to compute; the
-    other entries of o and hT are left NaN (used for sampled parity)."""
+    other entries of o and hT are left NaN (used for sampled parity).
+    ``qk_l2norm``: normalise every q and k row first (see ``_l2norm_rows``)."""
     B, T, H, K = _shape(q)
     V = _shape(v)[-1]
     segs = _segments(B, T, cu_seqlens)
@@ -114,7 +134,10 @@ def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, units=None, n
     for i, (n, h) in enumerate(sel):
         b, t0, t1 = segs[n]
         L = t1 - t0
-        bufs = dict(q=_f64(q[b, t0:t1, h]), k=_f64(k[b, t0:t1, h]), v=_f64(v[b, t0:t1, h]),
+        qu, ku = _f64(q[b, t0:t1, h]), _f64(k[b, t0:t1, h])
+        if qk_l2norm:
+            qu, ku = np.ascontiguousarray(_l2norm_rows(qu)[0]), np.ascontiguousarray(_l2norm_rows(ku)[0])
+        bufs = dict(q=qu, k=ku, v=_f64(v[b, t0:t1, h]),
                     g=_f64(g[b, t0:t1, h]), beta=_f64(beta[b, t0:t1, h]),
                     h0=None if h0 is None else _f64(h0[n, h]),
                     o=np.zeros((max(L, 1), V)), hT=np.zeros((K, V)))
@@ -132,9 +155,11 @@ def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, units=None, n
 
 
 def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0, units=None,
-            nthreads=None):
+            nthreads=None, qk_l2norm=False):
     """Token-by-token backward of o and hT with upstream gradients do (B,T,H,V)
-    and dhT (N,H,K,V) or None.  Returns dq, dk, dv, dg, dbeta, dh0 in fp64."""
+    and dhT (N,H,K,V) or None.  Returns dq, dk, dv, dg, dbeta, dh0 in fp64.
+    With ``qk_l2norm`` dq and dk are the gradients w.r.t. the raw (unnormalised)
+    q and k."""
     B, T, H, K = _shape(q)
     V = _shape(v)[-1]
     segs = _segments(B, T, cu_seqlens)
@@ -148,12 +173,18 @@ def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0,
         b, t0, t1 = segs[n]
         L = max(t1 - t0, 1)
         c = _f64
-        bufs = dict(q=c(q[b, t0:t1, h]), k=c(k[b, t0:t1, h]), v=c(v[b, t0:t1, h]),
+        qu, ku = c(q[b, t0:t1, h]), c(k[b, t0:t1, h])
+        if qk_l2norm:
+            (qu, qn), (ku, kn) = _l2norm_rows(qu), _l2norm_rows(ku)
+            qu, ku = np.ascontiguousarray(qu), np.ascontiguousarray(ku)
+        bufs = dict(q=qu, k=ku, v=c(v[b, t0:t1, h]),
                     g=c(g[b, t0:t1, h]), beta=c(beta[b, t0:t1, h]),
                     h0=None if h0 is None else c(h0[n, h]),
                     do_=c(do[b, t0:t1, h]), dhT=None if dhT is None else c(dhT[n, h]),
                     dq=np.zeros((L, K)), dk=np.zeros((L, K)), dv=np.zeros((L, V)),
                     dg=np.zeros(L), dbeta=np.zeros(L), dh0=np.zeros((K, V)))
+        if qk_l2norm:
+            bufs["norms"] = (qn, kn)
         keep.append(bufs)
         arr[i] = _Unit(t1 - t0, _ptr(bufs["q"]), _ptr(bufs["k"]), _ptr(bufs["v"]), _ptr(bufs["g"]),
                        _ptr(bufs["beta"]), _ptr(bufs["h0"]), None, None, _ptr(bufs["do_"]),
@@ -165,6 +196,10 @@ def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0,
     for (n, h), bufs in zip(sel, keep):
         b, t0, t1 = segs[n]
         L = t1 - t0
+        if qk_l2norm and L > 0:
+            qn, kn = bufs["norms"]
+            bufs["dq"][:L] = _l2norm_back(bufs["q"], qn, bufs["dq"][:L])
+            bufs["dk"][:L] = _l2norm_back(bufs["k"], kn, bufs["dk"][:L])
         for name in ("dq", "dk", "dv"):
             out[name][b, t0:t1, h] = bufs[name][:L]
         out["dg"][b, t0:t1, h] = bufs["dg"][:L]

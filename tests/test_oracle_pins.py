@@ -260,3 +260,87 @@ def test_sampled_units_match_full_run():
     np.testing.assert_array_equal(os_[1, :, 2], o[1, :, 2])
     np.testing.assert_array_equal(hs[0, 0], hT[0, 0])
     assert np.isnan(os_[0, :, 1]).all()
+
+
+# ---- optional q/k L2 normalisation inside the layer (jax-linear-attention 0.1.0,
+# "Quick start": use_qk_l2norm=True; the pages give no formula: x / |x| per token
+# and head is the reading taken)
+def _l2(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def test_l2norm_is_identity_on_unit_rows():
+    rng = np.random.default_rng(21)
+    B, T, H, K, V = 1, 30, 2, 5, 4
+    q, k = _l2(rng.standard_normal((B, T, H, K))), _l2(rng.standard_normal((B, T, H, K)))
+    v = rng.standard_normal((B, T, H, V)); g = -rng.random((B, T, H)) * 0.3
+    beta = rng.random((B, T, H)); h0 = rng.standard_normal((B, H, K, V))
+    o0, h0T = oracle.gdn_fwd(q, k, v, g, beta, h0=h0)
+    o1, h1T = oracle.gdn_fwd(q, k, v, g, beta, h0=h0, qk_l2norm=True)
+    np.testing.assert_allclose(o1, o0, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(h1T, h0T, rtol=1e-12, atol=1e-13)
+
+
+def test_l2norm_scale_invariance_and_zero_rows():
+    rng = np.random.default_rng(22)
+    B, T, H, K, V = 1, 25, 1, 6, 3
+    q, k = rng.standard_normal((B, T, H, K)), rng.standard_normal((B, T, H, K))
+    v = rng.standard_normal((B, T, H, V)); g = -rng.random((B, T, H)) * 0.3
+    beta = rng.random((B, T, H)); do = rng.standard_normal((B, T, H, V))
+    c = np.exp(rng.standard_normal((B, T, H, 1)))  # positive per-row factors
+    o, _ = oracle.gdn_fwd(q, k, v, g, beta, qk_l2norm=True)
+    oc, _ = oracle.gdn_fwd(q * c, k * c[::-1], v, g, beta, qk_l2norm=True)
+    np.testing.assert_allclose(oc, o, rtol=1e-11, atol=1e-12)
+    dq, dk, *_ = oracle.gdn_bwd(q, k, v, g, beta, do, qk_l2norm=True)
+    dqc, dkc, *_ = oracle.gdn_bwd(q * c, k * c[::-1], v, g, beta, do, qk_l2norm=True)
+    np.testing.assert_allclose(dqc * c, dq, rtol=1e-10, atol=1e-12)   # d/d(cx) = (1/c) d/dx
+    np.testing.assert_allclose(dkc * c[::-1], dk, rtol=1e-10, atol=1e-12)
+    # a zero query row reads nothing; a zero key row writes nothing
+    q0, k0 = q.copy(), k.copy()
+    q0[0, 7] = 0.0
+    k0[0, 3] = 0.0
+    oz, _ = oracle.gdn_fwd(q0, k0, v, g, beta, qk_l2norm=True)
+    assert np.all(oz[0, 7] == 0.0)
+    dqz, dkz, *_ = oracle.gdn_bwd(q0, k0, v, g, beta, do, qk_l2norm=True)
+    assert np.all(dqz[0, 7] == 0.0) and np.all(dkz[0, 3] == 0.0)
+    # a zero key row acts as a zero write strength (only the decay remains)
+    b0 = beta.copy()
+    b0[0, 3] = 0.0
+    ref, _ = oracle.gdn_fwd(q0, k, v, g, b0, qk_l2norm=True)
+    np.testing.assert_allclose(oz, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_l2norm_backward_finite_differences():
+    rng = np.random.default_rng(23)
+    lens = [11, 8]
+    T, H, K, V = sum(lens), 1, 4, 3
+    cu = np.cumsum([0] + lens)
+    x = dict(q=rng.standard_normal((1, T, H, K)), k=rng.standard_normal((1, T, H, K)),
+             v=rng.standard_normal((1, T, H, V)), g=-rng.random((1, T, H)) * 0.5,
+             beta=rng.random((1, T, H)), h0=rng.standard_normal((2, H, K, V)) * 0.5)
+    do = rng.standard_normal((1, T, H, V)); dhT = rng.standard_normal((2, H, K, V)) * 0.5
+
+    def loss(y):
+        o, hT = oracle.gdn_fwd(y["q"], y["k"], y["v"], y["g"], y["beta"], cu_seqlens=cu,
+                               h0=y["h0"], scale=0.7, qk_l2norm=True)
+        return float(np.sum(o * do) + np.sum(hT * dhT))
+
+    dq, dk, dv, dg, db, dh0 = oracle.gdn_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], do,
+                                             cu_seqlens=cu, h0=x["h0"], dhT=dhT, scale=0.7,
+                                             qk_l2norm=True)
+    eps = 1e-6
+    for name, gr in dict(q=dq, k=dk, v=dv, g=dg, beta=db, h0=dh0).items():
+        fd = np.zeros_like(gr)
+        it = np.nditer(x[name], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = {kk: vv.copy() for kk, vv in x.items()}
+            xm = {kk: vv.copy() for kk, vv in x.items()}
+            xp[name][idx] += eps
+            xm[name][idx] -= eps
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * eps)
+        err = np.max(np.abs(fd - gr)) / np.max(np.abs(gr))
+        assert err < 1e-7, (name, err)
+    # rows of dq and dk are orthogonal to their q and k rows (scale invariance)
+    np.testing.assert_allclose(np.sum(dq * x["q"], axis=-1), 0.0, atol=1e-12)
+    np.testing.assert_allclose(np.sum(dk * x["k"], axis=-1), 0.0, atol=1e-12)
