@@ -37,6 +37,7 @@ class GdnDesc(ctypes.Structure):
                 ("reserved", ctypes.c_int32)]
 
 GDN_FLAG_PIECE_SCAN = 1
+GDN_FLAG_QK_L2NORM = 2
 
 
 _lock = threading.Lock()
@@ -139,14 +140,16 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, output_final_state=True,
-            o=None, hT=None, workspace=None, cu_seqlens_host=None, stream=None, piece_scan=False):
+            o=None, hT=None, workspace=None, cu_seqlens_host=None, stream=None, piece_scan=False,
+            qk_l2norm=False):
     """Forward of the gated delta rule through the C ABI.  Returns (o, hT);
     hT is None when output_final_state is False.  piece_scan sets
-    GDN_FLAG_PIECE_SCAN (parallel pieces of long dense rows, joined exactly)."""
+    GDN_FLAG_PIECE_SCAN (parallel pieces of long dense rows, joined exactly);
+    qk_l2norm sets GDN_FLAG_QK_L2NORM (q and k rows divided by their norms)."""
     L = lib()
     cu_dev, cu_host = _seqlens(cu_seqlens, cu_seqlens_host, q.device)
-    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale,
-                                              GDN_FLAG_PIECE_SCAN if piece_scan else 0)
+    flags = (GDN_FLAG_PIECE_SCAN if piece_scan else 0) | (GDN_FLAG_QK_L2NORM if qk_l2norm else 0)
+    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale, flags)
     N = n_seqs if n_seqs else B
     _check(q, "q", q.dtype, (B, T, H, K)); _check(k, "k", q.dtype, (B, T, H, K))
     _check(v, "v", q.dtype, (B, T, H, V))
@@ -172,11 +175,13 @@ def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, output_final_
 
 
 def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0, grads=None,
-            workspace=None, cu_seqlens_host=None, stream=None, want_dh0=True):
-    """Backward through the C ABI.  Returns (dq, dk, dv, dg, dbeta, dh0)."""
+            workspace=None, cu_seqlens_host=None, stream=None, want_dh0=True, qk_l2norm=False):
+    """Backward through the C ABI.  Returns (dq, dk, dv, dg, dbeta, dh0); with
+    qk_l2norm, dq and dk are the gradients w.r.t. the raw (unnormalised) q and k."""
     L = lib()
     cu_dev, cu_host = _seqlens(cu_seqlens, cu_seqlens_host, q.device)
-    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale)
+    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale,
+                                              GDN_FLAG_QK_L2NORM if qk_l2norm else 0)
     N = n_seqs if n_seqs else B
     _check(q, "q", q.dtype, (B, T, H, K)); _check(k, "k", q.dtype, (B, T, H, K))
     _check(v, "v", q.dtype, (B, T, H, V)); _check(do, "do", q.dtype, (B, T, H, V))
@@ -202,12 +207,13 @@ def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0,
     return dq, dk, dv, dg, dbeta, dh0
 
 
-def gdn_decode(q, k, v, g, beta, state, scale=1.0, o=None, stream=None):
+def gdn_decode(q, k, v, g, beta, state, scale=1.0, o=None, stream=None, qk_l2norm=False):
     """Recurrent decode through the C ABI: advances ``state`` ([B][H][dk][dv]
     fp32, updated in place) through the T tokens of q, k, v ([B][T][H][D]) and
     returns o."""
     L = lib()
-    desc, (B, T, H, K, V, _) = _desc_from(q, v, None, scale)
+    desc, (B, T, H, K, V, _) = _desc_from(q, v, None, scale,
+                                         GDN_FLAG_QK_L2NORM if qk_l2norm else 0)
     _check(q, "q", q.dtype, (B, T, H, K)); _check(k, "k", q.dtype, (B, T, H, K))
     _check(v, "v", q.dtype, (B, T, H, V))
     _check(g, "g", torch.float32, (B, T, H)); _check(beta, "beta", torch.float32, (B, T, H))

@@ -7,7 +7,10 @@
 //   S <- a_t (S - b_t (S k_t) k_t^T) + b_t v_t k_t^T,   a_t = exp(g_t)
 //   o_t = scale S q_t
 //
-// with S = state^T kept in fp32.  One CTA per (sequence, head); thread v owns
+// with S = state^T kept in fp32 (with GDN_FLAG_QK_L2NORM, q_t and k_t are first
+// divided by their norms, as the pages' API option use_qk_l2norm does; the
+// factors 1/|q_t| and 1/|k_t| are applied where q_t and k_t enter).  One CTA per
+// (sequence, head); thread v owns
 // row v of S in registers (d_k values), so the state is read once and written
 // once per call and every step is thread-local arithmetic.  HBM bound: the
 // state (2 d_k d_v 4 bytes per sequence and head) dominates the traffic.
@@ -33,7 +36,7 @@ template <typename T, int K>
 __global__ void __launch_bounds__(128) decode_kernel(const T *q, const T *k, const T *v,
                                                      const float *g, const float *beta,
                                                      float *state, T *o, int Tn, int H, int V,
-                                                     float scale) {
+                                                     float scale, int l2n) {
     __shared__ float qs[K], ks[K];
     const int bh = blockIdx.x, b = bh / H, h = bh % H, vi = threadIdx.x;
     const bool active = vi < V;
@@ -51,21 +54,33 @@ __global__ void __launch_bounds__(128) decode_kernel(const T *q, const T *k, con
         __syncthreads();
         const float a = expf(g[row]), bt = beta[row];
         const float vv = active ? ldf(v, row * V + vi) : 0.f;
+        float iq = 1.f, ik = 1.f;  // 1/|q_t|, 1/|k_t| (zero rows stay zero)
+        if (l2n) {
+            float nq = 0.f, nk = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < K; ++kk) {
+                nq = fmaf(qs[kk], qs[kk], nq);
+                nk = fmaf(ks[kk], ks[kk], nk);
+            }
+            iq = nq > 0.f ? 1.f / sqrtf(nq) : 0.f;
+            ik = nk > 0.f ? 1.f / sqrtf(nk) : 0.f;
+        }
         float sk0 = 0.f, sk1 = 0.f;
 #pragma unroll
         for (int kk = 0; kk < K; kk += 2) {
             sk0 = fmaf(S[kk], ks[kk], sk0);
             sk1 = fmaf(S[kk + 1], ks[kk + 1], sk1);
         }
-        const float sk = sk0 + sk1;
+        const float sk = ik * (sk0 + sk1);
+        const float c1 = bt * sk * ik, c2 = bt * vv * ik;
         float o0 = 0.f, o1 = 0.f;
 #pragma unroll
         for (int kk = 0; kk < K; ++kk) {
-            S[kk] = a * (S[kk] - bt * sk * ks[kk]) + bt * vv * ks[kk];
+            S[kk] = a * (S[kk] - c1 * ks[kk]) + c2 * ks[kk];
             if (kk & 1) o1 = fmaf(S[kk], qs[kk], o1);
             else o0 = fmaf(S[kk], qs[kk], o0);
         }
-        if (active) stf(o, row * V + vi, scale * (o0 + o1));
+        if (active) stf(o, row * V + vi, scale * iq * (o0 + o1));
     }
     if (active) {
 #pragma unroll
@@ -78,16 +93,17 @@ cudaError_t launch_typed(const gdn_desc *d, const void *q, const void *k, const 
                          const float *g, const float *beta, float *state, void *o,
                          cudaStream_t s) {
     const int nbh = (int)(d->B * d->H), Tn = (int)d->T, H = (int)d->H, V = (int)d->dv;
+    const int l2n = (d->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     if (d->dk == 128) {
         GDN_LAUNCH(kKDecode, s,
                    decode_kernel<T, 128><<<nbh, 128, 0, s>>>(
                        (const T *)q, (const T *)k, (const T *)v, g, beta, state, (T *)o, Tn, H,
-                       V, d->scale));
+                       V, d->scale, l2n));
     } else {
         GDN_LAUNCH(kKDecode, s,
                    decode_kernel<T, 64><<<nbh, 128, 0, s>>>(
                        (const T *)q, (const T *)k, (const T *)v, g, beta, state, (T *)o, Tn, H,
-                       V, d->scale));
+                       V, d->scale, l2n));
     }
     return cudaSuccess;
 }
@@ -108,6 +124,8 @@ extern "C" gdn_status gdn_decode(const gdn_desc *d, const void *q, const void *k
     if (d->B * d->H >= (int64_t(1) << 31) || d->B * d->T >= (int64_t(1) << 31))
         return GDN_ERR_INVALID_ARG;
     if (!(d->scale == d->scale)) return GDN_ERR_INVALID_ARG;
+    if (d->reserved != 0 || (d->flags & ~(GDN_FLAG_PIECE_SCAN | GDN_FLAG_QK_L2NORM)))
+        return GDN_ERR_INVALID_ARG;
     if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, g, beta, state, o};
     for (const void *p : ptrs)

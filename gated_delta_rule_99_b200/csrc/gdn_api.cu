@@ -35,7 +35,9 @@ gdn_status describe(const gdn_desc *d, Problem *p) {
     p->NC = 0;
     p->dtype = d->dtype;
     p->scale = d->scale;
-    if (d->reserved != 0 || (d->flags & ~GDN_FLAG_PIECE_SCAN)) return GDN_ERR_INVALID_ARG;
+    if (d->reserved != 0 || (d->flags & ~(GDN_FLAG_PIECE_SCAN | GDN_FLAG_QK_L2NORM)))
+        return GDN_ERR_INVALID_ARG;
+    p->l2norm = (d->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     p->P = 1;
     p->L = 0;
     if ((d->flags & GDN_FLAG_PIECE_SCAN) && d->n_seqs == 0 && d->dtype == GDN_BF16 &&
@@ -105,6 +107,7 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.BT = pb.BT;
     p.scale = d->scale;
     p.bf16 = d->dtype == GDN_BF16;
+    p.l2norm = pb.l2norm;
     p.cu = d->n_seqs > 0 ? cu_dev : nullptr;
     char *base = static_cast<char *>(ws);
     p.hdr = reinterpret_cast<WsHeader *>(base);
@@ -138,6 +141,22 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.tMp = f(L.tMp);
     p.tBp = f(L.tBp);
     return p;
+}
+
+// Normalisation pass of the fp32 path: q and k rows divided by their norms into
+// the workspace copies, which the kernels then read in place of q and k.
+bool normalise_qk(const Problem &pb, const Layout &L, void *ws, Params *p, cudaStream_t s) {
+    if (pb.BT == 0) return true;
+    char *base = static_cast<char *>(ws);
+    const int64_t rows = pb.BT * pb.H;
+    if (launch_l2norm_rows(p->q, base + L.qn, reinterpret_cast<float *>(base + L.qinv), rows,
+                           (int)pb.K, p->bf16, s) != cudaSuccess ||
+        launch_l2norm_rows(p->k, base + L.kn, reinterpret_cast<float *>(base + L.kinv), rows,
+                           (int)pb.K, p->bf16, s) != cudaSuccess)
+        return false;
+    p->q = base + L.qn;
+    p->k = base + L.kn;
+    return true;
 }
 
 bool use_tc(const Problem &pb, bool bwd) {
@@ -198,6 +217,13 @@ Layout make_layout(const Problem &pb, bool bwd) {
         // one scratch slot per CTA of the chunk-parallel kernels (grid = min(NC*H, kSimtSlots))
         const size_t slots = nch < (size_t)kSimtSlots ? (nch > 0 ? nch : 1) : (size_t)kSimtSlots;
         L.scratch = take(slots * kSimtScratchFloats * f);
+        if (pb.l2norm) {  // normalised copies of q and k, and their inverse norms
+            const size_t rows = (size_t)pb.BT * pb.H, es = pb.dtype == GDN_BF16 ? 2 : 4;
+            L.qn = take(rows * pb.K * es);
+            L.kn = take(rows * pb.K * es);
+            L.qinv = take(rows * f);
+            L.kinv = take(rows * f);
+        }
     }
     L.total = off;
     return L;
@@ -252,8 +278,10 @@ gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.h0 = h0;
     p.o = o;
     p.hT = hT;
+    const bool tc = use_tc(pb, false);
     if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
-    cudaError_t e = use_tc(pb, false) ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
+    if (!tc && pb.l2norm && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;
+    cudaError_t e = tc ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -293,8 +321,20 @@ gdn_status gdn_bwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.dg = dg;
     p.dbeta = dbeta;
     p.dh0 = dh0;
+    const bool tc = use_tc(pb, true);
     if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
-    cudaError_t e = use_tc(pb, true) ? launch_tc_bwd(p, pb, s) : launch_simt_bwd(p, s);
+    const bool pre = !tc && pb.l2norm;
+    if (pre && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;
+    cudaError_t e = tc ? launch_tc_bwd(p, pb, s) : launch_simt_bwd(p, s);
+    if (e == cudaSuccess && pre && pb.BT > 0) {  // gradients w.r.t. the raw q and k
+        char *base = static_cast<char *>(workspace);
+        const int64_t rows = pb.BT * pb.H;
+        e = launch_l2norm_back(base + L.qn, reinterpret_cast<float *>(base + L.qinv), dq, rows,
+                               (int)pb.K, p.bf16, s);
+        if (e == cudaSuccess)
+            e = launch_l2norm_back(base + L.kn, reinterpret_cast<float *>(base + L.kinv), dk,
+                                   rows, (int)pb.K, p.bf16, s);
+    }
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

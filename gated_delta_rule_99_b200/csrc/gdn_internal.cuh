@@ -38,6 +38,7 @@ struct Params {
     int64_t BT;                    // tokens over all rows
     float scale;
     int32_t bf16;                  // 1: q/k/v/o/do/dq/dk/dv are bf16, 0: fp32
+    int32_t l2norm;                // 1: q and k rows are divided by their norms first
     // inputs
     const void *q, *k, *v, *do_;
     const float *g, *beta, *h0, *dhT;
@@ -76,6 +77,7 @@ struct Problem {
     int dtype;
     float scale;
     int64_t P, L;   // pieces per sequence (1 = no piece scan) and chunks per piece
+    int l2norm;     // GDN_FLAG_QK_L2NORM
 };
 
 // Workspace layout: offsets in bytes from the workspace base.
@@ -83,6 +85,7 @@ struct Layout {
     size_t chunks, seq_first;
     size_t W, Ut, A, U, Hs, dUloc, dU, dHn, scratch;
     size_t tW, tUt, tKd, tS, tUT, tQg, tdUL, tdSn, tdUT, tG, tA, tHin, tMp, tBp;
+    size_t qn, kn, qinv, kinv;  // normalised q, k copies and 1/|row| (passes of the fp32 path)
     size_t total;
 };
 
@@ -93,6 +96,12 @@ cudaError_t launch_build_chunks(const Params &p, cudaStream_t stream);
 cudaError_t launch_simt_fwd(const Params &p, cudaStream_t stream);
 cudaError_t launch_simt_bwd(const Params &p, cudaStream_t stream);
 bool tc_supported(const Problem &p);
+// Normalisation pass: xn = x / |x| per row of K values (dtype of x), inv = 1/|x|.
+cudaError_t launch_l2norm_rows(const void *x, void *xn, float *inv, int64_t rows, int K,
+                               bool bf16, cudaStream_t stream);
+// Projection pass, in place: dx <- (dx - xn (xn . dx)) * inv per row.
+cudaError_t launch_l2norm_back(const void *xn, const float *inv, void *dx, int64_t rows, int K,
+                               bool bf16, cudaStream_t stream);
 bool tc_bwd_ready();
 cudaError_t launch_tc_fwd(const Params &p, const Problem &pb, cudaStream_t stream);
 cudaError_t launch_tc_bwd(const Params &p, const Problem &pb, cudaStream_t stream);
@@ -116,6 +125,8 @@ enum KernelId : int32_t {
     kKTcPieceA,
     kKTcPieceScan,
     kKTcPieceC,
+    kKL2Norm,
+    kKL2NormBack,
     kKernelCount
 };
 

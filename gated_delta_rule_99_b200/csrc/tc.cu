@@ -216,6 +216,11 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
     }
     cp_async_wait<0>();
     operands_ready();
+    if (p.l2norm) {  // q and k rows divided by their norms
+        l2norm_tile_rows(QK, D, 0, nullptr);
+        l2norm_tile_rows(QK, D, C, nullptr);
+        operands_ready();
+    }
     const uint32_t tmem = tslot;
     if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
         const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);

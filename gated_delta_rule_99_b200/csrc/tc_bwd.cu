@@ -64,6 +64,11 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
     chunk_gates(G, nullptr, p, ci, h);
     cp_async_wait<0>();
     operands_ready();
+    if (p.l2norm) {  // q and k rows divided by their norms
+        l2norm_tile_rows(QK, D, 0, nullptr);
+        l2norm_tile_rows(QK, D, C, nullptr);
+        operands_ready();
+    }
     const uint32_t tmem = tslot;
     if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
         const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
@@ -408,6 +413,29 @@ __device__ __forceinline__ void warp_colsum(float *v, float *wsum, int w4, int c
     if (!(l & 1)) wsum[w4 * 64 + cb + q] = v[0];
 }
 
+// Backward of the optional row normalisation for this thread's column of 16
+// tokens i = cb + q (x holds the gradient w.r.t. the normalised rows u):
+// x <- (x - u (u . x)) / |row|, the dot products over the 128 columns summed by
+// warp butterflies and four warp partials.  Called by every thread of the CTA.
+__device__ __forceinline__ void project_rows(float *x, const ColSw &u, const float *inv,
+                                             float *dot, float *wsum, int w4, int cb, int l) {
+    float y[CW];
+#pragma unroll
+    for (int q = 0; q < CW; ++q) y[q] = u.at(cb, q) * x[q];
+    warp_colsum(y, wsum, w4, cb, l);
+    __syncthreads();
+    if (threadIdx.x < C) {
+        const int t = threadIdx.x;
+        dot[t] = (wsum[t] + wsum[64 + t]) + (wsum[128 + t] + wsum[192 + t]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < CW; ++q) {
+        const int i = cb + q;
+        x[q] = (x[q] - u.at(cb, q) * dot[i]) * inv[i];
+    }
+}
+
 // CW consecutive fp32 columns of this thread's TMEM lane (quadrant w % 4).
 __device__ __forceinline__ void ldcw(uint32_t tmem, int col, float *d) {
     tmem_ld16(tmq(tmem, col), d);
@@ -433,7 +461,8 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     float *vec = reinterpret_cast<float *>(sm + S_::kVec);
     float *G = vec, *bta = vec + 64, *gam = vec + 128, *e = vec + 192, *dB = vec + 256,
           *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576,
-          *dbl2 = vec + 640;
+          *dbl2 = vec + 640, *qinv = vec + 896, *kinv = vec + 960, *qdot = vec + 1024,
+          *kdot = vec + 1088;
     float *wsum = reinterpret_cast<float *>(sm + S_::kRed);  // [3][4 warps][64 columns]
     const int w4 = (tid >> 5) & 3;
     float *PE = reinterpret_cast<float *>(sm + S_::kPE);
@@ -493,6 +522,11 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         }
     }
     operands_ready();
+    if (p.l2norm) {  // q rows (threads 0-127) and k rows (128-255) divided by their norms
+        l2norm_tile_rows(QK, D, 0, qinv, 0);
+        l2norm_tile_rows(QK, D, C, kinv, 2 * C);
+        operands_ready();
+    }
     const uint32_t tmem = tslot;
     const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128, dob = smem_u32(DO), vb = smem_u32(VT),
                    scb = smem_u32(SC), dsb = smem_u32(DSN), utb = smem_u32(UT),
@@ -772,10 +806,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         tmem_ld16(tmq(tmem, cDQ + cb), a);
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < CW; ++q) {
-            const int i = cb + q;
-            sq[i * D + r] = __float2bfloat16_rn(p.scale * (gam[i] * d[q] + a[q]));
-        }
+        for (int q = 0; q < CW; ++q) d[q] = p.scale * (gam[cb + q] * d[q] + a[q]);
+        if (p.l2norm) project_rows(d, qcol, qinv, qdot, wsum, w4, cb, l);
+#pragma unroll
+        for (int q = 0; q < CW; ++q) sq[(cb + q) * D + r] = __float2bfloat16_rn(d[q]);
         tmem_ld16(tmq(tmem, cX2 + cb), d);
         tmem_ld16(tmq(tmem, cZ + cb), a);
         tmem_ld_wait();
@@ -786,7 +820,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         for (int q = 0; q < CW; ++q) d[q] += p.scale * a[q];
         ldcw(tmem, cDK + cb, a);
 #pragma unroll
-        for (int q = 0; q < CW; ++q) sk[(cb + q) * D + r] = __float2bfloat16_rn(d[q] + a[q]);
+        for (int q = 0; q < CW; ++q) d[q] += a[q];
+        if (p.l2norm) project_rows(d, kcol, kinv, kdot, wsum + 256, w4, cb, l);
+#pragma unroll
+        for (int q = 0; q < CW; ++q) sk[(cb + q) * D + r] = __float2bfloat16_rn(d[q]);
         __syncthreads();
         store_rows(static_cast<bf16 *>(p.dq), DO, ci.tok0, ci.len, h, H);
         store_rows(static_cast<bf16 *>(p.dk), VT, ci.tok0, ci.len, h, H);

@@ -135,5 +135,39 @@ inline cudaError_t set_smem(Kern k, int bytes) {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// The layer's optional q/k normalisation inside a kernel (jax-linear-attention
+// 0.1.0, "Quick start": use_qk_l2norm=True): rows [row0, row0 + 64) of a bf16
+// SW128 tile with R rows and 128 columns are divided by their Euclidean norms
+// (fp32 sums of squares in a fixed order; a zero row stays zero) and rounded
+// back to bf16 in place; 1/|row| goes to inv[] when it is given.  Threads
+// [tbase, tbase + 128) take two per row.  Every kernel that loads a q or k tile
+// runs this same code, so all see bit-identical normalised rows.
+__device__ __forceinline__ void l2norm_tile_rows(uint8_t *tile, int R, int row0, float *inv,
+                                                 int tbase = 0) {
+    const int t = (int)threadIdx.x - tbase;
+    if (t < 0 || t >= 2 * C) return;
+    const int r = t >> 1, half = t & 1;
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4 *>(tile + sw128_chunk(R, row0 + r, 8 * half + j)), f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) s = fmaf(f[q], f[q], s);
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    const float rn = s > 0.f ? 1.f / sqrtf(s) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint4 *ch = reinterpret_cast<uint4 *>(tile + sw128_chunk(R, row0 + r, 8 * half + j));
+        float f[8];
+        unpack8(*ch, f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] *= rn;
+        *ch = pack8(f);
+    }
+    if (inv && half == 0) inv[r] = rn;
+}
+
 }  // namespace tc
 }  // namespace gdn

@@ -53,6 +53,10 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     chunk_gates(G, bta, p, ci, h);
     cp_async_wait<0>();
     operands_ready();
+    if (p.l2norm) {  // k rows divided by their norms
+        l2norm_tile_rows(Kt, C, 0, nullptr);
+        operands_ready();
+    }
     const uint32_t tmem = tslot;
     uint32_t phase = 0;
     bool ok = true;

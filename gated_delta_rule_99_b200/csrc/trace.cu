@@ -8,7 +8,7 @@ thread_local bool g_open = false;
 
 const char *const kNames[kKernelCount] = {
     "build_chunks", "simt_prep", "simt_state_fwd", "simt_out", "simt_duloc", "simt_state_bwd",
-    "simt_grads", "tc_prep", "tc_state_fwd", "tc_out", "tc_chains", "tc_grads", "tc_prep_local", "decode", "tc_piece_a", "tc_piece_scan", "tc_piece_c"};
+    "simt_grads", "tc_prep", "tc_state_fwd", "tc_out", "tc_chains", "tc_grads", "tc_prep_local", "decode", "tc_piece_a", "tc_piece_scan", "tc_piece_c", "l2norm", "l2norm_back"};
 }  // namespace
 
 void trace_before(int32_t id, cudaStream_t stream) {

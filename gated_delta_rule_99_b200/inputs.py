@@ -83,11 +83,14 @@ def _l2norm(x: torch.Tensor) -> torch.Tensor:
 def make_inputs(B: int, T: int, H: int, K: int, V: int, dtype: str = "bf16", seed: int = 0,
                 gate_scale: float = 0.1, h0_std: float = 0.02, lengths=None, packed=None,
                 bwd: bool = True, dhT_std: float = 0.01, scale: float = 1.0,
-                device: str = "cpu", **_ignored) -> Inputs:
+                device: str = "cpu", raw_qk: bool = False, **_ignored) -> Inputs:
     """Draw one workload.  ``lengths`` (explicit document lengths) or ``packed``
     ((lo, hi) for random lengths) make a packed row; this needs B == 1.
     ``device`` picks where the generator runs (the draws differ between CPU
-    and CUDA generators, so the oracle must be fed the same tensors)."""
+    and CUDA generators, so the oracle must be fed the same tensors).
+    ``raw_qk`` leaves q and k unnormalised, each row scaled by its own factor
+    exp(N(0, 1)) (inputs for the layer's own normalisation option); the other
+    tensors are the same draws as without it."""
     tdt = {"bf16": torch.bfloat16, "fp32": torch.float32}[dtype]
     if packed is not None and lengths is None:
         lengths = doc_lengths(T, packed[0], packed[1], seed)
@@ -98,8 +101,10 @@ def make_inputs(B: int, T: int, H: int, K: int, V: int, dtype: str = "bf16", see
     N = B if cu is None else cu.numel() - 1
     gen = torch.Generator(device=device).manual_seed(seed)
     f32 = dict(generator=gen, device=device, dtype=torch.float32)
-    q = _l2norm(torch.randn(B, T, H, K, **f32)).to(tdt)
-    k = _l2norm(torch.randn(B, T, H, K, **f32)).to(tdt)
+    q = torch.randn(B, T, H, K, **f32)
+    k = torch.randn(B, T, H, K, **f32)
+    if not raw_qk:
+        q, k = _l2norm(q).to(tdt), _l2norm(k).to(tdt)
     v = torch.randn(B, T, H, V, **f32).to(tdt)
     g = -torch.nn.functional.softplus(torch.randn(B, T, H, **f32)) * gate_scale
     beta = torch.sigmoid(torch.randn(B, T, H, **f32))
@@ -108,6 +113,9 @@ def make_inputs(B: int, T: int, H: int, K: int, V: int, dtype: str = "bf16", see
     if bwd:
         do = torch.randn(B, T, H, V, **f32).to(tdt)
         dhT = torch.randn(N, H, K, V, **f32) * dhT_std if dhT_std > 0 else None
+    if raw_qk:
+        q = (q * torch.exp(torch.randn(B, T, H, 1, **f32))).to(tdt)
+        k = (k * torch.exp(torch.randn(B, T, H, 1, **f32))).to(tdt)
     return Inputs(q, k, v, g, beta, h0, cu, do, dhT, scale,
                   dict(B=B, T=T, H=H, K=K, V=V, dtype=dtype, seed=seed))
 

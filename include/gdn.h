@@ -99,6 +99,19 @@ typedef struct gdn_desc {
  * bf16, d_k = d_v = 128 forward on dense rows; ignored elsewhere. */
 #define GDN_FLAG_PIECE_SCAN 1
 
+/* Option for gdn_fwd, gdn_fwd_noalloc, gdn_bwd and gdn_decode: the layer first
+ * divides every q and k row (one token and head, d_k values) by its Euclidean
+ * norm, in fp32, rounding the result to the input dtype (a zero row stays
+ * zero); gdn_bwd then returns dq and dk with respect to the raw q and k,
+ * dq = (dq^ - q^ (q^ . dq^)) / |q| with q^ the normalised row and dq^ the
+ * gradient with respect to it.  The pages' API names the option
+ * (jax-linear-attention 0.1.0, "Quick start": use_qk_l2norm=True) without a
+ * formula; x / |x| is the reading taken.  On the bf16 d_k = d_v = 128 path the
+ * kernels that load q and k normalise their tiles themselves; elsewhere a
+ * normalisation pass runs first (and, in gdn_bwd, a projection pass last), with
+ * the normalised copies in the workspace. */
+#define GDN_FLAG_QK_L2NORM 2
+
 /* Library version (major * 10000 + minor * 100 + patch). */
 int gdn_version(void);
 

@@ -52,6 +52,31 @@ def test_workspace_size_rejects_bad_descriptors(bad, code):
     assert rc == code
 
 
+def test_flags_match_header_and_unknown_bits_are_rejected():
+    import re
+    hdr = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    defs = dict(re.findall(r"#define (GDN_FLAG_\w+) (\d+)", hdr))
+    assert int(defs["GDN_FLAG_PIECE_SCAN"]) == gdn.GDN_FLAG_PIECE_SCAN
+    assert int(defs["GDN_FLAG_QK_L2NORM"]) == gdn.GDN_FLAG_QK_L2NORM
+    ok = gdn.make_desc(2, 100, 3, 64, 128, flags=gdn.GDN_FLAG_QK_L2NORM | gdn.GDN_FLAG_PIECE_SCAN)
+    assert gdn.fwd_workspace_size(ok) > 0
+    bad = gdn.make_desc(2, 100, 3, 64, 128, flags=4)
+    assert gdn.fwd_workspace_size(bad) == 0 and _fwd(bad, ws_bytes=1 << 40) == 1
+
+
+def test_l2norm_workspace_holds_normalised_copies_only_off_the_tensor_core_path():
+    for dt, K, V, grows in ((1, 64, 128, True), (0, 64, 64, True), (0, 128, 128, False)):
+        plain = gdn.make_desc(2, 300, 3, K, V, dtype=dt)
+        l2 = gdn.make_desc(2, 300, 3, K, V, dtype=dt, flags=gdn.GDN_FLAG_QK_L2NORM)
+        for size in (gdn.fwd_workspace_size, gdn.bwd_workspace_size):
+            a, b = size(plain), size(l2)
+            if grows:  # two copies of (B*T*H, K) rows in the input dtype plus two norm vectors
+                es = 4 if dt == 1 else 2
+                assert b - a >= 2 * 2 * 300 * 3 * K * es + 2 * 4 * 2 * 300 * 3
+            else:
+                assert a == b
+
+
 def test_workspace_sizes_grow():
     a = gdn.fwd_workspace_size(gdn.make_desc(1, 64, 1, 64, 64))
     b = gdn.fwd_workspace_size(gdn.make_desc(1, 128, 1, 64, 64))
