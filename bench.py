@@ -551,25 +551,33 @@ def run_report(args, rank, world, local_rank):
     import torch
 
     import gated_delta_rule_99_b200 as gdn
-    from gated_delta_rule_99_b200.inputs import WORKLOADS, workload
+    from gated_delta_rule_99_b200.inputs import WORKLOADS, make_inputs, workload
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     pk = peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    runs = [(i, False) for i in sorted(WORKLOADS)] + [(4, True)]  # long row: also piece scan
-    for idx, piece in runs:
-        w = WORKLOADS[idx]
-        inp = workload(idx, device="cuda" if idx == 4 else "cpu")
+    # every workload; the long row also with the piece scan; the benchmark workload also with
+    # the layer's own q/k normalisation (raw q, k); head dim 64 dense and packed (tensor cores)
+    d64 = dict(WORKLOADS[2], K=64, V=64, name="gdn_fwdbwd_bf16_B4_T4096_H16_d64")
+    p64 = dict(WORKLOADS[3], K=64, V=64, name=WORKLOADS[3]["name"].replace("d128", "d64"))
+    runs = ([(i, dict(WORKLOADS[i]), False, False) for i in sorted(WORKLOADS)] +
+            [(4, dict(WORKLOADS[4]), True, False), (2, dict(WORKLOADS[2]), False, True),
+             (None, d64, False, False), (None, p64, False, False)])
+    for idx, w, piece, l2 in runs:
+        if idx is not None and not l2:
+            inp = workload(idx, device="cuda" if idx == 4 else "cpu")
+        else:
+            inp = make_inputs(**dict(w, raw_qk=l2))
         d = inp.to(dev)
         cu = inp.cu_seqlens
         cu_dev = None if cu is None else cu.to(dev)
         bwd = w["bwd"]
         B, T, H, K, V = w["B"], w["T"], w["H"], w["K"], w["V"]
         n = inp.n_seqs
+        flags = (gdn.GDN_FLAG_PIECE_SCAN if piece else 0) | (gdn.GDN_FLAG_QK_L2NORM if l2 else 0)
         desc = gdn.make_desc(B, T, H, K, V, 0 if cu is None else n,
-                             gdn.GDN_BF16 if w["dtype"] == "bf16" else gdn.GDN_FP32,
-                             flags=gdn.GDN_FLAG_PIECE_SCAN if piece else 0)
+                             gdn.GDN_BF16 if w["dtype"] == "bf16" else gdn.GDN_FP32, flags=flags)
         ws = gdn.alloc_workspace(max(gdn.fwd_workspace_size(desc),
                                      gdn.bwd_workspace_size(desc) if bwd else 0), dev)
         o = torch.empty_like(d.v)
@@ -582,14 +590,15 @@ def run_report(args, rank, world, local_rank):
 
         def step():
             gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=cu_dev, cu_seqlens_host=cu,
-                        h0=d.h0, o=o, hT=hT, workspace=ws, piece_scan=piece)
+                        h0=d.h0, o=o, hT=hT, workspace=ws, piece_scan=piece, qk_l2norm=l2)
             if bwd:
                 gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, cu_seqlens=cu_dev,
-                            cu_seqlens_host=cu, h0=d.h0, dhT=d.dhT, grads=grads, workspace=ws)
+                            cu_seqlens_host=cu, h0=d.h0, dhT=d.dhT, grads=grads, workspace=ws,
+                            qk_l2norm=l2)
 
         for _ in range(3):
             step()
-        steps = 3 if idx == 4 else max(5, args.steps)
+        steps = 3 if T > 100000 else max(5, args.steps)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(steps)]
         torch.cuda.synchronize()
@@ -611,11 +620,11 @@ def run_report(args, rank, world, local_rank):
         t_bound = max(flops / (pk["tc_sus"] * 1e12), bytes_ / (pk["hbm"] * 1e9))
         if rank == 0:
             print(json.dumps({
-                "workload": w["name"] + ("+piece_scan" if piece else ""),
+                "workload": w["name"] + ("+piece_scan" if piece else "") + ("+qk_l2norm" if l2 else ""),
                 "pass": "fwd+bwd" if bwd else "fwd",
                 "tokens_per_s": B * T / (ms / 1e3), "ms_per_call": ms,
                 "roofline_frac": t_bound * 1e3 / ms, "roofline_us": t_bound * 1e6,
-                "path": "tensor-core" if (w["dtype"] == "bf16" and K == V == 128) else "fp32",
+                "path": "tensor-core" if w["dtype"] == "bf16" else "fp32",
                 "peaks": pk["src"]}), flush=True)
         del d, ws, o, hT, grads
         torch.cuda.empty_cache()

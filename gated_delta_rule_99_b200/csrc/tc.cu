@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(NT, 1) tc_piece_a_kernel(Params p) {
     ChainFwd a;
     a.h = h;
     a.where = 31;
+    a.init_user = 1;  // h0 (piece 0); the middle pieces start from zero or the identity
+    a.out_user = 0;   // tHin, tBp, tMp are internal [128][128] blocks
     int piece;
     if (r == 0) {
         piece = 0;
@@ -171,6 +173,8 @@ __global__ void __launch_bounds__(NT, 1) tc_piece_c_kernel(Params p) {
     ChainFwd a;
     a.h = h;
     a.where = 35;
+    a.init_user = 0;  // tHin
+    a.out_user = 1;   // hT
     a.init = p.tHin + ((size_t)unit * p.P + piece) * DD;
     a.init_identity = 0;
     a.zero_ut = 0;
@@ -192,7 +196,7 @@ constexpr int kOutSmem = OutSmem::kEnd + 1024;
 __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
+    __shared__ uint64_t mbar, lbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
@@ -200,29 +204,39 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
     uint8_t *QK = sm + OutSmem::kQK, *Ss = sm + OutSmem::kS, *UTs = sm + OutSmem::kUT;
     uint8_t *QG = sm + OutSmem::kQG, *Ps = sm + OutSmem::kP;
     float *G = reinterpret_cast<float *>(sm + OutSmem::kG);
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
-    load_image_async(Ss, static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128, kImg128);
-    load_image_async(UTs, static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT);
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, p.K);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K);
     cp_async_commit();
-    if (tid < C) G[tid] = p.tG[(size_t)ch * C + tid];
-    if (tid == 0) {
+    if (tid == 0) {  // the state and U^T images by bulk copies
         mbar_init(&mbar, 1);
+        mbar_init(&lbar, 1);
         fence_mbar_init();
+        mbar_arrive_expect_tx(&lbar, (uint32_t)(kImg128 + kImgUT));
+        bulk_load(smem_u32(Ss), static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128,
+                  (uint32_t)kImg128, &lbar);
+        bulk_load(smem_u32(UTs), static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT,
+                  (uint32_t)kImgUT, &lbar);
     }
+    if (tid < C) G[tid] = p.tG[(size_t)ch * C + tid];
     if (tid < 32) {
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
+    __syncthreads();  // thread 0's mbarrier inits are visible before any thread waits on them
     cp_async_wait<0>();
+    bool ok = __syncthreads_and(mbar_wait(&lbar, 0, kWaitLimit));
+    if (!ok && tid == 0) {
+        record_timeout(p, 7);
+        mbar_wait(&lbar, 0, kWaitLimit);  // no copy left in flight
+    }
     operands_ready();
-    if (p.l2norm) {  // q and k rows divided by their norms
+    if (ok && p.l2norm) {  // q and k rows divided by their norms
         l2norm_tile_rows(QK, D, 0, nullptr);
         l2norm_tile_rows(QK, D, C, nullptr);
         operands_ready();
     }
     const uint32_t tmem = tslot;
-    if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
+    if (ok && tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
         const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
@@ -230,7 +244,7 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
         mma_commit(&mbar);
     }
     // scale * gam_i * q_i as a K-major operand (rows i)
-    for (int t = tid; t < C * 16; t += NT) {
+    for (int t = tid; ok && t < C * 16; t += NT) {
         const int r = t >> 4, j = t & 15;
         float f[8];
         unpack8(*reinterpret_cast<const uint4 *>(QK + sw128_chunk(D, r, j)), f);
@@ -239,7 +253,7 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
         for (int q = 0; q < 8; ++q) f[q] *= s;
         *reinterpret_cast<uint4 *>(QG + sw128_chunk(C, r, j)) = pack8(f);
     }
-    bool ok = cta_wait(&mbar, 0, p, 5);
+    if (ok) ok = cta_wait(&mbar, 0, p, 5);
     if (ok) {
         const int i = m64_row();
         for (int c0 = 0; c0 < C; c0 += 16) {
@@ -284,8 +298,8 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
         bf16 *o = static_cast<bf16 *>(p.o);
         for (int t = tid; t < C * 16; t += NT) {
             const int i = t >> 4, j = t & 15;
-            if (i < ci.len)
-                *reinterpret_cast<uint4 *>(o + ((int64_t)(ci.tok0 + i) * H + h) * D + j * 8) =
+            if (i < ci.len && j * 8 < p.V)
+                *reinterpret_cast<uint4 *>(o + ((int64_t)(ci.tok0 + i) * H + h) * p.V + j * 8) =
                     *reinterpret_cast<const uint4 *>(QK + i * 256 + j * 16);
         }
     }
@@ -297,7 +311,10 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
 
 }  // namespace
 
-bool tc_supported(const Problem &pb) { return pb.K == 128 && pb.V == 128; }
+// Head dims 64 run on the 128-wide tiles zero-padded in shared memory.
+bool tc_supported(const Problem &pb) {
+    return (pb.K == 64 || pb.K == 128) && (pb.V == 64 || pb.V == 128);
+}
 
 bool tc_bwd_ready() { return true; }
 

@@ -49,9 +49,9 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
     const ChunkInfo ci = p.chunks[c];
     uint8_t *QK = sm + LocalSmem::kQK, *DO = sm + LocalSmem::kDO, *Ps = sm + LocalSmem::kP;
     float *G = reinterpret_cast<float *>(sm + LocalSmem::kG);
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
-    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H);
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, p.K);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K);
+    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H, p.V);
     cp_async_commit();
     if (tid == 0) {
         mbar_init(&mbar, 1);
@@ -167,7 +167,7 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
                   static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT, kImgUT, bar);
         bulk_load(smem_u32(b + SbwdSmem::kG), p.tG + ch * C, C * 4, bar);
     }
-    load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H);
+    load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H, p.V);
     cp_async_commit();
 }
 
@@ -180,10 +180,10 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     if (p.hdr->status) return;
     const int H = p.H, n = blk / H, h = blk % H, v = threadIdx.x;
     float S[D];  // dS row v (gradient of the state leaving the current chunk)
-    if (p.dhT) {
-        const float *g0 = p.dhT + ((size_t)n * H + h) * D * D;
+    if (p.dhT) {  // [K][V] blocks; rows and columns past them are zero
+        const float *g0 = p.dhT + ((size_t)n * H + h) * p.K * p.V;
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = g0[kk * D + v];
+        for (int kk = 0; kk < D; ++kk) S[kk] = (kk < p.K && v < p.V) ? g0[kk * p.V + v] : 0.f;
     } else {
 #pragma unroll
         for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
@@ -256,9 +256,8 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         }
         if (!cta_wait(&mbar, phase, p, 13)) break;
         phase ^= 1;
-        {  // dU^T = dS Kd^T + local dU^T ; -dU^T is the next operand, +dU^T an image for tc_grads
+        {  // dU^T = dS Kd^T + local dU^T: the next operand, and (bulk-stored) an image for tc_grads
             const uint8_t *dul = b + SbwdSmem::kDUL;  // local dU^T, swizzled rows
-            uint8_t *img = static_cast<uint8_t *>(p.tdUT) + ch * kImgUT;
 #pragma unroll
             for (int c16 = 0; c16 < C; c16 += 16) {
                 float d[16], l[16];
@@ -269,21 +268,19 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
                         l + 8);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) d[q] += l[q];
-                *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, c16 / 8)) = pack8(d);
-                *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) d[q] = -d[q];
                 *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8)) = pack8(d);
                 *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
             }
         }
         operands_ready();
-        if (v == 0) {  // - dU^T W: M = 128 (v), N = 128 keys, K = 64 tokens
+        if (v == 0) {  // + dU^T (-W): M = 128 (v), N = 128 keys, K = 64 tokens (W image negated)
             const uint32_t ub = smem_u32(dUs), wb = smem_u32(b + SbwdSmem::kW);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(wb, C, s), idy, 1);
             mma_commit(&mbar);
+            bulk_store(static_cast<uint8_t *>(p.tdUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
+            bulk_commit();
         }
         if (!cta_wait(&mbar, phase, p, 14)) break;
         phase ^= 1;
@@ -307,9 +304,12 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         bulk_wait_all();
     }
     if (p.dh0) {
-        float *g0 = p.dh0 + ((size_t)n * H + h) * D * D;
+        float *g0 = p.dh0 + ((size_t)n * H + h) * p.K * p.V;
+        if (v < p.V) {
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) g0[kk * D + v] = S[kk];
+            for (int kk = 0; kk < D; ++kk)
+                if (kk < p.K) g0[kk * p.V + v] = S[kk];
+        }
     }
     cp_async_wait<0>();
     tc_fence_before();
@@ -366,14 +366,15 @@ struct ColSw {
     }
 };
 
-// Copies rows [0, len) of a 64 x 128 bf16 staging tile (plain rows) to one
-// chunk and head of a [tokens][H][128] tensor with 16-byte stores.
+// Copies rows [0, len) and columns [0, width) of a 64 x 128 bf16 staging tile
+// (plain rows) to one chunk and head of a [tokens][H][width] tensor with
+// 16-byte stores.
 __device__ __forceinline__ void store_rows(bf16 *dst, const uint8_t *stage, int64_t tok0, int len,
-                                           int h, int H) {
+                                           int h, int H, int width) {
     for (int t = threadIdx.x; t < C * 16; t += NG) {
         const int i = t >> 4, j = t & 15;
-        if (i < len)
-            *reinterpret_cast<uint4 *>(dst + ((tok0 + i) * H + h) * D + j * 8) =
+        if (i < len && j * 8 < width)
+            *reinterpret_cast<uint4 *>(dst + ((tok0 + i) * H + h) * width + j * 8) =
                 *reinterpret_cast<const uint4 *>(stage + i * 256 + j * 16);
     }
 }
@@ -487,10 +488,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
                   &lbar);
     }
     // q, k, v, do rows by cp.async into the swizzled layout
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, NG);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, NG);
-    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H, NG);
-    load_rows_async(VT, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H, NG);
+    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, p.K, NG);
+    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K, NG);
+    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H, p.V, NG);
+    load_rows_async(VT, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H, p.V, NG);
     cp_async_commit();
     if (tid < C) {
         const int64_t idx = (int64_t)(ci.tok0 + tid) * H + h;
@@ -636,7 +637,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         (k == 0 ? dB : k == 1 ? qx : kx)[i] = (w[0] + w[64]) + (w[128] + w[192]);
     }
     __syncthreads();
-    store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H);
+    store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H, p.V);
     ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
 #pragma unroll
     for (int q = 0; q < CW / 8; ++q)
@@ -825,8 +826,8 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
 #pragma unroll
         for (int q = 0; q < CW; ++q) sk[(cb + q) * D + r] = __float2bfloat16_rn(d[q]);
         __syncthreads();
-        store_rows(static_cast<bf16 *>(p.dq), DO, ci.tok0, ci.len, h, H);
-        store_rows(static_cast<bf16 *>(p.dk), VT, ci.tok0, ci.len, h, H);
+        store_rows(static_cast<bf16 *>(p.dq), DO, ci.tok0, ci.len, h, H, p.K);
+        store_rows(static_cast<bf16 *>(p.dk), VT, ci.tok0, ci.len, h, H, p.K);
     }
 done:
     tc_fence_before();

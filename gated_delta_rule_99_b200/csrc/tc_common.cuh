@@ -49,28 +49,22 @@ __device__ __forceinline__ void operands_ready() {
     tc_fence_after();
 }
 
-// Loads rows [0, 64) of one chunk and head of a [tokens][H][128] bf16 tensor
-// into an SW128 tile with R rows (block stride), starting at row `row0`;
-// rows at or past `len` are zero.  Asynchronous (cp.async).
+// Loads rows [0, 64) of one chunk and head of a [tokens][H][width] bf16 tensor
+// (width 64 or 128) into the 128 columns of an SW128 tile with R rows (block
+// stride), starting at row `row0`; rows at or past `len` and columns at or past
+// `width` are zero (a head dim of 64 runs on the 128-wide tiles: the zero
+// columns add nothing to any product, and the state's padded rows and columns
+// stay zero).  Asynchronous (cp.async).
 __device__ __forceinline__ void load_rows_async(uint8_t *tile, int R, int row0, const bf16 *src,
-                                                int64_t tok0, int len, int h, int H,
+                                                int64_t tok0, int len, int h, int H, int width,
                                                 int nthreads = NT) {
     const uint32_t base = smem_u32(tile);
     for (int t = threadIdx.x; t < C * 16; t += nthreads) {
         const int r = t >> 4, j = t & 15;
-        const bool valid = r < len;
-        const bf16 *g = valid ? src + ((tok0 + r) * H + h) * D + j * 8 : src;
+        const bool valid = r < len && j * 8 < width;
+        const bf16 *g = valid ? src + ((tok0 + r) * H + h) * width + j * 8 : src;
         cp_async16_zfill(base + sw128_chunk(R, row0 + r, j), g, valid);
     }
-}
-
-// Linear copy of a tile image (bytes multiple of 16 * NT).
-__device__ __forceinline__ void load_image_async(uint8_t *tile, const void *img, size_t bytes,
-                                                 int nthreads = NT) {
-    const uint32_t base = smem_u32(tile);
-    const uint8_t *g = static_cast<const uint8_t *>(img);
-    for (size_t off = (size_t)threadIdx.x * 16; off < bytes; off += (size_t)nthreads * 16)
-        cp_async16(base + (uint32_t)off, g + off);
 }
 
 // In-chunk cumulative log-decay (zero gates past len), summed in token order by

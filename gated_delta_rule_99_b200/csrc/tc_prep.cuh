@@ -39,8 +39,8 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     float *F = reinterpret_cast<float *>(sm + PrepSmem::kF);
     const int tid = threadIdx.x;
 
-    load_rows_async(Kt, C, 0, (const bf16 *)p.k, ci.tok0, ci.len, h, H);
-    load_rows_async(Vt, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H);
+    load_rows_async(Kt, C, 0, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K);
+    load_rows_async(Vt, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H, p.V);
     cp_async_commit();
     if (tid == 0) {
         mbar_init(&mbar, 1);
@@ -250,7 +250,9 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
                 float w[16];
                 tmem_ld16(tm(tmem, c0), w);
                 tmem_ld_wait();
-                if (i >= 0) {
+                if (i >= 0) {  // stored negated: both chains subtract W products
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) w[q] = -w[q];
                     *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8)) = pack8(w);
                     *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(w + 8);
                 }

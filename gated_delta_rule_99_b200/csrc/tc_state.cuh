@@ -36,11 +36,13 @@ __device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, 
 // One run of the forward chain over chunks [c0, c1) of one head.
 struct ChainFwd {
     int h, c0, c1;
-    const float *init;   // state H entering chunk c0 ([d_k][d_v] fp32), or nullptr for zero
+    const float *init;   // state H entering chunk c0 (fp32), or nullptr for zero
+    int init_user;       // init is a caller's [K][V] block (else an internal [128][128] one)
     int init_identity;   // start from H = I (the transition-matrix run of the piece scan)
     int zero_ut;         // take Ut as zero (the transition-matrix run)
     int snapshots;       // write the state entering every chunk and U^T (tile images)
-    float *final_out;    // state leaving chunk c1 - 1 ([d_k][d_v] fp32), or nullptr
+    float *final_out;    // state leaving chunk c1 - 1 (fp32), or nullptr
+    int out_user;        // final_out is a caller's [K][V] block (else [128][128])
     int where;           // tag recorded if a bounded wait gives up
 };
 
@@ -54,8 +56,9 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     const int H = p.H, h = a.h, v = threadIdx.x;
     float S[D];
     if (a.init) {
+        const int ik = a.init_user ? p.K : D, iv = a.init_user ? p.V : D;
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = a.init[kk * D + v];
+        for (int kk = 0; kk < D; ++kk) S[kk] = (kk < ik && v < iv) ? a.init[kk * iv + v] : 0.f;
     } else {
 #pragma unroll
         for (int kk = 0; kk < D; ++kk) S[kk] = (a.init_identity && kk == v) ? 1.f : 0.f;
@@ -132,7 +135,7 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-                d[q] = (with_ut ? __bfloat162float(Ut[(c32 + q) * D + v]) : 0.f) - d[q];
+                d[q] = (with_ut ? __bfloat162float(Ut[(c32 + q) * D + v]) : 0.f) + d[q];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
@@ -172,8 +175,12 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         if (a.snapshots) bulk_wait_all();
     }
     if (a.final_out) {
+        const int ok = a.out_user ? p.K : D, ov = a.out_user ? p.V : D;
+        if (v < ov) {
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) a.final_out[kk * D + v] = S[kk];
+            for (int kk = 0; kk < D; ++kk)
+                if (kk < ok) a.final_out[kk * ov + v] = S[kk];
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -188,11 +195,13 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
     a.h = h;
     a.c0 = p.seq_first[n];
     a.c1 = p.seq_first[n + 1];
-    a.init = p.h0 ? p.h0 + ((size_t)n * H + h) * D * D : nullptr;
+    a.init = p.h0 ? p.h0 + ((size_t)n * H + h) * p.K * p.V : nullptr;
+    a.init_user = 1;
     a.init_identity = 0;
     a.zero_ut = 0;
     a.snapshots = 1;
-    a.final_out = p.hT ? p.hT + ((size_t)n * H + h) * D * D : nullptr;
+    a.final_out = p.hT ? p.hT + ((size_t)n * H + h) * p.K * p.V : nullptr;
+    a.out_user = 1;
     a.where = 3;
     chain_fwd(p, a);
 }

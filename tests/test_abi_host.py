@@ -65,7 +65,8 @@ def test_flags_match_header_and_unknown_bits_are_rejected():
 
 
 def test_l2norm_workspace_holds_normalised_copies_only_off_the_tensor_core_path():
-    for dt, K, V, grows in ((1, 64, 128, True), (0, 64, 64, True), (0, 128, 128, False)):
+    for dt, K, V, grows in ((1, 64, 128, True), (1, 128, 128, True), (0, 64, 64, False),
+                            (0, 128, 128, False)):
         plain = gdn.make_desc(2, 300, 3, K, V, dtype=dt)
         l2 = gdn.make_desc(2, 300, 3, K, V, dtype=dt, flags=gdn.GDN_FLAG_QK_L2NORM)
         for size in (gdn.fwd_workspace_size, gdn.bwd_workspace_size):

@@ -41,8 +41,9 @@ def test_tensor_core_path_packed_ragged():
     _check(inp, TOL["bf16"])
 
 
-@pytest.mark.parametrize("dtype,K,V", [("fp32", 64, 128), ("bf16", 64, 64), ("fp32", 128, 64)])
-def test_pass_path(dtype, K, V):
+@pytest.mark.parametrize("dtype,K,V", [("fp32", 64, 128), ("bf16", 64, 64), ("fp32", 128, 64),
+                                       ("bf16", 128, 64)])
+def test_other_head_dims_and_fp32(dtype, K, V):
     inp = make_inputs(B=2, T=150, H=2, K=K, V=V, dtype=dtype, seed=62, raw_qk=True)
     _check(inp, TOL[dtype])
 

@@ -209,3 +209,30 @@ def test_tc_zero_write_strength_and_no_initial_state():
     inp = make_inputs(B=1, T=129, H=2, K=128, V=128, dtype="bf16", seed=23, h0_std=0.0)
     inp.beta[:, 40:90] = 0.0
     check_all(inp, TOL["bf16"])
+
+
+# ---- head dims of 64 on the tensor-core path (the 128-wide tiles zero-padded)
+@pytest.mark.parametrize("K,V", [(64, 64), (64, 128), (128, 64)])
+def test_tc_head_dim_64_packed_ragged(K, V):
+    lengths = [1, 0, 63, 64, 65, 130, 7, 200]
+    inp = make_inputs(B=1, T=sum(lengths), H=3, K=K, V=V, dtype="bf16", seed=24 + K + V,
+                      lengths=lengths, scale=0.25)
+    check_all(inp, TOL["bf16"])
+
+
+def test_tc_head_dim_64_dense_rows_full_size_sampled():
+    inp = make_inputs(B=4, T=4096, H=16, K=64, V=64, dtype="bf16", seed=25)
+    check_all(inp, TOL["bf16"], units=[(0, 0), (3, 15), (1, 8)])
+
+
+def test_tc_head_dim_64_chained_halves_bitwise():
+    inp = make_inputs(B=2, T=1024, H=2, K=64, V=128, dtype="bf16", seed=26, bwd=False)
+    d = inp.to("cuda")
+    o, hT = gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, h0=d.h0)
+    sl = lambda x, a, b: x[:, a:b].contiguous()
+    oa, ha = gdn.gdn_fwd(sl(d.q, 0, 512), sl(d.k, 0, 512), sl(d.v, 0, 512), sl(d.g, 0, 512),
+                         sl(d.beta, 0, 512), h0=d.h0)
+    ob, hb = gdn.gdn_fwd(sl(d.q, 512, 1024), sl(d.k, 512, 1024), sl(d.v, 512, 1024),
+                         sl(d.g, 512, 1024), sl(d.beta, 512, 1024), h0=ha)
+    torch.cuda.synchronize()
+    assert torch.equal(o[:, :512], oa) and torch.equal(o[:, 512:], ob) and torch.equal(hT, hb)
