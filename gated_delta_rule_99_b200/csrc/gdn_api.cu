@@ -1,6 +1,9 @@
 // C ABI of the Gated DeltaNet layer: validation, workspace layout and launch
 // sequencing on the caller's stream.  Declared in include/gdn.h.
+#include <cudaTypedefs.h>
+
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "gdn_internal.cuh"
@@ -143,6 +146,37 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     return p;
 }
 
+// The driver's tensor-map encoder, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        else
+            (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// [tokens][H][width] bf16 viewed as a 3-d tensor (element, head, token); a box is
+// 64 elements x 1 head x 64 tokens (128-byte rows in the operand tiles' swizzle).
+bool encode_rows(CUtensorMap *m, const void *ptr, int64_t BT, int64_t H, int64_t width) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+    if (!fn || !ptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)BT};
+    cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)H * width * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estride[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+              estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Normalisation pass of the fp32 path: q and k rows divided by their norms into
 // the workspace copies, which the kernels then read in place of q and k.
 bool normalise_qk(const Problem &pb, const Layout &L, void *ws, Params *p, cudaStream_t s) {
@@ -164,6 +198,13 @@ bool use_tc(const Problem &pb, bool bwd) {
 }
 
 }  // namespace
+
+bool encode_row_maps(Params &p, bool bwd) {
+    if (p.BT <= 0) return true;  // nothing is loaded
+    return encode_rows(&p.tm_q, p.q, p.BT, p.H, p.K) && encode_rows(&p.tm_k, p.k, p.BT, p.H, p.K) &&
+           encode_rows(&p.tm_v, p.v, p.BT, p.H, p.V) &&
+           (!bwd || encode_rows(&p.tm_do, p.do_, p.BT, p.H, p.V));
+}
 
 // Workspace layout.  The SIMT path (fp32) keeps fp32 per-(chunk, head)
 // intermediates; the tensor-core path (bf16) has its own region.
@@ -279,6 +320,7 @@ gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.o = o;
     p.hT = hT;
     const bool tc = use_tc(pb, false);
+    if (tc && !encode_row_maps(p, false)) return GDN_ERR_CUDA;
     if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
     if (!tc && pb.l2norm && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;
     cudaError_t e = tc ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
@@ -322,6 +364,7 @@ gdn_status gdn_bwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.dbeta = dbeta;
     p.dh0 = dh0;
     const bool tc = use_tc(pb, true);
+    if (tc && !encode_row_maps(p, true)) return GDN_ERR_CUDA;
     if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
     const bool pre = !tc && pb.l2norm;
     if (pre && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;

@@ -1,6 +1,7 @@
 // Internal declarations shared by the C ABI (gdn_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -64,6 +65,10 @@ struct Params {
     // (sequence, head, piece) the entering state, the composed transition and offset
     int32_t P, L;
     float *tHin, *tMp, *tBp;
+    // tensor maps of the bf16 [tokens][H][d] inputs for the tensor-core path: a box is 64
+    // tokens x 64 elements of one head, written to shared memory with the operand tiles'
+    // 128-byte swizzle (encoded on the host for every call)
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;
 };
 
 // Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).
@@ -104,6 +109,8 @@ cudaError_t launch_l2norm_back(const void *xn, const float *inv, void *dx, int64
                                bool bf16, cudaStream_t stream);
 bool tc_bwd_ready();
 cudaError_t launch_tc_fwd(const Params &p, const Problem &pb, cudaStream_t stream);
+// Encodes p.tm_q, tm_k, tm_v (and tm_do for the backward) from p.q, p.k, p.v, p.do_.
+bool encode_row_maps(Params &p, bool bwd);
 cudaError_t launch_tc_bwd(const Params &p, const Problem &pb, cudaStream_t stream);
 
 // Kernel ids recorded by the launch trace (gdn_trace_install).

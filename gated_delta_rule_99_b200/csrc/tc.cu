@@ -28,7 +28,7 @@ namespace {
 using namespace tc;
 
 // ============================================================ tc_prep
-__global__ void __launch_bounds__(NT) tc_prep_kernel(Params p, int want_A) {
+__global__ void __launch_bounds__(NT) tc_prep_kernel(const __grid_constant__ Params p, int want_A) {
     prep_body(p, blockIdx.x, want_A);
 }
 
@@ -193,7 +193,7 @@ struct OutSmem {
 };
 constexpr int kOutSmem = OutSmem::kEnd + 1024;
 
-__global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
+__global__ void __launch_bounds__(NT) tc_out_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar, lbar;
@@ -204,14 +204,13 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
     uint8_t *QK = sm + OutSmem::kQK, *Ss = sm + OutSmem::kS, *UTs = sm + OutSmem::kUT;
     uint8_t *QG = sm + OutSmem::kQG, *Ps = sm + OutSmem::kP;
     float *G = reinterpret_cast<float *>(sm + OutSmem::kG);
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, p.K);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K);
-    cp_async_commit();
-    if (tid == 0) {  // the state and U^T images by bulk copies
+    if (tid == 0) {  // q and k rows by the tensor engine, the state and U^T images by bulk copies
         mbar_init(&mbar, 1);
         mbar_init(&lbar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&lbar, (uint32_t)(kImg128 + kImgUT));
+        mbar_arrive_expect_tx(&lbar, 2 * row_tile_bytes(p.K) + (uint32_t)(kImg128 + kImgUT));
+        load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
+        load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
         bulk_load(smem_u32(Ss), static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128,
                   (uint32_t)kImg128, &lbar);
         bulk_load(smem_u32(UTs), static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT,
@@ -223,11 +222,10 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(Params p) {
         tmem_relinquish();
     }
     __syncthreads();  // thread 0's mbarrier inits are visible before any thread waits on them
-    cp_async_wait<0>();
-    bool ok = __syncthreads_and(mbar_wait(&lbar, 0, kWaitLimit));
-    if (!ok && tid == 0) {
-        record_timeout(p, 7);
-        mbar_wait(&lbar, 0, kWaitLimit);  // no copy left in flight
+    bool ok = copies_arrived(&lbar, p, 7);
+    if (ok) {
+        fix_rows(QK, D, 0, ci.len, p.K);
+        fix_rows(QK, D, C, ci.len, p.K);
     }
     operands_ready();
     if (ok && p.l2norm) {  // q and k rows divided by their norms

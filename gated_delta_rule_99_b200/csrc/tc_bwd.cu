@@ -42,42 +42,48 @@ constexpr int kLocalSmem = LocalSmem::kEnd + 1024;
 __device__ __forceinline__ void local_body(const Params &p, int ch) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
+    __shared__ uint64_t mbar, lbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, c = ch / H, h = ch % H, tid = threadIdx.x;
     const ChunkInfo ci = p.chunks[c];
     uint8_t *QK = sm + LocalSmem::kQK, *DO = sm + LocalSmem::kDO, *Ps = sm + LocalSmem::kP;
     float *G = reinterpret_cast<float *>(sm + LocalSmem::kG);
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, p.K);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K);
-    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H, p.V);
-    cp_async_commit();
-    if (tid == 0) {
+    if (tid == 0) {  // q, k and dO rows by the tensor engine
         mbar_init(&mbar, 1);
+        mbar_init(&lbar, 1);
         fence_mbar_init();
+        mbar_arrive_expect_tx(&lbar, 2 * row_tile_bytes(p.K) + row_tile_bytes(p.V));
+        load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
+        load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
+        load_rows_tma(DO, C, 0, &p.tm_do, ci.tok0, h, p.V, &lbar);
     }
     if (tid < 32) {
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
-    chunk_gates(G, nullptr, p, ci, h);
-    cp_async_wait<0>();
+    chunk_gates(G, nullptr, p, ci, h);  // its barriers also publish the mbarrier inits
+    bool ok = copies_arrived(&lbar, p, 32);
+    if (ok) {
+        fix_rows(QK, D, 0, ci.len, p.K);
+        fix_rows(QK, D, C, ci.len, p.K);
+        fix_rows(DO, C, 0, ci.len, p.V);
+    }
     operands_ready();
-    if (p.l2norm) {  // q and k rows divided by their norms
+    if (ok && p.l2norm) {  // q and k rows divided by their norms
         l2norm_tile_rows(QK, D, 0, nullptr);
         l2norm_tile_rows(QK, D, C, nullptr);
         operands_ready();
     }
     const uint32_t tmem = tslot;
-    if (tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
+    if (ok && tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
         const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
             mma_bf16(tmem, desc_kmajor(qb, D, s), desc_kmajor(kb, D, s), id, s > 0);
         mma_commit(&mbar);
     }
-    {  // Qg = scale diag(gam) Q: an operand of the reverse state pass (tile image)
+    if (ok) {  // Qg = scale diag(gam) Q: an operand of the reverse state pass (tile image)
         uint8_t *img = static_cast<uint8_t *>(p.tQg) + (size_t)ch * kImg64;
         for (int t = tid; t < C * 16; t += NT) {
             const int r = t >> 4, j = t & 15;
@@ -89,7 +95,7 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
             *reinterpret_cast<uint4 *>(img + sw128_chunk(C, r, j)) = pack8(f);
         }
     }
-    bool ok = cta_wait(&mbar, 0, p, 11);
+    if (ok) ok = cta_wait(&mbar, 0, p, 11);
     if (ok) {
         const int i = m64_row();
         for (int c0 = 0; c0 < C; c0 += 16) {
@@ -133,7 +139,7 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
 
 // tc_prep (with A for the backward) on CTAs [0, NC*H) and tc_local on
 // [NC*H, 2*NC*H): independent chunk-parallel steps in one launch.
-__global__ void __launch_bounds__(NT, 4) tc_prep_local_kernel(Params p) {
+__global__ void __launch_bounds__(NT, 4) tc_prep_local_kernel(const __grid_constant__ Params p) {
     const int nch = p.NC * p.H;
     if ((int)blockIdx.x < nch) prep_body(p, blockIdx.x, 1);
     else local_body(p, blockIdx.x - nch);
@@ -149,14 +155,15 @@ struct SbwdSmem {
 };
 constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
 
-// Chunk ch's Kd, W and Qg images, local dU^T image and gate row by bulk copies
-// (thread 0, completing on `bar`); its dO rows by cp.async (one commit group).
+// Chunk ch's Kd, W and Qg images, local dU^T image and gate row by bulk copies,
+// its dO rows by the tensor engine (thread 0, all completing on `bar`).
 __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
                                               const ChunkInfo &ci, int h, const Params &p,
                                               uint64_t *bar) {
     uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
     if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(bar, 3u * (uint32_t)kImg64 + (uint32_t)kImgUT + C * 4u);
+        mbar_arrive_expect_tx(bar, 3u * (uint32_t)kImg64 + (uint32_t)kImgUT + C * 4u +
+                                       row_tile_bytes(p.V));
         bulk_load(smem_u32(b + SbwdSmem::kKd), static_cast<const uint8_t *>(p.tKd) + ch * kImg64,
                   kImg64, bar);
         bulk_load(smem_u32(b + SbwdSmem::kW), static_cast<const uint8_t *>(p.tW) + ch * kImg64,
@@ -166,9 +173,8 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
         bulk_load(smem_u32(b + SbwdSmem::kDUL),
                   static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT, kImgUT, bar);
         bulk_load(smem_u32(b + SbwdSmem::kG), p.tG + ch * C, C * 4, bar);
+        load_rows_tma(b + SbwdSmem::kDO, C, 0, &p.tm_do, ci.tok0, h, p.V, bar);
     }
-    load_rows_async(b + SbwdSmem::kDO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, p.H, p.V);
-    cp_async_commit();
 }
 
 // Body of the reverse state pass for CTA `blk` (sequence blk / H, head blk % H).
@@ -219,12 +225,10 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         if (c - 1 >= c0) {
             sbwd_prefetch(sm, buf ^ 1, ch - H, p.chunks[c - 1], h, p, &lbar[buf ^ 1]);
             pend |= 2u >> buf;
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
         }
         const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, kWaitLimit);
         uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
+        if (lok) fix_rows(b + SbwdSmem::kDO, C, 0, p.chunks[c].len, p.V);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
@@ -311,7 +315,6 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
                 if (kk < p.K) g0[kk * p.V + v] = S[kk];
         }
     }
-    cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
     if (v < 32) tmem_dealloc(tmem, 256);
@@ -320,7 +323,8 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
 // Both chains of the backward in one launch: CTAs [0, N*H) recompute the
 // forward states (pf has no final-state output), CTAs [N*H, 2*N*H) run the
 // reverse pass.  They are independent, so each gets its own SMs.
-__global__ void __launch_bounds__(NT, 1) tc_chains_kernel(Params pf, Params pb) {
+__global__ void __launch_bounds__(NT, 1) tc_chains_kernel(const __grid_constant__ Params pf,
+                                                           const __grid_constant__ Params pb) {
     const int nh = pb.N * pb.H;
     if ((int)blockIdx.x < nh) state_fwd_body(pf, blockIdx.x);
     else state_bwd_body(pb, blockIdx.x - nh);
@@ -443,7 +447,7 @@ __device__ __forceinline__ void ldcw(uint32_t tmem, int col, float *d) {
     tmem_ld_wait();
 }
 
-__global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
+__global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar;
@@ -475,7 +479,8 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
     if (tid == 0) {  // the tile images and A by bulk copies (one instruction each)
         mbar_init(&lbar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&lbar, 2 * kImg128 + 2 * kImgUT + kImgA);
+        mbar_arrive_expect_tx(&lbar, 2 * kImg128 + 2 * kImgUT + kImgA + 2 * row_tile_bytes(p.K) +
+                                         2 * row_tile_bytes(p.V));
         bulk_load(smem_u32(SC), static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128,
                   kImg128, &lbar);
         bulk_load(smem_u32(DSN), static_cast<const uint8_t *>(p.tdSn) + (size_t)ch * kImg128,
@@ -486,13 +491,12 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
                   kImgUT, &lbar);
         bulk_load(smem_u32(AB), static_cast<const uint8_t *>(p.tA) + (size_t)ch * kImgA, kImgA,
                   &lbar);
+        // q, k, dO, v rows by the tensor engine
+        load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
+        load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
+        load_rows_tma(DO, C, 0, &p.tm_do, ci.tok0, h, p.V, &lbar);
+        load_rows_tma(VT, C, 0, &p.tm_v, ci.tok0, h, p.V, &lbar);
     }
-    // q, k, v, do rows by cp.async into the swizzled layout
-    load_rows_async(QK, D, 0, (const bf16 *)p.q, ci.tok0, ci.len, h, H, p.K, NG);
-    load_rows_async(QK, D, C, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K, NG);
-    load_rows_async(DO, C, 0, (const bf16 *)p.do_, ci.tok0, ci.len, h, H, p.V, NG);
-    load_rows_async(VT, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H, p.V, NG);
-    cp_async_commit();
     if (tid < C) {
         const int64_t idx = (int64_t)(ci.tok0 + tid) * H + h;
         G[tid] = p.tG[(size_t)ch * C + tid];
@@ -511,17 +515,16 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(Params p) {
         gam[tid] = expf(G[tid]);
         e[tid] = expf(G[C - 1] - G[tid]);
     }
-    cp_async_wait<0>();
-    {  // the bulk copies (bounded wait, decided by the whole CTA)
-        const bool lok = __syncthreads_and(mbar_wait(&lbar, 0, kWaitLimit));
-        if (!lok) {
-            if (tid == 0) record_timeout(p, 20);
-            tc_fence_before();
-            __syncthreads();
-            if (tid < 32) tmem_dealloc(tslot, 512);
-            return;
-        }
+    if (!copies_arrived(&lbar, p, 20)) {  // (the barrier above published the inits)
+        tc_fence_before();
+        __syncthreads();
+        if (tid < 32) tmem_dealloc(tslot, 512);
+        return;
     }
+    fix_rows(QK, D, 0, ci.len, p.K, NG);
+    fix_rows(QK, D, C, ci.len, p.K, NG);
+    fix_rows(DO, C, 0, ci.len, p.V, NG);
+    fix_rows(VT, C, 0, ci.len, p.V, NG);
     operands_ready();
     if (p.l2norm) {  // q rows (threads 0-127) and k rows (128-255) divided by their norms
         l2norm_tile_rows(QK, D, 0, qinv, 0);

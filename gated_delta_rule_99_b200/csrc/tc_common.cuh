@@ -49,22 +49,52 @@ __device__ __forceinline__ void operands_ready() {
     tc_fence_after();
 }
 
-// Loads rows [0, 64) of one chunk and head of a [tokens][H][width] bf16 tensor
-// (width 64 or 128) into the 128 columns of an SW128 tile with R rows (block
-// stride), starting at row `row0`; rows at or past `len` and columns at or past
-// `width` are zero (a head dim of 64 runs on the 128-wide tiles: the zero
-// columns add nothing to any product, and the state's padded rows and columns
-// stay zero).  Asynchronous (cp.async).
-__device__ __forceinline__ void load_rows_async(uint8_t *tile, int R, int row0, const bf16 *src,
-                                                int64_t tok0, int len, int h, int H, int width,
-                                                int nthreads = NT) {
-    const uint32_t base = smem_u32(tile);
+// Bytes one load_rows_tma call completes on its mbarrier (one 64 x 64 box per
+// 64 columns of the source rows).
+__device__ __forceinline__ uint32_t row_tile_bytes(int width) { return width == D ? 16384u : 8192u; }
+
+// Rows [0, 64) of one chunk and head (tokens tok0..tok0+63 of head h) of a
+// [tokens][H][width] bf16 tensor (width 64 or 128) into the first width/64
+// column blocks of an SW128 tile with R rows, starting at row `row0` (0 or 64):
+// one 64 x 64 box per block by the tensor engine, row_tile_bytes(width) on
+// `bar`.  One thread issues it.  Tokens past the tensor arrive as zeros; the
+// rows past the chunk's end and the columns past `width` are cleared by
+// fix_rows once the copy has landed.
+__device__ __forceinline__ void load_rows_tma(uint8_t *tile, int R, int row0,
+                                              const CUtensorMap *map, int64_t tok0, int h,
+                                              int width, uint64_t *bar) {
+    const uint32_t base = smem_u32(tile) + (uint32_t)row0 * 128u;
+    tma_load_3d(base, map, 0, h, (int)tok0, bar);
+    if (width == D) tma_load_3d(base + (uint32_t)R * 128u, map, 64, h, (int)tok0, bar);
+}
+
+// Zeroes, in the tile block load_rows_tma filled, the rows at or past `len`
+// (in a chunk shorter than 64 they hold the next sequence's tokens) and, for a
+// head dim of 64, the second 64-column block (a head dim of 64 runs on the
+// 128-wide tiles: the zero columns add nothing to any product, and the state's
+// padded rows and columns stay zero).
+__device__ __forceinline__ void fix_rows(uint8_t *tile, int R, int row0, int len, int width,
+                                         int nthreads = NT) {
+    if (len >= C && width == D) return;
     for (int t = threadIdx.x; t < C * 16; t += nthreads) {
         const int r = t >> 4, j = t & 15;
-        const bool valid = r < len && j * 8 < width;
-        const bf16 *g = valid ? src + ((tok0 + r) * H + h) * width + j * 8 : src;
-        cp_async16_zfill(base + sw128_chunk(R, row0 + r, j), g, valid);
+        if (r >= len || j * 8 >= width)
+            *reinterpret_cast<uint4 *>(tile + sw128_chunk(R, row0 + r, j)) = make_uint4(0, 0, 0, 0);
     }
+}
+
+// Bounded wait for phase 0 of `bar` (a CTA's input copies), decided by the
+// whole CTA (a barrier); the caller must have made the mbarrier's init visible
+// to every thread (a barrier after it) first.  On failure records `where` and
+// waits once more, bounded, so that no copy is left in flight when the CTA
+// gives up.
+__device__ __forceinline__ bool copies_arrived(uint64_t *bar, const Params &p, int where) {
+    const bool ok = __syncthreads_and(mbar_wait(bar, 0, kWaitLimit));
+    if (!ok && threadIdx.x == 0) {
+        record_timeout(p, where);
+        mbar_wait(bar, 0, kWaitLimit);
+    }
+    return ok;
 }
 
 // In-chunk cumulative log-decay (zero gates past len), summed in token order by

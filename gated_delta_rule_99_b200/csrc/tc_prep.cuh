@@ -26,7 +26,7 @@ constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 colu
 __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
+    __shared__ uint64_t mbar, lbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, c = ch / H, h = ch % H;
@@ -39,30 +39,34 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     float *F = reinterpret_cast<float *>(sm + PrepSmem::kF);
     const int tid = threadIdx.x;
 
-    load_rows_async(Kt, C, 0, (const bf16 *)p.k, ci.tok0, ci.len, h, H, p.K);
-    load_rows_async(Vt, C, 0, (const bf16 *)p.v, ci.tok0, ci.len, h, H, p.V);
-    cp_async_commit();
-    if (tid == 0) {
+    if (tid == 0) {  // K and V rows by the tensor engine
         mbar_init(&mbar, 1);
+        mbar_init(&lbar, 1);
         fence_mbar_init();
+        mbar_arrive_expect_tx(&lbar, row_tile_bytes(p.K) + row_tile_bytes(p.V));
+        load_rows_tma(Kt, C, 0, &p.tm_k, ci.tok0, h, p.K, &lbar);
+        load_rows_tma(Vt, C, 0, &p.tm_v, ci.tok0, h, p.V, &lbar);
     }
     if (tid < 32) {
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
-    chunk_gates(G, bta, p, ci, h);
-    cp_async_wait<0>();
+    chunk_gates(G, bta, p, ci, h);  // its barriers also publish the mbarrier inits
+    bool ok = copies_arrived(&lbar, p, 31);
+    if (ok) {
+        fix_rows(Kt, C, 0, ci.len, p.K);
+        fix_rows(Vt, C, 0, ci.len, p.V);
+    }
     operands_ready();
-    if (p.l2norm) {  // k rows divided by their norms
+    if (ok && p.l2norm) {  // k rows divided by their norms
         l2norm_tile_rows(Kt, C, 0, nullptr);
         operands_ready();
     }
     const uint32_t tmem = tslot;
     uint32_t phase = 0;
-    bool ok = true;
 
     // K K^T (M = 64 rows i, N = 64 cols j, K = 128)
-    if (tid == 0) {
+    if (ok && tid == 0) {
         const uint32_t kb = smem_u32(Kt), id = idesc_bf16(64, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
@@ -70,7 +74,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         mma_commit(&mbar);
     }
     // meanwhile: Kd = diag(e) K as a tile image, and G
-    {
+    if (ok) {
         const float Gn = G[C - 1];
         uint8_t *dst = static_cast<uint8_t *>(p.tKd) + (size_t)ch * kImg64;
         for (int t = tid; t < C * 16; t += NT) {
@@ -87,7 +91,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             F[tid] = expf(G[tid | 15] - G[tid]);
         }
     }
-    ok = cta_wait(&mbar, phase, p, 1);
+    if (ok) ok = cta_wait(&mbar, phase, p, 1);
     phase ^= 1;
     if (ok) {
         // L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32)

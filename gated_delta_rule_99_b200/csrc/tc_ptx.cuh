@@ -1,6 +1,6 @@
 // Hand-written sm_100a PTX wrappers: tcgen05 (TMEM alloc, MMA, commit, ld),
-// mbarrier with bounded waits, async-proxy fences, cp.async staging, and the
-// 128-byte-swizzled shared-memory tile format the MMAs read.
+// mbarrier with bounded waits, async-proxy fences, bulk and tensor-map (TMA)
+// copies, and the 128-byte-swizzled shared-memory tile format the MMAs read.
 //
 // Tile format ("SW128 tile"): a tile of R rows x (64 * nb) bf16 columns is
 // stored as nb column blocks of R rows x 128 bytes; block b starts at
@@ -10,6 +10,7 @@
 // MN-major operand (reduction along its rows; columns are M or N).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -154,27 +155,21 @@ __device__ __forceinline__ void bulk_load(uint32_t sdst, const void *gsrc, uint3
         :: "r"(sdst), "l"(gsrc), "r"(bytes), "r"(smem_u32(mbar)) : "memory");
 }
 
+// Tensor-map (TMA) load of one 3-d box into this CTA's shared memory at `sdst`
+// (1024-byte aligned for the 128-byte swizzle), completing its bytes on the
+// mbarrier; coordinates innermost first.  No multicast.
+__device__ __forceinline__ void tma_load_3d(uint32_t sdst, const CUtensorMap *map, int x, int y,
+                                            int z, uint64_t *mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];"
+        :: "r"(sdst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
+           "r"(smem_u32(mbar)) : "memory");
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (MMA reads).
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// ---------------------------------------------------------------- cp.async
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *gptr) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(saddr), "l"(gptr) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
-}
-
-// 16-byte cp.async that writes zeros (reads nothing) when `valid` is false.
-__device__ __forceinline__ void cp_async16_zfill(uint32_t saddr, const void *gptr, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                 :: "r"(saddr), "l"(gptr), "r"(valid ? 16 : 0) : "memory");
 }
 
 // Bulk (async-proxy) copy shared -> global of `bytes` (multiple of 16, both 16-byte aligned).
