@@ -10,9 +10,8 @@
 // with S = state^T kept in fp32 (with GDN_FLAG_QK_L2NORM, q_t and k_t are first
 // divided by their norms, as the pages' API option use_qk_l2norm does; the
 // factors 1/|q_t| and 1/|k_t| are applied where q_t and k_t enter).  One CTA per
-// (sequence, head); thread v owns
-// row v of S in registers (d_k values), so the state is read once and written
-// once per call and every step is thread-local arithmetic.  HBM bound: the
+// (sequence, head); the state is read once and written once per call and
+// lives in registers in between (two threads per row of S).  HBM bound: the
 // state (2 d_k d_v 4 bytes per sequence and head) dominates the traffic.
 #include "gdn_internal.cuh"
 
@@ -32,22 +31,28 @@ __device__ __forceinline__ void stf(__nv_bfloat16 *p, int64_t i, float x) {
     p[i] = __float2bfloat16_rn(x);
 }
 
+// 256 threads per (sequence, head): thread t owns half t / 128 of the keys
+// (K / 2 entries) of state row v = t % 128, so a row's state lives in two
+// threads' registers; the halves' dot products meet in shared memory, added in a
+// fixed order.
 template <typename T, int K>
-__global__ void __launch_bounds__(128) decode_kernel(const T *q, const T *k, const T *v,
+__global__ void __launch_bounds__(256) decode_kernel(const T *q, const T *k, const T *v,
                                                      const float *g, const float *beta,
                                                      float *state, T *o, int Tn, int H, int V,
                                                      float scale, int l2n) {
-    __shared__ float qs[K], ks[K];
-    const int bh = blockIdx.x, b = bh / H, h = bh % H, vi = threadIdx.x;
+    constexpr int KH = K / 2;
+    __shared__ float qs[K], ks[K], red_k[2][128], red_o[2][128];
+    const int bh = blockIdx.x, b = bh / H, h = bh % H, t = threadIdx.x;
+    const int vi = t & 127, half = t >> 7, k0 = half * KH;
     const bool active = vi < V;
     float *st = state + (size_t)bh * K * V;
-    float S[K];
+    float S[KH];
 #pragma unroll
-    for (int kk = 0; kk < K; ++kk) S[kk] = active ? st[(size_t)kk * V + vi] : 0.f;
-    for (int t = 0; t < Tn; ++t) {
-        const int64_t row = ((int64_t)b * Tn + t) * H + h;
-        __syncthreads();  // previous token's q/k no longer read
-        for (int kk = threadIdx.x; kk < K; kk += blockDim.x) {
+    for (int j = 0; j < KH; ++j) S[j] = active ? st[(size_t)(k0 + j) * V + vi] : 0.f;
+    for (int tk = 0; tk < Tn; ++tk) {
+        const int64_t row = ((int64_t)b * Tn + tk) * H + h;
+        __syncthreads();  // the previous token's q, k and partial sums are no longer read
+        for (int kk = t; kk < K; kk += 256) {
             qs[kk] = ldf(q, row * K + kk);
             ks[kk] = ldf(k, row * K + kk);
         }
@@ -67,24 +72,30 @@ __global__ void __launch_bounds__(128) decode_kernel(const T *q, const T *k, con
         }
         float sk0 = 0.f, sk1 = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < K; kk += 2) {
-            sk0 = fmaf(S[kk], ks[kk], sk0);
-            sk1 = fmaf(S[kk + 1], ks[kk + 1], sk1);
+        for (int j = 0; j < KH; j += 2) {
+            sk0 = fmaf(S[j], ks[k0 + j], sk0);
+            sk1 = fmaf(S[j + 1], ks[k0 + j + 1], sk1);
         }
-        const float sk = ik * (sk0 + sk1);
+        red_k[half][vi] = sk0 + sk1;
+        __syncthreads();
+        const float sk = ik * (red_k[0][vi] + red_k[1][vi]);
         const float c1 = bt * sk * ik, c2 = bt * vv * ik;
         float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < K; ++kk) {
-            S[kk] = a * (S[kk] - c1 * ks[kk]) + c2 * ks[kk];
-            if (kk & 1) o1 = fmaf(S[kk], qs[kk], o1);
-            else o0 = fmaf(S[kk], qs[kk], o0);
+        for (int j = 0; j < KH; ++j) {
+            const float kj = ks[k0 + j];
+            S[j] = a * (S[j] - c1 * kj) + c2 * kj;
+            if (j & 1) o1 = fmaf(S[j], qs[k0 + j], o1);
+            else o0 = fmaf(S[j], qs[k0 + j], o0);
         }
-        if (active) stf(o, row * V + vi, scale * iq * (o0 + o1));
+        red_o[half][vi] = o0 + o1;
+        __syncthreads();
+        if (half == 0 && active)
+            stf(o, row * V + vi, scale * iq * (red_o[0][vi] + red_o[1][vi]));
     }
     if (active) {
 #pragma unroll
-        for (int kk = 0; kk < K; ++kk) st[(size_t)kk * V + vi] = S[kk];
+        for (int j = 0; j < KH; ++j) st[(size_t)(k0 + j) * V + vi] = S[j];
     }
 }
 
@@ -96,12 +107,12 @@ cudaError_t launch_typed(const gdn_desc *d, const void *q, const void *k, const 
     const int l2n = (d->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     if (d->dk == 128) {
         GDN_LAUNCH(kKDecode, s,
-                   decode_kernel<T, 128><<<nbh, 128, 0, s>>>(
+                   decode_kernel<T, 128><<<nbh, 256, 0, s>>>(
                        (const T *)q, (const T *)k, (const T *)v, g, beta, state, (T *)o, Tn, H,
                        V, d->scale, l2n));
     } else {
         GDN_LAUNCH(kKDecode, s,
-                   decode_kernel<T, 64><<<nbh, 128, 0, s>>>(
+                   decode_kernel<T, 64><<<nbh, 256, 0, s>>>(
                        (const T *)q, (const T *)k, (const T *)v, g, beta, state, (T *)o, Tn, H,
                        V, d->scale, l2n));
     }

@@ -542,7 +542,6 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     uint32_t phase = 0;
     bool ok;
     float d[CW];
-    const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
     if (tid == 0) {
         const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
                        i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
@@ -625,14 +624,17 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         }
         warp_colsum(d, wsum, w4, cb, l);
     }
-    ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
+    {  // column readers of q and k are built where used (they cost 8 registers each)
+        const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
+        ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
 #pragma unroll
-    for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
-    warp_colsum(d, wsum + 256, w4, cb, l);
-    ldcw(tmem, cX2 + cb, d);  // partial k . X2
+        for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
+        warp_colsum(d, wsum + 256, w4, cb, l);
+        ldcw(tmem, cX2 + cb, d);  // partial k . X2
 #pragma unroll
-    for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
-    warp_colsum(d, wsum + 512, w4, cb, l);
+        for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
+        warp_colsum(d, wsum + 512, w4, cb, l);
+    }
     __syncthreads();
     if (tid < 3 * C) {
         const int k = tid >> 6, i = tid & 63;
@@ -688,10 +690,13 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
         }
     }
-    ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
+    {
+        const ColSw kcol(QK + C * 128, D, r);
+        ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
 #pragma unroll
-    for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
-    warp_colsum(d, wsum, w4, cb, l);
+        for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
+        warp_colsum(d, wsum, w4, cb, l);
+    }
     __syncthreads();
     if (tid < C) kz[tid] = (wsum[tid] + wsum[64 + tid]) + (wsum[128 + tid] + wsum[192 + tid]);
     operands_ready();
@@ -805,6 +810,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     {  // dq = scale (diag(gam) X1 + dPG K) ; dk = diag(e) X2 + diag(b gam) Z + dPG^T Q' + dL terms
         // staged as rows in the consumed dO and V tiles, then 16-byte stores
         bf16 *sq = reinterpret_cast<bf16 *>(DO), *sk = reinterpret_cast<bf16 *>(VT);
+        const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
         float a[CW];
         tmem_ld16(tmq(tmem, cX1 + cb), d);
         tmem_ld16(tmq(tmem, cDQ + cb), a);
