@@ -537,8 +537,9 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                    dub = smem_u32(DUT), ab = smem_u32(AB), x3b = smem_u32(X3), dab = smem_u32(DA),
                    t1b = smem_u32(T1), dpb = smem_u32(DPG), dlb = smem_u32(DLG);
     // TMEM columns
+    // (Y2 takes X3's columns once X3 is read, T1 then Y2's; dL takes Q K^T's once P is formed)
     constexpr int cQK = 0, cX1 = 64, cX2 = 128, cX3 = 192, cDP = 256, cAU = 320, cY1 = 384,
-                  cY2 = 0, cZ = 448, cT1 = 192, cDL = 0, cDQ = 256, cDK = 320, cDKA = 384;
+                  cY2 = 192, cZ = 448, cT1 = 192, cDL = 0, cDQ = 256, cDK = 320, cDKA = 384;
     uint32_t phase = 0;
     bool ok;
     float d[CW];
@@ -596,6 +597,22 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         Gam[gidx(i, j)] = j <= i ? expf(G[i] - G[j]) : 0.f;
     }
     __syncthreads();
+    ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
+#pragma unroll
+    for (int q = 0; q < CW / 8; ++q)
+        *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
+    operands_ready();
+    if (tid == 0) {  // issued now; the SIMT work below runs while they execute
+        const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
+            mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)  // Zp^T = X3^T A   (Z = -Zp)
+            mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
+        mma_commit(&mbar);
+    }
+    // meanwhile: P, Gam . K K^T, dv and the column sums, dP
     // P (scaled, lower incl. diagonal) and Gam . K K^T (strictly lower), fp32
     ldcw(tmem, cQK + cb, d);
     if (r < 64) {
@@ -643,10 +660,6 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     }
     __syncthreads();
     store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H, p.V);
-    ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
-#pragma unroll
-    for (int q = 0; q < CW / 8; ++q)
-        *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
     ldcw(tmem, cDP + cb, d);  // dP: dPG = dP . Gam as an operand tile; PE <- dP . P
     if (i64 >= 0) {
 #pragma unroll
@@ -659,17 +672,6 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
 #pragma unroll
         for (int q = 0; q < CW / 8; ++q)
             *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
-    }
-    operands_ready();
-    if (tid == 0) {
-        const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
-            mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // Zp^T = X3^T A   (Z = -Zp)
-            mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
-        mma_commit(&mbar);
     }
     ok = cta_wait(&mbar, phase, p, 22);
     phase ^= 1;
@@ -690,6 +692,15 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
         }
     }
+    operands_ready();
+    if (tid == 0) {  // T1 = A^T dA (M = 64)
+        const uint32_t id = idesc_bf16(64, 64, 1, 1);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_bf16(tmem + cT1, desc_mnmajor(ab, C, s), desc_mnmajor(dab, C, s), id, s > 0);
+        mma_commit(&mbar);
+    }
+    // meanwhile: k . Z
     {
         const ColSw kcol(QK + C * 128, D, r);
         ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
@@ -699,14 +710,6 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     }
     __syncthreads();
     if (tid < C) kz[tid] = (wsum[tid] + wsum[64 + tid]) + (wsum[128 + tid] + wsum[192 + tid]);
-    operands_ready();
-    if (tid == 0) {  // T1 = A^T dA (M = 64)
-        const uint32_t id = idesc_bf16(64, 64, 1, 1);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            mma_bf16(tmem + cT1, desc_mnmajor(ab, C, s), desc_mnmajor(dab, C, s), id, s > 0);
-        mma_commit(&mbar);
-    }
     ok = cta_wait(&mbar, phase, p, 23);
     phase ^= 1;
     if (!ok) goto done;
