@@ -193,6 +193,14 @@ bool normalise_qk(const Problem &pb, const Layout &L, void *ws, Params *p, cudaS
     return true;
 }
 
+// Packed documents: the chunk table, built and checked on the device (which also
+// resets the workspace's status word).  Dense rows: no table (kernels use the
+// closed form), only the status word reset.
+cudaError_t start_call(const Params &p, const gdn_desc *d, cudaStream_t s) {
+    if (d->n_seqs > 0) return launch_build_chunks(p, s);
+    return cudaMemsetAsync(p.hdr, 0, 16, s);
+}
+
 bool use_tc(const Problem &pb, bool bwd) {
     return pb.dtype == GDN_BF16 && tc_supported(pb) && (!bwd || tc_bwd_ready());
 }
@@ -321,7 +329,7 @@ gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.hT = hT;
     const bool tc = use_tc(pb, false);
     if (tc && !encode_row_maps(p, false)) return GDN_ERR_CUDA;
-    if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (start_call(p, desc, s) != cudaSuccess) return GDN_ERR_CUDA;
     if (!tc && pb.l2norm && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;
     cudaError_t e = tc ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
@@ -365,7 +373,7 @@ gdn_status gdn_bwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.dh0 = dh0;
     const bool tc = use_tc(pb, true);
     if (tc && !encode_row_maps(p, true)) return GDN_ERR_CUDA;
-    if (launch_build_chunks(p, s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (start_call(p, desc, s) != cudaSuccess) return GDN_ERR_CUDA;
     const bool pre = !tc && pb.l2norm;
     if (pre && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;
     cudaError_t e = tc ? launch_tc_bwd(p, pb, s) : launch_simt_bwd(p, s);

@@ -74,6 +74,36 @@ struct Params {
 // Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).
 constexpr size_t kSimtScratchFloats = 64 * 128 * 14 + 64 * 64 * 10 + 64 * 8;
 
+// Chunk c of the call: from the table build_chunks writes for packed documents,
+// or in closed form for dense rows (row c / n, chunk c % n of a row, n = ceil(T / 64)),
+// which then need no table.
+__device__ __forceinline__ ChunkInfo chunk_at(const Params &p, int c) {
+    if (p.cu) return p.chunks[c];
+    const int npr = (p.T + kChunk - 1) / kChunk, row = c / npr, j = c - row * npr;
+    ChunkInfo ci;
+    ci.seq = row;
+    ci.tok0 = row * p.T + j * kChunk;
+    ci.len = p.T - j * kChunk < kChunk ? p.T - j * kChunk : kChunk;
+    ci.idx = j;
+    return ci;
+}
+// Chunk c of sequence n whose first chunk is c0 (no division: for the loops
+// that walk one sequence's chunks).
+__device__ __forceinline__ ChunkInfo chunk_in_seq(const Params &p, int n, int c0, int c) {
+    if (p.cu) return p.chunks[c];
+    const int j = c - c0;
+    ChunkInfo ci;
+    ci.seq = n;
+    ci.tok0 = n * p.T + j * kChunk;
+    ci.len = p.T - j * kChunk < kChunk ? p.T - j * kChunk : kChunk;
+    ci.idx = j;
+    return ci;
+}
+// First chunk of sequence n (n = N gives the chunk count).
+__device__ __forceinline__ int seq_first_at(const Params &p, int n) {
+    return p.cu ? p.seq_first[n] : n * ((p.T + kChunk - 1) / kChunk);
+}
+
 // Host-side problem summary after validation.
 struct Problem {
     int64_t B, T, H, K, V, N, BT;

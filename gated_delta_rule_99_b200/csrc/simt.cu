@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads) simt_prep_kernel(Params p) {
     float *M = bv + C * 128, *G = M + C * C, *bta = G + C;
     for (int ch = blockIdx.x; ch < p.NC * H; ch += gridDim.x) {
         const int c = ch / H, h = ch % H;
-        const ChunkInfo ci = p.chunks[c];
+        const ChunkInfo ci = chunk_at(p, c);
         load_rows(fk, p.k, p.bf16, ci.tok0, ci.len, h, H, K, 1.f);
         load_rows(fv, p.v, p.bf16, ci.tok0, ci.len, h, H, V, 1.f);
         load_gate(G, bta, p, ci, h);
@@ -172,9 +172,9 @@ __global__ void __launch_bounds__(kThreads) simt_state_fwd_kernel(Params p) {
         Hsl[e] = p.h0 ? p.h0[(((int64_t)n * H + h) * K + kk) * V + v0 + j] : 0.f;
     }
     __syncthreads();
-    const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
+    const int c0 = seq_first_at(p, n), c1 = seq_first_at(p, n + 1);
     for (int c = c0; c < c1; ++c) {
-        const ChunkInfo ci = p.chunks[c];
+        const ChunkInfo ci = chunk_at(p, c);
         const size_t ch = (size_t)c * H + h;
         load_gate(G, nullptr, p, ci, h);
         const float gC = expf(G[C - 1]);
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads) simt_out_kernel(Params p) {
     float *fq = slot(p), *fk = fq + C * 128, *O = fk + C * 128, *P = O + C * 128, *G = P + C * C;
     for (int ch = blockIdx.x; ch < p.NC * H; ch += gridDim.x) {
         const int c = ch / H, h = ch % H;
-        const ChunkInfo ci = p.chunks[c];
+        const ChunkInfo ci = chunk_at(p, c);
         load_rows(fq, p.q, p.bf16, ci.tok0, ci.len, h, H, K, p.scale);
         load_rows(fk, p.k, p.bf16, ci.tok0, ci.len, h, H, K, 1.f);
         load_gate(G, nullptr, p, ci, h);
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads) simt_duloc_kernel(Params p) {
           *G = P + C * C;
     for (int ch = blockIdx.x; ch < p.NC * H; ch += gridDim.x) {
         const int c = ch / H, h = ch % H;
-        const ChunkInfo ci = p.chunks[c];
+        const ChunkInfo ci = chunk_at(p, c);
         load_rows(fq, p.q, p.bf16, ci.tok0, ci.len, h, H, K, p.scale);
         load_rows(fk, p.k, p.bf16, ci.tok0, ci.len, h, H, K, 1.f);
         load_rows(fdo, p.do_, p.bf16, ci.tok0, ci.len, h, H, V, 1.f);
@@ -276,9 +276,9 @@ __global__ void __launch_bounds__(kThreads) simt_state_bwd_kernel(Params p) {
         dHsl[e] = p.dhT ? p.dhT[(((int64_t)n * H + h) * K + kk) * V + v0 + j] : 0.f;
     }
     __syncthreads();
-    const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
+    const int c0 = seq_first_at(p, n), c1 = seq_first_at(p, n + 1);
     for (int c = c1 - 1; c >= c0; --c) {
-        const ChunkInfo ci = p.chunks[c];
+        const ChunkInfo ci = chunk_at(p, c);
         const size_t ch = (size_t)c * H + h;
         load_gate(G, nullptr, p, ci, h);
         const float gC = expf(G[C - 1]);
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kThreads) simt_grads_kernel(Params p) {
     float *G = dLG + T4, *bta = G + C, *gam = bta + C, *e = gam + C, *dG = e + C, *red = dG + C;
     for (int ch = blockIdx.x; ch < p.NC * H; ch += gridDim.x) {
         const int c = ch / H, h = ch % H;
-        const ChunkInfo ci = p.chunks[c];
+        const ChunkInfo ci = chunk_at(p, c);
         const float *Hs = p.Hs + (size_t)ch * K * V, *dHn = p.dHn + (size_t)ch * K * V;
         const float *U = p.U + (size_t)ch * C * V, *dU = p.dU + (size_t)ch * C * V;
         const float *A = p.A + (size_t)ch * C * C;

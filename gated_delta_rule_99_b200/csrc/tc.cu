@@ -41,8 +41,8 @@ __global__ void __launch_bounds__(NT, 1) tc_state_fwd_kernel(Params p) {
 // Chunks [c0, c1) of piece `piece` of dense row n (pieces of p.L chunks; the
 // last may be shorter or empty).
 __device__ __forceinline__ void piece_range(const Params &p, int n, int piece, int *c0, int *c1) {
-    const int end = p.seq_first[n + 1];
-    int a = p.seq_first[n] + piece * p.L;
+    const int end = seq_first_at(p, n + 1);
+    int a = seq_first_at(p, n) + piece * p.L;
     a = a < end ? a : end;
     const int b = a + p.L < end ? a + p.L : end;
     *c0 = a;
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(const __grid_constant__ Para
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
-    const ChunkInfo ci = p.chunks[c];
+    const ChunkInfo ci = chunk_at(p, c);
     uint8_t *QK = sm + OutSmem::kQK, *Ss = sm + OutSmem::kS, *UTs = sm + OutSmem::kUT;
     uint8_t *QG = sm + OutSmem::kQG, *Ps = sm + OutSmem::kP;
     float *G = reinterpret_cast<float *>(sm + OutSmem::kG);

@@ -46,7 +46,7 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, c = ch / H, h = ch % H, tid = threadIdx.x;
-    const ChunkInfo ci = p.chunks[c];
+    const ChunkInfo ci = chunk_at(p, c);
     uint8_t *QK = sm + LocalSmem::kQK, *DO = sm + LocalSmem::kDO, *Ps = sm + LocalSmem::kP;
     float *G = reinterpret_cast<float *>(sm + LocalSmem::kG);
     if (tid == 0) {  // q, k and dO rows by the tensor engine
@@ -208,12 +208,13 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
-    const int c0 = p.seq_first[n], c1 = p.seq_first[n + 1];
+    const int c0 = seq_first_at(p, n), c1 = seq_first_at(p, n + 1);
     uint32_t phase = 0;
     // per buffer b (bit b): bulk copies in flight, and the parity of their next completion
     uint32_t pend = 0, lpar = 0;
     if (c0 < c1) {
-        sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, p.chunks[c1 - 1], h, p, &lbar[0]);
+        sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, chunk_in_seq(p, n, c0, c1 - 1), h, p,
+                      &lbar[0]);
         pend = 1;
     }
     uint8_t *dSs = sm + SbwdSmem::kdS, *dUs = sm + SbwdSmem::kdU;
@@ -223,12 +224,13 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         const int buf = (c1 - 1 - c) & 1;
         const size_t ch = (size_t)c * H + h;
         if (c - 1 >= c0) {
-            sbwd_prefetch(sm, buf ^ 1, ch - H, p.chunks[c - 1], h, p, &lbar[buf ^ 1]);
+            sbwd_prefetch(sm, buf ^ 1, ch - H, chunk_in_seq(p, n, c0, c - 1), h, p,
+                          &lbar[buf ^ 1]);
             pend |= 2u >> buf;
         }
         const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, kWaitLimit);
         uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
-        if (lok) fix_rows(b + SbwdSmem::kDO, C, 0, p.chunks[c].len, p.V);
+        if (lok) fix_rows(b + SbwdSmem::kDO, C, 0, chunk_in_seq(p, n, c0, c).len, p.V);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
     const int wg = tid >> 7, r = tid & 127, cb = CW * wg;
     const int l = tid & 31, i64 = l < 16 ? ((tid >> 5) & 3) * 16 + l : -1;  // M = 64 row
-    const ChunkInfo ci = p.chunks[c];
+    const ChunkInfo ci = chunk_at(p, c);
     using S_ = GradSmem;
     uint8_t *QK = sm + S_::kQK, *DO = sm + S_::kDO, *VT = sm + S_::kV, *SC = sm + S_::kSC,
             *DSN = sm + S_::kDSN, *UT = sm + S_::kUT, *DUT = sm + S_::kDUT, *AB = sm + S_::kAB,

@@ -30,7 +30,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, c = ch / H, h = ch % H;
-    const ChunkInfo ci = p.chunks[c];
+    const ChunkInfo ci = chunk_at(p, c);
     uint8_t *Kt = sm + PrepSmem::kK, *Vt = sm + PrepSmem::kV;
     uint8_t *Ab = sm + PrepSmem::kAb, *Ac = sm + PrepSmem::kAc;
     float *L = reinterpret_cast<float *>(sm + PrepSmem::kL);

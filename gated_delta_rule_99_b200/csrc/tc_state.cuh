@@ -193,8 +193,8 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
     const int H = p.H, n = blk / H, h = blk % H;
     ChainFwd a;
     a.h = h;
-    a.c0 = p.seq_first[n];
-    a.c1 = p.seq_first[n + 1];
+    a.c0 = seq_first_at(p, n);
+    a.c1 = seq_first_at(p, n + 1);
     a.init = p.h0 ? p.h0 + ((size_t)n * H + h) * p.K * p.V : nullptr;
     a.init_user = 1;
     a.init_identity = 0;
