@@ -137,6 +137,7 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.tdSn = b(L.tdSn);
     p.tdUT = b(L.tdUT);
     p.tG = f(L.tG);
+    p.tB = f(L.tB);
     p.tA = b(L.tA);
     p.P = (int32_t)pb.P;
     p.L = (int32_t)pb.L;
@@ -211,7 +212,10 @@ bool encode_row_maps(Params &p, bool bwd) {
     if (p.BT <= 0) return true;  // nothing is loaded
     return encode_rows(&p.tm_q, p.q, p.BT, p.H, p.K) && encode_rows(&p.tm_k, p.k, p.BT, p.H, p.K) &&
            encode_rows(&p.tm_v, p.v, p.BT, p.H, p.V) &&
-           (!bwd || encode_rows(&p.tm_do, p.do_, p.BT, p.H, p.V));
+           (!bwd || (encode_rows(&p.tm_do, p.do_, p.BT, p.H, p.V) &&
+                     encode_rows(&p.tm_dq, p.dq, p.BT, p.H, p.K) &&
+                     encode_rows(&p.tm_dk, p.dk, p.BT, p.H, p.K) &&
+                     encode_rows(&p.tm_dv, p.dv, p.BT, p.H, p.V)));
 }
 
 // Workspace layout.  The SIMT path (fp32) keeps fp32 per-(chunk, head)
@@ -247,6 +251,7 @@ Layout make_layout(const Problem &pb, bool bwd) {
         }
         if (bwd) {
             L.tA = take(nch * kChunk * kChunk * 2);  // bf16 tile image of A
+            L.tB = take(nch * kChunk * f);
             L.tQg = take(nch * img64);
             L.tdUL = take(nch * img64);
             L.tdSn = take(nch * img128);

@@ -60,6 +60,7 @@ struct Params {
     void *tS, *tUT;                // 128x128 image of the state entering the chunk, 128x64 U^T image
     void *tQg, *tdUL, *tdSn, *tdUT;  // backward: scaled-q image, local dU^T, dS image, dU^T image
     float *tG;                     // 64 cumulative gates per (chunk, head)
+    float *tB;                     // 64 write strengths per (chunk, head), 0 past its end
     void *tA;                      // 64x64 bf16 tile image of A (backward)
     // piece scan of long rows (forward): pieces per sequence, chunks per piece, and per
     // (sequence, head, piece) the entering state, the composed transition and offset
@@ -68,7 +69,7 @@ struct Params {
     // tensor maps of the bf16 [tokens][H][d] inputs for the tensor-core path: a box is 64
     // tokens x 64 elements of one head, written to shared memory with the operand tiles'
     // 128-byte swizzle (encoded on the host for every call)
-    CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv;
 };
 
 // Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).
@@ -119,7 +120,7 @@ struct Problem {
 struct Layout {
     size_t chunks, seq_first;
     size_t W, Ut, A, U, Hs, dUloc, dU, dHn, scratch;
-    size_t tW, tUt, tKd, tS, tUT, tQg, tdUL, tdSn, tdUT, tG, tA, tHin, tMp, tBp;
+    size_t tW, tUt, tKd, tS, tUT, tQg, tdUL, tdSn, tdUT, tG, tB, tA, tHin, tMp, tBp;
     size_t qn, kn, qinv, kinv;  // normalised q, k copies and 1/|row| (passes of the fp32 path)
     size_t total;
 };
@@ -139,7 +140,8 @@ cudaError_t launch_l2norm_back(const void *xn, const float *inv, void *dx, int64
                                bool bf16, cudaStream_t stream);
 bool tc_bwd_ready();
 cudaError_t launch_tc_fwd(const Params &p, const Problem &pb, cudaStream_t stream);
-// Encodes p.tm_q, tm_k, tm_v (and tm_do for the backward) from p.q, p.k, p.v, p.do_.
+// Encodes p.tm_q, tm_k, tm_v (and tm_do, tm_dq, tm_dk, tm_dv for the backward) from
+// p.q, p.k, p.v, p.do_, p.dq, p.dk, p.dv.
 bool encode_row_maps(Params &p, bool bwd);
 cudaError_t launch_tc_bwd(const Params &p, const Problem &pb, cudaStream_t stream);
 

@@ -13,7 +13,11 @@
 //                 and writes dS (the gradient of the state leaving the chunk)
 //                 and dU^T as tile images
 //   tc_grads      chunk-parallel: every chunk-local gradient (dq, dk, dv, dg,
-//                 dbeta) from the recomputed and propagated pieces.
+//                 dbeta) from the recomputed and propagated pieces; one
+//                 persistent CTA per SM walks its (chunk, head) units and
+//                 fetches each input group of the next unit into the buffers
+//                 the current one has finished with, so the copies run under
+//                 the compute; dq, dk, dv leave by tensor-map stores.
 //
 // Products run in transposed form wherever that lets the accumulator use all
 // 128 TMEM lanes (M = 128 over the key or value dim); 64 x 64 products use the
@@ -339,20 +343,14 @@ constexpr int NG = 512;
 constexpr int CW = 16;  // columns per warpgroup
 
 struct GradSmem {
-    static constexpr int kQK = 0, kDO = 32768, kV = 49152, kSC = 65536, kDSN = 98304,
-                         kUT = 131072, kDUT = 147456, kAB = 163840, kX3 = 172032,
-                         kDA = 188416, kT1 = 196608, kDPG = 204800, kDLG = 212992,
-                         kVec = 221184, kEnd = kVec + 24 * 256;
-    // reused once the first products have consumed the images there: fp32
-    // 64 x 65 P (then dP.P + dL.L) and Gam.KK^T, per-warp partial column sums
-    // [3][4][64], and the 64 x 64 decay matrix Gam (columns xor-swizzled by row)
-    static constexpr int kPE = kSC, kKKG = kSC + 64 * 65 * 4, kRed = kDSN + 1024,
-                         kGam = kDUT;
+    // q rows 0-63 and k rows 64-127 form one 128-row tile, dO and v another
+    static constexpr int kQK = 0, kDV = 32768, kSC = 65536, kDSN = 98304, kUT = 131072,
+                         kDUT = 147456, kAB = 163840, kX3 = 172032, kDA = 188416,
+                         kT1 = 196608, kDPG = 204800, kDLG = 212992, kVec = 221184,
+                         kVecFloats = 2432, kEnd = kVec + kVecFloats * 4;
 };
 constexpr int kGradSmem = GradSmem::kEnd + 1024;
-constexpr int LP = 65;  // padded row stride (floats) of the fp32 scratch
-
-__device__ __forceinline__ int gidx(int i, int j) { return i * 64 + (j ^ (i & 31)); }
+static_assert(GradSmem::kT1 == GradSmem::kDA + C * 128, "[dA; T1] is one 128-row operand tile");
 
 // Column c of an SW128 tile with R rows, read row by row: the swizzle term
 // depends on the row only through row % 8, so it is computed once.
@@ -372,19 +370,108 @@ struct ColSw {
     }
 };
 
-// Copies rows [0, len) and columns [0, width) of a 64 x 128 bf16 staging tile
-// (plain rows) to one chunk and head of a [tokens][H][width] tensor with
-// 16-byte stores.
-__device__ __forceinline__ void store_rows(bf16 *dst, const uint8_t *stage, int64_t tok0, int len,
-                                           int h, int H, int width) {
+// Writes this thread's column (tokens cb + q, column `col`) into a 64-row SW128
+// bf16 tile (the layout of the row loads and stores).
+__device__ __forceinline__ void stage_col(uint8_t *tile, const float *x, int cb, int col) {
+    uint8_t *c0 = tile + (col >> 6) * C * 128 + (col & 7) * 2;
+    const int cp = (col & 63) >> 3;
+#pragma unroll
+    for (int q = 0; q < CW; ++q)  // row cb + q, whose swizzle term is q % 8 (cb is a multiple of 8)
+        *reinterpret_cast<bf16 *>(c0 + (cb + q) * 128 + ((cp ^ (q & 7)) << 4)) =
+            __float2bfloat16_rn(x[q]);
+}
+
+// Stores rows [0, len) and columns [0, width) of a staged 64-row SW128 tile to
+// one chunk and head of a [tokens][H][width] bf16 tensor.  A full chunk goes
+// out by tensor-map stores (one box per 64 columns) issued by thread 0 (which
+// must wait for their reads before the tile is rewritten); a shorter chunk by
+// 16-byte stores of every thread, so that no row past its end is written.  The
+// staged rows must have been fenced for the async proxy and published by a
+// barrier.
+__device__ __forceinline__ void store_tile(const CUtensorMap *map, bf16 *dst, const uint8_t *tile,
+                                           int64_t tok0, int len, int h, int H, int width) {
+    if (len == C) {
+        if (threadIdx.x == 0) {
+            tma_store_3d(map, 0, h, (int)tok0, smem_u32(tile));
+            if (width == D) tma_store_3d(map, 64, h, (int)tok0, smem_u32(tile) + C * 128);
+            bulk_commit();
+        }
+        return;
+    }
     for (int t = threadIdx.x; t < C * 16; t += NG) {
         const int i = t >> 4, j = t & 15;
         if (i < len && j * 8 < width)
             *reinterpret_cast<uint4 *>(dst + ((tok0 + i) * H + h) * width + j * 8) =
-                *reinterpret_cast<const uint4 *>(stage + i * 256 + j * 16);
+                *reinterpret_cast<const uint4 *>(tile + sw128_chunk(C, i, j));
     }
 }
 
+// Input groups of one tc_grads unit, each completing on its own mbarrier (bit b
+// of a mask is group b): the state images with G and b, the dO and v rows, A,
+// and the q and k rows.
+enum : uint32_t { kGrpImg = 1, kGrpDV = 2, kGrpA = 4, kGrpQK = 8, kGrpAll = 15 };
+constexpr int kGrpCount = 4;
+
+// Issues (one thread) the copies of the groups in `mask` for unit u, whose
+// chunk is cn; G and b land in [G | b] slot `gslot` of the vector area.
+__device__ __forceinline__ void grads_fetch(const Params &p, uint8_t *sm, int u,
+                                            const ChunkInfo &cn, uint32_t mask, int gslot,
+                                            uint64_t *bars) {
+    using S_ = GradSmem;
+    constexpr uint32_t kImgA = C * C * 2;
+    const int h = u % p.H;
+    if (mask & kGrpImg) {
+        uint64_t *bar = &bars[0];
+        mbar_arrive_expect_tx(bar, 2 * kImg128 + 2 * kImgUT + 2 * C * 4);
+        bulk_load(smem_u32(sm + S_::kSC), static_cast<const uint8_t *>(p.tS) + (size_t)u * kImg128,
+                  kImg128, bar);
+        bulk_load(smem_u32(sm + S_::kDSN),
+                  static_cast<const uint8_t *>(p.tdSn) + (size_t)u * kImg128, kImg128, bar);
+        bulk_load(smem_u32(sm + S_::kUT), static_cast<const uint8_t *>(p.tUT) + (size_t)u * kImgUT,
+                  kImgUT, bar);
+        bulk_load(smem_u32(sm + S_::kDUT),
+                  static_cast<const uint8_t *>(p.tdUT) + (size_t)u * kImgUT, kImgUT, bar);
+        float *gb = reinterpret_cast<float *>(sm + S_::kVec) + gslot * 128;
+        bulk_load(smem_u32(gb), p.tG + (size_t)u * C, C * 4, bar);
+        bulk_load(smem_u32(gb + C), p.tB + (size_t)u * C, C * 4, bar);
+    }
+    if (mask & kGrpDV) {
+        uint64_t *bar = &bars[1];
+        mbar_arrive_expect_tx(bar, 2 * row_tile_bytes(p.V));
+        load_rows_tma(sm + S_::kDV, D, 0, &p.tm_do, cn.tok0, h, p.V, bar);
+        load_rows_tma(sm + S_::kDV, D, C, &p.tm_v, cn.tok0, h, p.V, bar);
+    }
+    if (mask & kGrpA) {
+        uint64_t *bar = &bars[2];
+        mbar_arrive_expect_tx(bar, kImgA);
+        bulk_load(smem_u32(sm + S_::kAB), static_cast<const uint8_t *>(p.tA) + (size_t)u * kImgA,
+                  kImgA, bar);
+    }
+    if (mask & kGrpQK) {
+        uint64_t *bar = &bars[3];
+        mbar_arrive_expect_tx(bar, 2 * row_tile_bytes(p.K));
+        load_rows_tma(sm + S_::kQK, D, 0, &p.tm_q, cn.tok0, h, p.K, bar);
+        load_rows_tma(sm + S_::kQK, D, C, &p.tm_k, cn.tok0, h, p.K, bar);
+    }
+}
+
+// Bounded wait of the whole CTA for the groups in `mask` to complete phase
+// `parity`; records `where` on failure.
+__device__ __forceinline__ bool groups_arrived(uint64_t *bars, uint32_t mask, uint32_t parity,
+                                               const Params &p, int where) {
+    bool ok = true;
+    for (int g = 0; g < kGrpCount; ++g)
+        if ((mask >> g) & 1) ok = ok && mbar_wait(&bars[g], parity, kWaitLimit);
+    const bool all = __syncthreads_and(ok);
+    if (!all && threadIdx.x == 0) record_timeout(p, where);
+    return all;
+}
+
+// After a failed wait: one more bounded wait for the groups still in flight.
+__device__ __forceinline__ void groups_drain(uint64_t *bars, uint32_t mask, uint32_t parity) {
+    for (int g = 0; g < kGrpCount; ++g)
+        if ((mask >> g) & 1) mbar_wait(&bars[g], parity, kWaitLimit);
+}
 
 // Column sums over the 32 lanes of a warp of the CW = 16 values v[q] that each
 // thread holds (lane l of the warp is row l of a 32-row slice; v[q] belongs to
@@ -452,398 +539,400 @@ __device__ __forceinline__ void ldcw(uint32_t tmem, int col, float *d) {
 __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
+    // MMA completions: mbar_a the first two products (X3, A^T dU), mbar_z Y2 and
+    // Zp, mbar the others in order (one phase in flight on each)
+    __shared__ uint64_t mbar, mbar_a, mbar_z, lbar[kGrpCount];
     __shared__ uint32_t tslot;
     __shared__ float s_hd;
     if (p.hdr->status) return;
-    const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
-    const int wg = tid >> 7, r = tid & 127, cb = CW * wg;
-    const int l = tid & 31, i64 = l < 16 ? ((tid >> 5) & 3) * 16 + l : -1;  // M = 64 row
-    const ChunkInfo ci = chunk_at(p, c);
+    const int H = p.H, nunits = p.NC * H, tid = threadIdx.x;
+    const int wg = tid >> 7, r = tid & 127, cb = CW * wg, l = tid & 31, w4 = (tid >> 5) & 3;
+    const int i64 = l < 16 ? w4 * 16 + l : -1;  // M = 64 row of this thread's lane
     using S_ = GradSmem;
-    uint8_t *QK = sm + S_::kQK, *DO = sm + S_::kDO, *VT = sm + S_::kV, *SC = sm + S_::kSC,
-            *DSN = sm + S_::kDSN, *UT = sm + S_::kUT, *DUT = sm + S_::kDUT, *AB = sm + S_::kAB,
+    uint8_t *QK = sm + S_::kQK, *DV = sm + S_::kDV, *SC = sm + S_::kSC, *DSN = sm + S_::kDSN,
             *X3 = sm + S_::kX3, *DA = sm + S_::kDA, *T1 = sm + S_::kT1, *DPG = sm + S_::kDPG,
             *DLG = sm + S_::kDLG;
     float *vec = reinterpret_cast<float *>(sm + S_::kVec);
-    float *G = vec, *bta = vec + 64, *gam = vec + 128, *e = vec + 192, *dB = vec + 256,
-          *qx = vec + 320, *kx = vec + 384, *kz = vec + 448, *dG = vec + 512, *tmp = vec + 576,
-          *dbl2 = vec + 640, *qinv = vec + 896, *kinv = vec + 960, *qdot = vec + 1024,
-          *kdot = vec + 1088;
-    float *wsum = reinterpret_cast<float *>(sm + S_::kRed);  // [3][4 warps][64 columns]
-    const int w4 = (tid >> 5) & 3;
-    float *PE = reinterpret_cast<float *>(sm + S_::kPE);
-    float *KKG = reinterpret_cast<float *>(sm + S_::kKKG);
-    float *Gam = reinterpret_cast<float *>(sm + S_::kGam);
-
-    __shared__ uint64_t lbar;
-    constexpr uint32_t kImgA = C * C * 2;
-    if (tid == 0) {  // the tile images and A by bulk copies (one instruction each)
-        mbar_init(&lbar, 1);
-        fence_mbar_init();
-        mbar_arrive_expect_tx(&lbar, 2 * kImg128 + 2 * kImgUT + kImgA + 2 * row_tile_bytes(p.K) +
-                                         2 * row_tile_bytes(p.V));
-        bulk_load(smem_u32(SC), static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128,
-                  kImg128, &lbar);
-        bulk_load(smem_u32(DSN), static_cast<const uint8_t *>(p.tdSn) + (size_t)ch * kImg128,
-                  kImg128, &lbar);
-        bulk_load(smem_u32(UT), static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT, kImgUT,
-                  &lbar);
-        bulk_load(smem_u32(DUT), static_cast<const uint8_t *>(p.tdUT) + (size_t)ch * kImgUT,
-                  kImgUT, &lbar);
-        bulk_load(smem_u32(AB), static_cast<const uint8_t *>(p.tA) + (size_t)ch * kImgA, kImgA,
-                  &lbar);
-        // q, k, dO, v rows by the tensor engine
-        load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
-        load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
-        load_rows_tma(DO, C, 0, &p.tm_do, ci.tok0, h, p.V, &lbar);
-        load_rows_tma(VT, C, 0, &p.tm_v, ci.tok0, h, p.V, &lbar);
-    }
-    if (tid < C) {
-        const int64_t idx = (int64_t)(ci.tok0 + tid) * H + h;
-        G[tid] = p.tG[(size_t)ch * C + tid];
-        bta[tid] = tid < ci.len ? p.beta[idx] : 0.f;
-    }
+    // vec + 0: two [G | b] slots of 128 floats, the current unit's and the prefetched one's
+    float *gam = vec + 256, *e = vec + 320, *dB = vec + 384, *qx = vec + 448, *kx = vec + 512,
+          *kz = vec + 576, *dG = vec + 640, *tmp = vec + 704, *dbl2 = vec + 768,
+          *qinv = vec + 1024, *kinv = vec + 1088, *rowp = vec + 1152;
+    // per-warp partial column sums, four sets of [4 warps][64 columns]
+    float *wsum = vec + 1408;
+    float *qdot = rowp, *kdot = rowp + 64;  // (the row partials are consumed before the epilogue)
+    const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128, dvb = smem_u32(DV), vb = dvb + C * 128,
+                   scb = smem_u32(SC), dsb = smem_u32(DSN), utb = smem_u32(sm + S_::kUT),
+                   dub = smem_u32(sm + S_::kDUT), ab = smem_u32(sm + S_::kAB),
+                   x3b = smem_u32(X3), dab = smem_u32(DA), dpb = smem_u32(DPG),
+                   dlb = smem_u32(DLG);
     if (tid == 0) {
+        for (int g = 0; g < kGrpCount; ++g) mbar_init(&lbar[g], 1);
         mbar_init(&mbar, 1);
+        mbar_init(&mbar_a, 1);
+        mbar_init(&mbar_z, 1);
         fence_mbar_init();
     }
     if (tid < 32) {
         tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
-    __syncthreads();
-    if (tid < C) {
-        gam[tid] = expf(G[tid]);
-        e[tid] = expf(G[C - 1] - G[tid]);
-    }
-    if (!copies_arrived(&lbar, p, 20)) {  // (the barrier above published the inits)
-        tc_fence_before();
-        __syncthreads();
-        if (tid < 32) tmem_dealloc(tslot, 512);
-        return;
-    }
-    fix_rows(QK, D, 0, ci.len, p.K, NG);
-    fix_rows(QK, D, C, ci.len, p.K, NG);
-    fix_rows(DO, C, 0, ci.len, p.V, NG);
-    fix_rows(VT, C, 0, ci.len, p.V, NG);
-    operands_ready();
-    if (p.l2norm) {  // q rows (threads 0-127) and k rows (128-255) divided by their norms
-        l2norm_tile_rows(QK, D, 0, qinv, 0);
-        l2norm_tile_rows(QK, D, C, kinv, 2 * C);
-        operands_ready();
-    }
+    __syncthreads();  // publishes the mbarrier inits and the TMEM address
     const uint32_t tmem = tslot;
-    const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128, dob = smem_u32(DO), vb = smem_u32(VT),
-                   scb = smem_u32(SC), dsb = smem_u32(DSN), utb = smem_u32(UT),
-                   dub = smem_u32(DUT), ab = smem_u32(AB), x3b = smem_u32(X3), dab = smem_u32(DA),
-                   t1b = smem_u32(T1), dpb = smem_u32(DPG), dlb = smem_u32(DLG);
-    // TMEM columns
-    // (Y2 takes X3's columns once X3 is read, T1 then Y2's; dL takes Q K^T's once P is formed)
-    constexpr int cQK = 0, cX1 = 64, cX2 = 128, cX3 = 192, cDP = 256, cAU = 320, cY1 = 384,
-                  cY2 = 192, cZ = 448, cT1 = 192, cDL = 0, cDQ = 256, cDK = 320, cDKA = 384;
-    uint32_t phase = 0;
-    bool ok;
-    float d[CW];
-    if (tid == 0) {
-        const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
-                       i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
-                       i64km = idesc_bf16(64, 64, 0, 1), i64mk = idesc_bf16(64, 64, 1, 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
-            mma_bf16(tmem + cQK, desc_kmajor(qkb, D, s), desc_kmajor(kb, D, s), i128, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // X1^T = S^T dO^T  (over v)
-            mma_bf16(tmem + cX1, desc_mnmajor(scb, D, s), desc_kmajor(dob, C, s), i128mk, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // X2^T = dSn^T U^T
-            mma_bf16(tmem + cX2, desc_mnmajor(dsb, D, s), desc_mnmajor(utb, D, s), i128mm, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // X3^T = S^T dU^T
-            mma_bf16(tmem + cX3, desc_mnmajor(scb, D, s), desc_mnmajor(dub, D, s), i128mm, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // dP = dO U^T (M = 64)
-            mma_bf16(tmem + cDP, desc_kmajor(dob, C, s), desc_mnmajor(utb, D, s), i64km, s > 0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // (A^T dU)^T = dU^T A
-            mma_bf16(tmem + cAU, desc_kmajor(dub, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // Y1 = dU V^T (M = 64)
-            mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, C, s), i64mk, s > 0);
-        mma_commit(&mbar);
+    // The CTA runs units (chunk, head) blockIdx.x, + gridDim.x, ...  Each input
+    // group of the next unit is fetched as soon as the current unit has
+    // consumed that group's buffers, so the copies run under the compute.
+    int unit = blockIdx.x;
+    if (tid == 0 && unit < nunits) {
+        const ChunkInfo cn = chunk_at(p, unit / H);
+        grads_fetch(p, sm, unit, cn, kGrpAll, 0, lbar);
     }
-    {  // <S, dSn> (elementwise over identically laid out images) while the products run
-        float s = 0.f;
-        for (int t = tid; t < D * D / 8; t += NG) {
-            float a[8], b[8];
-            unpack8(*reinterpret_cast<const uint4 *>(SC + t * 16), a);
-            unpack8(*reinterpret_cast<const uint4 *>(DSN + t * 16), b);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) s = fmaf(a[q], b[q], s);
+    uint32_t pend = kGrpAll, ppar = 0;  // load groups in flight and the phase they complete
+    uint32_t phase = 0;                 // MMA-completion barrier
+    bool ok = true;
+    for (int it = 0; unit < nunits; ++it, unit += gridDim.x) {
+        const int c = unit / H, h = unit % H, next = unit + (int)gridDim.x;
+        const bool more = next < nunits;
+        const ChunkInfo ci = chunk_at(p, c);
+        const float *G = vec + (it & 1) * 128, *bta = G + 64;
+        ok = groups_arrived(lbar, pend, ppar, p, 20);
+        if (!ok) break;
+        pend = 0;
+        if (tid < C) {
+            gam[tid] = expf(G[tid]);
+            e[tid] = expf(G[C - 1] - G[tid]);
         }
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (l == 0) tmp[tid >> 5] = s;
-        __syncthreads();
-        if (tid == 0) {
-            float a = 0.f;
-            for (int w = 0; w < NG / 32; ++w) a += tmp[w];
-            s_hd = a;  // read after the barrier of the wait below
+        fix_rows(QK, D, 0, ci.len, p.K, NG);
+        fix_rows(QK, D, C, ci.len, p.K, NG);
+        fix_rows(DV, D, 0, ci.len, p.V, NG);
+        fix_rows(DV, D, C, ci.len, p.V, NG);
+        operands_ready();
+        if (p.l2norm) {  // q rows (threads 0-127) and k rows (128-255) divided by their norms
+            l2norm_tile_rows(QK, D, 0, qinv, 0);
+            l2norm_tile_rows(QK, D, C, kinv, 2 * C);
+            operands_ready();
         }
-    }
-    ok = cta_wait(&mbar, phase, p, 21);
-    phase ^= 1;
-    if (!ok) goto done;
-    // the decay matrix, once (the dU^T image there is consumed)
-    for (int t = tid; t < C * C; t += NG) {
-        const int i = t >> 6, j = t & 63;
-        Gam[gidx(i, j)] = j <= i ? expf(G[i] - G[j]) : 0.f;
-    }
-    __syncthreads();
-    ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
+        // TMEM columns.  [Q;K] K^T stays to the end (P in lanes 0-63, K K^T in lanes
+        // 64-127); Y2 takes X3's columns once X3 is read, T1 then Y2's, dL then T1's.
+        constexpr int cQK = 0, cX1 = 64, cX2 = 128, cX3 = 192, cDP = 256, cAU = 320, cY1 = 384,
+                      cY2 = 192, cZ = 448, cT1 = 192, cDL = 192, cDQ = 256, cDK = 320, cDKA = 384;
+        float d[CW];
+        if (tid == 0) {  // the products the SIMT work needs first, then the rest
+            const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
+                           i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
+                           i64mk = idesc_bf16(64, 64, 1, 0);
 #pragma unroll
-    for (int q = 0; q < CW / 8; ++q)
-        *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
-    operands_ready();
-    if (tid == 0) {  // issued now; the SIMT work below runs while they execute
-        const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1);
+            for (int s = 0; s < 8; ++s)  // X3^T = S^T dU^T
+                mma_bf16(tmem + cX3, desc_mnmajor(scb, D, s), desc_mnmajor(dub, D, s), i128mm,
+                         s > 0);
 #pragma unroll
-        for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
-            mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
+            for (int s = 0; s < 4; ++s)  // (A^T dU)^T = dU^T A
+                mma_bf16(tmem + cAU, desc_kmajor(dub, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
+            mma_commit(&mbar_a);
 #pragma unroll
-        for (int s = 0; s < 4; ++s)  // Zp^T = X3^T A   (Z = -Zp)
-            mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
-        mma_commit(&mbar);
-    }
-    // meanwhile: P, Gam . K K^T, dv and the column sums, dP
-    // P (scaled, lower incl. diagonal) and Gam . K K^T (strictly lower), fp32
-    ldcw(tmem, cQK + cb, d);
-    if (r < 64) {
+            for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
+                mma_bf16(tmem + cQK, desc_kmajor(qkb, D, s), desc_kmajor(kb, D, s), i128, s > 0);
 #pragma unroll
-        for (int q = 0; q < CW; ++q) {
-            const int j = cb + q;
-            PE[r * LP + j] = j <= r ? p.scale * Gam[gidx(r, j)] * d[q] : 0.f;
+            for (int s = 0; s < 8; ++s)  // X1^T = S^T dO^T  (over v)
+                mma_bf16(tmem + cX1, desc_mnmajor(scb, D, s), desc_kmajor(dvb, D, s), i128mk,
+                         s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // X2^T = dSn^T U^T
+                mma_bf16(tmem + cX2, desc_mnmajor(dsb, D, s), desc_mnmajor(utb, D, s), i128mm,
+                         s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // [dO; V] U^T: lanes 0-63 dP = dO U^T, next to P
+                mma_bf16(tmem + cDP, desc_kmajor(dvb, D, s), desc_mnmajor(utb, D, s), i128km,
+                         s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // Y1 = dU V^T (M = 64)
+                mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, D, s), i64mk, s > 0);
+            mma_commit(&mbar);
+        } else if (tid >= 32) {  // <S, dSn> (identically laid out images) by warps 1-15
+            float s = 0.f;
+            for (int t = tid - 32; t < D * D / 8; t += NG - 32) {
+                float a[8], b[8];
+                unpack8(*reinterpret_cast<const uint4 *>(SC + t * 16), a);
+                unpack8(*reinterpret_cast<const uint4 *>(DSN + t * 16), b);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) s = fmaf(a[q], b[q], s);
+            }
+            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (l == 0) tmp[(tid >> 5) - 1] = s;
+            bar_sync(1, NG - 32);
+            if (tid == 32) {
+                float a = 0.f;
+                for (int w = 0; w < NG / 32 - 1; ++w) a += tmp[w];
+                s_hd = a;  // read after later barriers
+            }
         }
-    } else {
-        const int i = r - 64;
-#pragma unroll
-        for (int q = 0; q < CW; ++q) {
-            const int j = cb + q;
-            KKG[i * LP + j] = j < i ? Gam[gidx(i, j)] * d[q] : 0.f;
-        }
-    }
-    {  // dv = diag(b) A^T dU (staged as rows in the consumed dO tile); partial v . (A^T dU)
-        bf16 *stage = reinterpret_cast<bf16 *>(DO);
-        const ColSw vcol(VT, C, r);
-        ldcw(tmem, cAU + cb, d);
-#pragma unroll
-        for (int q = 0; q < CW; ++q) {
-            const int i = cb + q;
-            stage[i * D + r] = __float2bfloat16_rn(bta[i] * d[q]);
-            d[q] *= vcol.at(cb, q);
-        }
-        warp_colsum(d, wsum, w4, cb, l);
-    }
-    {  // column readers of q and k are built where used (they cost 8 registers each)
-        const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
-        ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
-#pragma unroll
-        for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
-        warp_colsum(d, wsum + 256, w4, cb, l);
-        ldcw(tmem, cX2 + cb, d);  // partial k . X2
-#pragma unroll
-        for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
-        warp_colsum(d, wsum + 512, w4, cb, l);
-    }
-    __syncthreads();
-    if (tid < 3 * C) {
-        const int k = tid >> 6, i = tid & 63;
-        const float *w = wsum + k * 256 + i;
-        (k == 0 ? dB : k == 1 ? qx : kx)[i] = (w[0] + w[64]) + (w[128] + w[192]);
-    }
-    __syncthreads();
-    store_rows(static_cast<bf16 *>(p.dv), DO, ci.tok0, ci.len, h, H, p.V);
-    ldcw(tmem, cDP + cb, d);  // dP: dPG = dP . Gam as an operand tile; PE <- dP . P
-    if (i64 >= 0) {
-#pragma unroll
-        for (int q = 0; q < CW; ++q) {
-            const int j = cb + q;
-            const float dp = j <= i64 ? d[q] : 0.f;
-            PE[i64 * LP + j] *= dp;
-            d[q] = dp * Gam[gidx(i64, j)];
-        }
+        if (tid == 0) bulk_wait_read();  // the previous unit's rows staged in X3 and dA/T1 are out
+        ok = cta_wait(&mbar_a, it & 1, p, 26);
+        if (!ok) break;
+        ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
 #pragma unroll
         for (int q = 0; q < CW / 8; ++q)
-            *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
-    }
-    ok = cta_wait(&mbar, phase, p, 22);
-    phase ^= 1;
-    if (!ok) goto done;
-    {  // dA = (dU V^T) diag(b) - (X3 K^T) diag(b gam)
-        float y2[CW];
-        tmem_ld16(tmq(tmem, cY1 + cb), d);
-        tmem_ld16(tmq(tmem, cY2 + cb), y2);
-        tmem_ld_wait();
-        if (i64 >= 0) {
+            *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
+        operands_ready();
+        if (tid == 0) {  // issued now; the SIMT work below runs while they execute
+            const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
+                mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)  // Zp^T = X3^T A   (Z = -Zp)
+                mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
+            mma_commit(&mbar_z);
+        }
+        {  // dv = diag(b) A^T dU, staged in dA/T1 (thread r holds column r); partial v . (A^T dU)
+            const ColSw vcol(DV + C * 128, D, r);
+            ldcw(tmem, cAU + cb, d);
+            float y[CW];
 #pragma unroll
             for (int q = 0; q < CW; ++q) {
-                const int m = cb + q;
-                d[q] = bta[m] * d[q] - bta[m] * gam[m] * y2[q];
+                y[q] = bta[cb + q] * d[q];
+                d[q] *= vcol.at(cb, q);
+            }
+            stage_col(DA, y, cb, r);
+            warp_colsum(d, wsum, w4, cb, l);
+        }
+        ok = cta_wait(&mbar, phase, p, 21);
+        phase ^= 1;
+        if (!ok) break;
+        if (more) {  // S, dSn, U^T, dU^T, G and b of the next unit (their buffers are consumed)
+            if (tid == 0) grads_fetch(p, sm, next, ci, kGrpImg, (it + 1) & 1, lbar);
+            pend |= kGrpImg;
+            ppar = (it + 1) & 1;
+        }
+        {  // column readers of q and k are built where used (they cost 8 registers each)
+            const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
+            ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
+            warp_colsum(d, wsum + 256, w4, cb, l);
+            ldcw(tmem, cX2 + cb, d);  // partial k . X2
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
+            warp_colsum(d, wsum + 512, w4, cb, l);
+        }
+        if (w4 < 2) {  // row i = r of P and dP: P . dP (row and column partials), dPG = dP . Gam
+            float pq[CW];
+            tmem_ld16(tmq(tmem, cQK + cb), pq);
+            tmem_ld16(tmq(tmem, cDP + cb), d);
+            tmem_ld_wait();
+            const float gi = G[r];
+            float rs = 0.f;
+#pragma unroll
+            for (int q = 0; q < CW; ++q) {
+                const int j = cb + q;
+                const float gm = expf(j <= r ? gi - G[j] : -INFINITY);  // Gam (0 above diagonal)
+                const float dp = j <= r ? d[q] : 0.f;
+                pq[q] = (p.scale * gm * pq[q]) * dp;
+                rs += pq[q];
+                d[q] = dp * gm;
+            }
+            rowp[wg * 64 + r] = rs;
+#pragma unroll
+            for (int q = 0; q < CW / 8; ++q)
+                *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, r, cb / 8 + q)) = pack8(d + 8 * q);
+            warp_colsum(pq, wsum + 768, w4, cb, l);
+        }
+        fence_async_smem();  // the staged dv rows leave by bulk copies
+        __syncthreads();
+        if (more) {  // dO and v rows of the next unit (read by the first products and the dv sums)
+            if (tid == 0) grads_fetch(p, sm, next, chunk_at(p, next / H), kGrpDV, 0, lbar);
+            pend |= kGrpDV;
+        }
+        store_tile(&p.tm_dv, static_cast<bf16 *>(p.dv), DA, ci.tok0, ci.len, h, H, p.V);
+        if (tid < 3 * C) {
+            const int k = tid >> 6, i = tid & 63;
+            const float *w = wsum + k * 256 + i;
+            (k == 0 ? dB : k == 1 ? qx : kx)[i] = (w[0] + w[64]) + (w[128] + w[192]);
+        }
+        if (tid == 0) bulk_wait_read();  // dA/T1 are written next
+        ok = cta_wait(&mbar_z, it & 1, p, 22);
+        if (!ok) break;
+        {  // dA = (dU V^T) diag(b) - (X3 K^T) diag(b gam)
+            float y2[CW];
+            tmem_ld16(tmq(tmem, cY1 + cb), d);
+            tmem_ld16(tmq(tmem, cY2 + cb), y2);
+            tmem_ld_wait();
+            if (i64 >= 0) {
+#pragma unroll
+                for (int q = 0; q < CW; ++q) {
+                    const int m = cb + q;
+                    d[q] = bta[m] * d[q] - bta[m] * gam[m] * y2[q];
+                }
+#pragma unroll
+                for (int q = 0; q < CW / 8; ++q)
+                    *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i64, cb / 8 + q)) =
+                        pack8(d + 8 * q);
+            }
+        }
+        operands_ready();
+        if (tid == 0) {  // T1 = A^T dA (M = 64)
+            const uint32_t id = idesc_bf16(64, 64, 1, 1);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + cT1, desc_mnmajor(ab, C, s), desc_mnmajor(dab, C, s), id, s > 0);
+            mma_commit(&mbar);
+        }
+        // meanwhile: k . Z
+        {
+            const ColSw kcol(QK + C * 128, D, r);
+            ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
+            warp_colsum(d, wsum, w4, cb, l);
+        }
+        __syncthreads();
+        if (tid < C) kz[tid] = (wsum[tid] + wsum[64 + tid]) + (wsum[128 + tid] + wsum[192 + tid]);
+        ok = cta_wait(&mbar, phase, p, 23);
+        phase ^= 1;
+        if (!ok) break;
+        ldcw(tmem, cT1 + cb, d);
+        if (i64 >= 0) {
+#pragma unroll
+            for (int q = 0; q < CW / 8; ++q)
+                *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
+        }
+        operands_ready();
+        if (tid == 0) {  // [dA; T1] A^T (M = 128): lanes 64-127 hold T1 A^T = -dL, next to K K^T
+            const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + cDL, desc_kmajor(dab, D, s), desc_kmajor(ab, C, s), id, s > 0);
+            mma_commit(&mbar);
+        }
+        ok = cta_wait(&mbar, phase, p, 24);
+        phase ^= 1;
+        if (!ok) break;
+        if (more) {  // A of the next unit (its last product is done)
+            if (tid == 0) grads_fetch(p, sm, next, ci, kGrpA, 0, lbar);
+            pend |= kGrpA;
+        }
+        if (w4 >= 2) {  // row i = r - 64: dL (strictly lower), Gam . K K^T; dLG = diag(b) dL . Gam
+            const int i = r - C;
+            float kk[CW];
+            tmem_ld16(tmq(tmem, cQK + cb), kk);
+            tmem_ld16(tmq(tmem, cDL + cb), d);
+            tmem_ld_wait();
+            const float bi = bta[i], gi = G[i];
+            float dbl = 0.f;
+#pragma unroll
+            for (int q = 0; q < CW; ++q) {
+                const int j = cb + q;
+                const float gm = expf(j < i ? gi - G[j] : -INFINITY);
+                const float dl = j < i ? -d[q] : 0.f;
+                const float kkg = gm * kk[q];
+                kk[q] = dl * bi * kkg;
+                dbl = fmaf(dl, kkg, dbl);
+                d[q] = bi * dl * gm;
             }
 #pragma unroll
             for (int q = 0; q < CW / 8; ++q)
-                *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
+                *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i, cb / 8 + q)) = pack8(d + 8 * q);
+            dbl2[wg * 64 + i] = dbl;
+            warp_colsum(kk, wsum + 768, w4, cb, l);
         }
-    }
-    operands_ready();
-    if (tid == 0) {  // T1 = A^T dA (M = 64)
-        const uint32_t id = idesc_bf16(64, 64, 1, 1);
+        operands_ready();
+        if (tid == 0) {
+            const uint32_t imk = idesc_bf16(128, 64, 1, 0), imm = idesc_bf16(128, 64, 1, 1);
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            mma_bf16(tmem + cT1, desc_mnmajor(ab, C, s), desc_mnmajor(dab, C, s), id, s > 0);
-        mma_commit(&mbar);
-    }
-    // meanwhile: k . Z
-    {
-        const ColSw kcol(QK + C * 128, D, r);
-        ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
+            for (int s = 0; s < 4; ++s)  // (dPG K)^T = K^T dPG^T
+                mma_bf16(tmem + cDQ, desc_mnmajor(kb, D, s), desc_kmajor(dpb, C, s), imk, s > 0);
 #pragma unroll
-        for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
-        warp_colsum(d, wsum, w4, cb, l);
-    }
-    __syncthreads();
-    if (tid < C) kz[tid] = (wsum[tid] + wsum[64 + tid]) + (wsum[128 + tid] + wsum[192 + tid]);
-    ok = cta_wait(&mbar, phase, p, 23);
-    phase ^= 1;
-    if (!ok) goto done;
-    ldcw(tmem, cT1 + cb, d);
-    if (i64 >= 0) {
+            for (int s = 0; s < 4; ++s)  // (dPG^T Q)^T = Q^T dPG
+                mma_bf16(tmem + cDKA, desc_mnmajor(qkb, D, s), desc_mnmajor(dpb, C, s), imm, s > 0);
 #pragma unroll
-        for (int q = 0; q < CW / 8; ++q)
-            *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
-    }
-    operands_ready();
-    if (tid == 0) {  // T1 A^T = -dL (M = 64)
-        const uint32_t id = idesc_bf16(64, 64, 0, 0);
+            for (int s = 0; s < 4; ++s)  // (diag(b) dLG K)^T
+                mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_kmajor(dlb, C, s), imk, s > 0);
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            mma_bf16(tmem + cDL, desc_kmajor(t1b, C, s), desc_kmajor(ab, C, s), id, s > 0);
-        mma_commit(&mbar);
-    }
-    ok = cta_wait(&mbar, phase, p, 24);
-    phase ^= 1;
-    if (!ok) goto done;
-    ldcw(tmem, cDL + cb, d);  // dL (strictly lower); diag(b) dL . Gam tile; PE += dL . L
-    if (i64 >= 0) {
-        float dbl = 0.f;
-        const float bi = bta[i64];
-#pragma unroll
-        for (int q = 0; q < CW; ++q) {
-            const int j = cb + q;
-            const float dl = j < i64 ? -d[q] : 0.f;
-            const float kkg = KKG[i64 * LP + j];
-            PE[i64 * LP + j] += dl * bi * kkg;
-            dbl = fmaf(dl, kkg, dbl);
-            d[q] = bi * dl * Gam[gidx(i64, j)];
+            for (int s = 0; s < 4; ++s)  // ((diag(b) dLG)^T K)^T
+                mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_mnmajor(dlb, C, s), imm, 1);
+            mma_commit(&mbar);
         }
-#pragma unroll
-        for (int q = 0; q < CW / 8; ++q)
-            *reinterpret_cast<uint4 *>(DLG + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
-        dbl2[wg * 64 + i64] = dbl;
-    }
-    operands_ready();
-    if (tid == 0) {
-        const uint32_t imk = idesc_bf16(128, 64, 1, 0), imm = idesc_bf16(128, 64, 1, 1);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // (dPG K)^T = K^T dPG^T
-            mma_bf16(tmem + cDQ, desc_mnmajor(kb, D, s), desc_kmajor(dpb, C, s), imk, s > 0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // (dPG^T Q)^T = Q^T dPG
-            mma_bf16(tmem + cDKA, desc_mnmajor(qkb, D, s), desc_mnmajor(dpb, C, s), imm, s > 0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // (diag(b) dLG K)^T
-            mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_kmajor(dlb, C, s), imk, s > 0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // ((diag(b) dLG)^T K)^T
-            mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_mnmajor(dlb, C, s), imm, 1);
-        mma_commit(&mbar);
-    }
-    // meanwhile: dbeta and dG (rows), then dg = reverse cumulative sum of dG
-    {  // row and column sums of PE: eight threads per token, eight entries each
-        const int i = tid >> 3, part = tid & 7;
-        float rs = 0.f, cs = 0.f;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            rs += PE[i * LP + part * 8 + t];
-            cs += PE[(part * 8 + t) * LP + i];
+        // meanwhile: dbeta and dG (rows), then dg = reverse cumulative sum of dG.  The
+        // row sums of P . dP + dL . L are the row partials plus b times the dL rows'
+        // sums; the column sums come from the last set of warp partials.
+        if (tid < C) {
+            const int i = tid;
+            const float *w = wsum + 768 + i;
+            const float dbs = (dbl2[i] + dbl2[64 + i]) + (dbl2[128 + i] + dbl2[192 + i]);
+            const float rsum = ((rowp[i] + rowp[64 + i]) + (rowp[128 + i] + rowp[192 + i])) +
+                               bta[i] * dbs;
+            const float csum = (w[0] + w[64]) + (w[128] + w[192]);
+            dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + (rsum - csum) + bta[i] * gam[i] * kz[i];
+            dB[i] += dbs + gam[i] * kz[i];
         }
-        float x = rs - cs;
-#pragma unroll
-        for (int off = 1; off < 8; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-        if (part == 0) {
-            dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + x + bta[i] * gam[i] * kz[i];
-            dB[i] += (dbl2[i] + dbl2[64 + i]) + (dbl2[128 + i] + dbl2[192 + i]) + gam[i] * kz[i];
-        }
-    }
-    __syncthreads();
-    if (tid < 32) {  // dg = reverse cumulative sum of dG (+ the terms of the last token)
-        const float a = dG[2 * l], b = dG[2 * l + 1];
-        float s = e[2 * l] * kx[2 * l] + e[2 * l + 1] * kx[2 * l + 1];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        const float extra = gam[C - 1] * s_hd + s;
-        float x = a + b;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float t = __shfl_down_sync(0xffffffffu, x, off);
-            if (l + off < 32) x += t;
-        }
-        const int i0 = 2 * l;
-        if (i0 < ci.len) {
-            const int64_t o = (int64_t)(ci.tok0 + i0) * H + h;
-            p.dg[o] = x + extra;
-            p.dbeta[o] = dB[i0];
-        }
-        if (i0 + 1 < ci.len) {
-            const int64_t o = (int64_t)(ci.tok0 + i0 + 1) * H + h;
-            p.dg[o] = (x - a) + extra;
-            p.dbeta[o] = dB[i0 + 1];
-        }
-    }
-    ok = cta_wait(&mbar, phase, p, 25);
-    phase ^= 1;
-    if (!ok) goto done;
-    {  // dq = scale (diag(gam) X1 + dPG K) ; dk = diag(e) X2 + diag(b gam) Z + dPG^T Q' + dL terms
-        // staged as rows in the consumed dO and V tiles, then 16-byte stores
-        bf16 *sq = reinterpret_cast<bf16 *>(DO), *sk = reinterpret_cast<bf16 *>(VT);
-        const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
-        float a[CW];
-        tmem_ld16(tmq(tmem, cX1 + cb), d);
-        tmem_ld16(tmq(tmem, cDQ + cb), a);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < CW; ++q) d[q] = p.scale * (gam[cb + q] * d[q] + a[q]);
-        if (p.l2norm) project_rows(d, qcol, qinv, qdot, wsum, w4, cb, l);
-#pragma unroll
-        for (int q = 0; q < CW; ++q) sq[(cb + q) * D + r] = __float2bfloat16_rn(d[q]);
-        tmem_ld16(tmq(tmem, cX2 + cb), d);
-        tmem_ld16(tmq(tmem, cZ + cb), a);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < CW; ++q) d[q] = e[cb + q] * d[q] - bta[cb + q] * gam[cb + q] * a[q];
-        ldcw(tmem, cDKA + cb, a);
-#pragma unroll
-        for (int q = 0; q < CW; ++q) d[q] += p.scale * a[q];
-        ldcw(tmem, cDK + cb, a);
-#pragma unroll
-        for (int q = 0; q < CW; ++q) d[q] += a[q];
-        if (p.l2norm) project_rows(d, kcol, kinv, kdot, wsum + 256, w4, cb, l);
-#pragma unroll
-        for (int q = 0; q < CW; ++q) sk[(cb + q) * D + r] = __float2bfloat16_rn(d[q]);
         __syncthreads();
-        store_rows(static_cast<bf16 *>(p.dq), DO, ci.tok0, ci.len, h, H, p.K);
-        store_rows(static_cast<bf16 *>(p.dk), VT, ci.tok0, ci.len, h, H, p.K);
+        if (tid < 32) {  // dg = reverse cumulative sum of dG (+ the terms of the last token)
+            const float a = dG[2 * l], b = dG[2 * l + 1];
+            float s = e[2 * l] * kx[2 * l] + e[2 * l + 1] * kx[2 * l + 1];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            const float extra = gam[C - 1] * s_hd + s;
+            float x = a + b;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float t = __shfl_down_sync(0xffffffffu, x, off);
+                if (l + off < 32) x += t;
+            }
+            const int i0 = 2 * l;
+            if (i0 < ci.len) {
+                const int64_t o = (int64_t)(ci.tok0 + i0) * H + h;
+                p.dg[o] = x + extra;
+                p.dbeta[o] = dB[i0];
+            }
+            if (i0 + 1 < ci.len) {
+                const int64_t o = (int64_t)(ci.tok0 + i0 + 1) * H + h;
+                p.dg[o] = (x - a) + extra;
+                p.dbeta[o] = dB[i0 + 1];
+            }
+        }
+        ok = cta_wait(&mbar, phase, p, 25);
+        phase ^= 1;
+        if (!ok) break;
+        if (more && !p.l2norm) {  // q and k rows of the next unit (the epilogue reads only TMEM)
+            if (tid == 0) grads_fetch(p, sm, next, chunk_at(p, next / H), kGrpQK, 0, lbar);
+            pend |= kGrpQK;
+        }
+        {  // dq = scale (diag(gam) X1 + dPG K); dk = diag(e) X2 + diag(b gam) Z + dPG^T Q'
+           // + dL terms; staged (thread r holds column r): dq in X3, dk in dA/T1
+            float a[CW];
+            tmem_ld16(tmq(tmem, cX1 + cb), d);
+            tmem_ld16(tmq(tmem, cDQ + cb), a);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] = p.scale * (gam[cb + q] * d[q] + a[q]);
+            if (p.l2norm) project_rows(d, ColSw(QK, D, r), qinv, qdot, wsum, w4, cb, l);
+            stage_col(X3, d, cb, r);
+            tmem_ld16(tmq(tmem, cX2 + cb), d);
+            tmem_ld16(tmq(tmem, cZ + cb), a);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] = e[cb + q] * d[q] - bta[cb + q] * gam[cb + q] * a[q];
+            ldcw(tmem, cDKA + cb, a);
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] += p.scale * a[q];
+            ldcw(tmem, cDK + cb, a);
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] += a[q];
+            if (p.l2norm)
+                project_rows(d, ColSw(QK + C * 128, D, r), kinv, kdot, wsum + 256, w4, cb, l);
+            stage_col(DA, d, cb, r);
+        }
+        fence_async_smem();
+        __syncthreads();  // the unit's reads are done and the staged rows are visible
+        if (more && p.l2norm) {
+            if (tid == 0) grads_fetch(p, sm, next, chunk_at(p, next / H), kGrpQK, 0, lbar);
+            pend |= kGrpQK;
+        }
+        store_tile(&p.tm_dq, static_cast<bf16 *>(p.dq), X3, ci.tok0, ci.len, h, H, p.K);
+        store_tile(&p.tm_dk, static_cast<bf16 *>(p.dk), DA, ci.tok0, ci.len, h, H, p.K);
+        if (ci.len < C) __syncthreads();  // (the next unit rewrites the tiles)
     }
-done:
+    if (!ok && tid == 0) groups_drain(lbar, pend, ppar);  // leave no copy in flight
+    if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (tid < 32) tmem_dealloc(tmem, 512);
@@ -869,7 +958,11 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
     }
     if (nch > 0) {
         if ((e = set_smem(tc_grads_kernel, kGradSmem))) return e;
-        GDN_LAUNCH(kKTcGrads, stream, tc_grads_kernel<<<nch, NG, kGradSmem, stream>>>(p));
+        int dev = 0, nsm = 0;  // one persistent CTA per SM (or per unit, if fewer)
+        if ((e = cudaGetDevice(&dev))) return e;
+        if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev))) return e;
+        const int grid = nch < nsm ? nch : nsm;
+        GDN_LAUNCH(kKTcGrads, stream, tc_grads_kernel<<<grid, NG, kGradSmem, stream>>>(p));
     }
     return cudaSuccess;
 }

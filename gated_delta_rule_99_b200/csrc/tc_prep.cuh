@@ -88,6 +88,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         }
         if (tid < C) {
             p.tG[(size_t)ch * C + tid] = G[tid];
+            if (p.tB) p.tB[(size_t)ch * C + tid] = bta[tid];
             F[tid] = expf(G[tid | 15] - G[tid]);
         }
     }

@@ -172,6 +172,14 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Tensor-map store of one box from shared memory at tensor coordinates
+// (x, y, z), committed with the bulk groups of the issuing thread.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, int x, int y, int z,
+                                             uint32_t ssrc) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 :: "l"(map), "r"(ssrc), "r"(x), "r"(y), "r"(z) : "memory");
+}
+
 // Bulk (async-proxy) copy shared -> global of `bytes` (multiple of 16, both 16-byte aligned).
 __device__ __forceinline__ void bulk_store(void *gdst, uint32_t ssrc, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
