@@ -28,7 +28,7 @@ namespace {
 using namespace tc;
 
 // ============================================================ tc_prep
-__global__ void __launch_bounds__(NT) tc_prep_kernel(const __grid_constant__ Params p, int want_A) {
+__global__ void __launch_bounds__(NT, 4) tc_prep_kernel(const __grid_constant__ Params p, int want_A) {
     prep_body(p, blockIdx.x, want_A);
 }
 

@@ -22,6 +22,14 @@ struct PrepSmem {
 constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
 constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 columns each)
 
+// acc += a x (four columns)
+__device__ __forceinline__ void fma4(float4 &acc, float a, const float4 x) {
+    acc.x = fmaf(a, x.x, acc.x);
+    acc.y = fmaf(a, x.y, acc.y);
+    acc.z = fmaf(a, x.z, acc.z);
+    acc.w = fmaf(a, x.w, acc.w);
+}
+
 // Body of the prep step for CTA `ch` (chunk ch / H, head ch % H).
 __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     extern __shared__ uint8_t smem_raw[];
@@ -151,56 +159,63 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             }
             __syncthreads();
         }
+        // Row blocks ib = 1..3: unit u = tid + NT n of row block ib is block j = u / 64,
+        // row r = (u / 4) % 16, columns c4 .. c4 + 3 (c4 = 4 (u % 4)); a thread forms its
+        // four columns from float4 rows (the 32 units of a warp share j, so the k loop
+        // bound is uniform; rows r of stride LS = 68 floats fall in distinct banks).
 #pragma unroll
         for (int ib = 1; ib < 4; ++ib) {
-            // elements e = tid + 128 n of the ib blocks (j, r, c) left of the diagonal
-            float t[6];
+            float4 t[2];
 #pragma unroll
-            for (int n = 0; n < 2 * ib; ++n) {
-                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            for (int n = 0; n < 2; ++n) {  // T_ij = sum_{k=j}^{ib-1} L_ik A_kj
+                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib) continue;
                 const float *Lr = L + (16 * ib + r) * LS;
-                float s0 = 0.f, s1 = 0.f;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int k = j; k < ib; ++k) {
-                    const float *Ak = L + (16 * k) * LS + 16 * j + c;
+                    const float *Ak = L + (16 * k) * LS + 16 * j + c4;
 #pragma unroll
                     for (int m = 0; m < 16; m += 4) {
                         const float4 l4 = *reinterpret_cast<const float4 *>(Lr + 16 * k + m);
-                        s0 = fmaf(l4.x, Ak[m * LS], s0);
-                        s1 = fmaf(l4.y, Ak[(m + 1) * LS], s1);
-                        s0 = fmaf(l4.z, Ak[(m + 2) * LS], s0);
-                        s1 = fmaf(l4.w, Ak[(m + 3) * LS], s1);
+                        fma4(acc, l4.x, *reinterpret_cast<const float4 *>(Ak + m * LS));
+                        fma4(acc, l4.y, *reinterpret_cast<const float4 *>(Ak + (m + 1) * LS));
+                        fma4(acc, l4.z, *reinterpret_cast<const float4 *>(Ak + (m + 2) * LS));
+                        fma4(acc, l4.w, *reinterpret_cast<const float4 *>(Ak + (m + 3) * LS));
                     }
                 }
-                t[n] = s0 + s1;
+                t[n] = acc;
             }
             __syncthreads();  // every product of this row block has read its L blocks
 #pragma unroll
-            for (int n = 0; n < 2 * ib; ++n) {
-                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                L[(16 * ib + r) * LS + 16 * j + c] = t[n];
+            for (int n = 0; n < 2; ++n) {
+                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib) continue;
+                *reinterpret_cast<float4 *>(L + (16 * ib + r) * LS + 16 * j + c4) = t[n];
             }
             __syncthreads();
 #pragma unroll
-            for (int n = 0; n < 2 * ib; ++n) {
-                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                const float *Ai = L + (16 * ib + r) * LS + 16 * ib;       // row r of A_ii
-                const float *Tc = L + (16 * ib) * LS + 16 * j + c;        // column c of T_ij
-                float s0 = 0.f, s1 = 0.f;
+            for (int n = 0; n < 2; ++n) {  // A_ij = -A_ii T_ij
+                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib) continue;
+                const float *Ai = L + (16 * ib + r) * LS + 16 * ib;  // row r of A_ii
+                const float *Tj = L + (16 * ib) * LS + 16 * j + c4;  // T_ij, columns c4 ..
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int m = 0; m < 16; m += 4) {
                     const float4 a4 = *reinterpret_cast<const float4 *>(Ai + m);
-                    s0 = fmaf(a4.x, Tc[m * LS], s0);
-                    s1 = fmaf(a4.y, Tc[(m + 1) * LS], s1);
-                    s0 = fmaf(a4.z, Tc[(m + 2) * LS], s0);
-                    s1 = fmaf(a4.w, Tc[(m + 3) * LS], s1);
+                    fma4(acc, a4.x, *reinterpret_cast<const float4 *>(Tj + m * LS));
+                    fma4(acc, a4.y, *reinterpret_cast<const float4 *>(Tj + (m + 1) * LS));
+                    fma4(acc, a4.z, *reinterpret_cast<const float4 *>(Tj + (m + 2) * LS));
+                    fma4(acc, a4.w, *reinterpret_cast<const float4 *>(Tj + (m + 3) * LS));
                 }
-                t[n] = -(s0 + s1);
+                t[n] = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
             __syncthreads();
 #pragma unroll
-            for (int n = 0; n < 2 * ib; ++n) {
-                const int e = tid + NT * n, j = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                L[(16 * ib + r) * LS + 16 * j + c] = t[n];
+            for (int n = 0; n < 2; ++n) {
+                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib) continue;
+                *reinterpret_cast<float4 *>(L + (16 * ib + r) * LS + 16 * j + c4) = t[n];
             }
             __syncthreads();
         }
