@@ -253,21 +253,7 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(const __grid_constant__ Para
     }
     if (ok) ok = cta_wait(&mbar, 0, p, 5);
     if (ok) {
-        const int i = m64_row();
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, c0), d);
-            tmem_ld_wait();
-            if (i >= 0) {
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int j = c0 + q;
-                    d[q] = j <= i ? p.scale * expf(G[i] - G[j]) * d[q] : 0.f;
-                }
-                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8)) = pack8(d);
-                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
-            }
-        }
+        build_p_tile(tmem, G, p.scale, Ps);
         operands_ready();
         if (tid == 0) {
             const uint32_t id = idesc_bf16(128, 64, 0, 0);

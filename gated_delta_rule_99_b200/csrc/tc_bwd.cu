@@ -101,21 +101,7 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
     }
     if (ok) ok = cta_wait(&mbar, 0, p, 11);
     if (ok) {
-        const int i = m64_row();
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, c0), d);
-            tmem_ld_wait();
-            if (i >= 0) {
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int j = c0 + q;
-                    d[q] = j <= i ? p.scale * expf(G[i] - G[j]) * d[q] : 0.f;
-                }
-                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8)) = pack8(d);
-                *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(d + 8);
-            }
-        }
+        build_p_tile(tmem, G, p.scale, Ps);
         operands_ready();
         if (tid == 0) {  // local dU^T[v][j] = sum_i dO[i][v] P[i][j]: M = 128, N = 64, K = 64
             const uint32_t db = smem_u32(DO), pb = smem_u32(Ps), id = idesc_bf16(128, 64, 1, 1);

@@ -193,5 +193,36 @@ __device__ __forceinline__ void l2norm_tile_rows(uint8_t *tile, int R, int row0,
     if (inv && half == 0) inv[r] = rn;
 }
 
+// P = scale lower(Q K^T . Gam), diagonal included, from the M = 64 accumulator at
+// TMEM column 0 into a 64 x 64 bf16 SW128 tile (CTAs of four warps).  The rows
+// of a warp lie in one 16-block, so the blocks above it are written as zeros
+// without evaluating their decays.
+__device__ __forceinline__ void build_p_tile(uint32_t tmem, const float *G, float scale,
+                                             uint8_t *Ps) {
+    const int i = m64_row();
+    float d[4][16];
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm(tmem, 16 * cb), d[cb]);
+    tmem_ld_wait();
+    if (i < 0) return;
+    const int ib = i >> 4;
+    const float gi = G[i];
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb) {
+        if (cb <= ib) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int j = 16 * cb + q;
+                d[cb][q] = j <= i ? scale * expf(gi - G[j]) * d[cb][q] : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) d[cb][q] = 0.f;
+        }
+        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, 2 * cb)) = pack8(d[cb]);
+        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(C, i, 2 * cb + 1)) = pack8(d[cb] + 8);
+    }
+}
+
 }  // namespace tc
 }  // namespace gdn

@@ -15,9 +15,11 @@ constexpr int LS = 68;  // row stride (floats) of L: 16-byte aligned rows for ve
 struct PrepSmem {
     // L (fp32 64 x 68) becomes A in place; once A is read out, its bytes hold
     // the two bf16 operand tiles A diag(b gam) and A diag(b).  F: per-column
-    // decay factors exp(G_e - G_j) to the end e of column j's 16-block.
+    // decay factors exp(G_e - G_j) to the end e of column j's 16-block; E: exp(G_j);
+    // EK: exp(G_n - G_j), n the chunk's last token.
     static constexpr int kK = 0, kV = kK + 16384, kL = kV + 16384, kAb = kL, kAc = kL + 8192,
-                         kG = kL + C * LS * 4, kB = kG + 256, kF = kB + 256, kEnd = kF + 256;
+                         kG = kL + C * LS * 4, kB = kG + 256, kF = kB + 256, kE = kF + 256,
+                         kEK = kE + 256, kEnd = kEK + 256;
 };
 constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
 constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 columns each)
@@ -45,6 +47,8 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     float *G = reinterpret_cast<float *>(sm + PrepSmem::kG);
     float *bta = reinterpret_cast<float *>(sm + PrepSmem::kB);
     float *F = reinterpret_cast<float *>(sm + PrepSmem::kF);
+    float *E = reinterpret_cast<float *>(sm + PrepSmem::kE);
+    float *EK = reinterpret_cast<float *>(sm + PrepSmem::kEK);
     const int tid = threadIdx.x;
 
     if (tid == 0) {  // K and V rows by the tensor engine
@@ -60,6 +64,11 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         tmem_relinquish();
     }
     chunk_gates(G, bta, p, ci, h);  // its barriers also publish the mbarrier inits
+    if (tid < C) {  // the decay factors, once (published by the barrier of the wait below)
+        F[tid] = expf(G[tid | 15] - G[tid]);
+        E[tid] = expf(G[tid]);
+        EK[tid] = expf(G[C - 1] - G[tid]);
+    }
     bool ok = copies_arrived(&lbar, p, 31);
     if (ok) {
         fix_rows(Kt, C, 0, ci.len, p.K);
@@ -83,13 +92,12 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     }
     // meanwhile: Kd = diag(e) K as a tile image, and G
     if (ok) {
-        const float Gn = G[C - 1];
         uint8_t *dst = static_cast<uint8_t *>(p.tKd) + (size_t)ch * kImg64;
         for (int t = tid; t < C * 16; t += NT) {
             const int off = t * 16, r = (off & 8191) >> 7;
             float f[8];
             unpack8(*reinterpret_cast<const uint4 *>(Kt + off), f);
-            const float e = expf(Gn - G[r]);
+            const float e = EK[r];
 #pragma unroll
             for (int i = 0; i < 8; ++i) f[i] *= e;
             *reinterpret_cast<uint4 *>(dst + off) = pack8(f);
@@ -97,32 +105,44 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         if (tid < C) {
             p.tG[(size_t)ch * C + tid] = G[tid];
             if (p.tB) p.tB[(size_t)ch * C + tid] = bta[tid];
-            F[tid] = expf(G[tid | 15] - G[tid]);
         }
     }
     if (ok) ok = cta_wait(&mbar, phase, p, 1);
     phase ^= 1;
     if (ok) {
-        // L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32)
+        // L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32).  The rows of a
+        // warp lie in one 16-block (M = 64 layout), so the three cases are warp-uniform.
         const int i = m64_row();
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, c0), d);
-            tmem_ld_wait();
-            if (i >= 0) {
-                // Gam_ij = exp(G_i - G_e) exp(G_e - G_j), e = c0 + 15, for blocks left of the
-                // diagonal block (both factors <= 1); the diagonal block directly
-                if (c0 + 15 < i) {
-                    const float ri = bta[i] * expf(G[i] - G[c0 + 15]);
+        float d[4][16];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) L[i * LS + c0 + q] = ri * F[c0 + q] * d[q];
-                } else {
+        for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm(tmem, 16 * cb), d[cb]);
+        tmem_ld_wait();
+        if (i >= 0) {
+            const int ib = i >> 4;
+            const float bi = bta[i];
+            float *Li = L + i * LS;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                const int c0 = 16 * cb;
+                float x[16];
+                if (cb < ib) {  // Gam_ij = exp(G_i - G_e) exp(G_e - G_j), e = c0 + 15 (both <= 1)
+                    const float ri = bi * expf(G[i] - G[c0 + 15]);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) x[q] = ri * F[c0 + q] * d[cb][q];
+                } else if (cb == ib) {  // the diagonal block directly
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const int j = c0 + q;
-                        L[i * LS + j] = j < i ? bta[i] * expf(G[i] - G[j]) * d[q] : 0.f;
+                        x[q] = j < i ? bi * expf(G[i] - G[j]) * d[cb][q] : 0.f;
                     }
+                } else {  // above the diagonal
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) x[q] = 0.f;
                 }
+#pragma unroll
+                for (int q = 0; q < 16; q += 4)
+                    *reinterpret_cast<float4 *>(Li + c0 + q) =
+                        make_float4(x[q], x[q + 1], x[q + 2], x[q + 3]);
             }
         }
         tc_fence_before();
@@ -240,7 +260,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
                 for (int q = 0; q < 8; ++q) {
                     const int c = 8 * cc + q;
                     fc[q] = av[n][q] * bta[c];
-                    fb[q] = fc[q] * expf(G[c]);
+                    fb[q] = fc[q] * E[c];
                 }
                 *reinterpret_cast<uint4 *>(Ab + sw128_chunk(C, r, cc)) = pack8(fb);
                 *reinterpret_cast<uint4 *>(Ac + sw128_chunk(C, r, cc)) = pack8(fc);
