@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
 #pragma unroll
             for (int q = 0; q < CW; ++q) {
                 const int j = cb + q;
-                const float gm = expf(j <= r ? gi - G[j] : -INFINITY);  // Gam (0 above diagonal)
+                const float gm = __expf(j <= r ? gi - G[j] : -INFINITY);  // Gam (0 above diagonal)
                 const float dp = j <= r ? d[q] : 0.f;
                 pq[q] = (p.scale * gm * pq[q]) * dp;
                 rs += pq[q];
@@ -807,7 +807,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
 #pragma unroll
             for (int q = 0; q < CW; ++q) {
                 const int j = cb + q;
-                const float gm = expf(j < i ? gi - G[j] : -INFINITY);
+                const float gm = __expf(j < i ? gi - G[j] : -INFINITY);
                 const float dl = j < i ? -d[q] : 0.f;
                 const float kkg = gm * kk[q];
                 kk[q] = dl * bi * kkg;

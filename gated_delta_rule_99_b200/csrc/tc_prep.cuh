@@ -179,17 +179,19 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             }
             __syncthreads();
         }
-        // Row blocks ib = 1..3: unit u = tid + NT n of row block ib is block j = u / 64,
-        // row r = (u / 4) % 16, columns c4 .. c4 + 3 (c4 = 4 (u % 4)); a thread forms its
-        // four columns from float4 rows (the 32 units of a warp share j, so the k loop
-        // bound is uniform; rows r of stride LS = 68 floats fall in distinct banks).
+        // Row blocks ib = 1..3: unit u of row block ib is block j = u / 64, row
+        // r = (u / 4) % 16, columns c4 .. c4 + 3 (c4 = 4 (u % 4)); thread t takes unit t
+        // and, for ib = 3, threads 64-127 also unit t + 64 (block j = 2, the shortest
+        // sum).  A thread forms its four columns from float4 rows (the 32 units of a warp
+        // share j, so the k loop bound is uniform; rows r of stride LS = 68 floats fall
+        // in distinct banks).
 #pragma unroll
         for (int ib = 1; ib < 4; ++ib) {
             float4 t[2];
 #pragma unroll
             for (int n = 0; n < 2; ++n) {  // T_ij = sum_{k=j}^{ib-1} L_ik A_kj
-                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
-                if (u >= 64 * ib) continue;
+                const int u = tid + 64 * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib || (n && tid < 64)) continue;
                 const float *Lr = L + (16 * ib + r) * LS;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int k = j; k < ib; ++k) {
@@ -208,15 +210,15 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             __syncthreads();  // every product of this row block has read its L blocks
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
-                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
-                if (u >= 64 * ib) continue;
+                const int u = tid + 64 * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib || (n && tid < 64)) continue;
                 *reinterpret_cast<float4 *>(L + (16 * ib + r) * LS + 16 * j + c4) = t[n];
             }
             __syncthreads();
 #pragma unroll
             for (int n = 0; n < 2; ++n) {  // A_ij = -A_ii T_ij
-                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
-                if (u >= 64 * ib) continue;
+                const int u = tid + 64 * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib || (n && tid < 64)) continue;
                 const float *Ai = L + (16 * ib + r) * LS + 16 * ib;  // row r of A_ii
                 const float *Tj = L + (16 * ib) * LS + 16 * j + c4;  // T_ij, columns c4 ..
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -233,8 +235,8 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             __syncthreads();
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
-                const int u = tid + NT * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
-                if (u >= 64 * ib) continue;
+                const int u = tid + 64 * n, j = u >> 6, r = (u >> 2) & 15, c4 = (u & 3) * 4;
+                if (u >= 64 * ib || (n && tid < 64)) continue;
                 *reinterpret_cast<float4 *>(L + (16 * ib + r) * LS + 16 * j + c4) = t[n];
             }
             __syncthreads();
