@@ -48,6 +48,17 @@ def test_other_head_dims_and_fp32(dtype, K, V):
     _check(inp, TOL[dtype])
 
 
+def test_many_units_per_cta_head_dim_64():
+    """Packed ragged documents with more (chunk, head) units than SMs at d_k = 64:
+    the persistent gradient kernel's prefetched q/k tiles are normalised and
+    padded per unit."""
+    import numpy as np
+    lengths = [int(x) for x in np.random.default_rng(65).integers(1, 151, size=48)]
+    inp = make_inputs(B=1, T=sum(lengths), H=8, K=64, V=128, dtype="bf16", seed=65,
+                      lengths=lengths, raw_qk=True)
+    _check(inp, TOL["bf16"])
+
+
 def test_zero_rows_and_gradients_orthogonal_to_rows():
     inp = make_inputs(B=1, T=130, H=2, K=128, V=128, dtype="bf16", seed=63, raw_qk=True)
     inp.q[0, 5] = 0

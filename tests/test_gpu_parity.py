@@ -160,6 +160,55 @@ def test_packed_equals_per_document_runs_bitwise():
         assert torch.equal(got[5][n:n + 1], gn[5])
 
 
+def _ragged_lengths(n, seed):
+    rng = np.random.default_rng(seed)
+    return [int(x) for x in rng.integers(1, 151, size=n)]
+
+
+@pytest.mark.parametrize("case", ["packed", "dense"])
+def test_tc_many_units_per_cta(case):
+    """More (chunk, head) units than SMs, so every persistent CTA of the gradient
+    kernel walks several units and prefetches the next one's inputs; short chunks
+    (packed documents of 1-150 tokens, or a 40-token tail per dense row) take the
+    row-store path between full ones.  Every element against the oracle."""
+    if case == "packed":
+        lengths = _ragged_lengths(56, 27)
+        inp = make_inputs(B=1, T=sum(lengths), H=8, K=128, V=128, dtype="bf16", seed=27,
+                          lengths=lengths)
+    else:
+        inp = make_inputs(B=3, T=1000, H=16, K=128, V=128, dtype="bf16", seed=28)
+    check_all(inp, TOL["bf16"])
+
+
+def test_tc_many_units_split_call_bitwise():
+    """The same documents in one packed call and in two calls (first half, second
+    half): each document's outputs are bitwise equal, whichever CTA and slot of
+    the persistent kernel handled its units."""
+    lengths = _ragged_lengths(40, 29)
+    inp = make_inputs(B=1, T=sum(lengths), H=8, K=128, V=128, dtype="bf16", seed=29,
+                      lengths=lengths)
+    o, hT = run_fwd(inp)
+    got = run_bwd(inp)
+    cu = inp.cu_seqlens.tolist()
+    half = len(lengths) // 2
+    for n0, n1 in ((0, half), (half, len(lengths))):
+        t0, t1 = cu[n0], cu[n1]
+        sub = inp.to("cpu")
+        sl = lambda x: x[:, t0:t1].contiguous()
+        sub.q, sub.k, sub.v, sub.g, sub.beta, sub.do = map(sl, (inp.q, inp.k, inp.v, inp.g,
+                                                                 inp.beta, inp.do))
+        sub.h0 = inp.h0[n0:n1].contiguous()
+        sub.dhT = inp.dhT[n0:n1].contiguous()
+        sub.cu_seqlens = torch.tensor([c - t0 for c in cu[n0:n1 + 1]], dtype=torch.int32)
+        on, hn = run_fwd(sub)
+        assert torch.equal(o[:, t0:t1], on)
+        assert torch.equal(hT[n0:n1], hn)
+        gn = run_bwd(sub)
+        for a, b in zip(got[:5], gn[:5]):
+            assert torch.equal(a[:, t0:t1], b)
+        assert torch.equal(got[5][n0:n1], gn[5])
+
+
 def test_run_to_run_determinism():
     inp = make_inputs(B=2, T=500, H=4, K=128, V=128, dtype="bf16", seed=17)
     a = run_fwd(inp) + run_bwd(inp)
