@@ -133,7 +133,7 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.tS = b(L.tS);
     p.tUT = b(L.tUT);
     p.tQg = b(L.tQg);
-    p.tdUL = b(L.tdUL);
+    p.tP = b(L.tP);
     p.tdSn = b(L.tdSn);
     p.tdUT = b(L.tdUT);
     p.tG = f(L.tG);
@@ -253,7 +253,7 @@ Layout make_layout(const Problem &pb, bool bwd) {
             L.tA = take(nch * kChunk * kChunk * 2);  // bf16 tile image of A
             L.tB = take(nch * kChunk * f);
             L.tQg = take(nch * img64);
-            L.tdUL = take(nch * img64);
+            L.tP = take(nch * kChunk * kChunk * 2);  // bf16 tile image of P
             L.tdSn = take(nch * img128);
             L.tdUT = take(nch * img64);
         }

@@ -58,7 +58,7 @@ struct Params {
     // (128-byte-swizzled, as the MMAs read them) and plain rows
     void *tW, *tUt, *tKd;          // 64x128 W image, 64x128 Ut rows, 64x128 diag(e)K image
     void *tS, *tUT;                // 128x128 image of the state entering the chunk, 128x64 U^T image
-    void *tQg, *tdUL, *tdSn, *tdUT;  // backward: scaled-q image, local dU^T, dS image, dU^T image
+    void *tQg, *tP, *tdSn, *tdUT;  // backward: scaled-q image, P tile, dS image, dU^T image
     float *tG;                     // 64 cumulative gates per (chunk, head)
     float *tB;                     // 64 write strengths per (chunk, head), 0 past its end
     void *tA;                      // 64x64 bf16 tile image of A (backward)
@@ -120,7 +120,7 @@ struct Problem {
 struct Layout {
     size_t chunks, seq_first;
     size_t W, Ut, A, U, Hs, dUloc, dU, dHn, scratch;
-    size_t tW, tUt, tKd, tS, tUT, tQg, tdUL, tdSn, tdUT, tG, tB, tA, tHin, tMp, tBp;
+    size_t tW, tUt, tKd, tS, tUT, tQg, tP, tdSn, tdUT, tG, tB, tA, tHin, tMp, tBp;
     size_t qn, kn, qinv, kinv;  // normalised q, k copies and 1/|row| (passes of the fp32 path)
     size_t total;
 };

@@ -36,7 +36,7 @@ using namespace tc;
 // ============================================================ tc_local
 struct LocalSmem {
     // P overwrites the Q half of the [Q; K] tile once Q K^T and Qg have consumed it
-    static constexpr int kQK = 0, kDO = kQK + 32768, kP = kQK, kG = kDO + 16384, kEnd = kG + 256;
+    static constexpr int kQK = 0, kP = kQK, kG = kQK + 32768, kEnd = kG + 256;
 };
 constexpr int kLocalSmem = LocalSmem::kEnd + 1024;
 
@@ -51,16 +51,15 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
     if (p.hdr->status) return;
     const int H = p.H, c = ch / H, h = ch % H, tid = threadIdx.x;
     const ChunkInfo ci = chunk_at(p, c);
-    uint8_t *QK = sm + LocalSmem::kQK, *DO = sm + LocalSmem::kDO, *Ps = sm + LocalSmem::kP;
+    uint8_t *QK = sm + LocalSmem::kQK, *Ps = sm + LocalSmem::kP;
     float *G = reinterpret_cast<float *>(sm + LocalSmem::kG);
-    if (tid == 0) {  // q, k and dO rows by the tensor engine
+    if (tid == 0) {  // q and k rows by the tensor engine
         mbar_init(&mbar, 1);
         mbar_init(&lbar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&lbar, 2 * row_tile_bytes(p.K) + row_tile_bytes(p.V));
+        mbar_arrive_expect_tx(&lbar, 2 * row_tile_bytes(p.K));
         load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
         load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
-        load_rows_tma(DO, C, 0, &p.tm_do, ci.tok0, h, p.V, &lbar);
     }
     if (tid < 32) {
         tmem_alloc(&tslot, 128);
@@ -71,7 +70,6 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
     if (ok) {
         fix_rows(QK, D, 0, ci.len, p.K);
         fix_rows(QK, D, C, ci.len, p.K);
-        fix_rows(DO, C, 0, ci.len, p.V);
     }
     operands_ready();
     if (ok && p.l2norm) {  // q and k rows divided by their norms
@@ -100,26 +98,15 @@ __device__ __forceinline__ void local_body(const Params &p, int ch) {
         }
     }
     if (ok) ok = cta_wait(&mbar, 0, p, 11);
-    if (ok) {
+    if (ok) {  // P as a tile image: the reverse state pass forms the local dU^T = dO^T P itself
         build_p_tile(tmem, G, p.scale, Ps);
-        operands_ready();
-        if (tid == 0) {  // local dU^T[v][j] = sum_i dO[i][v] P[i][j]: M = 128, N = 64, K = 64
-            const uint32_t db = smem_u32(DO), pb = smem_u32(Ps), id = idesc_bf16(128, 64, 1, 1);
-#pragma unroll
-            for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 64, desc_mnmajor(db, C, s), desc_mnmajor(pb, C, s), id, s > 0);
-            mma_commit(&mbar);
-        }
-        ok = cta_wait(&mbar, 1, p, 12);
-    }
-    if (ok) {
-        uint8_t *dul = static_cast<uint8_t *>(p.tdUL) + (size_t)ch * kImgUT;
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float d[16];
-            tmem_ld16(tm(tmem, 64 + c0), d);
-            tmem_ld_wait();
-            *reinterpret_cast<uint4 *>(dul + sw128_chunk(D, tid, c0 / 8)) = pack8(d);
-            *reinterpret_cast<uint4 *>(dul + sw128_chunk(D, tid, c0 / 8 + 1)) = pack8(d + 8);
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(static_cast<uint8_t *>(p.tP) + (size_t)ch * C * C * 2, smem_u32(Ps),
+                       (uint32_t)(C * C * 2));
+            bulk_commit();
+            bulk_wait_all();
         }
     }
     tc_fence_before();
@@ -138,9 +125,9 @@ __global__ void __launch_bounds__(NT, 4) tc_prep_local_kernel(const __grid_const
 // ============================================================ tc_state_bwd
 struct SbwdSmem {
     static constexpr int kdS = 0, kdU = kdS + 32768, kBuf = kdU + 16384;
-    // per buffer: Kd image, W image, Qg image, dO tile, local dU^T rows, gates
-    static constexpr int kKd = 0, kW = 16384, kQg = 32768, kDO = 49152, kDUL = 65536,
-                         kG = 81920, kBufBytes = 81920 + 1024;
+    // per buffer: Kd image, W image, Qg image, dO tile, P tile, gates
+    static constexpr int kKd = 0, kW = 16384, kQg = 32768, kDO = 49152, kP = 65536,
+                         kG = 73728, kBufBytes = 73728 + 1024;
     static constexpr int kEnd = kBuf + 2 * kBufBytes;
 };
 constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
@@ -152,7 +139,7 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
                                               uint64_t *bar) {
     uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
     if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(bar, 3u * (uint32_t)kImg64 + (uint32_t)kImgUT + C * 4u +
+        mbar_arrive_expect_tx(bar, 3u * (uint32_t)kImg64 + (uint32_t)(C * C * 2) + C * 4u +
                                        row_tile_bytes(p.V));
         bulk_load(smem_u32(b + SbwdSmem::kKd), static_cast<const uint8_t *>(p.tKd) + ch * kImg64,
                   kImg64, bar);
@@ -160,8 +147,8 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
                   kImg64, bar);
         bulk_load(smem_u32(b + SbwdSmem::kQg), static_cast<const uint8_t *>(p.tQg) + ch * kImg64,
                   kImg64, bar);
-        bulk_load(smem_u32(b + SbwdSmem::kDUL),
-                  static_cast<const uint8_t *>(p.tdUL) + ch * kImgUT, kImgUT, bar);
+        bulk_load(smem_u32(b + SbwdSmem::kP),
+                  static_cast<const uint8_t *>(p.tP) + ch * (size_t)(C * C * 2), C * C * 2, bar);
         bulk_load(smem_u32(b + SbwdSmem::kG), p.tG + ch * C, C * 4, bar);
         load_rows_tma(b + SbwdSmem::kDO, C, 0, &p.tm_do, ci.tok0, h, p.V, bar);
     }
@@ -209,7 +196,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     }
     uint8_t *dSs = sm + SbwdSmem::kdS, *dUs = sm + SbwdSmem::kdU;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), idx = idesc_bf16(128, 128, 1, 1),
-                   idy = idesc_bf16(128, 128, 0, 1);
+                   idy = idesc_bf16(128, 128, 0, 1), idp = idesc_bf16(128, 64, 1, 1);
     for (int c = c1 - 1; c >= c0; --c) {
         const int buf = (c1 - 1 - c) & 1;
         const size_t ch = (size_t)c * H + h;
@@ -220,7 +207,25 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         }
         const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, kWaitLimit);
         uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
-        if (lok) fix_rows(b + SbwdSmem::kDO, C, 0, chunk_in_seq(p, n, c0, c).len, p.V);
+        const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
+                       qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO),
+                       pb = smem_u32(b + SbwdSmem::kP);
+        // dO^T P (the local dU^T; M = 128 (v), N = 64, K = 64 tokens) and dO^T Qg (M = 128,
+        // N = 128 keys, K = 64) do not depend on dS: on a full chunk (whose dO rows need no
+        // clearing) thread 0 issues them as soon as its copies landed, under the dS image
+        // writes below
+        const int len = chunk_in_seq(p, n, c0, c).len;
+        const bool early = len == C && p.V == D;
+        auto issue_local = [&]() {
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem, desc_mnmajor(ob, C, s), desc_mnmajor(pb, C, s), idp, s > 0);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + 64, desc_mnmajor(ob, C, s), desc_mnmajor(qb, C, s), idx, s > 0);
+        };
+        if (v == 0 && lok && early) issue_local();
+        if (lok && !early) fix_rows(b + SbwdSmem::kDO, C, 0, len, p.V);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
@@ -236,37 +241,26 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         lpar ^= 1u << buf;
         const float gC = expf(reinterpret_cast<const float *>(b + SbwdSmem::kG)[C - 1]);
         if (v == 0) {
-            const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
-                           qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO);
-            // dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
+            if (!early) issue_local();
+            // + dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, s > 0);
-            // dO^T Qg: M = 128 (v), N = 128 keys, K = 64 tokens
-#pragma unroll
-            for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 64, desc_mnmajor(ob, C, s), desc_mnmajor(qb, C, s), idx, s > 0);
+                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, 1);
             mma_commit(&mbar);
             bulk_store(static_cast<uint8_t *>(p.tdSn) + ch * kImg128, sb, (uint32_t)kImg128);
             bulk_commit();
         }
         if (!cta_wait(&mbar, phase, p, 13)) break;
         phase ^= 1;
-        {  // dU^T = dS Kd^T + local dU^T: the next operand, and (bulk-stored) an image for tc_grads
-            const uint8_t *dul = b + SbwdSmem::kDUL;  // local dU^T, swizzled rows
 #pragma unroll
-            for (int c16 = 0; c16 < C; c16 += 16) {
-                float d[16], l[16];
-                tmem_ld16(tm(tmem, c16), d);
-                tmem_ld_wait();
-                unpack8(*reinterpret_cast<const uint4 *>(dul + sw128_chunk(D, v, c16 / 8)), l);
-                unpack8(*reinterpret_cast<const uint4 *>(dul + sw128_chunk(D, v, c16 / 8 + 1)),
-                        l + 8);
+        for (int c32 = 0; c32 < C; c32 += 32) {  // dU^T: the next operand, and an image for tc_grads
+            float d[32];
+            tmem_ld16(tm(tmem, c32), d);
+            tmem_ld16(tm(tmem, c32 + 16), d + 16);
+            tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < 16; ++q) d[q] += l[q];
-                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8)) = pack8(d);
-                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c16 / 8 + 1)) = pack8(d + 8);
-            }
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
         }
         operands_ready();
         if (v == 0) {  // + dU^T (-W): M = 128 (v), N = 128 keys, K = 64 tokens (W image negated)
