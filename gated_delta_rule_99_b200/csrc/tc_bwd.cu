@@ -516,12 +516,20 @@ __device__ __forceinline__ void ldcw(uint32_t tmem, int col, float *d) {
     tmem_ld_wait();
 }
 
+// Bounded wait of one thread for an MMA-completion phase, after which it may
+// read the products (the CTA decides on a failure at its next barrier).
+__device__ __forceinline__ bool thread_wait(uint64_t *bar, uint32_t parity) {
+    const bool ok = mbar_wait(bar, parity, kWaitLimit);
+    tc_fence_after();
+    return ok;
+}
+
 __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    // MMA completions: mbar_a the first two products (X3, A^T dU), mbar_z Y2 and
-    // Zp, mbar the others in order (one phase in flight on each)
-    __shared__ uint64_t mbar, mbar_a, mbar_z, lbar[kGrpCount];
+    // MMA completions (one phase in flight on each): mbar_a X3^T and (A^T dU)^T;
+    // mbar_c X1^T, X2^T and Y1; mbar_z Y2 and Zp; mbar the others in order
+    __shared__ uint64_t mbar, mbar_a, mbar_c, mbar_z, lbar[kGrpCount];
     __shared__ uint32_t tslot;
     __shared__ float s_hd;
     if (p.hdr->status) return;
@@ -549,6 +557,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         for (int g = 0; g < kGrpCount; ++g) mbar_init(&lbar[g], 1);
         mbar_init(&mbar, 1);
         mbar_init(&mbar_a, 1);
+        mbar_init(&mbar_c, 1);
         mbar_init(&mbar_z, 1);
         fence_mbar_init();
     }
@@ -596,10 +605,9 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         constexpr int cQK = 0, cX1 = 64, cX2 = 128, cX3 = 192, cDP = 256, cAU = 320, cY1 = 384,
                       cY2 = 192, cZ = 448, cT1 = 192, cDL = 192, cDQ = 256, cDK = 320, cDKA = 384;
         float d[CW];
-        if (tid == 0) {  // the products the SIMT work needs first, then the rest
-            const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mk = idesc_bf16(128, 64, 1, 0),
-                           i128mm = idesc_bf16(128, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1),
-                           i64mk = idesc_bf16(64, 64, 1, 0);
+        if (tid == 0) {  // the products the SIMT work needs first (the rest come after X3)
+            const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mm = idesc_bf16(128, 64, 1, 1),
+                           i128km = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
             for (int s = 0; s < 8; ++s)  // X3^T = S^T dU^T
                 mma_bf16(tmem + cX3, desc_mnmajor(scb, D, s), desc_mnmajor(dub, D, s), i128mm,
@@ -612,20 +620,9 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
                 mma_bf16(tmem + cQK, desc_kmajor(qkb, D, s), desc_kmajor(kb, D, s), i128, s > 0);
 #pragma unroll
-            for (int s = 0; s < 8; ++s)  // X1^T = S^T dO^T  (over v)
-                mma_bf16(tmem + cX1, desc_mnmajor(scb, D, s), desc_kmajor(dvb, D, s), i128mk,
-                         s > 0);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)  // X2^T = dSn^T U^T
-                mma_bf16(tmem + cX2, desc_mnmajor(dsb, D, s), desc_mnmajor(utb, D, s), i128mm,
-                         s > 0);
-#pragma unroll
             for (int s = 0; s < 8; ++s)  // [dO; V] U^T: lanes 0-63 dP = dO U^T, next to P
                 mma_bf16(tmem + cDP, desc_kmajor(dvb, D, s), desc_mnmajor(utb, D, s), i128km,
                          s > 0);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)  // Y1 = dU V^T (M = 64)
-                mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, D, s), i64mk, s > 0);
             mma_commit(&mbar);
         } else if (tid >= 32) {  // <S, dSn> (identically laid out images) by warps 1-15
             float s = 0.f;
@@ -653,8 +650,21 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         for (int q = 0; q < CW / 8; ++q)
             *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
         operands_ready();
-        if (tid == 0) {  // issued now; the SIMT work below runs while they execute
-            const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1);
+        if (tid == 2 * 32) {  // warp 2 (rows 64-95) has no part in the P . dP phase below
+            const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1),
+                           i128mk = idesc_bf16(128, 64, 1, 0), i128mm = idesc_bf16(128, 64, 1, 1);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // X1^T = S^T dO^T  (over v)
+                mma_bf16(tmem + cX1, desc_mnmajor(scb, D, s), desc_kmajor(dvb, D, s), i128mk,
+                         s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // X2^T = dSn^T U^T
+                mma_bf16(tmem + cX2, desc_mnmajor(dsb, D, s), desc_mnmajor(utb, D, s), i128mm,
+                         s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // Y1 = dU V^T (M = 64)
+                mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, D, s), i64mk, s > 0);
+            mma_commit(&mbar_c);
 #pragma unroll
             for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
                 mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
@@ -663,37 +673,11 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
             mma_commit(&mbar_z);
         }
-        {  // dv = diag(b) A^T dU, staged in dA/T1 (thread r holds column r); partial v . (A^T dU)
-            const ColSw vcol(DV + C * 128, D, r);
-            ldcw(tmem, cAU + cb, d);
-            float y[CW];
-#pragma unroll
-            for (int q = 0; q < CW; ++q) {
-                y[q] = bta[cb + q] * d[q];
-                d[q] *= vcol.at(cb, q);
-            }
-            stage_col(DA, y, cb, r);
-            warp_colsum(d, wsum, w4, cb, l);
-        }
-        ok = cta_wait(&mbar, phase, p, 21);
+        // meanwhile, each thread waiting for what it reads itself (no barrier waits on the
+        // issuing warp); the CTA decides on a failed wait at the barrier after them
+        bool fine = true;
+        if (w4 < 2) fine = thread_wait(&mbar, phase);  // Q K^T and dP
         phase ^= 1;
-        if (!ok) break;
-        if (more) {  // S, dSn, U^T, dU^T, G and b of the next unit (their buffers are consumed)
-            if (tid == 0) grads_fetch(p, sm, next, ci, kGrpImg, (it + 1) & 1, lbar);
-            pend |= kGrpImg;
-            ppar = (it + 1) & 1;
-        }
-        {  // column readers of q and k are built where used (they cost 8 registers each)
-            const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
-            ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
-#pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
-            warp_colsum(d, wsum + 256, w4, cb, l);
-            ldcw(tmem, cX2 + cb, d);  // partial k . X2
-#pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
-            warp_colsum(d, wsum + 512, w4, cb, l);
-        }
         if (w4 < 2) {  // row i = r of P and dP: P . dP (row and column partials), dPG = dP . Gam
             float pq[CW];
             tmem_ld16(tmq(tmem, cQK + cb), pq);
@@ -716,8 +700,42 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, r, cb / 8 + q)) = pack8(d + 8 * q);
             warp_colsum(pq, wsum + 768, w4, cb, l);
         }
+        {  // dv = diag(b) A^T dU, staged in dA/T1 (thread r holds column r); partial v . (A^T dU)
+            const ColSw vcol(DV + C * 128, D, r);
+            ldcw(tmem, cAU + cb, d);
+            float y[CW];
+#pragma unroll
+            for (int q = 0; q < CW; ++q) {
+                y[q] = bta[cb + q] * d[q];
+                d[q] *= vcol.at(cb, q);
+            }
+            stage_col(DA, y, cb, r);
+            warp_colsum(d, wsum, w4, cb, l);
+        }
+        fine = thread_wait(&mbar_c, it & 1) && fine;  // X1, X2, Y1
+        if (more) {  // S, dSn, U^T, dU^T, G and b of the next unit (every product reading
+                     // them is complete: thread 0 waited for all three barriers)
+            if (tid == 0) grads_fetch(p, sm, next, ci, kGrpImg, (it + 1) & 1, lbar);
+            pend |= kGrpImg;
+            ppar = (it + 1) & 1;
+        }
+        {  // column readers of q and k are built where used (they cost 8 registers each)
+            const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
+            ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
+            warp_colsum(d, wsum + 256, w4, cb, l);
+            ldcw(tmem, cX2 + cb, d);  // partial k . X2
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
+            warp_colsum(d, wsum + 512, w4, cb, l);
+        }
         fence_async_smem();  // the staged dv rows leave by bulk copies
-        __syncthreads();
+        ok = __syncthreads_and(fine);
+        if (!ok) {
+            if (tid == 0) record_timeout(p, 21);
+            break;
+        }
         if (more) {  // dO and v rows of the next unit (read by the first products and the dv sums)
             if (tid == 0) grads_fetch(p, sm, next, chunk_at(p, next / H), kGrpDV, 0, lbar);
             pend |= kGrpDV;
