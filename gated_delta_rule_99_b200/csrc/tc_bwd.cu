@@ -833,7 +833,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             warp_colsum(kk, wsum + 768, w4, cb, l);
         }
         operands_ready();
-        if (tid == 0) {
+        if (tid == 2 * 32) {  // warp 2 has no part in the row sums and the scan below
             const uint32_t imk = idesc_bf16(128, 64, 1, 0), imm = idesc_bf16(128, 64, 1, 1);
 #pragma unroll
             for (int s = 0; s < 4; ++s)  // (dPG K)^T = K^T dPG^T
