@@ -92,8 +92,33 @@ def kernel_work(name, w, n_chunks):
     return None, None, None
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and blank lines (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":  # a literal, escapes included
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            while i < n and text[i] != "\n":
+                i += 1
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def csrc_hash() -> str:
-    """Hash of the CUDA sources and the ABI header (ties recorded ncu traffic to a build)."""
+    """Hash of the code (comments and blank lines aside) of the CUDA sources and the
+    ABI header: ties recorded ncu traffic to a build."""
     import glob
     import hashlib
     h = hashlib.sha1()
@@ -102,8 +127,8 @@ def csrc_hash() -> str:
                    glob.glob(os.path.join(ROOT, "include", "*.h")))
     for f in files:
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -4,11 +4,11 @@
 // pieces are recomputed (tc_prep keeps A in fp32; tc_state_fwd rewrites the
 // state entering every chunk and U^T), three kernels run:
 //
-//   tc_local      chunk-parallel: P = scale lower(Q K^T . Gam), the local
-//                 dU^T = dO^T P, and Qg = scale diag(gam) Q (a tile image)
+//   tc_local      chunk-parallel: P = scale lower(Q K^T . Gam) and
+//                 Qg = scale diag(gam) Q (tile images)
 //   tc_state_bwd  serial over the chunks of a sequence, in reverse; thread v
 //                 owns row v of dS = dH^T (fp32 registers); per chunk
-//                   dU^T = dS Kd^T + (local dU^T)
+//                   dU^T = dO^T P + dS Kd^T
 //                   dS  <- gam_n dS + dO^T Qg - dU^T W
 //                 and writes dS (the gradient of the state leaving the chunk)
 //                 and dU^T as tile images
@@ -132,7 +132,7 @@ struct SbwdSmem {
 };
 constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
 
-// Chunk ch's Kd, W and Qg images, local dU^T image and gate row by bulk copies,
+// Chunk ch's Kd, W, Qg and P images and gate row by bulk copies,
 // its dO rows by the tensor engine (thread 0, all completing on `bar`).
 __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
                                               const ChunkInfo &ci, int h, const Params &p,
