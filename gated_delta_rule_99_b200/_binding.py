@@ -20,8 +20,10 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "mi
           4: "workspace missing or too small", 5: "CUDA runtime error",
           6: "device-side wait timed out"}
 EXPORTS = ("gdn_version", "gdn_chunk_size", "gdn_fwd_workspace_size", "gdn_bwd_workspace_size",
-           "gdn_fwd", "gdn_fwd_noalloc", "gdn_bwd", "gdn_decode", "gdn_device_status", "gdn_status_string", "gdn_trace_install",
-           "gdn_kernel_name")
+           "gdn_fwd", "gdn_fwd_noalloc", "gdn_fwd_noalloc_status", "gdn_bwd", "gdn_decode",
+           "gdn_device_status", "gdn_status_string", "gdn_trace_install", "gdn_kernel_name",
+           "gdn_set_wait_limit", "gdn_set_test_hook")
+GDN_TEST_STALL_COPY, GDN_TEST_FAIL_LAUNCH = 1, 2
 
 
 class GdnError(RuntimeError):
@@ -63,6 +65,12 @@ def lib() -> ctypes.CDLL:
             L.gdn_fwd.argtypes = [dp, vp, vp, vp, fp, fp, i32p, i32p, fp, vp, fp, vp, sz, vp]
             L.gdn_fwd_noalloc.restype = ctypes.c_int
             L.gdn_fwd_noalloc.argtypes = [dp, vp, vp, vp, fp, fp, i32p, i32p, fp, vp, fp, vp]
+            L.gdn_fwd_noalloc_status.restype = ctypes.c_int
+            L.gdn_fwd_noalloc_status.argtypes = [vp]
+            L.gdn_set_wait_limit.restype = None
+            L.gdn_set_wait_limit.argtypes = [ctypes.c_uint32]
+            L.gdn_set_test_hook.restype = None
+            L.gdn_set_test_hook.argtypes = [ctypes.c_int32]
             L.gdn_bwd.restype = ctypes.c_int
             L.gdn_bwd.argtypes = [dp, vp, vp, vp, fp, fp, i32p, i32p, fp, vp, fp, vp, vp, vp, fp,
                                   fp, fp, vp, sz, vp]
@@ -230,6 +238,18 @@ def gdn_decode(q, k, v, g, beta, state, scale=1.0, o=None, stream=None, qk_l2nor
 
 def device_status(workspace, stream=None) -> int:
     return int(lib().gdn_device_status(_ptr(workspace), _stream(stream)))
+
+
+def set_wait_limit(polls: int) -> None:
+    """Testing hook: device-side waits of later calls from this thread give up
+    after ``polls`` polls (0 restores the built-in limit)."""
+    lib().gdn_set_wait_limit(int(polls))
+
+
+def set_test_hook(hook: int) -> None:
+    """Testing hook: plant GDN_TEST_STALL_COPY or GDN_TEST_FAIL_LAUNCH in later
+    calls from this thread (0 removes it)."""
+    lib().gdn_set_test_hook(int(hook))
 
 
 class GdnTrace(ctypes.Structure):

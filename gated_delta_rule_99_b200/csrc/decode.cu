@@ -132,7 +132,10 @@ extern "C" gdn_status gdn_decode(const gdn_desc *d, const void *q, const void *k
     if (d->B < 1 || d->T < 1 || d->H < 1 || d->n_seqs != 0) return GDN_ERR_INVALID_ARG;
     if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return GDN_ERR_UNSUPPORTED;
     if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN_ERR_UNSUPPORTED;
-    if (d->B * d->H >= (int64_t(1) << 31) || d->B * d->T >= (int64_t(1) << 31))
+    // range checks before any product is formed (no signed overflow on huge inputs)
+    constexpr int64_t kLim = int64_t(1) << 31;
+    if (d->B >= kLim || d->T >= kLim || d->H >= kLim || d->H >= kLim / d->B ||
+        d->T >= kLim / d->B)
         return GDN_ERR_INVALID_ARG;
     if (!(d->scale == d->scale)) return GDN_ERR_INVALID_ARG;
     if (d->reserved != 0 || (d->flags & ~(GDN_FLAG_PIECE_SCAN | GDN_FLAG_QK_L2NORM)))
@@ -142,6 +145,7 @@ extern "C" gdn_status gdn_decode(const gdn_desc *d, const void *q, const void *k
     for (const void *p : ptrs)
         if (mis(p)) return GDN_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    arm_planted_failure();
     cudaError_t e = d->dtype == GDN_BF16
                         ? launch_typed<__nv_bfloat16>(d, q, k, v, g, beta, state, o, s)
                         : launch_typed<float>(d, q, k, v, g, beta, state, o, s);

@@ -23,7 +23,11 @@ gdn_status describe(const gdn_desc *d, Problem *p) {
     if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return GDN_ERR_UNSUPPORTED;
     if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN_ERR_UNSUPPORTED;
     if (d->n_seqs > 0 && d->B != 1) return GDN_ERR_INVALID_ARG;
-    if (d->B * d->T >= (int64_t(1) << 31) || d->H >= (1 << 16)) return GDN_ERR_INVALID_ARG;
+    // range checks before any product is formed (no signed overflow on huge inputs)
+    constexpr int64_t kLim = int64_t(1) << 31;
+    if (d->B >= kLim || d->T >= kLim || d->T >= kLim / d->B || d->H >= (1 << 16) ||
+        d->n_seqs >= kLim)
+        return GDN_ERR_INVALID_ARG;
     if (!(d->scale == d->scale)) return GDN_ERR_INVALID_ARG;  // NaN scale
     p->B = d->B;
     p->T = d->T;
@@ -35,6 +39,8 @@ gdn_status describe(const gdn_desc *d, Problem *p) {
     if (p->N >= (int64_t(1) << 30)) return GDN_ERR_INVALID_ARG;
     p->NCmax = d->n_seqs > 0 ? (d->T + kChunk - 1) / kChunk + d->n_seqs
                              : d->B * ((d->T + kChunk - 1) / kChunk);
+    // grids of (chunk, head) and (sequence, head) CTAs are formed in int32
+    if (p->NCmax * p->H >= (int64_t(1) << 30)) return GDN_ERR_INVALID_ARG;
     p->NC = 0;
     p->dtype = d->dtype;
     p->scale = d->scale;
@@ -111,6 +117,8 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.scale = d->scale;
     p.bf16 = d->dtype == GDN_BF16;
     p.l2norm = pb.l2norm;
+    p.wait_limit = call_wait_limit();
+    p.test_hook = call_test_hook();
     p.cu = d->n_seqs > 0 ? cu_dev : nullptr;
     char *base = static_cast<char *>(ws);
     p.hdr = reinterpret_cast<WsHeader *>(base);
@@ -334,6 +342,7 @@ gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.hT = hT;
     const bool tc = use_tc(pb, false);
     if (tc && !encode_row_maps(p, false)) return GDN_ERR_CUDA;
+    arm_planted_failure();
     if (start_call(p, desc, s) != cudaSuccess) return GDN_ERR_CUDA;
     if (!tc && pb.l2norm && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;
     cudaError_t e = tc ? launch_tc_fwd(p, pb, s) : launch_simt_fwd(p, s);
@@ -378,6 +387,7 @@ gdn_status gdn_bwd(const gdn_desc *desc, const void *q, const void *k, const voi
     p.dh0 = dh0;
     const bool tc = use_tc(pb, true);
     if (tc && !encode_row_maps(p, true)) return GDN_ERR_CUDA;
+    arm_planted_failure();
     if (start_call(p, desc, s) != cudaSuccess) return GDN_ERR_CUDA;
     const bool pre = !tc && pb.l2norm;
     if (pre && !normalise_qk(pb, L, workspace, &p, s)) return GDN_ERR_CUDA;

@@ -15,6 +15,10 @@ namespace gdn {
 constexpr int kChunk = 64;        // tokens per chunk (the chunkwise form's block length)
 constexpr int kSimtSlots = 512;   // CTAs of the SIMT chunk-parallel kernels (each owns a scratch slot)
 constexpr int kSimtVSlice = 32;   // value columns per CTA in the SIMT state passes
+// Polls of a bounded mbarrier wait (about a second) unless gdn_set_wait_limit
+// lowered it; the waits that drain copies still in flight after a failure
+// always use this one.
+constexpr uint32_t kWaitLimit = 1u << 23;
 
 // One chunk of one sequence: tokens [tok0, tok0 + len) of the flattened B*T rows.
 struct ChunkInfo {
@@ -40,6 +44,8 @@ struct Params {
     float scale;
     int32_t bf16;                  // 1: q/k/v/o/do/dq/dk/dv are bf16, 0: fp32
     int32_t l2norm;                // 1: q and k rows are divided by their norms first
+    uint32_t wait_limit;           // polls of a bounded mbarrier wait before it gives up
+    int32_t test_hook;             // planted failure for the tests (GDN_TEST_*), 0 = none
     // inputs
     const void *q, *k, *v, *do_;
     const float *g, *beta, *h0, *dhT;
@@ -173,10 +179,20 @@ enum KernelId : int32_t {
 void trace_before(int32_t id, cudaStream_t stream);
 void trace_after(cudaStream_t stream);
 
+// Per-host-thread settings of the testing hooks (gdn_set_wait_limit,
+// gdn_set_test_hook): the wait limit and hook the next call's kernels get,
+// arming the planted launch failure at the start of an ABI call, and taking it
+// (true once per armed call) before a launch.
+uint32_t call_wait_limit();
+int32_t call_test_hook();
+void arm_planted_failure();
+bool take_planted_failure();
+
 // Launches `...` (a kernel<<<>>>(...) expression) inside a trace bracket and
 // returns its launch error from the enclosing function.
 #define GDN_LAUNCH(id, stream, ...)                              \
     do {                                                         \
+        if (::gdn::take_planted_failure()) return cudaErrorLaunchFailure; \
         ::gdn::trace_before((id), (stream));                     \
         __VA_ARGS__;                                             \
         ::gdn::trace_after((stream));                            \

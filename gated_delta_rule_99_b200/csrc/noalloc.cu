@@ -51,3 +51,20 @@ extern "C" gdn_status gdn_fwd_noalloc(const gdn_desc *desc, const void *q, const
     return gdn_fwd(desc, q, k, v, g, beta, cu_seqlens, cu_seqlens_host, h0, o, hT, scratch,
                    (size_t)GDN_NOALLOC_MAX_WORKSPACE, stream);
 }
+
+// The status word heads the scratch (it is gdn_fwd's workspace header there),
+// so it is read and cleared through the symbol itself: no address lookup, and
+// a device that never ran gdn_fwd_noalloc reads its zero-initialised word.
+extern "C" gdn_status gdn_fwd_noalloc_status(void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    int32_t status = 0;
+    if (cudaMemcpyFromSymbol(&status, g_noalloc_scratch, sizeof(status)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (status != 0) {
+        const int32_t zero = 0;
+        if (cudaMemcpyToSymbol(g_noalloc_scratch, &zero, sizeof(zero)) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    return status == 0 ? GDN_OK : static_cast<gdn_status>(status);
+}

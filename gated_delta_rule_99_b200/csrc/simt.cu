@@ -1,7 +1,9 @@
 // fp32 SIMT kernels of the chunkwise Gated DeltaNet forward and backward.
 //
-// This is the exact-precision path (fp32 inputs) and the algebraic reference
-// the tensor-core path is checked against.  It follows the chunkwise form of
+// This is the path of fp32 inputs (fp32 CUDA-core FMAs throughout; the bf16
+// tensor-core path is a separate implementation of the same algebra, and both
+// are checked against the fp64 oracle, not against each other).  It follows the
+// chunkwise form of
 // the recurrence S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T,
 // o_t = scale S_t q_t (the pages name the method and its chunk-parallel
 // form -- jax-linear-attention 0.1.0, "How it works" -- without printing it).

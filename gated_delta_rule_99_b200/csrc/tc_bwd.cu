@@ -205,7 +205,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
                           &lbar[buf ^ 1]);
             pend |= 2u >> buf;
         }
-        const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, kWaitLimit);
+        const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
         uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
         const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
                        qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO),
@@ -441,7 +441,7 @@ __device__ __forceinline__ bool groups_arrived(uint64_t *bars, uint32_t mask, ui
                                                const Params &p, int where) {
     bool ok = true;
     for (int g = 0; g < kGrpCount; ++g)
-        if ((mask >> g) & 1) ok = ok && mbar_wait(&bars[g], parity, kWaitLimit);
+        if ((mask >> g) & 1) ok = ok && mbar_wait(&bars[g], parity, p.wait_limit);
     const bool all = __syncthreads_and(ok);
     if (!all && threadIdx.x == 0) record_timeout(p, where);
     return all;
@@ -518,8 +518,8 @@ __device__ __forceinline__ void ldcw(uint32_t tmem, int col, float *d) {
 
 // Bounded wait of one thread for an MMA-completion phase, after which it may
 // read the products (the CTA decides on a failure at its next barrier).
-__device__ __forceinline__ bool thread_wait(uint64_t *bar, uint32_t parity) {
-    const bool ok = mbar_wait(bar, parity, kWaitLimit);
+__device__ __forceinline__ bool thread_wait(uint64_t *bar, uint32_t parity, uint32_t limit) {
+    const bool ok = mbar_wait(bar, parity, limit);
     tc_fence_after();
     return ok;
 }
@@ -676,7 +676,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         // meanwhile, each thread waiting for what it reads itself (no barrier waits on the
         // issuing warp); the CTA decides on a failed wait at the barrier after them
         bool fine = true;
-        if (w4 < 2) fine = thread_wait(&mbar, phase);  // Q K^T and dP
+        if (w4 < 2) fine = thread_wait(&mbar, phase, p.wait_limit);  // Q K^T and dP
         phase ^= 1;
         if (w4 < 2) {  // row i = r of P and dP: P . dP (row and column partials), dPG = dP . Gam
             float pq[CW];
@@ -712,7 +712,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             stage_col(DA, y, cb, r);
             warp_colsum(d, wsum, w4, cb, l);
         }
-        fine = thread_wait(&mbar_c, it & 1) && fine;  // X1, X2, Y1
+        fine = thread_wait(&mbar_c, it & 1, p.wait_limit) && fine;  // X1, X2, Y1
         if (more) {  // S, dSn, U^T, dU^T, G and b of the next unit (every product reading
                      // them is complete: thread 0 waited for all three barriers)
             if (tid == 0) grads_fetch(p, sm, next, ci, kGrpImg, (it + 1) & 1, lbar);

@@ -16,7 +16,6 @@ using bf16 = __nv_bfloat16;
 constexpr int C = kChunk;      // 64
 constexpr int D = 128;         // d_k = d_v
 constexpr int NT = 128;        // threads per CTA
-constexpr uint32_t kWaitLimit = 1u << 23;
 
 constexpr size_t kImg64 = (size_t)C * D * 2;   // 64 x 128 bf16 tile image (16 KB)
 constexpr size_t kImg128 = (size_t)D * D * 2;  // 128 x 128 (32 KB)
@@ -34,7 +33,7 @@ __device__ __forceinline__ void record_timeout(const Params &p, int where) {
 // Bounded wait on an MMA-completion barrier, decided uniformly by the CTA.
 __device__ __forceinline__ bool cta_wait(uint64_t *mbar, uint32_t parity, const Params &p,
                                          int where) {
-    const bool ok = mbar_wait(mbar, parity, kWaitLimit);
+    const bool ok = mbar_wait(mbar, parity, p.wait_limit);
     const bool all_ok = __syncthreads_and(ok);
     if (!all_ok && threadIdx.x == 0) record_timeout(p, where);
     tc_fence_after();
@@ -89,7 +88,7 @@ __device__ __forceinline__ void fix_rows(uint8_t *tile, int R, int row0, int len
 // waits once more, bounded, so that no copy is left in flight when the CTA
 // gives up.
 __device__ __forceinline__ bool copies_arrived(uint64_t *bar, const Params &p, int where) {
-    const bool ok = __syncthreads_and(mbar_wait(bar, 0, kWaitLimit));
+    const bool ok = __syncthreads_and(mbar_wait(bar, 0, p.wait_limit));
     if (!ok && threadIdx.x == 0) {
         record_timeout(p, where);
         mbar_wait(bar, 0, kWaitLimit);
@@ -97,23 +96,27 @@ __device__ __forceinline__ bool copies_arrived(uint64_t *bar, const Params &p, i
     return ok;
 }
 
-// In-chunk cumulative log-decay (zero gates past len), summed in token order by
-// one thread so every kernel gets bit-identical values; also the write strengths.
+// In-chunk cumulative log-decay (zero gates past len) and the write strengths.
+// Threads 0-63 hold one token each: an inclusive shuffle scan inside each warp
+// (five steps, each lane adding in the same fixed order), then the second warp
+// adds the first warp's total.  Every kernel runs this same code, so all get
+// bit-identical values.  Called by the whole CTA (it ends with a barrier).
 __device__ __forceinline__ void chunk_gates(float *G, float *bta, const Params &p, const ChunkInfo &ci, int h) {
     const int r = threadIdx.x;
     if (r < C) {
         const int64_t idx = (int64_t)(ci.tok0 + r) * p.H + h;
-        G[r] = r < ci.len ? p.g[idx] : 0.f;
+        float x = r < ci.len ? p.g[idx] : 0.f;
         if (bta) bta[r] = r < ci.len ? p.beta[idx] : 0.f;
+        const int l = r & 31;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (l >= off) x += y;
+        }
+        G[r] = x;
     }
     __syncthreads();
-    if (r == 0) {
-        float s = 0.f;
-        for (int i = 0; i < C; ++i) {
-            s += G[i];
-            G[i] = s;
-        }
-    }
+    if (r >= 32 && r < C) G[r] += G[31];
     __syncthreads();
 }
 

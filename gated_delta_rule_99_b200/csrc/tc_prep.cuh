@@ -55,7 +55,10 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         mbar_init(&mbar, 1);
         mbar_init(&lbar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&lbar, row_tile_bytes(p.K) + row_tile_bytes(p.V));
+        // (the planted stall of the tests: 16 bytes more than the copies bring, on the
+        // first (chunk, head) only, so its bounded wait runs out after they have landed)
+        const uint32_t planted = (p.test_hook == GDN_TEST_STALL_COPY && ch == 0) ? 16u : 0u;
+        mbar_arrive_expect_tx(&lbar, row_tile_bytes(p.K) + row_tile_bytes(p.V) + planted);
         load_rows_tma(Kt, C, 0, &p.tm_k, ci.tok0, h, p.K, &lbar);
         load_rows_tma(Vt, C, 0, &p.tm_v, ci.tok0, h, p.V, &lbar);
     }

@@ -95,7 +95,7 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
             state_prefetch(sm, buf ^ 1, ch + H, p, with_ut, &lbar[buf ^ 1]);
             pend |= 2u >> buf;
         }
-        const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, kWaitLimit);
+        const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
         // the state entering this chunk, as bf16 operand rows
 #pragma unroll
         for (int j = 0; j < 16; ++j)

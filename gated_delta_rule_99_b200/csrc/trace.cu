@@ -5,6 +5,10 @@ namespace gdn {
 namespace {
 thread_local gdn_trace *g_trace = nullptr;
 thread_local bool g_open = false;
+// testing hooks (gdn_set_wait_limit, gdn_set_test_hook)
+thread_local uint32_t g_wait_limit = 0;
+thread_local int32_t g_hook = 0;
+thread_local bool g_fail_armed = false;
 
 const char *const kNames[kKernelCount] = {
     "build_chunks", "simt_prep", "simt_state_fwd", "simt_out", "simt_duloc", "simt_state_bwd",
@@ -41,9 +45,28 @@ void trace_after(cudaStream_t stream) {
     g_open = false;
 }
 
+uint32_t call_wait_limit() { return g_wait_limit ? g_wait_limit : kWaitLimit; }
+
+int32_t call_test_hook() { return g_hook; }
+
+void arm_planted_failure() { g_fail_armed = g_hook == GDN_TEST_FAIL_LAUNCH; }
+
+bool take_planted_failure() {
+    const bool f = g_fail_armed;
+    g_fail_armed = false;
+    return f;
+}
+
 }  // namespace gdn
 
 extern "C" {
+
+void gdn_set_wait_limit(uint32_t polls) { gdn::g_wait_limit = polls; }
+
+void gdn_set_test_hook(int32_t hook) {
+    gdn::g_hook = hook;
+    gdn::g_fail_armed = false;
+}
 
 void gdn_trace_install(gdn_trace *trace) {
     gdn::g_trace = trace;

@@ -143,14 +143,23 @@ gdn_status gdn_fwd(const gdn_desc *desc, const void *q, const void *k, const voi
  * call on each device looks up the array's device address with that device
  * current, so make the first call before any stream capture.  All calls share
  * the one array: calls that overlap on the GPU (other streams, other host
- * threads) race and corrupt each other's results, so serialise them.  Device-
- * side status is not reported for this entry point.  No allocation of any
- * kind is made. */
+ * threads) race and corrupt each other's results, so serialise them.  The
+ * device-side status of these calls lives in the array's header: read it with
+ * gdn_fwd_noalloc_status.  No allocation of any kind is made. */
 #define GDN_NOALLOC_MAX_WORKSPACE (64u * 1024u * 1024u)
 gdn_status gdn_fwd_noalloc(const gdn_desc *desc, const void *q, const void *k, const void *v,
                            const float *g, const float *beta, const int32_t *cu_seqlens,
                            const int32_t *cu_seqlens_host, const float *h0, void *o, float *hT,
                            void *stream);
+
+/* gdn_device_status for gdn_fwd_noalloc on the current device: synchronises
+ * the stream, then returns and clears the device-side status the last
+ * gdn_fwd_noalloc call on this device recorded in the library's static
+ * scratch (GDN_OK, GDN_ERR_TIMEOUT, or GDN_ERR_INVALID_ARG when the device copy
+ * of cu_seqlens disagreed with the host mirror).  GDN_OK if gdn_fwd_noalloc has
+ * not run on this device yet; GDN_ERR_CUDA if the stream failed.  It copies a
+ * few bytes between host and device and allocates nothing. */
+gdn_status gdn_fwd_noalloc_status(void *stream);
 
 /* Backward of (o, hT) given do_ and dhT (NULL means zero): writes dq, dk, dv,
  * dg, dbeta and dh0 (dh0 may be NULL to skip it).  The per-chunk states are
@@ -181,6 +190,30 @@ gdn_status gdn_device_status(void *workspace, void *stream);
 
 /* Static English name of a status code. */
 const char *gdn_status_string(gdn_status status);
+
+/* Testing hooks, per host thread (they let the tests drive the failure paths
+ * without faulting a GPU).  Both apply to every later call from the calling
+ * thread until changed; the defaults are 0.
+ *
+ * gdn_set_wait_limit: every bounded device-side wait of the tensor-core
+ * kernels gives up after `polls` polls of its mbarrier instead of the built-in
+ * 2^23 (about a second); 0 restores the built-in limit.  A wait that gives up
+ * records GDN_ERR_TIMEOUT, and the kernels of the call that start after it
+ * return at once (read it with gdn_device_status).
+ *
+ * gdn_set_test_hook: plants one failure in each later call.
+ *   GDN_TEST_STALL_COPY  the first (chunk, head) CTA of the call's tensor-core
+ *                        preparation step arms its input-copy mbarrier for 16
+ *                        bytes more than its copies bring: every copy lands,
+ *                        the wait runs out, and the call records
+ *                        GDN_ERR_TIMEOUT (outputs are then undefined).
+ *   GDN_TEST_FAIL_LAUNCH the call's first kernel launch is skipped and treated
+ *                        as a failed launch: the call returns GDN_ERR_CUDA.
+ * 0 removes the hook. */
+#define GDN_TEST_STALL_COPY 1
+#define GDN_TEST_FAIL_LAUNCH 2
+void gdn_set_wait_limit(uint32_t polls);
+void gdn_set_test_hook(int32_t hook);
 
 /* Optional launch tracing (profiling aid).  While a trace is installed on the
  * calling host thread, every kernel that gdn_fwd / gdn_bwd launch from that

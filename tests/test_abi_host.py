@@ -169,3 +169,31 @@ def test_decode_rejects_bad_arguments():
                         None) == 1
     assert L.gdn_decode(ctypes.byref(ok), *p, None, FAKE, None) == 1
     assert L.gdn_decode(ctypes.byref(ok), *p, FAKE + 4, FAKE, None) == 3
+
+
+def test_testing_hooks_match_header_and_are_callable_without_a_gpu():
+    hdr = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    defs = dict(re.findall(r"#define (GDN_TEST_\w+) (\d+)", hdr))
+    assert int(defs["GDN_TEST_STALL_COPY"]) == gdn.GDN_TEST_STALL_COPY
+    assert int(defs["GDN_TEST_FAIL_LAUNCH"]) == gdn.GDN_TEST_FAIL_LAUNCH
+    # per-thread settings only: setting and clearing them touches no device
+    gdn.set_wait_limit(1000)
+    gdn.set_test_hook(gdn.GDN_TEST_FAIL_LAUNCH)
+    gdn.set_test_hook(0)
+    gdn.set_wait_limit(0)
+    # an argument error still comes first, hook or not
+    gdn.set_test_hook(gdn.GDN_TEST_FAIL_LAUNCH)
+    try:
+        assert _fwd(gdn.make_desc(B=0, T=10, H=1, dk=64, dv=64), ws_bytes=1 << 20) == 1
+    finally:
+        gdn.set_test_hook(0)
+
+
+def test_descriptor_products_are_range_checked_before_they_are_formed():
+    # B * T would overflow a signed 64-bit product; both are rejected first
+    for B, T in ((1 << 40, 1 << 40), (3, (1 << 62)), (1 << 62, 2)):
+        d = gdn.make_desc(B=B, T=T, H=1, dk=64, dv=64)
+        assert gdn.fwd_workspace_size(d) == 0
+    # (chunk, head) grids must stay within int32
+    d = gdn.make_desc(B=1, T=(1 << 31) - 64, H=1 << 10, dk=64, dv=64)
+    assert gdn.fwd_workspace_size(d) == 0

@@ -40,21 +40,14 @@ def test_piece_scan_matches_oracle_and_default_path(B, T, H, gate):
 
 
 def test_piece_scan_long_context_workload():
+    """The long-row workload on the piece scan equals the default sequential
+    path up to the bf16 rounding of the transition matrices (both are checked
+    against the fp64 oracle over the whole row in
+    test_gpu_parity.py::test_long_context_full_row_against_oracle)."""
     inp = workload(4, device="cuda")
     o_p, h_p = _fwd(inp, True)
     o_s, h_s = _fwd(inp, False)
     e_o = maxnorm_err(o_p.float(), o_s.float().cpu().numpy().astype(np.float64))
     e_h = maxnorm_err(h_p, h_s.cpu().numpy().astype(np.float64))
-    P = 4096
-    cpu = lambda x: x[:, -P:].cpu()
-    # the tail of the row, against the oracle run from the default path's state there is not
-    # allowed (no oracle input from the CUDA path): compare the head instead
-    ro, _ = oracle.gdn_fwd(inp.q[:, :P].cpu(), inp.k[:, :P].cpu(), inp.v[:, :P].cpu(),
-                           inp.g[:, :P].cpu(), inp.beta[:, :P].cpu(), h0=inp.h0.cpu(),
-                           units=[(0, 0), (0, 5)])
-    m = np.isfinite(ro)
-    e_head = maxnorm_err(np64(o_p[:, :P].cpu())[m], ro[m])
-    print("piece scan long row: o vs sequential %.2e, hT vs sequential %.2e, head vs oracle %.2e"
-          % (e_o, e_h, e_head))
-    assert e_o <= TOL and e_h <= TOL and e_head <= TOL
-    del cpu
+    print("piece scan long row: o vs sequential %.2e, hT vs sequential %.2e" % (e_o, e_h))
+    assert e_o <= TOL and e_h <= TOL

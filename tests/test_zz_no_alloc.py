@@ -60,3 +60,25 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     rc = gdn.lib().gdn_fwd_noalloc(ctypes.byref(desc), p, p, p, p, p, None, None, None, p, None,
                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == 4  # GDN_ERR_WORKSPACE, returned before any launch
+
+
+def test_noalloc_status_reports_and_clears_device_side_failures():
+    """The device-side status of gdn_fwd_noalloc lives in the library's static
+    scratch; gdn_fwd_noalloc_status reads and clears it.  A device copy of
+    cu_seqlens that disagrees with the host mirror is caught on the device."""
+    inp = make_inputs(B=1, T=200, H=1, K=64, V=64, dtype="bf16", seed=19, lengths=[100, 100])
+    d = inp.to("cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    L = gdn.lib()
+    o = torch.empty_like(d.v)
+    hT = torch.empty(2, 1, 64, 64, device="cuda")
+    bad_dev = torch.tensor([0, 201, 200], dtype=torch.int32, device="cuda")
+    assert _noalloc(d, bad_dev, inp.cu_seqlens, o, hT) == 0  # accepted on the host
+    assert L.gdn_fwd_noalloc_status(stream) == 1             # GDN_ERR_INVALID_ARG on the device
+    assert L.gdn_fwd_noalloc_status(stream) == 0             # cleared by the read
+    assert _noalloc(d, inp.cu_seqlens.cuda(), inp.cu_seqlens, o, hT) == 0
+    assert L.gdn_fwd_noalloc_status(stream) == 0
+    ref_o, ref_h = gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, cu_seqlens=inp.cu_seqlens.cuda(),
+                               cu_seqlens_host=inp.cu_seqlens, h0=d.h0)
+    torch.cuda.synchronize()
+    assert maxnorm_err(o, ref_o) <= TOL["bf16"] and maxnorm_err(hT, ref_h) <= TOL["bf16"]
