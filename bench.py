@@ -133,7 +133,8 @@ def csrc_hash() -> str:
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from profiles/traffic.md, or None if the sources changed."""
+    """DRAM bytes of all of a kernel's launches in one step, from profiles/traffic.md,
+    or None if the sources changed since the capture."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.md")) as f:
             lines = f.read().splitlines()
@@ -467,9 +468,16 @@ def run_ours(args, rank, world, local_rank):
     dom = max(per_kernel.items(), key=lambda kv: kv[1][1]) if per_kernel else None
     roof = None
     if dom:
+        # a kernel may launch several times per step (the forward runs in parts of every
+        # row): the work of all its launches in a step over their summed event time
         name, (n, ms) = dom
         per_launch_s = ms / n / 1e3
+        per_step = n / args.steps
         bound, amount, unit = kernel_work(name, w, n_chunks)
+        if amount is not None:  # algorithmic work of one launch: the passes a step makes
+            # over the whole workload (the fp32 path's prep and forward chain run in both
+            # gdn_fwd and gdn_bwd) spread over the step's launches
+            amount *= {"simt_prep": 2, "simt_state_fwd": 2}.get(name, 1) / per_step
         if bound == "alu":
             peak = alu_peak_tflops(pk["sm_mhz"])
             ach = amount / per_launch_s / 1e12
@@ -482,11 +490,12 @@ def run_ours(args, rank, world, local_rank):
             ach = amount / per_launch_s / (1e9 if bound == "hbm" else 1e12)
             wl = ("gdn_fwdbwd_bf16_B4_T4096_H16_d128" if not args.shape else
                   "gdn_fwdbwd_bf16_B%d_T%d_H%d_d128" % (B, T, H))
+            tr = recorded_traffic(name, wl)
             roof = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak,
                     "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": ach / peak,
-                    "traffic": recorded_traffic(name, wl),
+                    "traffic": None if tr is None else tr / per_step,
                     "algorithmic": amount, "peak_source": pk["src"],
-                    "ms_per_launch": per_launch_s * 1e3}
+                    "ms_per_launch": per_launch_s * 1e3, "launches_per_step": per_step}
     sr = step_roofline(w, pk)
     cpu = None
     if not args.no_cpu_baseline and world == 1:

@@ -40,6 +40,7 @@ class GdnDesc(ctypes.Structure):
 
 GDN_FLAG_PIECE_SCAN = 1
 GDN_FLAG_QK_L2NORM = 2
+GDN_FLAG_VALUE_SLICES = 4
 
 
 _lock = threading.Lock()
@@ -149,14 +150,16 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, output_final_state=True,
             o=None, hT=None, workspace=None, cu_seqlens_host=None, stream=None, piece_scan=False,
-            qk_l2norm=False):
+            qk_l2norm=False, value_slices=False):
     """Forward of the gated delta rule through the C ABI.  Returns (o, hT);
     hT is None when output_final_state is False.  piece_scan sets
     GDN_FLAG_PIECE_SCAN (parallel pieces of long dense rows, joined exactly);
-    qk_l2norm sets GDN_FLAG_QK_L2NORM (q and k rows divided by their norms)."""
+    qk_l2norm sets GDN_FLAG_QK_L2NORM (q and k rows divided by their norms);
+    value_slices sets GDN_FLAG_VALUE_SLICES (chains split by value columns)."""
     L = lib()
     cu_dev, cu_host = _seqlens(cu_seqlens, cu_seqlens_host, q.device)
-    flags = (GDN_FLAG_PIECE_SCAN if piece_scan else 0) | (GDN_FLAG_QK_L2NORM if qk_l2norm else 0)
+    flags = ((GDN_FLAG_PIECE_SCAN if piece_scan else 0) | (GDN_FLAG_QK_L2NORM if qk_l2norm else 0)
+             | (GDN_FLAG_VALUE_SLICES if value_slices else 0))
     desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale, flags)
     N = n_seqs if n_seqs else B
     _check(q, "q", q.dtype, (B, T, H, K)); _check(k, "k", q.dtype, (B, T, H, K))

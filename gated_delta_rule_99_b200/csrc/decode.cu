@@ -138,7 +138,8 @@ extern "C" gdn_status gdn_decode(const gdn_desc *d, const void *q, const void *k
         d->T >= kLim / d->B)
         return GDN_ERR_INVALID_ARG;
     if (!(d->scale == d->scale)) return GDN_ERR_INVALID_ARG;
-    if (d->reserved != 0 || (d->flags & ~(GDN_FLAG_PIECE_SCAN | GDN_FLAG_QK_L2NORM)))
+    if (d->reserved != 0 ||
+        (d->flags & ~(GDN_FLAG_PIECE_SCAN | GDN_FLAG_QK_L2NORM | GDN_FLAG_VALUE_SLICES)))
         return GDN_ERR_INVALID_ARG;
     if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, g, beta, state, o};

@@ -44,9 +44,11 @@ gdn_status describe(const gdn_desc *d, Problem *p) {
     p->NC = 0;
     p->dtype = d->dtype;
     p->scale = d->scale;
-    if (d->reserved != 0 || (d->flags & ~(GDN_FLAG_PIECE_SCAN | GDN_FLAG_QK_L2NORM)))
+    if (d->reserved != 0 ||
+        (d->flags & ~(GDN_FLAG_PIECE_SCAN | GDN_FLAG_QK_L2NORM | GDN_FLAG_VALUE_SLICES)))
         return GDN_ERR_INVALID_ARG;
     p->l2norm = (d->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    p->vslice = (d->flags & GDN_FLAG_VALUE_SLICES) ? 1 : 0;
     p->P = 1;
     p->L = 0;
     if ((d->flags & GDN_FLAG_PIECE_SCAN) && d->n_seqs == 0 && d->dtype == GDN_BF16 &&
@@ -117,6 +119,7 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.scale = d->scale;
     p.bf16 = d->dtype == GDN_BF16;
     p.l2norm = pb.l2norm;
+    p.vslice = pb.vslice;
     p.wait_limit = call_wait_limit();
     p.test_hook = call_test_hook();
     p.cu = d->n_seqs > 0 ? cu_dev : nullptr;

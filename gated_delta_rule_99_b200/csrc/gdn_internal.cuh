@@ -44,6 +44,7 @@ struct Params {
     float scale;
     int32_t bf16;                  // 1: q/k/v/o/do/dq/dk/dv are bf16, 0: fp32
     int32_t l2norm;                // 1: q and k rows are divided by their norms first
+    int32_t vslice;                // 1: the forward chains run by value slices (GDN_FLAG_VALUE_SLICES)
     uint32_t wait_limit;           // polls of a bounded mbarrier wait before it gives up
     int32_t test_hook;             // planted failure for the tests (GDN_TEST_*), 0 = none
     // inputs
@@ -120,6 +121,7 @@ struct Problem {
     float scale;
     int64_t P, L;   // pieces per sequence (1 = no piece scan) and chunks per piece
     int l2norm;     // GDN_FLAG_QK_L2NORM
+    int vslice;     // GDN_FLAG_VALUE_SLICES
 };
 
 // Workspace layout: offsets in bytes from the workspace base.

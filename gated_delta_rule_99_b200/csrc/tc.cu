@@ -33,8 +33,10 @@ __global__ void __launch_bounds__(NT, 4) tc_prep_kernel(const __grid_constant__ 
 }
 
 // ============================================================ tc_state_fwd
+// One CTA per (sequence, head), or per (sequence, head, value slice) with p.vslice.
 __global__ void __launch_bounds__(NT, 1) tc_state_fwd_kernel(Params p) {
-    state_fwd_body(p, blockIdx.x);
+    if (p.vslice) state_fwd_sliced_body(p, blockIdx.x);
+    else state_fwd_body(p, blockIdx.x);
 }
 
 // ============================================================ piece scan (long rows)
@@ -54,11 +56,13 @@ __device__ __forceinline__ void piece_range(const Params &p, int n, int piece, i
 // 1 <= q <= P - 2 runs once from zero (-> B_q, the offset of its affine map)
 // and once from the identity with Ut taken as zero (-> M_q, its transition).
 __global__ void __launch_bounds__(NT, 1) tc_piece_a_kernel(Params p) {
-    const int roles = 2 * p.P - 3, unit = blockIdx.x / roles, r = blockIdx.x % roles;
+    const int nsl = p.vslice ? value_slices(p) : 1, roles = 2 * p.P - 3, blk = blockIdx.x / nsl;
+    const int unit = blk / roles, r = blk % roles;
     const int n = unit / p.H, h = unit % p.H;
     const size_t u = (size_t)unit * p.P, DD = (size_t)D * D;
     ChainFwd a;
     a.h = h;
+    a.slice = blockIdx.x % nsl;
     a.where = 31;
     a.init_user = 1;  // h0 (piece 0); the middle pieces start from zero or the identity
     a.out_user = 0;   // tHin, tBp, tMp are internal [128][128] blocks
@@ -86,7 +90,8 @@ __global__ void __launch_bounds__(NT, 1) tc_piece_a_kernel(Params p) {
         a.final_out = p.tMp + (u + piece) * DD;
     }
     piece_range(p, n, piece, &a.c0, &a.c1);
-    chain_fwd(p, a);
+    if (p.vslice) chain_fwd_sliced(p, a);
+    else chain_fwd(p, a);
 }
 
 // Phase B: per (row, head), the entering state of piece q >= 2,
@@ -167,11 +172,13 @@ __global__ void __launch_bounds__(NT, 1) tc_piece_scan_kernel(Params p) {
 // Phase C: every piece q >= 1 reruns its chain from its entering state,
 // writing the per-chunk snapshots; the last piece writes hT.
 __global__ void __launch_bounds__(NT, 1) tc_piece_c_kernel(Params p) {
-    const int per = p.P - 1, unit = blockIdx.x / per, piece = 1 + blockIdx.x % per;
+    const int nsl = p.vslice ? value_slices(p) : 1, blk = blockIdx.x / nsl;
+    const int per = p.P - 1, unit = blk / per, piece = 1 + blk % per;
     const int n = unit / p.H, h = unit % p.H;
     const size_t DD = (size_t)D * D;
     ChainFwd a;
     a.h = h;
+    a.slice = blockIdx.x % nsl;
     a.where = 35;
     a.init_user = 0;  // tHin
     a.out_user = 1;   // hT
@@ -181,12 +188,16 @@ __global__ void __launch_bounds__(NT, 1) tc_piece_c_kernel(Params p) {
     a.snapshots = 1;
     a.final_out = (piece == p.P - 1 && p.hT) ? p.hT + (size_t)unit * DD : nullptr;
     piece_range(p, n, piece, &a.c0, &a.c1);
-    chain_fwd(p, a);
+    if (p.vslice) chain_fwd_sliced(p, a);
+    else chain_fwd(p, a);
 }
 
 // ============================================================ tc_out
 // O^T[v][i] = S[v][:] . (scale gam_i q_i) + sum_j U^T[v][j] P[i][j],
-// P = scale lower(Q K^T . Gam).  One CTA per (chunk, head).
+// P = scale lower(Q K^T . Gam).  One CTA per (chunk, head).  The snapshots come
+// as S (rows = values) and U^T tiles, read K-major, or, from the chain by value
+// slices (p.vslice), as H = S^T (rows = keys) and U (rows = tokens) tiles, read
+// MN-major: the same A operands of the two M = 128 products.
 struct OutSmem {
     static constexpr int kQK = 0, kS = kQK + 32768, kUT = kS + 32768, kQG = kUT + 16384,
                          kP = kQG + 16384, kG = kP + 8192, kEnd = kG + 256;
@@ -256,15 +267,25 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(const __grid_constant__ Para
         build_p_tile(tmem, G, p.scale, Ps);
         operands_ready();
         if (tid == 0) {
-            const uint32_t id = idesc_bf16(128, 64, 0, 0);
             const uint32_t sb = smem_u32(Ss), qg = smem_u32(QG), ub = smem_u32(UTs),
                            pb = smem_u32(Ps);
+            if (!p.vslice) {
+                const uint32_t id = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
-            for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tmem + 64, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
+                for (int s = 0; s < D / 16; ++s)
+                    mma_bf16(tmem + 64, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
 #pragma unroll
-            for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_kmajor(pb, C, s), id, 1);
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_kmajor(pb, C, s), id, 1);
+            } else {
+                const uint32_t id = idesc_bf16(128, 64, 1, 0);
+#pragma unroll
+                for (int s = 0; s < D / 16; ++s)
+                    mma_bf16(tmem + 64, desc_mnmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tmem + 64, desc_mnmajor(ub, C, s), desc_kmajor(pb, C, s), id, 1);
+            }
             mma_commit(&mbar);
         }
         ok = cta_wait(&mbar, 1, p, 6);
@@ -312,12 +333,17 @@ cudaError_t tc_launch_prep(const Params &p, int want_A, cudaStream_t stream) {
     return cudaSuccess;
 }
 
+// CTAs per forward chain, and their shared memory: one per (sequence, head), or one
+// per value slice with p.vslice.
+static int chain_slices(const Params &p) { return p.vslice ? (p.V + 63) / 64 : 1; }
+static int chain_smem(const Params &p) { return p.vslice ? kSliceSmem : kStateSmem; }
+
 cudaError_t tc_launch_state_fwd(const Params &p, cudaStream_t stream) {
-    const int nseq = p.N * p.H;
+    const int nseq = p.N * p.H * chain_slices(p), sm = chain_smem(p);
     if (nseq == 0) return cudaSuccess;
-    cudaError_t e = set_smem(tc_state_fwd_kernel, kStateSmem);
+    cudaError_t e = set_smem(tc_state_fwd_kernel, sm);
     if (e != cudaSuccess) return e;
-    GDN_LAUNCH(kKTcStateFwd, stream, tc_state_fwd_kernel<<<nseq, NT, kStateSmem, stream>>>(p));
+    GDN_LAUNCH(kKTcStateFwd, stream, tc_state_fwd_kernel<<<nseq, NT, sm, stream>>>(p));
     return cudaSuccess;
 }
 
@@ -325,16 +351,16 @@ cudaError_t launch_tc_fwd(const Params &p, const Problem &, cudaStream_t stream)
     cudaError_t e;
     if ((e = tc_launch_prep(p, 0, stream))) return e;
     if (p.P > 1 && p.N * p.H > 0) {  // piece scan of long rows
-        const int units = p.N * p.H;
-        if ((e = set_smem(tc_piece_a_kernel, kStateSmem))) return e;
+        const int units = p.N * p.H, nsl = chain_slices(p), sm = chain_smem(p);
+        if ((e = set_smem(tc_piece_a_kernel, sm))) return e;
         GDN_LAUNCH(kKTcPieceA, stream,
-                   tc_piece_a_kernel<<<units * (2 * p.P - 3), NT, kStateSmem, stream>>>(p));
+                   tc_piece_a_kernel<<<units * (2 * p.P - 3) * nsl, NT, sm, stream>>>(p));
         if ((e = set_smem(tc_piece_scan_kernel, kScanSmem))) return e;
         GDN_LAUNCH(kKTcPieceScan, stream,
                    tc_piece_scan_kernel<<<units, NT, kScanSmem, stream>>>(p));
-        if ((e = set_smem(tc_piece_c_kernel, kStateSmem))) return e;
+        if ((e = set_smem(tc_piece_c_kernel, sm))) return e;
         GDN_LAUNCH(kKTcPieceC, stream,
-                   tc_piece_c_kernel<<<units * (p.P - 1), NT, kStateSmem, stream>>>(p));
+                   tc_piece_c_kernel<<<units * (p.P - 1) * nsl, NT, sm, stream>>>(p));
     } else if ((e = tc_launch_state_fwd(p, stream))) {
         return e;
     }

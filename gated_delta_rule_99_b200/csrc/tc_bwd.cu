@@ -124,11 +124,13 @@ __global__ void __launch_bounds__(NT, 4) tc_prep_local_kernel(const __grid_const
 
 // ============================================================ tc_state_bwd
 struct SbwdSmem {
-    static constexpr int kdS = 0, kdU = kdS + 32768, kBuf = kdU + 16384;
-    // per buffer: Kd image, W image, Qg image, dO tile, P tile, gates
+    // two dS images (the next chunk's is written while the current one may still be
+    // read), dU^T, then per prefetch buffer: Kd image, W image, Qg image, dO tile,
+    // P tile; the buffers' gate rows last
+    static constexpr int kdS0 = 0, kdU = kdS0 + 2 * 32768, kBuf = kdU + 16384;
     static constexpr int kKd = 0, kW = 16384, kQg = 32768, kDO = 49152, kP = 65536,
-                         kG = 73728, kBufBytes = 73728 + 1024;
-    static constexpr int kEnd = kBuf + 2 * kBufBytes;
+                         kBufBytes = 73728;
+    static constexpr int kGr = kBuf + 2 * kBufBytes, kEnd = kGr + 2 * 256;
 };
 constexpr int kSbwdSmem = SbwdSmem::kEnd + 1024;
 
@@ -149,7 +151,7 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
                   kImg64, bar);
         bulk_load(smem_u32(b + SbwdSmem::kP),
                   static_cast<const uint8_t *>(p.tP) + ch * (size_t)(C * C * 2), C * C * 2, bar);
-        bulk_load(smem_u32(b + SbwdSmem::kG), p.tG + ch * C, C * 4, bar);
+        bulk_load(smem_u32(sm + SbwdSmem::kGr + buf * 256), p.tG + ch * C, C * 4, bar);
         load_rows_tma(b + SbwdSmem::kDO, C, 0, &p.tm_do, ci.tok0, h, p.V, bar);
     }
 }
@@ -181,6 +183,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         tmem_alloc(&tslot, 256);
         tmem_relinquish();
     }
+    state_image(sm + SbwdSmem::kdS0, S, v);  // dS leaving the last chunk
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -194,7 +197,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
                       &lbar[0]);
         pend = 1;
     }
-    uint8_t *dSs = sm + SbwdSmem::kdS, *dUs = sm + SbwdSmem::kdU;
+    uint8_t *dUs = sm + SbwdSmem::kdU;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0), idx = idesc_bf16(128, 128, 1, 1),
                    idy = idesc_bf16(128, 128, 0, 1), idp = idesc_bf16(128, 64, 1, 1);
     for (int c = c1 - 1; c >= c0; --c) {
@@ -207,13 +210,15 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         }
         const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
         uint8_t *b = sm + SbwdSmem::kBuf + buf * SbwdSmem::kBufBytes;
+        // the dS image this chunk reads (written by the previous chunk's update), and the
+        // one this chunk's update writes
+        uint8_t *dSs = sm + SbwdSmem::kdS0 + buf * 32768, *dSn = sm + SbwdSmem::kdS0 + (buf ^ 1) * 32768;
         const uint32_t sb = smem_u32(dSs), kb = smem_u32(b + SbwdSmem::kKd),
                        qb = smem_u32(b + SbwdSmem::kQg), ob = smem_u32(b + SbwdSmem::kDO),
                        pb = smem_u32(b + SbwdSmem::kP);
         // dO^T P (the local dU^T; M = 128 (v), N = 64, K = 64 tokens) and dO^T Qg (M = 128,
         // N = 128 keys, K = 64) do not depend on dS: on a full chunk (whose dO rows need no
-        // clearing) thread 0 issues them as soon as its copies landed, under the dS image
-        // writes below
+        // clearing) thread 0 issues them as soon as its copies landed
         const int len = chunk_in_seq(p, n, c0, c).len;
         const bool early = len == C && p.V == D;
         auto issue_local = [&]() {
@@ -226,9 +231,6 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         };
         if (v == 0 && lok && early) issue_local();
         if (lok && !early) fix_rows(b + SbwdSmem::kDO, C, 0, len, p.V);
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            *reinterpret_cast<uint4 *>(dSs + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
         fence_async_smem();
         tc_fence_before();
         const bool all = __syncthreads_and(lok);
@@ -239,7 +241,8 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         }
         pend &= ~(1u << buf);
         lpar ^= 1u << buf;
-        const float gC = expf(reinterpret_cast<const float *>(b + SbwdSmem::kG)[C - 1]);
+        const float gC =
+            expf(reinterpret_cast<const float *>(sm + SbwdSmem::kGr + buf * 256)[C - 1]);
         if (v == 0) {
             if (!early) issue_local();
             // + dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
@@ -249,6 +252,9 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
             mma_commit(&mbar);
             bulk_store(static_cast<uint8_t *>(p.tdSn) + ch * kImg128, sb, (uint32_t)kImg128);
             bulk_commit();
+            // the previous chunk's stores (dU^T, and the dS image this chunk's update
+            // rewrites) have read their sources
+            bulk_wait_read_n<1>();
         }
         if (!cta_wait(&mbar, phase, p, 13)) break;
         phase ^= 1;
@@ -282,8 +288,11 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)  // the next chunk's dS image
+                *reinterpret_cast<uint4 *>(dSn + sw128_chunk(D, v, c32 / 8 + q)) =
+                    pack8(S + c32 + 8 * q);
         }
-        if (v == 0) bulk_wait_read();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();

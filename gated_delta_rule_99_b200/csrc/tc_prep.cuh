@@ -9,7 +9,7 @@ namespace tc {
 
 // ============================================================ tc_prep
 // Per (chunk, head): gates, A = (I + L)^-1 (fp32, by 16 x 16 blocks), and the
-// tile images W, Kd and the plain rows of Ut that the state pass consumes.
+// tile images W, Kd and Ut that the state chains consume.
 constexpr int LS = 68;  // row stride (floats) of L: 16-byte aligned rows for vector loads
 
 struct PrepSmem {
@@ -316,16 +316,17 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             phase ^= 1;
         }
     }
-    if (ok) {
+    if (ok) {  // Ut as a 64 x 128 tile image (rows = tokens): an operand of the chains'
+               // first product, whose 64-column blocks are the two halves of the values
         const int i = m64_row();
-        bf16 *Ut = static_cast<bf16 *>(p.tUt) + (size_t)ch * C * D;
+        uint8_t *Ut = static_cast<uint8_t *>(p.tUt) + (size_t)ch * kImg64;
         for (int c0 = 0; c0 < D; c0 += 16) {
             float u[16];
             tmem_ld16(tm(tmem, c0), u);
             tmem_ld_wait();
             if (i >= 0) {
-                *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0) = pack8(u);
-                *reinterpret_cast<uint4 *>(Ut + (size_t)i * D + c0 + 8) = pack8(u + 8);
+                *reinterpret_cast<uint4 *>(Ut + sw128_chunk(C, i, c0 / 8)) = pack8(u);
+                *reinterpret_cast<uint4 *>(Ut + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(u + 8);
             }
         }
     }

@@ -11,14 +11,17 @@ namespace tc {
 // ============================================================ tc_state_fwd
 // One CTA per (sequence, head); thread v owns row v of S (fp32 registers).
 struct StateSmem {
-    static constexpr int kS = 0, kUT = kS + 32768, kW0 = kUT + 16384, kKd0 = kW0 + 2 * 16384,
-                         kUt0 = kKd0 + 2 * 16384, kG0 = kUt0 + 2 * 16384, kEnd = kG0 + 2 * 256;
+    // two images of the state (the next chunk's is written while the current one
+    // may still be read), U^T, the 64 x 64 identity block that adds Ut^T inside
+    // the first product, and per prefetch buffer the W, Kd and Ut images and gates
+    static constexpr int kS0 = 0, kUT = kS0 + 2 * 32768, kI = kUT + 16384, kW0 = kI + 8192,
+                         kKd0 = kW0 + 2 * 16384, kUt0 = kKd0 + 2 * 16384, kG0 = kUt0 + 2 * 16384,
+                         kEnd = kG0 + 2 * 256;
 };
 constexpr int kStateSmem = StateSmem::kEnd + 1024;
 
-// Bulk copies (thread 0) of chunk ch's W and Kd images, its Ut rows (unless
-// the run takes Ut as zero) and its gate row into buffer `buf`, completing
-// on `bar`.
+// Bulk copies (thread 0) of chunk ch's W, Kd and Ut images (Ut unless the run
+// takes it as zero) and its gate row into buffer `buf`, completing on `bar`.
 __device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p,
                                                bool with_ut, uint64_t *bar) {
     if (threadIdx.x != 0) return;
@@ -44,9 +47,31 @@ struct ChainFwd {
     float *final_out;    // state leaving chunk c1 - 1 (fp32), or nullptr
     int out_user;        // final_out is a caller's [K][V] block (else [128][128])
     int where;           // tag recorded if a bounded wait gives up
+    int slice;           // value columns [64 slice, 64 slice + 64) (chain_fwd_sliced only)
 };
 
+// Writes the 64 x 64 bf16 identity as an SW128 tile (all threads of the CTA).
+__device__ __forceinline__ void identity_tile(uint8_t *tile) {
+    for (int t = threadIdx.x; t < C * 8; t += NT) {
+        const int r = t >> 3, j = t & 7;
+        float f[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] = (r == 8 * j + q) ? 1.f : 0.f;
+        *reinterpret_cast<uint4 *>(tile + sw128_chunk(C, r, j)) = pack8(f);
+    }
+}
+
+// Row v of the state as bf16 operand row v of a 128 x 128 SW128 tile.
+__device__ __forceinline__ void state_image(uint8_t *img, const float *S, int v) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        *reinterpret_cast<uint4 *>(img + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
+}
+
 // The forward state chain: thread v owns row v of S = H^T (fp32 registers).
+// Per chunk the first product adds Ut^T through an identity block, so U^T
+// leaves the accumulator ready to be rounded; the state image of the next
+// chunk is written into the other image while the state is updated.
 __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
@@ -73,12 +98,14 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         tmem_alloc(&tslot, 256);
         tmem_relinquish();
     }
+    const bool with_ut = !a.zero_ut;
+    identity_tile(sm + StateSmem::kI);
+    state_image(sm + StateSmem::kS0, S, v);  // the state entering the first chunk
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
     const int c0 = a.c0, c1 = a.c1;
-    const bool with_ut = !a.zero_ut;
     uint32_t phase = 0;
     // per buffer b (bit b): a copy in flight, and the parity of its next completion
     uint32_t pend = 0, lpar = 0;
@@ -86,21 +113,19 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         state_prefetch(sm, 0, (size_t)c0 * H + h, p, with_ut, &lbar[0]);
         pend = 1;
     }
-    uint8_t *Ss = sm + StateSmem::kS, *UTs = sm + StateSmem::kUT;
-    const uint32_t id1 = idesc_bf16(128, 64, 0, 0), id2 = idesc_bf16(128, 128, 0, 1);
+    uint8_t *UTs = sm + StateSmem::kUT;
+    const uint32_t id1 = idesc_bf16(128, 64, 0, 0), idu = idesc_bf16(128, 64, 1, 0),
+                   id2 = idesc_bf16(128, 128, 0, 1), ib = smem_u32(sm + StateSmem::kI);
     for (int c = c0; c < c1; ++c) {
         const int buf = (c - c0) & 1;
         const size_t ch = (size_t)c * H + h;
+        uint8_t *Ss = sm + StateSmem::kS0 + buf * 32768, *Sn = sm + StateSmem::kS0 + (buf ^ 1) * 32768;
         if (c + 1 < c1) {
             state_prefetch(sm, buf ^ 1, ch + H, p, with_ut, &lbar[buf ^ 1]);
             pend |= 2u >> buf;
         }
         const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
-        // the state entering this chunk, as bf16 operand rows
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        fence_async_smem();
+        fence_async_smem();  // the state image written by the previous chunk's update
         tc_fence_before();
         const bool all = __syncthreads_and(lok);
         tc_fence_after();
@@ -112,30 +137,34 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         lpar ^= 1u << buf;
         const float gC =
             expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
-        if (v == 0) {
-            const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384);
+        if (v == 0) {  // U^T = S (-W)^T + Ut^T I  (the W image is stored negated)
+            const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384),
+                           ub = smem_u32(sm + StateSmem::kUt0 + buf * 16384);
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
                 mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
+            if (with_ut) {
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(ib, C, s), idu, 1);
+            }
             mma_commit(&mbar);
             if (a.snapshots) {
                 bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128, sb, (uint32_t)kImg128);
                 bulk_commit();
+                // the previous chunk's stores (U^T, and the state image that this chunk's
+                // update rewrites) have read their sources
+                bulk_wait_read_n<1>();
             }
         }
         if (!cta_wait(&mbar, phase, p, a.where)) break;
         phase ^= 1;
-        // U^T[v][i] = Ut[i][v] - (S W^T)[v][i]
-        const bf16 *Ut = reinterpret_cast<const bf16 *>(sm + StateSmem::kUt0 + buf * 16384);
 #pragma unroll
-        for (int c32 = 0; c32 < C; c32 += 32) {
+        for (int c32 = 0; c32 < C; c32 += 32) {  // U^T as an operand tile (row v)
             float d[32];
             tmem_ld16(tm(tmem, c32), d);
             tmem_ld16(tm(tmem, c32 + 16), d + 16);
             tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-                d[q] = (with_ut ? __bfloat162float(Ut[(c32 + q) * D + v]) : 0.f) + d[q];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
@@ -155,16 +184,18 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         if (!cta_wait(&mbar, phase, p, a.where + 1)) break;
         phase ^= 1;
 #pragma unroll
-        for (int c32 = 0; c32 < D; c32 += 32) {
+        for (int c32 = 0; c32 < D; c32 += 32) {  // S <- gam_n S + U^T Kd, and the next image
             float d[32];
             tmem_ld16(tm(tmem, 64 + c32), d);
             tmem_ld16(tm(tmem, 64 + c32 + 16), d + 16);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(Sn + sw128_chunk(D, v, c32 / 8 + q)) =
+                    pack8(S + c32 + 8 * q);
         }
-        // shared operands are rewritten next chunk: their bulk stores must have read them
-        if (v == 0 && a.snapshots) bulk_wait_read();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -187,6 +218,191 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     if (v < 32) tmem_dealloc(tmem, 256);
 }
 
+// ============================================================ chain by value slices
+// The value columns of the state evolve independently given a chunk's W, Kd,
+// gates and their own columns of Ut (rows of S = H^T do not mix), so a chain
+// can be split over CTAs by value columns.  chain_fwd_sliced runs the columns
+// [v0, v0 + 64) of one (sequence, head) in a CTA of its own, in the
+// untransposed form: thread k owns row k of H_s = H[:, v0:v0+64] (64 fp32
+// registers, half of chain_fwd's) and per chunk
+//
+//   U_s = Ut_s - W H_s          (M = 64 tokens, N = 64 values, K = 128 keys)
+//   H_s <- gam_n H_s + Kd^T U_s  (M = 128 keys, N = 64 values, K = 64 tokens)
+//
+// With snapshots it writes the state entering each chunk as block `slice` of a
+// 128 x 128 SW128 tile of H (rows = keys) and U_s as block `slice` of a
+// 64 x 128 tile of U (rows = tokens): the layouts tc_out reads.
+struct SliceSmem {
+    static constexpr int kH = 0, kU = kH + 16384, kI = kU + 8192, kW0 = kI + 8192,
+                         kKd0 = kW0 + 2 * 16384, kUt0 = kKd0 + 2 * 16384, kG0 = kUt0 + 2 * 8192,
+                         kEnd = kG0 + 2 * 256;
+};
+constexpr int kSliceSmem = SliceSmem::kEnd + 1024;
+
+// Bulk copies (thread 0) of chunk ch's W and Kd images, column block `sl` of
+// its Ut image (unless the run takes Ut as zero) and its gate row into buffer
+// `buf`, completing on `bar`.
+__device__ __forceinline__ void slice_prefetch(uint8_t *sm, int buf, size_t ch, int sl,
+                                               const Params &p, bool with_ut, uint64_t *bar) {
+    if (threadIdx.x != 0) return;
+    mbar_arrive_expect_tx(bar, 2u * (uint32_t)kImg64 + (with_ut ? 8192u : 0u) + C * 4u);
+    bulk_load(smem_u32(sm + SliceSmem::kW0 + buf * 16384),
+              static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64, bar);
+    bulk_load(smem_u32(sm + SliceSmem::kKd0 + buf * 16384),
+              static_cast<const uint8_t *>(p.tKd) + ch * kImg64, kImg64, bar);
+    if (with_ut)
+        bulk_load(smem_u32(sm + SliceSmem::kUt0 + buf * 8192),
+                  static_cast<const uint8_t *>(p.tUt) + ch * kImg64 + sl * 8192, 8192, bar);
+    bulk_load(smem_u32(sm + SliceSmem::kG0 + buf * 256), p.tG + ch * C, C * 4, bar);
+}
+
+__device__ __forceinline__ void chain_fwd_sliced(const Params &p, const ChainFwd &a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar, lbar[2];
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, h = a.h, k = threadIdx.x, sl = a.slice, v0 = 64 * sl;
+    float S[64];  // row k of H_s
+    if (a.init) {
+        const int ik = a.init_user ? p.K : D, iv = a.init_user ? p.V : D;
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+            S[j] = (k < ik && v0 + j < iv) ? a.init[(size_t)k * iv + v0 + j] : 0.f;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) S[j] = (a.init_identity && k == v0 + j) ? 1.f : 0.f;
+    }
+    if (k == 0) {
+        mbar_init(&mbar, 1);
+        mbar_init(&lbar[0], 1);
+        mbar_init(&lbar[1], 1);
+        fence_mbar_init();
+    }
+    if (k < 32) {
+        tmem_alloc(&tslot, 64);
+        tmem_relinquish();
+    }
+    identity_tile(sm + SliceSmem::kI);
+    tc_fence_before();
+    fence_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    // 64 TMEM columns: the first product (M = 64) is read out before the second
+    // (M = 128) overwrites the same columns
+    const uint32_t tmem = tslot;
+    const int c0 = a.c0, c1 = a.c1;
+    const bool with_ut = !a.zero_ut;
+    uint32_t phase = 0, pend = 0, lpar = 0;  // per buffer b (bit b): copy in flight, parity
+    if (c0 < c1) {
+        slice_prefetch(sm, 0, (size_t)c0 * H + h, sl, p, with_ut, &lbar[0]);
+        pend = 1;
+    }
+    uint8_t *Hs = sm + SliceSmem::kH, *Us = sm + SliceSmem::kU;
+    const uint32_t hb = smem_u32(Hs), ub = smem_u32(Us);
+    const uint32_t id1 = idesc_bf16(64, 64, 0, 1), id2 = idesc_bf16(128, 64, 1, 1);
+    for (int c = c0; c < c1; ++c) {
+        const int buf = (c - c0) & 1;
+        const size_t ch = (size_t)c * H + h;
+        if (c + 1 < c1) {
+            slice_prefetch(sm, buf ^ 1, ch + H, sl, p, with_ut, &lbar[buf ^ 1]);
+            pend |= 2u >> buf;
+        }
+        const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
+        // the state entering this chunk: row k of the H_s operand tile (128 bytes)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4 *>(Hs + sw128_chunk(D, k, j)) = pack8(S + 8 * j);
+        fence_async_smem();
+        tc_fence_before();
+        const bool all = __syncthreads_and(lok);
+        tc_fence_after();
+        if (!all) {
+            if (k == 0) record_timeout(p, 40 + a.where);
+            break;
+        }
+        pend &= ~(1u << buf);
+        lpar ^= 1u << buf;
+        const float gC =
+            expf(reinterpret_cast<const float *>(sm + SliceSmem::kG0 + buf * 256)[C - 1]);
+        if (k == 0) {  // U_s = -W H_s + I Ut_s (the W image is stored negated)
+            const uint32_t wb = smem_u32(sm + SliceSmem::kW0 + buf * 16384),
+                           utb = smem_u32(sm + SliceSmem::kUt0 + buf * 8192),
+                           ib = smem_u32(sm + SliceSmem::kI);
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(wb, C, s), desc_mnmajor(hb, D, s), id1, s > 0);
+            if (with_ut) {
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tmem, desc_kmajor(ib, C, s), desc_mnmajor(utb, C, s), id1, 1);
+            }
+            mma_commit(&mbar);
+            if (a.snapshots) {
+                bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128 + sl * 16384, hb, 16384u);
+                bulk_commit();
+            }
+        }
+        if (!cta_wait(&mbar, phase, p, a.where)) break;
+        phase ^= 1;
+        {  // U_s as an operand tile: row i on the M = 64 lanes
+            const int i = m64_row();
+            float d[64];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tmem_ld16(tm(tmem, 16 * q), d + 16 * q);
+            tmem_ld_wait();
+            if (i >= 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4 *>(Us + sw128_chunk(C, i, j)) = pack8(d + 8 * j);
+            }
+        }
+        operands_ready();  // (also orders the TMEM reads above before the product below)
+        if (k == 0) {  // Kd^T U_s
+            const uint32_t kb = smem_u32(sm + SliceSmem::kKd0 + buf * 16384);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem, desc_mnmajor(kb, C, s), desc_mnmajor(ub, C, s), id2, s > 0);
+            mma_commit(&mbar);
+            if (a.snapshots) {
+                bulk_store(static_cast<uint8_t *>(p.tUT) + ch * kImgUT + sl * 8192, ub, 8192u);
+                bulk_commit();
+            }
+        }
+        if (!cta_wait(&mbar, phase, p, a.where + 1)) break;
+        phase ^= 1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float d[16];
+            tmem_ld16(tm(tmem, 16 * q), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 16; ++x) S[16 * q + x] = fmaf(gC, S[16 * q + x], d[x]);
+        }
+        // the operand tiles are rewritten next chunk: their bulk stores must have read them
+        if (k == 0 && a.snapshots) bulk_wait_read();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if (k == 0) {  // copies still in flight after an early exit
+        for (int b = 0; b < 2; ++b)
+            if ((pend >> b) & 1u) mbar_wait(&lbar[b], (lpar >> b) & 1u, kWaitLimit);
+        if (a.snapshots) bulk_wait_all();
+    }
+    if (a.final_out) {
+        const int ok = a.out_user ? p.K : D, ov = a.out_user ? p.V : D;
+        if (k < ok) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (v0 + j < ov) a.final_out[(size_t)k * ov + v0 + j] = S[j];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (k < 32) tmem_dealloc(tmem, 64);
+}
+
 // Body of the forward state pass for CTA `blk` (sequence blk / H, head blk % H):
 // the whole sequence from h0, writing the per-chunk snapshots and hT.
 __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
@@ -203,7 +419,32 @@ __device__ __forceinline__ void state_fwd_body(const Params &p, int blk) {
     a.final_out = p.hT ? p.hT + ((size_t)n * H + h) * p.K * p.V : nullptr;
     a.out_user = 1;
     a.where = 3;
+    a.slice = 0;
     chain_fwd(p, a);
+}
+
+// Value slices of the forward chain's rows (64 value columns each).
+__device__ __forceinline__ int value_slices(const Params &p) { return (p.V + 63) / 64; }
+
+// The forward pass's state chain by value slices: CTA `blk` runs slice
+// blk % value_slices of (sequence, head) blk / value_slices, the whole sequence
+// from h0, writing the H and U snapshots tc_out reads and its columns of hT.
+__device__ __forceinline__ void state_fwd_sliced_body(const Params &p, int blk) {
+    const int nsl = value_slices(p), unit = blk / nsl, H = p.H, n = unit / H, h = unit % H;
+    ChainFwd a;
+    a.h = h;
+    a.slice = blk % nsl;
+    a.c0 = seq_first_at(p, n);
+    a.c1 = seq_first_at(p, n + 1);
+    a.init = p.h0 ? p.h0 + ((size_t)n * H + h) * p.K * p.V : nullptr;
+    a.init_user = 1;
+    a.init_identity = 0;
+    a.zero_ut = 0;
+    a.snapshots = 1;
+    a.final_out = p.hT ? p.hT + ((size_t)n * H + h) * p.K * p.V : nullptr;
+    a.out_user = 1;
+    a.where = 3;
+    chain_fwd_sliced(p, a);
 }
 
 }  // namespace tc

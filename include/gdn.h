@@ -112,6 +112,19 @@ typedef struct gdn_desc {
  * the normalised copies in the workspace. */
 #define GDN_FLAG_QK_L2NORM 2
 
+/* Forward option: run the forward state chains by value slices.  The rows of
+ * S (one per value column) evolve independently given a chunk's keys, write
+ * strengths and gates, so each (sequence, head) chain can be split over CTAs
+ * by value columns (the d_v slicing of the chunkwise form): two CTAs of 64
+ * value columns each, in the untransposed form in which the key dimension is
+ * the M = 128 side of the state update.  Same results up to the association
+ * of the products inside the tensor cores; not bitwise equal to the default.
+ * On a B200 it is not faster (a chain step is bound by the fixed latency of
+ * its two dependent tensor-core products, which does not shrink with their
+ * size), so it is off by default.  Applies to the bf16 forward (and the piece
+ * scan); ignored elsewhere, and by gdn_bwd and gdn_decode. */
+#define GDN_FLAG_VALUE_SLICES 4
+
 /* Library version (major * 10000 + minor * 100 + patch). */
 int gdn_version(void);
 

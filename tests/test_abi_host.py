@@ -58,9 +58,11 @@ def test_flags_match_header_and_unknown_bits_are_rejected():
     defs = dict(re.findall(r"#define (GDN_FLAG_\w+) (\d+)", hdr))
     assert int(defs["GDN_FLAG_PIECE_SCAN"]) == gdn.GDN_FLAG_PIECE_SCAN
     assert int(defs["GDN_FLAG_QK_L2NORM"]) == gdn.GDN_FLAG_QK_L2NORM
-    ok = gdn.make_desc(2, 100, 3, 64, 128, flags=gdn.GDN_FLAG_QK_L2NORM | gdn.GDN_FLAG_PIECE_SCAN)
+    assert int(defs["GDN_FLAG_VALUE_SLICES"]) == gdn.GDN_FLAG_VALUE_SLICES
+    every = gdn.GDN_FLAG_QK_L2NORM | gdn.GDN_FLAG_PIECE_SCAN | gdn.GDN_FLAG_VALUE_SLICES
+    ok = gdn.make_desc(2, 100, 3, 64, 128, flags=every)
     assert gdn.fwd_workspace_size(ok) > 0
-    bad = gdn.make_desc(2, 100, 3, 64, 128, flags=4)
+    bad = gdn.make_desc(2, 100, 3, 64, 128, flags=8)
     assert gdn.fwd_workspace_size(bad) == 0 and _fwd(bad, ws_bytes=1 << 40) == 1
 
 
