@@ -254,6 +254,8 @@ Layout make_layout(const Problem &pb, bool bwd) {
         L.tG = take(nch * kChunk * f);
         L.tS = take(nch * img128);
         L.tUT = take(nch * img64);
+        L.tQg = take(nch * img64);                   // bf16 tile image of scale diag(gam) Q
+        L.tP = take(nch * kChunk * kChunk * 2);      // bf16 tile image of P
         if (!bwd && pb.P > 1) {
             const size_t units = (size_t)pb.N * pb.H * pb.P, st = (size_t)128 * 128 * f;
             L.tHin = take(units * st);
@@ -263,8 +265,6 @@ Layout make_layout(const Problem &pb, bool bwd) {
         if (bwd) {
             L.tA = take(nch * kChunk * kChunk * 2);  // bf16 tile image of A
             L.tB = take(nch * kChunk * f);
-            L.tQg = take(nch * img64);
-            L.tP = take(nch * kChunk * kChunk * 2);  // bf16 tile image of P
             L.tdSn = take(nch * img128);
             L.tdUT = take(nch * img64);
         }

@@ -14,10 +14,11 @@
 //   U^T = Ut^T - S W^T        (M = 128 rows v, N = 64 tokens, K = 128)
 //   S  <- gam_n S + U^T Kd    (M = 128 rows v, N = 128 keys,  K = 64 tokens)
 //
-// Kernels: tc_prep (chunk-parallel: gates, K K^T, the blocked inverse A in
-// fp32, W, Ut, Kd = diag(e) K), tc_state_fwd (serial over the chunks of a
-// sequence; one CTA per (sequence, head); writes the state entering every
-// chunk and U^T as swizzled tile images), tc_out (chunk-parallel output).
+// Kernels: tc_prep (chunk-parallel: gates, [Q; K] K^T, the blocked inverse A
+// in fp32, W, Ut, Kd = diag(e) K, Qg = scale diag(gam) Q and P), tc_state_fwd
+// (serial over the chunks of a sequence; one CTA per (sequence, head); writes
+// the state entering every chunk and U^T as swizzled tile images), tc_out
+// (chunk-parallel output: one product over the four images).
 #include "tc_common.cuh"
 #include "tc_prep.cuh"
 #include "tc_state.cuh"
@@ -194,13 +195,14 @@ __global__ void __launch_bounds__(NT, 1) tc_piece_c_kernel(Params p) {
 
 // ============================================================ tc_out
 // O^T[v][i] = S[v][:] . (scale gam_i q_i) + sum_j U^T[v][j] P[i][j],
-// P = scale lower(Q K^T . Gam).  One CTA per (chunk, head).  The snapshots come
-// as S (rows = values) and U^T tiles, read K-major, or, from the chain by value
-// slices (p.vslice), as H = S^T (rows = keys) and U (rows = tokens) tiles, read
-// MN-major: the same A operands of the two M = 128 products.
+// P = scale lower(Q K^T . Gam).  One CTA per (chunk, head), one M = 128 product
+// over four tile images: the chain's snapshots S and U^T (read K-major), or,
+// from the chain by value slices (p.vslice), H = S^T (rows = keys) and U (rows =
+// tokens) read MN-major, the same A operands; and tc_prep's Qg = scale diag(gam) Q
+// and P.  73 KB of shared memory: three CTAs per SM.
 struct OutSmem {
-    static constexpr int kQK = 0, kS = kQK + 32768, kUT = kS + 32768, kQG = kUT + 16384,
-                         kP = kQG + 16384, kG = kP + 8192, kEnd = kG + 256;
+    static constexpr int kS = 0, kUT = kS + 32768, kQG = kUT + 16384, kP = kQG + 16384,
+                         kEnd = kP + 8192;
 };
 constexpr int kOutSmem = OutSmem::kEnd + 1024;
 
@@ -212,89 +214,57 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(const __grid_constant__ Para
     if (p.hdr->status) return;
     const int H = p.H, ch = blockIdx.x, c = ch / H, h = ch % H, tid = threadIdx.x;
     const ChunkInfo ci = chunk_at(p, c);
-    uint8_t *QK = sm + OutSmem::kQK, *Ss = sm + OutSmem::kS, *UTs = sm + OutSmem::kUT;
-    uint8_t *QG = sm + OutSmem::kQG, *Ps = sm + OutSmem::kP;
-    float *G = reinterpret_cast<float *>(sm + OutSmem::kG);
-    if (tid == 0) {  // q and k rows by the tensor engine, the state and U^T images by bulk copies
+    uint8_t *Ss = sm + OutSmem::kS, *UTs = sm + OutSmem::kUT, *QG = sm + OutSmem::kQG,
+            *Ps = sm + OutSmem::kP;
+    if (tid == 0) {  // the four images by bulk copies
         mbar_init(&mbar, 1);
         mbar_init(&lbar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&lbar, 2 * row_tile_bytes(p.K) + (uint32_t)(kImg128 + kImgUT));
-        load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
-        load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
+        mbar_arrive_expect_tx(&lbar, (uint32_t)(kImg128 + kImgUT + kImg64 + C * C * 2));
         bulk_load(smem_u32(Ss), static_cast<const uint8_t *>(p.tS) + (size_t)ch * kImg128,
                   (uint32_t)kImg128, &lbar);
         bulk_load(smem_u32(UTs), static_cast<const uint8_t *>(p.tUT) + (size_t)ch * kImgUT,
                   (uint32_t)kImgUT, &lbar);
+        bulk_load(smem_u32(QG), static_cast<const uint8_t *>(p.tQg) + (size_t)ch * kImg64,
+                  (uint32_t)kImg64, &lbar);
+        bulk_load(smem_u32(Ps), static_cast<const uint8_t *>(p.tP) + (size_t)ch * (C * C * 2),
+                  (uint32_t)(C * C * 2), &lbar);
     }
-    if (tid < C) G[tid] = p.tG[(size_t)ch * C + tid];
     if (tid < 32) {
-        tmem_alloc(&tslot, 128);
+        tmem_alloc(&tslot, 64);
         tmem_relinquish();
     }
     __syncthreads();  // thread 0's mbarrier inits are visible before any thread waits on them
     bool ok = copies_arrived(&lbar, p, 7);
-    if (ok) {
-        fix_rows(QK, D, 0, ci.len, p.K);
-        fix_rows(QK, D, C, ci.len, p.K);
-    }
-    operands_ready();
-    if (ok && p.l2norm) {  // q and k rows divided by their norms
-        l2norm_tile_rows(QK, D, 0, nullptr);
-        l2norm_tile_rows(QK, D, C, nullptr);
-        operands_ready();
-    }
+    tc_fence_after();
     const uint32_t tmem = tslot;
-    if (ok && tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
-        const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
+    if (ok && tid == 0) {
+        const uint32_t sb = smem_u32(Ss), qg = smem_u32(QG), ub = smem_u32(UTs), pb = smem_u32(Ps);
+        if (!p.vslice) {
+            const uint32_t id = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-            mma_bf16(tmem, desc_kmajor(qb, D, s), desc_kmajor(kb, D, s), id, s > 0);
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(ub, D, s), desc_kmajor(pb, C, s), id, 1);
+        } else {
+            const uint32_t id = idesc_bf16(128, 64, 1, 0);
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tmem, desc_mnmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(pb, C, s), id, 1);
+        }
         mma_commit(&mbar);
     }
-    // scale * gam_i * q_i as a K-major operand (rows i)
-    for (int t = tid; ok && t < C * 16; t += NT) {
-        const int r = t >> 4, j = t & 15;
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4 *>(QK + sw128_chunk(D, r, j)), f);
-        const float s = p.scale * expf(G[r]);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] *= s;
-        *reinterpret_cast<uint4 *>(QG + sw128_chunk(C, r, j)) = pack8(f);
-    }
-    if (ok) ok = cta_wait(&mbar, 0, p, 5);
-    if (ok) {
-        build_p_tile(tmem, G, p.scale, Ps);
-        operands_ready();
-        if (tid == 0) {
-            const uint32_t sb = smem_u32(Ss), qg = smem_u32(QG), ub = smem_u32(UTs),
-                           pb = smem_u32(Ps);
-            if (!p.vslice) {
-                const uint32_t id = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-                for (int s = 0; s < D / 16; ++s)
-                    mma_bf16(tmem + 64, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
-#pragma unroll
-                for (int s = 0; s < C / 16; ++s)
-                    mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_kmajor(pb, C, s), id, 1);
-            } else {
-                const uint32_t id = idesc_bf16(128, 64, 1, 0);
-#pragma unroll
-                for (int s = 0; s < D / 16; ++s)
-                    mma_bf16(tmem + 64, desc_mnmajor(sb, D, s), desc_kmajor(qg, C, s), id, s > 0);
-#pragma unroll
-                for (int s = 0; s < C / 16; ++s)
-                    mma_bf16(tmem + 64, desc_mnmajor(ub, C, s), desc_kmajor(pb, C, s), id, 1);
-            }
-            mma_commit(&mbar);
-        }
-        ok = cta_wait(&mbar, 1, p, 6);
-    }
-    if (ok) {  // O^T column v -> rows of a staging tile (the consumed Q K tile), 16-byte stores
-        bf16 *stage = reinterpret_cast<bf16 *>(QK);
+    if (ok) ok = cta_wait(&mbar, 0, p, 6);
+    if (ok) {  // O^T column v -> rows of a staging tile over the consumed S image, 16-byte stores
+        bf16 *stage = reinterpret_cast<bf16 *>(Ss);
         for (int c0 = 0; c0 < C; c0 += 16) {
             float d[16];
-            tmem_ld16(tm(tmem, 64 + c0), d);
+            tmem_ld16(tm(tmem, c0), d);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 16; ++q) stage[(c0 + q) * D + tid] = __float2bfloat16_rn(d[q]);
@@ -305,12 +275,12 @@ __global__ void __launch_bounds__(NT) tc_out_kernel(const __grid_constant__ Para
             const int i = t >> 4, j = t & 15;
             if (i < ci.len && j * 8 < p.V)
                 *reinterpret_cast<uint4 *>(o + ((int64_t)(ci.tok0 + i) * H + h) * p.V + j * 8) =
-                    *reinterpret_cast<const uint4 *>(QK + i * 256 + j * 16);
+                    *reinterpret_cast<const uint4 *>(Ss + i * 256 + j * 16);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (tid < 32) tmem_dealloc(tmem, 128);
+    if (tid < 32) tmem_dealloc(tmem, 64);
 }
 
 

@@ -4,8 +4,9 @@
 // pieces are recomputed (tc_prep keeps A in fp32; tc_state_fwd rewrites the
 // state entering every chunk and U^T), three kernels run:
 //
-//   tc_local      chunk-parallel: P = scale lower(Q K^T . Gam) and
-//                 Qg = scale diag(gam) Q (tile images)
+//   tc_prep_local chunk-parallel: the preparation step (tc_prep.cuh) with A
+//                 written too, and the tile images P = scale lower(Q K^T . Gam)
+//                 and Qg = scale diag(gam) Q
 //   tc_state_bwd  serial over the chunks of a sequence, in reverse; thread v
 //                 owns row v of dS = dH^T (fp32 registers); per chunk
 //                   dU^T = dO^T P + dS Kd^T
@@ -33,93 +34,11 @@ namespace {
 
 using namespace tc;
 
-// ============================================================ tc_local
-struct LocalSmem {
-    // P overwrites the Q half of the [Q; K] tile once Q K^T and Qg have consumed it
-    static constexpr int kQK = 0, kP = kQK, kG = kQK + 32768, kEnd = kG + 256;
-};
-constexpr int kLocalSmem = LocalSmem::kEnd + 1024;
-
-// Body of the local step for CTA `ch` (chunk ch / H, head ch % H).  It forms
-// the chunk gates itself (the same code as tc_prep, so bit-identical), which
-// makes it independent of tc_prep: the two share one launch.
-__device__ __forceinline__ void local_body(const Params &p, int ch) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar, lbar;
-    __shared__ uint32_t tslot;
-    if (p.hdr->status) return;
-    const int H = p.H, c = ch / H, h = ch % H, tid = threadIdx.x;
-    const ChunkInfo ci = chunk_at(p, c);
-    uint8_t *QK = sm + LocalSmem::kQK, *Ps = sm + LocalSmem::kP;
-    float *G = reinterpret_cast<float *>(sm + LocalSmem::kG);
-    if (tid == 0) {  // q and k rows by the tensor engine
-        mbar_init(&mbar, 1);
-        mbar_init(&lbar, 1);
-        fence_mbar_init();
-        mbar_arrive_expect_tx(&lbar, 2 * row_tile_bytes(p.K));
-        load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
-        load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
-    }
-    if (tid < 32) {
-        tmem_alloc(&tslot, 128);
-        tmem_relinquish();
-    }
-    chunk_gates(G, nullptr, p, ci, h);  // its barriers also publish the mbarrier inits
-    bool ok = copies_arrived(&lbar, p, 32);
-    if (ok) {
-        fix_rows(QK, D, 0, ci.len, p.K);
-        fix_rows(QK, D, C, ci.len, p.K);
-    }
-    operands_ready();
-    if (ok && p.l2norm) {  // q and k rows divided by their norms
-        l2norm_tile_rows(QK, D, 0, nullptr);
-        l2norm_tile_rows(QK, D, C, nullptr);
-        operands_ready();
-    }
-    const uint32_t tmem = tslot;
-    if (ok && tid == 0) {  // Q K^T: M = 64, N = 64, K = 128
-        const uint32_t qb = smem_u32(QK), kb = qb + C * 128, id = idesc_bf16(64, 64, 0, 0);
-#pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-            mma_bf16(tmem, desc_kmajor(qb, D, s), desc_kmajor(kb, D, s), id, s > 0);
-        mma_commit(&mbar);
-    }
-    if (ok) {  // Qg = scale diag(gam) Q: an operand of the reverse state pass (tile image)
-        uint8_t *img = static_cast<uint8_t *>(p.tQg) + (size_t)ch * kImg64;
-        for (int t = tid; t < C * 16; t += NT) {
-            const int r = t >> 4, j = t & 15;
-            float f[8];
-            unpack8(*reinterpret_cast<const uint4 *>(QK + sw128_chunk(D, r, j)), f);
-            const float s = p.scale * expf(G[r]);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) f[q] *= s;
-            *reinterpret_cast<uint4 *>(img + sw128_chunk(C, r, j)) = pack8(f);
-        }
-    }
-    if (ok) ok = cta_wait(&mbar, 0, p, 11);
-    if (ok) {  // P as a tile image: the reverse state pass forms the local dU^T = dO^T P itself
-        build_p_tile(tmem, G, p.scale, Ps);
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_store(static_cast<uint8_t *>(p.tP) + (size_t)ch * C * C * 2, smem_u32(Ps),
-                       (uint32_t)(C * C * 2));
-            bulk_commit();
-            bulk_wait_all();
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (tid < 32) tmem_dealloc(tmem, 128);
-}
-
-// tc_prep (with A for the backward) on CTAs [0, NC*H) and tc_local on
-// [NC*H, 2*NC*H): independent chunk-parallel steps in one launch.
+// ============================================================ tc_prep_local
+// The preparation step with A also written (the backward's gradient kernel reads
+// it); the same step writes the P and Qg images the reverse chain reads.
 __global__ void __launch_bounds__(NT, 4) tc_prep_local_kernel(const __grid_constant__ Params p) {
-    const int nch = p.NC * p.H;
-    if ((int)blockIdx.x < nch) prep_body(p, blockIdx.x, 1);
-    else local_body(p, blockIdx.x - nch);
+    prep_body(p, blockIdx.x, 1);
 }
 
 // ============================================================ tc_state_bwd
@@ -953,10 +872,9 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
     Params pf = p;
     pf.hT = nullptr;
     if (nch > 0) {
-        const int sm = kLocalSmem > kPrepSmemRequest ? kLocalSmem : kPrepSmemRequest;
-        if ((e = set_smem(tc_prep_local_kernel, sm))) return e;
+        if ((e = set_smem(tc_prep_local_kernel, kPrepSmemRequest))) return e;
         GDN_LAUNCH(kKTcLocal, stream,
-                   tc_prep_local_kernel<<<2 * nch, NT, sm, stream>>>(p));
+                   tc_prep_local_kernel<<<nch, NT, kPrepSmemRequest, stream>>>(p));
     }
     if (nseq > 0) {
         const int sm = kSbwdSmem > kStateSmem ? kSbwdSmem : kStateSmem;

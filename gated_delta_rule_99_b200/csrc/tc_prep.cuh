@@ -9,19 +9,25 @@ namespace tc {
 
 // ============================================================ tc_prep
 // Per (chunk, head): gates, A = (I + L)^-1 (fp32, by 16 x 16 blocks), and the
-// tile images W, Kd and Ut that the state chains consume.
+// tile images W, Kd and Ut that the state chains consume, and the images of
+// Qg = scale diag(gam) Q and P = scale lower(Q K^T . Gam) that the output and
+// the reverse chain consume.  One M = 128 product [Q; K] K^T gives Q K^T on
+// lanes 0-63 and K K^T on lanes 64-127, so P (threads 0-63) and L (threads
+// 64-127) are built in the same phase.
 constexpr int LS = 68;  // row stride (floats) of L: 16-byte aligned rows for vector loads
 
 struct PrepSmem {
-    // L (fp32 64 x 68) becomes A in place; once A is read out, its bytes hold
-    // the two bf16 operand tiles A diag(b gam) and A diag(b).  F: per-column
-    // decay factors exp(G_e - G_j) to the end e of column j's 16-block; E: exp(G_j);
-    // EK: exp(G_n - G_j), n the chunk's last token.
-    static constexpr int kK = 0, kV = kK + 16384, kL = kV + 16384, kAb = kL, kAc = kL + 8192,
+    // [Q; K] rows as one 128-row tile (Q rows 0-63, K rows 64-127); once Q is
+    // consumed, the V rows are loaded into its place.  L (fp32 64 x 68) becomes A
+    // in place; once A is read out, its bytes hold the two bf16 operand tiles
+    // A diag(b gam) and A diag(b).  F: per-column decay factors exp(G_e - G_j) to
+    // the end e of column j's 16-block; E: exp(G_j); EK: exp(G_n - G_j), n the
+    // chunk's last token.
+    static constexpr int kQK = 0, kL = kQK + 32768, kAb = kL, kAc = kL + 8192,
                          kG = kL + C * LS * 4, kB = kG + 256, kF = kB + 256, kE = kF + 256,
                          kEK = kE + 256, kEnd = kEK + 256;
 };
-constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 32;
+constexpr int kPrepSmem = PrepSmem::kEnd + 1024 + 48;
 constexpr int kPrepSmemRequest = 52 * 1024;  // four CTAs per SM (TMEM: 128 columns each)
 
 // acc += a x (four columns)
@@ -32,16 +38,23 @@ __device__ __forceinline__ void fma4(float4 &acc, float a, const float4 x) {
     acc.w = fmaf(a, x.w, acc.w);
 }
 
+// Byte offset, in a [Q; K] tile of 128 rows, of byte `off` of a 64-row tile image
+// (block off / 8192, row and chunk position within it) taken from rows
+// [row0, row0 + 64): the swizzle depends on the row only through row % 8.
+__device__ __forceinline__ uint32_t qk_src(int off, int row0) {
+    return (uint32_t)((off >> 13) * 16384 + row0 * 128 + (off & 8191));
+}
+
 // Body of the prep step for CTA `ch` (chunk ch / H, head ch % H).
 __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar, lbar;
+    __shared__ uint64_t mbar, lbar, vbar;
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, c = ch / H, h = ch % H;
     const ChunkInfo ci = chunk_at(p, c);
-    uint8_t *Kt = sm + PrepSmem::kK, *Vt = sm + PrepSmem::kV;
+    uint8_t *QK = sm + PrepSmem::kQK;
     uint8_t *Ab = sm + PrepSmem::kAb, *Ac = sm + PrepSmem::kAc;
     float *L = reinterpret_cast<float *>(sm + PrepSmem::kL);
     float *G = reinterpret_cast<float *>(sm + PrepSmem::kG);
@@ -50,17 +63,19 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     float *E = reinterpret_cast<float *>(sm + PrepSmem::kE);
     float *EK = reinterpret_cast<float *>(sm + PrepSmem::kEK);
     const int tid = threadIdx.x;
+    const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128;  // K rows: 64-127 of the tile
 
-    if (tid == 0) {  // K and V rows by the tensor engine
+    if (tid == 0) {  // Q and K rows by the tensor engine (V comes once Q is consumed)
         mbar_init(&mbar, 1);
         mbar_init(&lbar, 1);
+        mbar_init(&vbar, 1);
         fence_mbar_init();
         // (the planted stall of the tests: 16 bytes more than the copies bring, on the
         // first (chunk, head) only, so its bounded wait runs out after they have landed)
         const uint32_t planted = (p.test_hook == GDN_TEST_STALL_COPY && ch == 0) ? 16u : 0u;
-        mbar_arrive_expect_tx(&lbar, row_tile_bytes(p.K) + row_tile_bytes(p.V) + planted);
-        load_rows_tma(Kt, C, 0, &p.tm_k, ci.tok0, h, p.K, &lbar);
-        load_rows_tma(Vt, C, 0, &p.tm_v, ci.tok0, h, p.V, &lbar);
+        mbar_arrive_expect_tx(&lbar, 2 * row_tile_bytes(p.K) + planted);
+        load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
+        load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
     }
     if (tid < 32) {
         tmem_alloc(&tslot, 128);
@@ -74,36 +89,44 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     }
     bool ok = copies_arrived(&lbar, p, 31);
     if (ok) {
-        fix_rows(Kt, C, 0, ci.len, p.K);
-        fix_rows(Vt, C, 0, ci.len, p.V);
+        fix_rows(QK, D, 0, ci.len, p.K);
+        fix_rows(QK, D, C, ci.len, p.K);
     }
     operands_ready();
-    if (ok && p.l2norm) {  // k rows divided by their norms
-        l2norm_tile_rows(Kt, C, 0, nullptr);
+    if (ok && p.l2norm) {  // q and k rows divided by their norms
+        l2norm_tile_rows(QK, D, 0, nullptr);
+        l2norm_tile_rows(QK, D, C, nullptr);
         operands_ready();
     }
     const uint32_t tmem = tslot;
     uint32_t phase = 0;
+    bool v_pending = false;  // the V copy is in flight and not yet waited for
 
-    // K K^T (M = 64 rows i, N = 64 cols j, K = 128)
+    // [Q; K] K^T (M = 128 rows: Q K^T on lanes 0-63, K K^T on lanes 64-127; N = 64; K = 128)
     if (ok && tid == 0) {
-        const uint32_t kb = smem_u32(Kt), id = idesc_bf16(64, 64, 0, 0);
+        const uint32_t id = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-            mma_bf16(tmem, desc_kmajor(kb, C, s), desc_kmajor(kb, C, s), id, s > 0);
+            mma_bf16(tmem, desc_kmajor(qkb, D, s), desc_kmajor(kb, D, s), id, s > 0);
         mma_commit(&mbar);
     }
-    // meanwhile: Kd = diag(e) K as a tile image, and G
+    // meanwhile: the Kd = diag(e) K and Qg = scale diag(gam) Q images, G and b
     if (ok) {
-        uint8_t *dst = static_cast<uint8_t *>(p.tKd) + (size_t)ch * kImg64;
+        uint8_t *kd = static_cast<uint8_t *>(p.tKd) + (size_t)ch * kImg64;
+        uint8_t *qg = static_cast<uint8_t *>(p.tQg) + (size_t)ch * kImg64;
         for (int t = tid; t < C * 16; t += NT) {
             const int off = t * 16, r = (off & 8191) >> 7;
-            float f[8];
-            unpack8(*reinterpret_cast<const uint4 *>(Kt + off), f);
-            const float e = EK[r];
+            float f[8], g[8];
+            unpack8(*reinterpret_cast<const uint4 *>(QK + qk_src(off, C)), f);
+            unpack8(*reinterpret_cast<const uint4 *>(QK + qk_src(off, 0)), g);
+            const float e = EK[r], gq = p.scale * E[r];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] *= e;
-            *reinterpret_cast<uint4 *>(dst + off) = pack8(f);
+            for (int i = 0; i < 8; ++i) {
+                f[i] *= e;
+                g[i] *= gq;
+            }
+            *reinterpret_cast<uint4 *>(kd + off) = pack8(f);
+            *reinterpret_cast<uint4 *>(qg + off) = pack8(g);
         }
         if (tid < C) {
             p.tG[(size_t)ch * C + tid] = G[tid];
@@ -112,40 +135,54 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     }
     if (ok) ok = cta_wait(&mbar, phase, p, 1);
     phase ^= 1;
+    if (ok && tid == 0) {  // Q is consumed (the product and the Qg image): V rows in its place
+        fence_async_smem();
+        mbar_arrive_expect_tx(&vbar, row_tile_bytes(p.V));
+        load_rows_tma(QK, D, 0, &p.tm_v, ci.tok0, h, p.V, &vbar);
+    }
+    v_pending = ok;
     if (ok) {
-        // L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32).  The rows of a
-        // warp lie in one 16-block (M = 64 layout), so the three cases are warp-uniform.
-        const int i = m64_row();
+        // Rows of the [Q; K] K^T accumulator (M = 128: row = lane = thread).  Threads 0-63:
+        // P = scale lower(Q K^T . Gam), diagonal included, as a 64 x 64 tile image.
+        // Threads 64-127: L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32).
+        // The 16 rows of a half-warp lie in one 16-block, so the cases are warp-uniform.
+        // Gam_ij = exp(G_i - G_e) exp(G_e - G_j) below a row's diagonal block (e = the
+        // block's last column, both factors <= 1), directly inside it.
         float d[4][16];
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm(tmem, 16 * cb), d[cb]);
         tmem_ld_wait();
-        if (i >= 0) {
-            const int ib = i >> 4;
-            const float bi = bta[i];
-            float *Li = L + i * LS;
+        const bool lrow = tid >= C;
+        const int i = lrow ? tid - C : tid, ib = i >> 4;
+        const float ci0 = lrow ? bta[i] : p.scale;
+        uint8_t *Pimg = static_cast<uint8_t *>(p.tP) + (size_t)ch * (C * C * 2);
+        float *Li = L + i * LS;
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                const int c0 = 16 * cb;
-                float x[16];
-                if (cb < ib) {  // Gam_ij = exp(G_i - G_e) exp(G_e - G_j), e = c0 + 15 (both <= 1)
-                    const float ri = bi * expf(G[i] - G[c0 + 15]);
+        for (int cb = 0; cb < 4; ++cb) {
+            const int c0 = 16 * cb;
+            float x[16];
+            if (cb < ib) {
+                const float ri = ci0 * expf(G[i] - G[c0 + 15]);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) x[q] = ri * F[c0 + q] * d[cb][q];
-                } else if (cb == ib) {  // the diagonal block directly
+                for (int q = 0; q < 16; ++q) x[q] = ri * F[c0 + q] * d[cb][q];
+            } else if (cb == ib) {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int j = c0 + q;
-                        x[q] = j < i ? bi * expf(G[i] - G[j]) * d[cb][q] : 0.f;
-                    }
-                } else {  // above the diagonal
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) x[q] = 0.f;
+                for (int q = 0; q < 16; ++q) {
+                    const int j = c0 + q;
+                    x[q] = (lrow ? j < i : j <= i) ? ci0 * expf(G[i] - G[j]) * d[cb][q] : 0.f;
                 }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) x[q] = 0.f;
+            }
+            if (lrow) {
 #pragma unroll
                 for (int q = 0; q < 16; q += 4)
                     *reinterpret_cast<float4 *>(Li + c0 + q) =
                         make_float4(x[q], x[q + 1], x[q + 2], x[q + 3]);
+            } else {
+                *reinterpret_cast<uint4 *>(Pimg + sw128_chunk(C, i, 2 * cb)) = pack8(x);
+                *reinterpret_cast<uint4 *>(Pimg + sw128_chunk(C, i, 2 * cb + 1)) = pack8(x + 8);
             }
         }
         tc_fence_before();
@@ -280,10 +317,10 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         // one after the other in the same 128 TMEM columns
         const uint32_t id = idesc_bf16(64, 128, 0, 1);
         if (tid == 0) {
-            const uint32_t ab = smem_u32(Ab), kb = smem_u32(Kt);
+            const uint32_t ab = smem_u32(Ab);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem, desc_kmajor(ab, C, s), desc_mnmajor(kb, C, s), id, s > 0);
+                mma_bf16(tmem, desc_kmajor(ab, C, s), desc_mnmajor(kb, D, s), id, s > 0);
             mma_commit(&mbar);
         }
         ok = cta_wait(&mbar, phase, p, 2);
@@ -305,17 +342,23 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
-            if (tid == 0) {
-                const uint32_t ac = smem_u32(Ac), vb = smem_u32(Vt);
+            // the V rows (loaded into the Q rows' place after the first product)
+            ok = copies_arrived(&vbar, p, 34);
+            v_pending = false;
+            if (ok) fix_rows(QK, D, 0, ci.len, p.V);
+            operands_ready();
+            if (ok && tid == 0) {
+                const uint32_t ac = smem_u32(Ac);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    mma_bf16(tmem, desc_kmajor(ac, C, s), desc_mnmajor(vb, C, s), id, s > 0);
+                    mma_bf16(tmem, desc_kmajor(ac, C, s), desc_mnmajor(qkb, D, s), id, s > 0);
                 mma_commit(&mbar);
             }
-            ok = cta_wait(&mbar, phase, p, 2);
+            if (ok) ok = cta_wait(&mbar, phase, p, 2);
             phase ^= 1;
         }
     }
+    if (v_pending && tid == 0) mbar_wait(&vbar, 0, kWaitLimit);  // leave no copy in flight
     if (ok) {  // Ut as a 64 x 128 tile image (rows = tokens): an operand of the chains'
                // first product, whose 64-column blocks are the two halves of the values
         const int i = m64_row();
