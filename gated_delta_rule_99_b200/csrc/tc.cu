@@ -40,6 +40,13 @@ __global__ void __launch_bounds__(NT, 1) tc_state_fwd_kernel(Params p) {
     else state_fwd_body(p, blockIdx.x);
 }
 
+// ============================================================ tc_state_fwd_out
+// The forward chain with the output formed in the same CTA (the default forward
+// of sequences that run without the piece scan or value slices).
+__global__ void __launch_bounds__(kOutChainThreads, 1) tc_state_fwd_out_kernel(Params p) {
+    state_fwd_out_body(p, blockIdx.x);
+}
+
 // ============================================================ piece scan (long rows)
 // Chunks [c0, c1) of piece `piece` of dense row n (pieces of p.L chunks; the
 // last may be shorter or empty).
@@ -320,6 +327,14 @@ cudaError_t tc_launch_state_fwd(const Params &p, cudaStream_t stream) {
 cudaError_t launch_tc_fwd(const Params &p, const Problem &, cudaStream_t stream) {
     cudaError_t e;
     if ((e = tc_launch_prep(p, 0, stream))) return e;
+    if (p.P == 1 && !p.vslice) {  // the chain writes the output itself
+        const int nseq = p.N * p.H;
+        if (nseq == 0) return cudaSuccess;
+        if ((e = set_smem(tc_state_fwd_out_kernel, kOutChainSmem))) return e;
+        GDN_LAUNCH(kKTcStateFwd, stream,
+                   tc_state_fwd_out_kernel<<<nseq, kOutChainThreads, kOutChainSmem, stream>>>(p));
+        return cudaSuccess;
+    }
     if (p.P > 1 && p.N * p.H > 0) {  // piece scan of long rows
         const int units = p.N * p.H, nsl = chain_slices(p), sm = chain_smem(p);
         if ((e = set_smem(tc_piece_a_kernel, sm))) return e;
@@ -343,5 +358,6 @@ cudaError_t launch_tc_fwd(const Params &p, const Problem &, cudaStream_t stream)
 }
 
 static_assert(kPrepSmem <= kPrepSmemRequest, "prep shared memory");
+static_assert(kOutChainSmem <= 227 * 1024, "chain-with-output shared memory");
 
 }  // namespace gdn

@@ -218,6 +218,260 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     if (v < 32) tmem_dealloc(tmem, 256);
 }
 
+// ============================================================ chain with the output
+// The forward pass's chain with the output formed in the same CTA.  Each chunk's
+// state image S and U^T image are in shared memory anyway, so
+//   O^T = S Qg^T + U^T P^T    (M = 128 values, N = 64 tokens, K = 128 + 64)
+// over tc_prep's Qg and P images gives the chunk's output without S or U^T
+// leaving the SM.  Threads 0-127 (warpgroup 0) run the chain as chain_fwd does
+// (thread v owns row v of S; the state image is rewritten during the update).
+// Threads 128-255 (warpgroup 1) form the output: their leader issues S Qg^T once
+// the chain has issued the chunk's first product (m1bar) and U^T P^T once it has
+// issued the second (m2bar), so they run in the tensor pipe's gaps while the
+// chain's own issuing thread is not held up; then the warpgroup reads the
+// accumulator, stages it as token rows and stores them.  The chain waits for
+// sqbar (S Qg^T has read the state image) before rewriting the state image and
+// for obar (the chunk's output is complete) before rewriting the U^T image or
+// refilling the chunk's prefetch slot.  Every wait is bounded.
+struct OutChainSmem {
+    // the state image, U^T, the identity block, the output staging rows, then per
+    // prefetch slot the W, Kd, Ut and Qg images and the P tile; the slots' gate rows
+    static constexpr int kS = 0, kUT = kS + 32768, kI = kUT + 16384, kStage = kI + 8192,
+                         kBuf = kStage + 16384;
+    static constexpr int kW = 0, kKd = 16384, kUt = 32768, kQg = 49152, kP = 65536,
+                         kBufBytes = 73728;
+    static constexpr int kG0 = kBuf + 2 * kBufBytes, kEnd = kG0 + 2 * 256;
+};
+constexpr int kOutChainSmem = OutChainSmem::kEnd + 1024;
+constexpr int kOutChainThreads = 256;
+
+__device__ __forceinline__ void outchain_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p,
+                                                  uint64_t *bar) {
+    uint8_t *b = sm + OutChainSmem::kBuf + buf * OutChainSmem::kBufBytes;
+    mbar_arrive_expect_tx(bar, 4u * (uint32_t)kImg64 + (uint32_t)(C * C * 2) + C * 4u);
+    bulk_load(smem_u32(b + OutChainSmem::kW), static_cast<const uint8_t *>(p.tW) + ch * kImg64,
+              kImg64, bar);
+    bulk_load(smem_u32(b + OutChainSmem::kKd), static_cast<const uint8_t *>(p.tKd) + ch * kImg64,
+              kImg64, bar);
+    bulk_load(smem_u32(b + OutChainSmem::kUt), static_cast<const uint8_t *>(p.tUt) + ch * kImg64,
+              kImg64, bar);
+    bulk_load(smem_u32(b + OutChainSmem::kQg), static_cast<const uint8_t *>(p.tQg) + ch * kImg64,
+              kImg64, bar);
+    bulk_load(smem_u32(b + OutChainSmem::kP),
+              static_cast<const uint8_t *>(p.tP) + ch * (size_t)(C * C * 2), C * C * 2, bar);
+    bulk_load(smem_u32(sm + OutChainSmem::kG0 + buf * 256), p.tG + ch * C, C * 4, bar);
+}
+
+// Bounded wait of one warpgroup (named barrier `id`, 128 threads) on an mbarrier
+// phase, decided by the warpgroup.
+__device__ __forceinline__ bool wg_wait(uint64_t *bar, uint32_t parity, const Params &p, int id,
+                                        int where) {
+    const bool ok = bar_and(id, NT, mbar_wait(bar, parity, p.wait_limit));
+    if (!ok && (threadIdx.x & (NT - 1)) == 0) record_timeout(p, where);
+    tc_fence_after();
+    return ok;
+}
+
+// Body for CTA `blk` (sequence blk / H, head blk % H): the whole sequence from h0,
+// writing o and hT.
+__device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar, m1bar, m2bar, sqbar, lbar[2], obar[2];
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int H = p.H, n = blk / H, h = blk % H, tid = threadIdx.x;
+    const int c0 = seq_first_at(p, n), c1 = seq_first_at(p, n + 1);
+    if (tid == 0) {
+        mbar_init(&mbar, 1);
+        mbar_init(&m1bar, 1);
+        mbar_init(&m2bar, 1);
+        mbar_init(&sqbar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&lbar[b], 1);
+            mbar_init(&obar[b], 1);
+        }
+        fence_mbar_init();
+    }
+    if (tid < 32) {
+        tmem_alloc(&tslot, 512);
+        tmem_relinquish();
+    }
+    // TMEM columns: 0-63 U^T, 64-191 the state update, 256 + 64 b output buffer b
+    uint8_t *Ss = sm + OutChainSmem::kS, *UTs = sm + OutChainSmem::kUT;
+    if (tid < NT) identity_tile(sm + OutChainSmem::kI);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot, sb = smem_u32(Ss), utb = smem_u32(UTs);
+    const uint32_t id1 = idesc_bf16(128, 64, 0, 0);
+    if (tid < NT) {
+        // ---------------------------------------------------------- warpgroup 0: the chain
+        const int v = tid;
+        float S[D];
+        const float *init = p.h0 ? p.h0 + ((size_t)n * H + h) * p.K * p.V : nullptr;
+#pragma unroll
+        for (int kk = 0; kk < D; ++kk)
+            S[kk] = (init && kk < p.K && v < p.V) ? init[kk * p.V + v] : 0.f;
+        state_image(Ss, S, v);  // the state entering the first chunk
+        uint32_t phase = 0, pend = 0, lpar = 0;
+        if (c0 < c1 && v == 0) {
+            outchain_prefetch(sm, 0, (size_t)c0 * H + h, p, &lbar[0]);
+            pend = 1;
+        }
+        const uint32_t idu = idesc_bf16(128, 64, 1, 0), id2 = idesc_bf16(128, 128, 0, 1),
+                       ib = smem_u32(sm + OutChainSmem::kI);
+        for (int c = c0; c < c1; ++c) {
+            const int it = c - c0, buf = it & 1;
+            const size_t ch = (size_t)c * H + h;
+            uint8_t *b = sm + OutChainSmem::kBuf + buf * OutChainSmem::kBufBytes;
+            // the previous chunk's output is complete: its U^T image (rewritten below) and
+            // its prefetch slot (refilled now) are free
+            bool ok = it == 0 || mbar_wait(&obar[(it - 1) & 1], ((it - 1) >> 1) & 1, p.wait_limit);
+            if (v == 0 && c + 1 < c1 && ok) {
+                outchain_prefetch(sm, buf ^ 1, ch + H, p, &lbar[buf ^ 1]);
+                pend |= 2u >> buf;
+            }
+            const bool lok = ok && mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
+            fence_async_smem();  // the state image written by the previous chunk's update
+            tc_fence_before();
+            const bool all = bar_and(1, NT, lok);
+            tc_fence_after();
+            if (!all) {
+                if (v == 0) record_timeout(p, 50);
+                break;
+            }
+            pend &= ~(1u << buf);
+            lpar ^= 1u << buf;
+            const float gC =
+                expf(reinterpret_cast<const float *>(sm + OutChainSmem::kG0 + buf * 256)[C - 1]);
+            if (v == 0) {
+                const uint32_t wb = smem_u32(b + OutChainSmem::kW),
+                               ub = smem_u32(b + OutChainSmem::kUt);
+#pragma unroll
+                for (int s = 0; s < D / 16; ++s)  // U^T = S (-W)^T + Ut^T I
+                    mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(ib, C, s), idu, 1);
+                mma_commit(&mbar);
+                mbar_arrive(&m1bar);  // the state image and the slot are ready for S Qg^T
+            }
+            if (!wg_wait(&mbar, phase, p, 1, 51)) break;
+            phase ^= 1;
+#pragma unroll
+            for (int c32 = 0; c32 < C; c32 += 32) {  // U^T as an operand tile (row v)
+                float d[32];
+                tmem_ld16(tm(tmem, c32), d);
+                tmem_ld16(tm(tmem, c32 + 16), d + 16);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) =
+                        pack8(d + 8 * q);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            bar_sync(1, NT);
+            tc_fence_after();
+            if (v == 0) {
+                const uint32_t kb = smem_u32(b + OutChainSmem::kKd);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)  // S <- gam_n S + U^T Kd
+                    mma_bf16(tmem + 64, desc_kmajor(utb, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
+                mma_commit(&mbar);
+                mbar_arrive(&m2bar);  // the U^T image is ready for U^T P^T
+            }
+            if (!wg_wait(&mbar, phase, p, 1, 53)) break;
+            phase ^= 1;
+            // S Qg^T has read the state image before it is rewritten
+            if (!wg_wait(&sqbar, it & 1, p, 1, 52)) break;
+#pragma unroll
+            for (int c32 = 0; c32 < D; c32 += 32) {  // S <- gam_n S + U^T Kd, and its image
+                float d[32];
+                tmem_ld16(tm(tmem, 64 + c32), d);
+                tmem_ld16(tm(tmem, 64 + c32 + 16), d + 16);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, c32 / 8 + q)) =
+                        pack8(S + c32 + 8 * q);
+            }
+            tc_fence_before();
+            bar_sync(1, NT);
+            tc_fence_after();
+        }
+        if (v == 0) {  // copies still in flight after an early exit
+            for (int b2 = 0; b2 < 2; ++b2)
+                if ((pend >> b2) & 1u) mbar_wait(&lbar[b2], (lpar >> b2) & 1u, kWaitLimit);
+        }
+        if (p.hT && v < p.V) {
+            float *out = p.hT + ((size_t)n * H + h) * p.K * p.V;
+#pragma unroll
+            for (int kk = 0; kk < D; ++kk)
+                if (kk < p.K) out[kk * p.V + v] = S[kk];
+        }
+    } else {
+        // ---------------------------------------------------------- warpgroup 1: the output
+        const int r = tid - NT;  // row v = r of O^T (warp 4 + w reaches TMEM lane quadrant w)
+        bf16 *stage = reinterpret_cast<bf16 *>(sm + OutChainSmem::kStage);
+        bf16 *o = static_cast<bf16 *>(p.o);
+        for (int c = c0; c < c1; ++c) {
+            const int it = c - c0, buf = it & 1;
+            uint8_t *b = sm + OutChainSmem::kBuf + buf * OutChainSmem::kBufBytes;
+            const uint32_t ob = tmem + 256 + 64 * buf;
+            bool ok = true;
+            if (r == 0) {  // the leader issues the chunk's output product in two parts
+                ok = mbar_wait(&m1bar, it & 1, p.wait_limit);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t qg = smem_u32(b + OutChainSmem::kQg);
+#pragma unroll
+                    for (int s = 0; s < D / 16; ++s)
+                        mma_bf16(ob, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id1, s > 0);
+                    mma_commit(&sqbar);
+                    ok = mbar_wait(&m2bar, it & 1, p.wait_limit);
+                }
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t pb = smem_u32(b + OutChainSmem::kP);
+#pragma unroll
+                    for (int s = 0; s < C / 16; ++s)
+                        mma_bf16(ob, desc_kmajor(utb, D, s), desc_kmajor(pb, C, s), id1, 1);
+                    mma_commit(&obar[buf]);
+                } else {
+                    record_timeout(p, 55);
+                }
+            }
+            if (!bar_and(2, NT, ok)) break;
+            if (!wg_wait(&obar[buf], (it >> 1) & 1, p, 2, 54)) break;
+            for (int c16 = 0; c16 < C; c16 += 16) {
+                float d[16];
+                tmem_ld16(tmq(ob, c16), d);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) stage[(c16 + q) * D + r] = __float2bfloat16_rn(d[q]);
+            }
+            tc_fence_before();
+            bar_sync(2, NT);  // the staged rows are complete and buffer `buf` is read
+            const ChunkInfo ci = chunk_in_seq(p, n, c0, c);
+            for (int t = r; t < C * 16; t += NT) {
+                const int i = t >> 4, j = t & 15;
+                if (i < ci.len && j * 8 < p.V)
+                    *reinterpret_cast<uint4 *>(o + ((int64_t)(ci.tok0 + i) * H + h) * p.V + j * 8) =
+                        *reinterpret_cast<const uint4 *>(stage + i * D + j * 8);
+            }
+            bar_sync(2, NT);  // the stores have read the staging rows
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 32) tmem_dealloc(tmem, 512);
+}
+
 // ============================================================ chain by value slices
 // The value columns of the state evolve independently given a chunk's W, Kd,
 // gates and their own columns of Ut (rows of S = H^T do not mix), so a chain
