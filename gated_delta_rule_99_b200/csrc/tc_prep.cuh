@@ -83,9 +83,9 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     }
     chunk_gates(G, bta, p, ci, h);  // its barriers also publish the mbarrier inits
     if (tid < C) {  // the decay factors, once (published by the barrier of the wait below)
-        F[tid] = expf(G[tid | 15] - G[tid]);
-        E[tid] = expf(G[tid]);
-        EK[tid] = expf(G[C - 1] - G[tid]);
+        F[tid] = __expf(G[tid | 15] - G[tid]);
+        E[tid] = __expf(G[tid]);
+        EK[tid] = __expf(G[C - 1] - G[tid]);
     }
     bool ok = copies_arrived(&lbar, p, 31);
     if (ok) {
@@ -147,7 +147,9 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         // Threads 64-127: L = strict_lower(diag(b) K K^T . Gam) into shared memory (fp32).
         // The 16 rows of a half-warp lie in one 16-block, so the cases are warp-uniform.
         // Gam_ij = exp(G_i - G_e) exp(G_e - G_j) below a row's diagonal block (e = the
-        // block's last column, both factors <= 1), directly inside it.
+        // block's last column, both factors <= 1), directly inside it (the fast
+        // exponential: its relative error, a few units in the last place of fp32,
+        // is far below the bf16 rounding every product operand gets).
         float d[4][16];
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm(tmem, 16 * cb), d[cb]);
@@ -162,14 +164,14 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             const int c0 = 16 * cb;
             float x[16];
             if (cb < ib) {
-                const float ri = ci0 * expf(G[i] - G[c0 + 15]);
+                const float ri = ci0 * __expf(G[i] - G[c0 + 15]);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) x[q] = ri * F[c0 + q] * d[cb][q];
             } else if (cb == ib) {
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int j = c0 + q;
-                    x[q] = (lrow ? j < i : j <= i) ? ci0 * expf(G[i] - G[j]) * d[cb][q] : 0.f;
+                    x[q] = (lrow ? j < i : j <= i) ? ci0 * __expf(G[i] - G[j]) * d[cb][q] : 0.f;
                 }
             } else {
 #pragma unroll
@@ -328,15 +330,18 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         if (ok) {
             const int i = m64_row();
             uint8_t *Wimg = static_cast<uint8_t *>(p.tW) + (size_t)ch * kImg64;
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float w[16];
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                float w[32];
                 tmem_ld16(tm(tmem, c0), w);
+                tmem_ld16(tm(tmem, c0 + 16), w + 16);
                 tmem_ld_wait();
                 if (i >= 0) {  // stored negated: both chains subtract W products
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) w[q] = -w[q];
-                    *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8)) = pack8(w);
-                    *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(w + 8);
+                    for (int q = 0; q < 32; ++q) w[q] = -w[q];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + q)) =
+                            pack8(w + 8 * q);
                 }
             }
             tc_fence_before();
@@ -363,13 +368,15 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
                // first product, whose 64-column blocks are the two halves of the values
         const int i = m64_row();
         uint8_t *Ut = static_cast<uint8_t *>(p.tUt) + (size_t)ch * kImg64;
-        for (int c0 = 0; c0 < D; c0 += 16) {
-            float u[16];
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            float u[32];
             tmem_ld16(tm(tmem, c0), u);
+            tmem_ld16(tm(tmem, c0 + 16), u + 16);
             tmem_ld_wait();
             if (i >= 0) {
-                *reinterpret_cast<uint4 *>(Ut + sw128_chunk(C, i, c0 / 8)) = pack8(u);
-                *reinterpret_cast<uint4 *>(Ut + sw128_chunk(C, i, c0 / 8 + 1)) = pack8(u + 8);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(Ut + sw128_chunk(C, i, c0 / 8 + q)) = pack8(u + 8 * q);
             }
         }
     }
