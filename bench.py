@@ -80,13 +80,14 @@ def kernel_work(name, w, n_chunks):
     # tensor-core path: HBM-facing kernels report the tensors the method must
     # move through them (bytes per token-head), chain kernels their MMA flops
     hbm = {"tc_grads": 4 * 2 * K + 8 + 3 * 2 * K + 8,   # q,k,v,do + g,b in; dq,dk,dv + dg,db out
-           "tc_prep": 2 * (K + V) + 8,                  # k, v, g, b
-           "tc_out": 2 * (2 * K) + 4 + 2 * V,           # q, k, g in; o out
-           "tc_local": 2 * (2 * K + V) + 4,             # q, k, do
-           "tc_prep_local": 2 * (K + V) + 8 + 2 * (2 * K + V) + 4}  # both of the above
+           "tc_prep": 2 * (2 * K + V) + 8,              # q, k, v, g, b
+           "tc_prep_local": 2 * (2 * K + V) + 8,        # the same step in the backward
+           "tc_out": 2 * V}                             # o out (its inputs are intermediates)
     if name in hbm:
         return "hbm", float(hbm[name]) * th, "B"
-    chain = {"tc_state_fwd": 2 * f2(C, V, K), "tc_chains": 5 * f2(C, V, K)}
+    # the forward chain also forms the output: O^T = S Qg^T + U^T P^T per chunk
+    chain = {"tc_state_fwd": 2 * f2(C, V, K) + f2(C, V, K) + f2(C, V, C),
+             "tc_chains": 5 * f2(C, V, K)}
     if name in chain:
         return "tensor", chain[name] * ch, "flop"
     return None, None, None

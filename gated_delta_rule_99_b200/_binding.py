@@ -186,13 +186,16 @@ def gdn_fwd(q, k, v, g, beta, cu_seqlens=None, h0=None, scale=1.0, output_final_
 
 
 def gdn_bwd(q, k, v, g, beta, do, cu_seqlens=None, h0=None, dhT=None, scale=1.0, grads=None,
-            workspace=None, cu_seqlens_host=None, stream=None, want_dh0=True, qk_l2norm=False):
+            workspace=None, cu_seqlens_host=None, stream=None, want_dh0=True, qk_l2norm=False,
+            piece_scan=False):
     """Backward through the C ABI.  Returns (dq, dk, dv, dg, dbeta, dh0); with
-    qk_l2norm, dq and dk are the gradients w.r.t. the raw (unnormalised) q and k."""
+    qk_l2norm, dq and dk are the gradients w.r.t. the raw (unnormalised) q and k;
+    piece_scan sets GDN_FLAG_PIECE_SCAN (both chains of long dense rows in
+    parallel pieces, joined exactly)."""
     L = lib()
     cu_dev, cu_host = _seqlens(cu_seqlens, cu_seqlens_host, q.device)
-    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale,
-                                              GDN_FLAG_QK_L2NORM if qk_l2norm else 0)
+    flags = (GDN_FLAG_QK_L2NORM if qk_l2norm else 0) | (GDN_FLAG_PIECE_SCAN if piece_scan else 0)
+    desc, (B, T, H, K, V, n_seqs) = _desc_from(q, v, cu_host, scale, flags)
     N = n_seqs if n_seqs else B
     _check(q, "q", q.dtype, (B, T, H, K)); _check(k, "k", q.dtype, (B, T, H, K))
     _check(v, "v", q.dtype, (B, T, H, V)); _check(do, "do", q.dtype, (B, T, H, V))

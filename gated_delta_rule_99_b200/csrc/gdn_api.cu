@@ -155,6 +155,9 @@ Params base_params(const Problem &pb, const gdn_desc *d, void *ws, const Layout 
     p.tHin = f(L.tHin);
     p.tMp = f(L.tMp);
     p.tBp = f(L.tBp);
+    p.tdHin = f(L.tdHin);
+    p.tTr = f(L.tTr);
+    p.tBr = f(L.tBr);
     return p;
 }
 
@@ -256,11 +259,16 @@ Layout make_layout(const Problem &pb, bool bwd) {
         L.tUT = take(nch * img64);
         L.tQg = take(nch * img64);                   // bf16 tile image of scale diag(gam) Q
         L.tP = take(nch * kChunk * kChunk * 2);      // bf16 tile image of P
-        if (!bwd && pb.P > 1) {
+        if (pb.P > 1) {  // piece scan: each piece's entering state, transition and offset
             const size_t units = (size_t)pb.N * pb.H * pb.P, st = (size_t)128 * 128 * f;
             L.tHin = take(units * st);
             L.tMp = take(units * st);
             L.tBp = take(units * st);
+            if (bwd) {  // the same for the reverse chain
+                L.tdHin = take(units * st);
+                L.tTr = take(units * st);
+                L.tBr = take(units * st);
+            }
         }
         if (bwd) {
             L.tA = take(nch * kChunk * kChunk * 2);  // bf16 tile image of A

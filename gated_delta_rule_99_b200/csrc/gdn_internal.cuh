@@ -73,6 +73,9 @@ struct Params {
     // (sequence, head, piece) the entering state, the composed transition and offset
     int32_t P, L;
     float *tHin, *tMp, *tBp;
+    // and, for the backward's reverse chain, per (sequence, head, piece) the dS
+    // leaving the piece, the piece's transition and its offset
+    float *tdHin, *tTr, *tBr;
     // tensor maps of the bf16 [tokens][H][d] inputs for the tensor-core path: a box is 64
     // tokens x 64 elements of one head, written to shared memory with the operand tiles'
     // 128-byte swizzle (encoded on the host for every call)
@@ -129,6 +132,7 @@ struct Layout {
     size_t chunks, seq_first;
     size_t W, Ut, A, U, Hs, dUloc, dU, dHn, scratch;
     size_t tW, tUt, tKd, tS, tUT, tQg, tP, tdSn, tdUT, tG, tB, tA, tHin, tMp, tBp;
+    size_t tdHin, tTr, tBr;
     size_t qn, kn, qinv, kinv;  // normalised q, k copies and 1/|row| (passes of the fp32 path)
     size_t total;
 };

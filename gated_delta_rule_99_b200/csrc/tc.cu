@@ -48,156 +48,24 @@ __global__ void __launch_bounds__(kOutChainThreads, 1) tc_state_fwd_out_kernel(P
 }
 
 // ============================================================ piece scan (long rows)
-// Chunks [c0, c1) of piece `piece` of dense row n (pieces of p.L chunks; the
-// last may be shorter or empty).
-__device__ __forceinline__ void piece_range(const Params &p, int n, int piece, int *c0, int *c1) {
-    const int end = seq_first_at(p, n + 1);
-    int a = seq_first_at(p, n) + piece * p.L;
-    a = a < end ? a : end;
-    const int b = a + p.L < end ? a + p.L : end;
-    *c0 = a;
-    *c1 = b;
-}
-
-// Phase A: piece 0 of every (row, head) runs the ordinary chain from h0
-// (snapshots on; its final state enters piece 1); every middle piece
-// 1 <= q <= P - 2 runs once from zero (-> B_q, the offset of its affine map)
-// and once from the identity with Ut taken as zero (-> M_q, its transition).
+// Phase A: piece 0 of every (row, head) runs the ordinary chain from h0, every
+// middle piece once from zero and once from the identity (piece_a_fwd_role);
+// phase B joins them (piece_scan_body); phase C reruns every later piece from
+// its entering state (piece_c_fwd_role).  With p.vslice each role runs as value
+// slices.
 __global__ void __launch_bounds__(NT, 1) tc_piece_a_kernel(Params p) {
     const int nsl = p.vslice ? value_slices(p) : 1, roles = 2 * p.P - 3, blk = blockIdx.x / nsl;
-    const int unit = blk / roles, r = blk % roles;
-    const int n = unit / p.H, h = unit % p.H;
-    const size_t u = (size_t)unit * p.P, DD = (size_t)D * D;
-    ChainFwd a;
-    a.h = h;
-    a.slice = blockIdx.x % nsl;
-    a.where = 31;
-    a.init_user = 1;  // h0 (piece 0); the middle pieces start from zero or the identity
-    a.out_user = 0;   // tHin, tBp, tMp are internal [128][128] blocks
-    int piece;
-    if (r == 0) {
-        piece = 0;
-        a.init = p.h0 ? p.h0 + (size_t)unit * DD : nullptr;
-        a.init_identity = 0;
-        a.zero_ut = 0;
-        a.snapshots = 1;
-        a.final_out = p.tHin + (u + 1) * DD;
-    } else if (r & 1) {
-        piece = (r + 1) / 2;
-        a.init = nullptr;
-        a.init_identity = 0;
-        a.zero_ut = 0;
-        a.snapshots = 0;
-        a.final_out = p.tBp + (u + piece) * DD;
-    } else {
-        piece = r / 2;
-        a.init = nullptr;
-        a.init_identity = 1;
-        a.zero_ut = 1;
-        a.snapshots = 0;
-        a.final_out = p.tMp + (u + piece) * DD;
-    }
-    piece_range(p, n, piece, &a.c0, &a.c1);
-    if (p.vslice) chain_fwd_sliced(p, a);
-    else chain_fwd(p, a);
+    piece_a_fwd_role(p, blk / roles, blk % roles, blockIdx.x % nsl);
 }
-
-// Phase B: per (row, head), the entering state of piece q >= 2,
-//   H_in(q) = M_{q-1} H_in(q-1) + B_{q-1},
-// one tensor-core product per piece (thread v owns column v of H in fp32).
-constexpr int kScanSmem = 65536 + 1024;
 
 __global__ void __launch_bounds__(NT, 1) tc_piece_scan_kernel(Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar;
-    __shared__ uint32_t tslot;
-    if (p.hdr->status) return;
-    const int unit = blockIdx.x, v = threadIdx.x;
-    const size_t u = (size_t)unit * p.P, DD = (size_t)D * D;
-    uint8_t *Ss = sm, *Mt = sm + 32768;
-    float S[D];
-    const float *h1 = p.tHin + (u + 1) * DD;
-#pragma unroll
-    for (int kk = 0; kk < D; ++kk) S[kk] = h1[kk * D + v];
-    if (v == 0) {
-        mbar_init(&mbar, 1);
-        fence_mbar_init();
-    }
-    if (v < 32) {
-        tmem_alloc(&tslot, 128);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tslot, id = idesc_bf16(128, 128, 0, 0);
-    uint32_t phase = 0;
-    for (int q = 2; q < p.P; ++q) {
-        const float *M = p.tMp + (u + q - 1) * DD, *Bq = p.tBp + (u + q - 1) * DD;
-        for (int t = v; t < D * 16; t += NT) {  // M as a K-major operand: rows kk, columns j
-            const int r = t >> 4, j8 = t & 15;
-            const float4 a0 = *reinterpret_cast<const float4 *>(M + r * D + j8 * 8);
-            const float4 a1 = *reinterpret_cast<const float4 *>(M + r * D + j8 * 8 + 4);
-            const float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            *reinterpret_cast<uint4 *>(Mt + sw128_chunk(D, r, j8)) = pack8(f);
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, j)) = pack8(S + 8 * j);
-        operands_ready();
-        if (v == 0) {
-            const uint32_t sb = smem_u32(Ss), mb = smem_u32(Mt);
-#pragma unroll
-            for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(mb, D, s), id, s > 0);
-            mma_commit(&mbar);
-        }
-        if (!cta_wait(&mbar, phase, p, 33)) break;
-        phase ^= 1;
-        float *hq = p.tHin + (u + q) * DD;
-#pragma unroll
-        for (int c32 = 0; c32 < D; c32 += 32) {
-            float d[32];
-            tmem_ld16(tm(tmem, c32), d);
-            tmem_ld16(tm(tmem, c32 + 16), d + 16);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                S[c32 + x] = d[x] + Bq[(c32 + x) * D + v];
-                hq[(c32 + x) * D + v] = S[c32 + x];
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (v < 32) tmem_dealloc(tmem, 128);
+    // H_in(q) = M_{q-1} H_in(q-1) + B_{q-1} for q = 2 .. P - 1
+    piece_scan_body(p, blockIdx.x, p.tHin, p.tMp, p.tBp, 2, p.P - 1, 1, 33);
 }
 
-// Phase C: every piece q >= 1 reruns its chain from its entering state,
-// writing the per-chunk snapshots; the last piece writes hT.
 __global__ void __launch_bounds__(NT, 1) tc_piece_c_kernel(Params p) {
-    const int nsl = p.vslice ? value_slices(p) : 1, blk = blockIdx.x / nsl;
-    const int per = p.P - 1, unit = blk / per, piece = 1 + blk % per;
-    const int n = unit / p.H, h = unit % p.H;
-    const size_t DD = (size_t)D * D;
-    ChainFwd a;
-    a.h = h;
-    a.slice = blockIdx.x % nsl;
-    a.where = 35;
-    a.init_user = 0;  // tHin
-    a.out_user = 1;   // hT
-    a.init = p.tHin + ((size_t)unit * p.P + piece) * DD;
-    a.init_identity = 0;
-    a.zero_ut = 0;
-    a.snapshots = 1;
-    a.final_out = (piece == p.P - 1 && p.hT) ? p.hT + (size_t)unit * DD : nullptr;
-    piece_range(p, n, piece, &a.c0, &a.c1);
-    if (p.vslice) chain_fwd_sliced(p, a);
-    else chain_fwd(p, a);
+    const int nsl = p.vslice ? value_slices(p) : 1, blk = blockIdx.x / nsl, per = p.P - 1;
+    piece_c_fwd_role(p, blk / per, 1 + blk % per, blockIdx.x % nsl);
 }
 
 // ============================================================ tc_out

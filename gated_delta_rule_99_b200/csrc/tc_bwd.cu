@@ -75,22 +75,38 @@ __device__ __forceinline__ void sbwd_prefetch(uint8_t *sm, int buf, size_t ch,
     }
 }
 
-// Body of the reverse state pass for CTA `blk` (sequence blk / H, head blk % H).
-__device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
+// One run of the reverse chain over chunks [c0, c1) of one head, last chunk first.
+struct ChainBwd {
+    int n, h, c0, c1;    // sequence n (its first chunk gives the chunks' positions), range
+    const float *init;   // dS leaving chunk c1 - 1 (fp32), or nullptr for zero
+    int init_user;       // init is a caller's [K][V] block (else an internal [128][128] one)
+    int init_identity;   // start from dS = I (the transition run of the piece scan)
+    int zero_local;      // drop the dO terms (the transition run)
+    int snapshots;       // write dS leaving every chunk and dU^T (tile images)
+    float *final_out;    // dS entering chunk c0 (fp32), or nullptr
+    int out_user;        // final_out is a caller's [K][V] block (else [128][128])
+    int where;           // tag recorded if a bounded wait gives up
+};
+
+// The reverse chain: thread v owns row v of dS = dH^T (fp32 registers), the
+// gradient of the state leaving the current chunk; per chunk
+//   dU^T = dO^T P + dS Kd^T ;  dS <- gam_n dS + dO^T Qg - dU^T W.
+__device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
     __shared__ uint64_t mbar, lbar[2];
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
-    const int H = p.H, n = blk / H, h = blk % H, v = threadIdx.x;
+    const int H = p.H, n = a.n, h = a.h, v = threadIdx.x;
+    const int sq0 = seq_first_at(p, n);  // the sequence's first chunk (chunk positions)
     float S[D];  // dS row v (gradient of the state leaving the current chunk)
-    if (p.dhT) {  // [K][V] blocks; rows and columns past them are zero
-        const float *g0 = p.dhT + ((size_t)n * H + h) * p.K * p.V;
+    if (a.init) {  // [K][V] or [128][128] blocks; rows and columns past them are zero
+        const int ik = a.init_user ? p.K : D, iv = a.init_user ? p.V : D;
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = (kk < p.K && v < p.V) ? g0[kk * p.V + v] : 0.f;
+        for (int kk = 0; kk < D; ++kk) S[kk] = (kk < ik && v < iv) ? a.init[kk * iv + v] : 0.f;
     } else {
 #pragma unroll
-        for (int kk = 0; kk < D; ++kk) S[kk] = 0.f;
+        for (int kk = 0; kk < D; ++kk) S[kk] = (a.init_identity && kk == v) ? 1.f : 0.f;
     }
     if (v == 0) {
         mbar_init(&mbar, 1);
@@ -107,12 +123,13 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
-    const int c0 = seq_first_at(p, n), c1 = seq_first_at(p, n + 1);
+    const int c0 = a.c0, c1 = a.c1;
+    const bool local = !a.zero_local;
     uint32_t phase = 0;
     // per buffer b (bit b): bulk copies in flight, and the parity of their next completion
     uint32_t pend = 0, lpar = 0;
     if (c0 < c1) {
-        sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, chunk_in_seq(p, n, c0, c1 - 1), h, p,
+        sbwd_prefetch(sm, 0, (size_t)(c1 - 1) * H + h, chunk_in_seq(p, n, sq0, c1 - 1), h, p,
                       &lbar[0]);
         pend = 1;
     }
@@ -123,7 +140,7 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         const int buf = (c1 - 1 - c) & 1;
         const size_t ch = (size_t)c * H + h;
         if (c - 1 >= c0) {
-            sbwd_prefetch(sm, buf ^ 1, ch - H, chunk_in_seq(p, n, c0, c - 1), h, p,
+            sbwd_prefetch(sm, buf ^ 1, ch - H, chunk_in_seq(p, n, sq0, c - 1), h, p,
                           &lbar[buf ^ 1]);
             pend |= 2u >> buf;
         }
@@ -138,8 +155,8 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         // dO^T P (the local dU^T; M = 128 (v), N = 64, K = 64 tokens) and dO^T Qg (M = 128,
         // N = 128 keys, K = 64) do not depend on dS: on a full chunk (whose dO rows need no
         // clearing) thread 0 issues them as soon as its copies landed
-        const int len = chunk_in_seq(p, n, c0, c).len;
-        const bool early = len == C && p.V == D;
+        const int len = chunk_in_seq(p, n, sq0, c).len;
+        const bool early = local && len == C && p.V == D;
         auto issue_local = [&]() {
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
@@ -149,13 +166,13 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
                 mma_bf16(tmem + 64, desc_mnmajor(ob, C, s), desc_mnmajor(qb, C, s), idx, s > 0);
         };
         if (v == 0 && lok && early) issue_local();
-        if (lok && !early) fix_rows(b + SbwdSmem::kDO, C, 0, len, p.V);
+        if (lok && local && !early) fix_rows(b + SbwdSmem::kDO, C, 0, len, p.V);
         fence_async_smem();
         tc_fence_before();
         const bool all = __syncthreads_and(lok);
         tc_fence_after();
         if (!all) {
-            if (v == 0) record_timeout(p, 45);
+            if (v == 0) record_timeout(p, a.where);
             break;
         }
         pend &= ~(1u << buf);
@@ -163,19 +180,21 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
         const float gC =
             expf(reinterpret_cast<const float *>(sm + SbwdSmem::kGr + buf * 256)[C - 1]);
         if (v == 0) {
-            if (!early) issue_local();
+            if (local && !early) issue_local();
             // + dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, 1);
+                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, local || s > 0);
             mma_commit(&mbar);
-            bulk_store(static_cast<uint8_t *>(p.tdSn) + ch * kImg128, sb, (uint32_t)kImg128);
-            bulk_commit();
-            // the previous chunk's stores (dU^T, and the dS image this chunk's update
-            // rewrites) have read their sources
-            bulk_wait_read_n<1>();
+            if (a.snapshots) {
+                bulk_store(static_cast<uint8_t *>(p.tdSn) + ch * kImg128, sb, (uint32_t)kImg128);
+                bulk_commit();
+                // the previous chunk's stores (dU^T, and the dS image this chunk's update
+                // rewrites) have read their sources
+                bulk_wait_read_n<1>();
+            }
         }
-        if (!cta_wait(&mbar, phase, p, 13)) break;
+        if (!cta_wait(&mbar, phase, p, a.where + 1)) break;
         phase ^= 1;
 #pragma unroll
         for (int c32 = 0; c32 < C; c32 += 32) {  // dU^T: the next operand, and an image for tc_grads
@@ -192,12 +211,15 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
             const uint32_t ub = smem_u32(dUs), wb = smem_u32(b + SbwdSmem::kW);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(wb, C, s), idy, 1);
+                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(wb, C, s), idy,
+                         local || s > 0);
             mma_commit(&mbar);
-            bulk_store(static_cast<uint8_t *>(p.tdUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
-            bulk_commit();
+            if (a.snapshots) {
+                bulk_store(static_cast<uint8_t *>(p.tdUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
+                bulk_commit();
+            }
         }
-        if (!cta_wait(&mbar, phase, p, 14)) break;
+        if (!cta_wait(&mbar, phase, p, a.where + 2)) break;
         phase ^= 1;
 #pragma unroll
         for (int c32 = 0; c32 < D; c32 += 32) {
@@ -219,19 +241,128 @@ __device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
     if (v == 0) {  // copies still in flight after an early exit
         for (int q = 0; q < 2; ++q)
             if ((pend >> q) & 1u) mbar_wait(&lbar[q], (lpar >> q) & 1u, kWaitLimit);
-        bulk_wait_all();
+        if (a.snapshots) bulk_wait_all();
     }
-    if (p.dh0) {
-        float *g0 = p.dh0 + ((size_t)n * H + h) * p.K * p.V;
-        if (v < p.V) {
+    if (a.final_out) {
+        const int ok = a.out_user ? p.K : D, ov = a.out_user ? p.V : D;
+        if (v < ov) {
 #pragma unroll
             for (int kk = 0; kk < D; ++kk)
-                if (kk < p.K) g0[kk * p.V + v] = S[kk];
+                if (kk < ok) a.final_out[kk * ov + v] = S[kk];
         }
     }
     tc_fence_before();
     __syncthreads();
     if (v < 32) tmem_dealloc(tmem, 256);
+}
+
+// Body of the reverse state pass for CTA `blk` (sequence blk / H, head blk % H):
+// the whole sequence from dhT, writing the per-chunk snapshots and dh0.
+__device__ __forceinline__ void state_bwd_body(const Params &p, int blk) {
+    const int H = p.H, n = blk / H, h = blk % H;
+    ChainBwd a;
+    a.n = n;
+    a.h = h;
+    a.c0 = seq_first_at(p, n);
+    a.c1 = seq_first_at(p, n + 1);
+    a.init = p.dhT ? p.dhT + ((size_t)n * H + h) * p.K * p.V : nullptr;
+    a.init_user = 1;
+    a.init_identity = 0;
+    a.zero_local = 0;
+    a.snapshots = 1;
+    a.final_out = p.dh0 ? p.dh0 + ((size_t)n * H + h) * p.K * p.V : nullptr;
+    a.out_user = 1;
+    a.where = 45;
+    chain_bwd(p, a);
+}
+
+// ============================================================ piece scan (long rows)
+// The backward's piece scan: the forward chain's roles of the forward piece scan
+// (piece_a_fwd_role, piece_c_fwd_role, with snapshots for the gradient kernel
+// and no final state), and the mirrored roles of the reverse chain, whose chunk
+// map is affine in dS as well:
+//   dS_prev = dS (gam_n I - Kd^T W) + dO^T (Qg - P W).
+// Phase A: the last piece runs from dhT with snapshots (its result enters piece
+// P - 2); every middle piece runs once from zero (-> its offset, tBr) and once
+// from dS = I without its dO terms (-> its transition, tTr).
+__device__ __forceinline__ void piece_a_bwd_role(const Params &p, int unit, int r) {
+    const int n = unit / p.H, h = unit % p.H;
+    const size_t u = (size_t)unit * p.P, DD = (size_t)D * D;
+    ChainBwd a;
+    a.n = n;
+    a.h = h;
+    a.where = 60;
+    a.init_user = 1;  // dhT (the last piece); the middle pieces start from zero or the identity
+    a.out_user = 0;   // tdHin, tBr, tTr are internal [128][128] blocks
+    int piece;
+    if (r == 0) {
+        piece = p.P - 1;
+        a.init = p.dhT ? p.dhT + (size_t)unit * DD : nullptr;
+        a.init_identity = 0;
+        a.zero_local = 0;
+        a.snapshots = 1;
+        a.final_out = p.tdHin + (u + p.P - 2) * DD;
+    } else if (r & 1) {
+        piece = (r + 1) / 2;
+        a.init = nullptr;
+        a.init_identity = 0;
+        a.zero_local = 0;
+        a.snapshots = 0;
+        a.final_out = p.tBr + (u + piece) * DD;
+    } else {
+        piece = r / 2;
+        a.init = nullptr;
+        a.init_identity = 1;
+        a.zero_local = 1;
+        a.snapshots = 0;
+        a.final_out = p.tTr + (u + piece) * DD;
+    }
+    piece_range(p, n, piece, &a.c0, &a.c1);
+    chain_bwd(p, a);
+}
+
+// Phase C: piece `piece` <= P - 2 reruns the reverse chain from the dS leaving it
+// (tdHin) with snapshots; piece 0 writes dh0.
+__device__ __forceinline__ void piece_c_bwd_role(const Params &p, int unit, int piece) {
+    const int n = unit / p.H, h = unit % p.H;
+    const size_t DD = (size_t)D * D;
+    ChainBwd a;
+    a.n = n;
+    a.h = h;
+    a.where = 64;
+    a.init_user = 0;
+    a.out_user = 1;
+    a.init = p.tdHin + ((size_t)unit * p.P + piece) * DD;
+    a.init_identity = 0;
+    a.zero_local = 0;
+    a.snapshots = 1;
+    a.final_out = (piece == 0 && p.dh0) ? p.dh0 + (size_t)unit * DD : nullptr;
+    piece_range(p, n, piece, &a.c0, &a.c1);
+    chain_bwd(p, a);
+}
+
+// One launch per phase for both chains: CTAs [0, units * roles) take the forward
+// chain's roles (pf: no final state), the rest the reverse chain's.
+__global__ void __launch_bounds__(NT, 1) tc_bwd_piece_a_kernel(const __grid_constant__ Params pf,
+                                                                const __grid_constant__ Params p) {
+    const int roles = 2 * p.P - 3, nf = p.N * p.H * roles, blk = blockIdx.x;
+    if (blk < nf) piece_a_fwd_role(pf, blk / roles, blk % roles, 0);
+    else piece_a_bwd_role(p, (blk - nf) / roles, (blk - nf) % roles);
+}
+
+__global__ void __launch_bounds__(NT, 1) tc_bwd_piece_scan_kernel(const __grid_constant__ Params p) {
+    const int units = p.N * p.H;
+    if ((int)blockIdx.x < units)  // H_in(q) = M_{q-1} H_in(q-1) + B_{q-1}, q = 2 .. P - 1
+        piece_scan_body(p, blockIdx.x, p.tHin, p.tMp, p.tBp, 2, p.P - 1, 1, 33);
+    else  // dS leaving piece q = dS leaving piece q + 1, times T_{q+1}, plus its offset
+        piece_scan_body(p, blockIdx.x - units, p.tdHin, p.tTr, p.tBr, p.P - 3, 0, -1, 66);
+}
+
+__global__ void __launch_bounds__(NT, 1) tc_bwd_piece_c_kernel(const __grid_constant__ Params pf,
+                                                                const __grid_constant__ Params p) {
+    const int per = p.P - 1, nf = p.N * p.H * per, blk = blockIdx.x;
+    if (blk < nf) piece_c_fwd_role(pf, blk / per, 1 + blk % per, 0);
+    else piece_c_bwd_role(p, (blk - nf) / per, (blk - nf) % per);
 }
 
 // Both chains of the backward in one launch: CTAs [0, N*H) recompute the
@@ -876,8 +1007,20 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
         GDN_LAUNCH(kKTcLocal, stream,
                    tc_prep_local_kernel<<<nch, NT, kPrepSmemRequest, stream>>>(p));
     }
-    if (nseq > 0) {
-        const int sm = kSbwdSmem > kStateSmem ? kSbwdSmem : kStateSmem;
+    const int sm = kSbwdSmem > kStateSmem ? kSbwdSmem : kStateSmem;
+    if (nseq > 0 && p.P > 1) {  // piece scan of long rows, for both chains
+        pf.vslice = 0;
+        const int roles = 2 * p.P - 3;
+        if ((e = set_smem(tc_bwd_piece_a_kernel, sm))) return e;
+        GDN_LAUNCH(kKTcPieceA, stream,
+                   tc_bwd_piece_a_kernel<<<2 * nseq * roles, NT, sm, stream>>>(pf, p));
+        if ((e = set_smem(tc_bwd_piece_scan_kernel, kScanSmem))) return e;
+        GDN_LAUNCH(kKTcPieceScan, stream,
+                   tc_bwd_piece_scan_kernel<<<2 * nseq, NT, kScanSmem, stream>>>(p));
+        if ((e = set_smem(tc_bwd_piece_c_kernel, sm))) return e;
+        GDN_LAUNCH(kKTcPieceC, stream,
+                   tc_bwd_piece_c_kernel<<<2 * nseq * (p.P - 1), NT, sm, stream>>>(pf, p));
+    } else if (nseq > 0) {
         if ((e = set_smem(tc_chains_kernel, sm))) return e;
         GDN_LAUNCH(kKTcStateBwd, stream, tc_chains_kernel<<<2 * nseq, NT, sm, stream>>>(pf, p));
     }

@@ -701,5 +701,162 @@ __device__ __forceinline__ void state_fwd_sliced_body(const Params &p, int blk) 
     chain_fwd_sliced(p, a);
 }
 
+// ============================================================ piece scan roles
+constexpr int kScanSmem = 65536 + 1024;  // the scan's state and transition operand images
+
+// The exact piece scan of long dense rows: each chunk maps the state affinely,
+// H' = M_c H + B_c, so a row split into P pieces of p.L chunks is joined by
+// composing every piece's (transition, offset) pair.
+
+// Chunks [c0, c1) of piece `piece` of dense row n (pieces of p.L chunks; the
+// last may be shorter or empty).
+__device__ __forceinline__ void piece_range(const Params &p, int n, int piece, int *c0, int *c1) {
+    const int end = seq_first_at(p, n + 1);
+    int a = seq_first_at(p, n) + piece * p.L;
+    a = a < end ? a : end;
+    const int b = a + p.L < end ? a + p.L : end;
+    *c0 = a;
+    *c1 = b;
+}
+
+// Forward phase A, role r of (row, head) unit `unit`: r = 0 runs piece 0 from
+// h0 with snapshots (its final state enters piece 1: tHin[1]); odd r runs middle
+// piece (r + 1) / 2 from zero (-> its offset B, tBp); even r >= 2 runs middle
+// piece r / 2 from the identity with Ut taken as zero (-> its transition M, tMp).
+__device__ __forceinline__ void piece_a_fwd_role(const Params &p, int unit, int r, int slice) {
+    const int n = unit / p.H, h = unit % p.H;
+    const size_t u = (size_t)unit * p.P, DD = (size_t)D * D;
+    ChainFwd a;
+    a.h = h;
+    a.slice = slice;
+    a.where = 31;
+    a.init_user = 1;  // h0 (piece 0); the middle pieces start from zero or the identity
+    a.out_user = 0;   // tHin, tBp, tMp are internal [128][128] blocks
+    int piece;
+    if (r == 0) {
+        piece = 0;
+        a.init = p.h0 ? p.h0 + (size_t)unit * DD : nullptr;
+        a.init_identity = 0;
+        a.zero_ut = 0;
+        a.snapshots = 1;
+        a.final_out = p.tHin + (u + 1) * DD;
+    } else if (r & 1) {
+        piece = (r + 1) / 2;
+        a.init = nullptr;
+        a.init_identity = 0;
+        a.zero_ut = 0;
+        a.snapshots = 0;
+        a.final_out = p.tBp + (u + piece) * DD;
+    } else {
+        piece = r / 2;
+        a.init = nullptr;
+        a.init_identity = 1;
+        a.zero_ut = 1;
+        a.snapshots = 0;
+        a.final_out = p.tMp + (u + piece) * DD;
+    }
+    piece_range(p, n, piece, &a.c0, &a.c1);
+    if (p.vslice) chain_fwd_sliced(p, a);
+    else chain_fwd(p, a);
+}
+
+// Forward phase C: piece `piece` >= 1 of unit `unit` reruns its chain from its
+// entering state (tHin) with snapshots; the last piece writes hT (if given).
+__device__ __forceinline__ void piece_c_fwd_role(const Params &p, int unit, int piece, int slice) {
+    const int n = unit / p.H, h = unit % p.H;
+    const size_t DD = (size_t)D * D;
+    ChainFwd a;
+    a.h = h;
+    a.slice = slice;
+    a.where = 35;
+    a.init_user = 0;  // tHin
+    a.out_user = 1;   // hT
+    a.init = p.tHin + ((size_t)unit * p.P + piece) * DD;
+    a.init_identity = 0;
+    a.zero_ut = 0;
+    a.snapshots = 1;
+    a.final_out = (piece == p.P - 1 && p.hT) ? p.hT + (size_t)unit * DD : nullptr;
+    piece_range(p, n, piece, &a.c0, &a.c1);
+    if (p.vslice) chain_fwd_sliced(p, a);
+    else chain_fwd(p, a);
+}
+
+// Phase B for unit `unit`: X[q] = X[q - dir] * T[q - dir] + B[q - dir] for q from
+// q_first to q_last in steps of dir (+1 for the forward, -1 for the reverse
+// chain), one tensor-core product per piece.  X, T, B are [P][128][128] fp32
+// blocks per unit with element [k][v]; in S form (thread v owns row v of S = X^T)
+// the step is S <- S T^T + B^T, the transition read as a K-major operand with rows
+// k.  (For the reverse chain the blocks hold dS^T from a run started at dS = I,
+// and the step dS <- dS T + B reads them the same way.)
+__device__ __forceinline__ void piece_scan_body(const Params &p, int unit, float *X, const float *T,
+                                                const float *Bq, int q_first, int q_last, int dir,
+                                                int where) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1k(smem_raw);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    if (p.hdr->status) return;
+    const int v = threadIdx.x;
+    const size_t u = (size_t)unit * p.P, DD = (size_t)D * D;
+    uint8_t *Ss = sm, *Mt = sm + 32768;
+    float S[D];
+    const float *x0 = X + (u + q_first - dir) * DD;
+#pragma unroll
+    for (int kk = 0; kk < D; ++kk) S[kk] = x0[kk * D + v];
+    if (v == 0) {
+        mbar_init(&mbar, 1);
+        fence_mbar_init();
+    }
+    if (v < 32) {
+        tmem_alloc(&tslot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot, id = idesc_bf16(128, 128, 0, 0);
+    uint32_t phase = 0;
+    for (int q = q_first; dir > 0 ? q <= q_last : q >= q_last; q += dir) {
+        const float *M = T + (u + q - dir) * DD, *Bm = Bq + (u + q - dir) * DD;
+        for (int t = v; t < D * 16; t += NT) {  // the transition as a K-major operand: rows k
+            const int r = t >> 4, j8 = t & 15;
+            const float4 a0 = *reinterpret_cast<const float4 *>(M + r * D + j8 * 8);
+            const float4 a1 = *reinterpret_cast<const float4 *>(M + r * D + j8 * 8 + 4);
+            const float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            *reinterpret_cast<uint4 *>(Mt + sw128_chunk(D, r, j8)) = pack8(f);
+        }
+        state_image(Ss, S, v);
+        operands_ready();
+        if (v == 0) {
+            const uint32_t sb = smem_u32(Ss), mb = smem_u32(Mt);
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(mb, D, s), id, s > 0);
+            mma_commit(&mbar);
+        }
+        if (!cta_wait(&mbar, phase, p, where)) break;
+        phase ^= 1;
+        float *xq = X + (u + q) * DD;
+#pragma unroll
+        for (int c32 = 0; c32 < D; c32 += 32) {
+            float d[32];
+            tmem_ld16(tm(tmem, c32), d);
+            tmem_ld16(tm(tmem, c32 + 16), d + 16);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+                S[c32 + x] = d[x] + Bm[(c32 + x) * D + v];
+                xq[(c32 + x) * D + v] = S[c32 + x];
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (v < 32) tmem_dealloc(tmem, 128);
+}
+
 }  // namespace tc
 }  // namespace gdn

@@ -95,8 +95,12 @@ typedef struct gdn_desc {
  * splits them exactly; the FlashQLA article, "Skipping the warm-up", whose
  * split is approximate).  Results equal the default path up to the bf16
  * rounding of the transition matrices, so the default path's bitwise
- * one-call-equals-chained-calls property does not carry over.  Applies to the
- * bf16, d_k = d_v = 128 forward on dense rows; ignored elsewhere. */
+ * one-call-equals-chained-calls property does not carry over.  In gdn_bwd both
+ * chains are split: the recomputed forward chain as above, and the reverse
+ * chain, whose chunk map is affine in dS too, by the mirrored scheme (pieces run
+ * from a zero and an identity dS, a scan from the row's end, reruns).  Applies
+ * to bf16 dense rows with d_k = d_v = 128 in gdn_fwd and gdn_bwd; ignored
+ * elsewhere. */
 #define GDN_FLAG_PIECE_SCAN 1
 
 /* Option for gdn_fwd, gdn_fwd_noalloc, gdn_bwd and gdn_decode: the layer first

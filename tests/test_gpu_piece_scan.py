@@ -51,3 +51,31 @@ def test_piece_scan_long_context_workload():
     e_h = maxnorm_err(h_p, h_s.cpu().numpy().astype(np.float64))
     print("piece scan long row: o vs sequential %.2e, hT vs sequential %.2e" % (e_o, e_h))
     assert e_o <= TOL and e_h <= TOL
+
+
+def _bwd(d, piece_scan):
+    r = gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, h0=d.h0, dhT=d.dhT, scale=d.scale,
+                    piece_scan=piece_scan)
+    torch.cuda.synchronize()
+    return r
+
+
+@pytest.mark.parametrize("B,T,H,gate", [(1, 16384, 2, 0.1), (2, 64 * 50 + 17, 1, 0.02),
+                                        (1, 8192, 1, 0.005)])
+def test_piece_scan_backward_matches_oracle_and_default_path(B, T, H, gate):
+    """gdn_bwd with both chains split into pieces: every gradient against the
+    fp64 oracle, and against the default backward (they differ only by the bf16
+    rounding of the pieces' transition matrices)."""
+    inp = make_inputs(B=B, T=T, H=H, K=128, V=128, dtype="bf16", seed=80 + H, gate_scale=gate,
+                      scale=0.125)
+    d = inp.to("cuda")
+    got = _bwd(d, True)
+    seq = _bwd(d, False)
+    ref = oracle.gdn_bwd(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.do, h0=inp.h0, dhT=inp.dhT,
+                         scale=inp.scale)
+    errs = {}
+    for name, a, b, c in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), got, ref, seq):
+        errs[name] = maxnorm_err(a, b)
+        errs[name + "_vs_seq"] = maxnorm_err(a, np64(c))
+    print("piece scan backward B=%d T=%d H=%d: %s" % (B, T, H, errs))
+    assert max(errs.values()) <= TOL, errs
