@@ -598,14 +598,18 @@ def run_report(args, rank, world, local_rank):
     # the layer's own q/k normalisation (raw q, k); head dim 64 dense and packed (tensor cores)
     d64 = dict(WORKLOADS[2], K=64, V=64, name="gdn_fwdbwd_bf16_B4_T4096_H16_d64")
     p64 = dict(WORKLOADS[3], K=64, V=64, name=WORKLOADS[3]["name"].replace("d128", "d64"))
+    # a long single row forward + backward (a quarter of the long-context row, which is
+    # a forward workload), with and without the piece scan of both chains
+    lrow = dict(WORKLOADS[4], T=1 << 18, bwd=True, name="gdn_fwdbwd_bf16_B1_T262144_H8_d128")
     runs = ([(i, dict(WORKLOADS[i]), False, False) for i in sorted(WORKLOADS)] +
             [(4, dict(WORKLOADS[4]), True, False), (2, dict(WORKLOADS[2]), False, True),
-             (None, d64, False, False), (None, p64, False, False)])
+             (None, d64, False, False), (None, p64, False, False),
+             (None, lrow, False, False), (None, lrow, True, False)])
     for idx, w, piece, l2 in runs:
         if idx is not None and not l2:
             inp = workload(idx, device="cuda" if idx == 4 else "cpu")
         else:
-            inp = make_inputs(**dict(w, raw_qk=l2))
+            inp = make_inputs(**dict(w, raw_qk=l2, device="cuda" if w["T"] > 100000 else "cpu"))
         d = inp.to(dev)
         cu = inp.cu_seqlens
         cu_dev = None if cu is None else cu.to(dev)
@@ -631,7 +635,7 @@ def run_report(args, rank, world, local_rank):
             if bwd:
                 gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, cu_seqlens=cu_dev,
                             cu_seqlens_host=cu, h0=d.h0, dhT=d.dhT, grads=grads, workspace=ws,
-                            qk_l2norm=l2)
+                            qk_l2norm=l2, piece_scan=piece)
 
         for _ in range(3):
             step()
