@@ -18,7 +18,14 @@
 //                 persistent CTA per SM walks its (chunk, head) units and
 //                 fetches each input group of the next unit into the buffers
 //                 the current one has finished with, so the copies run under
-//                 the compute; dq, dk, dv leave by tensor-map stores.
+//                 the compute; dq and dk leave by tensor-map stores, dv by
+//                 stores of every thread.
+//
+// The gradient of L takes two dependent products, not four: with
+// M = diag(b) V - diag(b gam) K H, U = A M, and dA = dU M^T, so
+// dL = -A^T dA A^T = -A^T dU (A M)^T = -A^T (dU U^T); and the gradient of W's
+// K factor, A^T dW = -A^T dU H^T, is formed as (H (dU^T A))^T from the
+// product dU^T A that dv needs anyway.
 //
 // Products run in transposed form wherever that lets the accumulator use all
 // 128 TMEM lanes (M = 128 over the key or value dim); 64 x 64 products use the
@@ -382,14 +389,18 @@ constexpr int NG = 512;
 constexpr int CW = 16;  // columns per warpgroup
 
 struct GradSmem {
-    // q rows 0-63 and k rows 64-127 form one 128-row tile, dO and v another
+    // q rows 0-63 and k rows 64-127 form one 128-row tile, dO and v another; then the
+    // images S, dSn, U^T, dU^T, A; TA: the dU^T A operand tile, then dq's staged rows;
+    // DKS: dk's staged rows, whose second half first holds the Y = dU U^T operand tile
     static constexpr int kQK = 0, kDV = 32768, kSC = 65536, kDSN = 98304, kUT = 131072,
-                         kDUT = 147456, kAB = 163840, kX3 = 172032, kDA = 188416,
-                         kT1 = 196608, kDPG = 204800, kDLG = 212992, kVec = 221184,
+                         kDUT = 147456, kAB = 163840, kTA = 172032, kDKS = 188416,
+                         kY = kDKS + C * 128, kDPG = 204800, kDLG = 212992, kVec = 221184,
                          kVecFloats = 2432, kEnd = kVec + kVecFloats * 4;
 };
 constexpr int kGradSmem = GradSmem::kEnd + 1024;
-static_assert(GradSmem::kT1 == GradSmem::kDA + C * 128, "[dA; T1] is one 128-row operand tile");
+static_assert(GradSmem::kDPG == GradSmem::kDKS + 2 * C * 128, "dk's staged rows: 16 KB");
+static_assert(GradSmem::kAB == GradSmem::kDUT + 2 * C * 128 && GradSmem::kAB % 1024 == 0,
+              "the 8 KB before A (the second half of dU^T) are the unused rows of A^T Y");
 
 // Column c of an SW128 tile with R rows, read row by row: the swizzle term
 // depends on the row only through row % 8, so it is computed once.
@@ -583,11 +594,21 @@ __device__ __forceinline__ bool thread_wait(uint64_t *bar, uint32_t parity, uint
     return ok;
 }
 
+// Shared-memory addresses of tc_grads' operand tiles, from the aligned base.
+struct GradTiles {
+    uint32_t qk, k, dv, sc, dsn, ut, dut, a, ta, y, dpg, dlg;
+    __device__ __forceinline__ explicit GradTiles(uint32_t b)
+        : qk(b + GradSmem::kQK), k(b + GradSmem::kQK + C * 128), dv(b + GradSmem::kDV),
+          sc(b + GradSmem::kSC), dsn(b + GradSmem::kDSN), ut(b + GradSmem::kUT),
+          dut(b + GradSmem::kDUT), a(b + GradSmem::kAB), ta(b + GradSmem::kTA), y(b + GradSmem::kY),
+          dpg(b + GradSmem::kDPG), dlg(b + GradSmem::kDLG) {}
+};
+
 __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    // MMA completions (one phase in flight on each): mbar_a X3^T and (A^T dU)^T;
-    // mbar_c X1^T, X2^T and Y1; mbar_z Y2 and Zp; mbar the others in order
+    // MMA completions (one phase in flight on each): mbar_a Y and (A^T dU)^T; mbar
+    // [Q;K] K^T and dP, then the last products; mbar_z -dL and Zp; mbar_c X1^T, X2^T
     __shared__ uint64_t mbar, mbar_a, mbar_c, mbar_z, lbar[kGrpCount];
     __shared__ uint32_t tslot;
     __shared__ float s_hd;
@@ -597,7 +618,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     const int i64 = l < 16 ? w4 * 16 + l : -1;  // M = 64 row of this thread's lane
     using S_ = GradSmem;
     uint8_t *QK = sm + S_::kQK, *DV = sm + S_::kDV, *SC = sm + S_::kSC, *DSN = sm + S_::kDSN,
-            *X3 = sm + S_::kX3, *DA = sm + S_::kDA, *T1 = sm + S_::kT1, *DPG = sm + S_::kDPG,
+            *TA = sm + S_::kTA, *DKS = sm + S_::kDKS, *YT = sm + S_::kY, *DPG = sm + S_::kDPG,
             *DLG = sm + S_::kDLG;
     float *vec = reinterpret_cast<float *>(sm + S_::kVec);
     // vec + 0: two [G | b] slots of 128 floats, the current unit's and the prefetched one's
@@ -607,11 +628,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     // per-warp partial column sums, four sets of [4 warps][64 columns]
     float *wsum = vec + 1408;
     float *qdot = rowp, *kdot = rowp + 64;  // (the row partials are consumed before the epilogue)
-    const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128, dvb = smem_u32(DV), vb = dvb + C * 128,
-                   scb = smem_u32(SC), dsb = smem_u32(DSN), utb = smem_u32(sm + S_::kUT),
-                   dub = smem_u32(sm + S_::kDUT), ab = smem_u32(sm + S_::kAB),
-                   x3b = smem_u32(X3), dab = smem_u32(DA), dpb = smem_u32(DPG),
-                   dlb = smem_u32(DLG);
+    const uint32_t smb = smem_u32(sm);  // (the tiles' addresses are formed where issued)
     if (tid == 0) {
         for (int g = 0; g < kGrpCount; ++g) mbar_init(&lbar[g], 1);
         mbar_init(&mbar, 1);
@@ -659,28 +676,30 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             l2norm_tile_rows(QK, D, C, kinv, 2 * C);
             operands_ready();
         }
-        // TMEM columns.  [Q;K] K^T stays to the end (P in lanes 0-63, K K^T in lanes
-        // 64-127); Y2 takes X3's columns once X3 is read, T1 then Y2's, dL then T1's.
-        constexpr int cQK = 0, cX1 = 64, cX2 = 128, cX3 = 192, cDP = 256, cAU = 320, cY1 = 384,
-                      cY2 = 192, cZ = 448, cT1 = 192, cDL = 192, cDQ = 256, cDK = 320, cDKA = 384;
+        // TMEM columns (64 each).  [Q;K] K^T stays to the dL phase (P on lanes 0-63, K K^T
+        // on lanes 64-127).  Y = dU U^T (M = 64) is read into a tile, and its columns then
+        // take A^T Y = -dL; (A^T dU)^T's take Zp^T = (A^T dU H^T)^T once read; dP's take
+        // (dPG K)^T.
+        constexpr int cQK = 0, cX1 = 64, cX2 = 128, cDK = 192, cDP = 256, cAU = 320, cY = 384,
+                      cDKA = 448, cZ = cAU, cDL = cY, cDQ = cDP;
         float d[CW];
-        if (tid == 0) {  // the products the SIMT work needs first (the rest come after X3)
-            const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128mm = idesc_bf16(128, 64, 1, 1),
+        if (tid == 0) {  // the products the SIMT work needs first
+            const GradTiles t(smb);
+            const uint32_t i64mm = idesc_bf16(64, 64, 1, 1), i128 = idesc_bf16(128, 64, 0, 0),
                            i128km = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
-            for (int s = 0; s < 8; ++s)  // X3^T = S^T dU^T
-                mma_bf16(tmem + cX3, desc_mnmajor(scb, D, s), desc_mnmajor(dub, D, s), i128mm,
-                         s > 0);
+            for (int s = 0; s < 8; ++s)  // Y = dU U^T (M = 64, over v)
+                mma_bf16(tmem + cY, desc_mnmajor(t.dut, D, s), desc_mnmajor(t.ut, D, s), i64mm, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)  // (A^T dU)^T = dU^T A
-                mma_bf16(tmem + cAU, desc_kmajor(dub, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
+                mma_bf16(tmem + cAU, desc_kmajor(t.dut, D, s), desc_mnmajor(t.a, C, s), i128km, s > 0);
             mma_commit(&mbar_a);
 #pragma unroll
             for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
-                mma_bf16(tmem + cQK, desc_kmajor(qkb, D, s), desc_kmajor(kb, D, s), i128, s > 0);
+                mma_bf16(tmem + cQK, desc_kmajor(t.qk, D, s), desc_kmajor(t.k, D, s), i128, s > 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s)  // [dO; V] U^T: lanes 0-63 dP = dO U^T, next to P
-                mma_bf16(tmem + cDP, desc_kmajor(dvb, D, s), desc_mnmajor(utb, D, s), i128km,
+                mma_bf16(tmem + cDP, desc_kmajor(t.dv, D, s), desc_mnmajor(t.ut, D, s), i128km,
                          s > 0);
             mma_commit(&mbar);
         } else if (tid >= 32) {  // <S, dSn> (identically laid out images) by warps 1-15
@@ -701,36 +720,62 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 s_hd = a;  // read after later barriers
             }
         }
-        if (tid == 0) bulk_wait_read();  // the previous unit's rows staged in X3 and dA/T1 are out
+        if (tid == 0) bulk_wait_read();  // the previous unit's dq and dk rows staged in TA, DKS are out
         ok = cta_wait(&mbar_a, it & 1, p, 26);
         if (!ok) break;
-        ldcw(tmem, cX3 + cb, d);  // X3^T as an operand tile (row kk)
+        ldcw(tmem, cY + cb, d);  // Y as a 64 x 64 operand tile (rows of the M = 64 layout)
+        if (i64 >= 0) {
 #pragma unroll
-        for (int q = 0; q < CW / 8; ++q)
-            *reinterpret_cast<uint4 *>(X3 + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
+            for (int q = 0; q < CW / 8; ++q)
+                *reinterpret_cast<uint4 *>(YT + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
+        }
+        {  // (A^T dU)^T = dU^T A (thread r holds row v = r): as an operand tile in TA;
+           // dv = diag(b) A^T dU, stored from here; partial v . (A^T dU)
+            ldcw(tmem, cAU + cb, d);
+#pragma unroll
+            for (int q = 0; q < CW / 8; ++q)
+                *reinterpret_cast<uint4 *>(TA + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
+            if (r < p.V) {  // (each warp writes 64 contiguous bytes per token)
+                bf16 *dvp = static_cast<bf16 *>(p.dv) + ((int64_t)(ci.tok0 + cb) * H + h) * p.V + r;
+                const int64_t ts = (int64_t)H * p.V;
+#pragma unroll
+                for (int q = 0; q < CW; ++q)
+                    if (cb + q < ci.len) dvp[q * ts] = __float2bfloat16_rn(bta[cb + q] * d[q]);
+            }
+            {
+                const ColSw vcol(DV + C * 128, D, r);
+#pragma unroll
+                for (int q = 0; q < CW; ++q) d[q] *= vcol.at(cb, q);
+            }
+            warp_colsum(d, wsum, w4, cb, l);
+        }
         operands_ready();
         if (tid == 2 * 32) {  // warp 2 (rows 64-95) has no part in the P . dP phase below
-            const uint32_t i64mk = idesc_bf16(64, 64, 1, 0), i128km = idesc_bf16(128, 64, 0, 1),
-                           i128mk = idesc_bf16(128, 64, 1, 0), i128mm = idesc_bf16(128, 64, 1, 1);
+            const GradTiles t(smb);
+            const uint32_t i128mm = idesc_bf16(128, 64, 1, 1), i128mk = idesc_bf16(128, 64, 1, 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)  // A^T Y = -dL on rows 64-127 (M = 128: rows 0-63 of
+                                         // the A operand are the 8 KB before A, not used)
+                mma_bf16(tmem + cDL, desc_mnmajor(t.a - C * 128, C, s), desc_mnmajor(t.y, C, s),
+                         i128mm, s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)  // Zp^T = S^T (dU^T A) = (A^T X3)^T, X3 = dU H^T
+                mma_bf16(tmem + cZ, desc_mnmajor(t.sc, D, s), desc_mnmajor(t.ta, D, s), i128mm,
+                         s > 0);
+            mma_commit(&mbar_z);
 #pragma unroll
             for (int s = 0; s < 8; ++s)  // X1^T = S^T dO^T  (over v)
-                mma_bf16(tmem + cX1, desc_mnmajor(scb, D, s), desc_kmajor(dvb, D, s), i128mk,
+                mma_bf16(tmem + cX1, desc_mnmajor(t.sc, D, s), desc_kmajor(t.dv, D, s), i128mk,
                          s > 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s)  // X2^T = dSn^T U^T
-                mma_bf16(tmem + cX2, desc_mnmajor(dsb, D, s), desc_mnmajor(utb, D, s), i128mm,
+                mma_bf16(tmem + cX2, desc_mnmajor(t.dsn, D, s), desc_mnmajor(t.ut, D, s), i128mm,
                          s > 0);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)  // Y1 = dU V^T (M = 64)
-                mma_bf16(tmem + cY1, desc_mnmajor(dub, D, s), desc_kmajor(vb, D, s), i64mk, s > 0);
             mma_commit(&mbar_c);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)  // Y2 = X3 K^T (M = 64)
-                mma_bf16(tmem + cY2, desc_mnmajor(x3b, D, s), desc_kmajor(kb, D, s), i64mk, s > 0);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)  // Zp^T = X3^T A   (Z = -Zp)
-                mma_bf16(tmem + cZ, desc_kmajor(x3b, D, s), desc_mnmajor(ab, C, s), i128km, s > 0);
-            mma_commit(&mbar_z);
+        }
+        if (tid < C) {  // dbeta's share from Ut = A diag(b) V (the partials were published above)
+            const float *w = wsum + tid;
+            dB[tid] = (w[0] + w[64]) + (w[128] + w[192]);
         }
         // meanwhile, each thread waiting for what it reads itself (no barrier waits on the
         // issuing warp); the CTA decides on a failed wait at the barrier after them
@@ -759,114 +804,19 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, r, cb / 8 + q)) = pack8(d + 8 * q);
             warp_colsum(pq, wsum + 768, w4, cb, l);
         }
-        {  // dv = diag(b) A^T dU, staged in dA/T1 (thread r holds column r); partial v . (A^T dU)
-            const ColSw vcol(DV + C * 128, D, r);
-            ldcw(tmem, cAU + cb, d);
-            float y[CW];
-#pragma unroll
-            for (int q = 0; q < CW; ++q) {
-                y[q] = bta[cb + q] * d[q];
-                d[q] *= vcol.at(cb, q);
-            }
-            stage_col(DA, y, cb, r);
-            warp_colsum(d, wsum, w4, cb, l);
-        }
-        fine = thread_wait(&mbar_c, it & 1, p.wait_limit) && fine;  // X1, X2, Y1
-        if (more) {  // S, dSn, U^T, dU^T, G and b of the next unit (every product reading
-                     // them is complete: thread 0 waited for all three barriers)
-            if (tid == 0) grads_fetch(p, sm, next, ci, kGrpImg, (it + 1) & 1, lbar);
-            pend |= kGrpImg;
-            ppar = (it + 1) & 1;
-        }
-        {  // column readers of q and k are built where used (they cost 8 registers each)
-            const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
-            ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
-#pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
-            warp_colsum(d, wsum + 256, w4, cb, l);
-            ldcw(tmem, cX2 + cb, d);  // partial k . X2
-#pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
-            warp_colsum(d, wsum + 512, w4, cb, l);
-        }
-        fence_async_smem();  // the staged dv rows leave by bulk copies
         ok = __syncthreads_and(fine);
         if (!ok) {
             if (tid == 0) record_timeout(p, 21);
             break;
         }
-        if (more) {  // dO and v rows of the next unit (read by the first products and the dv sums)
-            if (tid == 0) grads_fetch(p, sm, next, chunk_at(p, next / H), kGrpDV, 0, lbar);
-            pend |= kGrpDV;
-        }
-        store_tile(&p.tm_dv, static_cast<bf16 *>(p.dv), DA, ci.tok0, ci.len, h, H, p.V);
-        if (tid < 3 * C) {
-            const int k = tid >> 6, i = tid & 63;
-            const float *w = wsum + k * 256 + i;
-            (k == 0 ? dB : k == 1 ? qx : kx)[i] = (w[0] + w[64]) + (w[128] + w[192]);
-        }
-        if (tid == 0) bulk_wait_read();  // dA/T1 are written next
-        ok = cta_wait(&mbar_z, it & 1, p, 22);
-        if (!ok) break;
-        {  // dA = (dU V^T) diag(b) - (X3 K^T) diag(b gam)
-            float y2[CW];
-            tmem_ld16(tmq(tmem, cY1 + cb), d);
-            tmem_ld16(tmq(tmem, cY2 + cb), y2);
-            tmem_ld_wait();
-            if (i64 >= 0) {
-#pragma unroll
-                for (int q = 0; q < CW; ++q) {
-                    const int m = cb + q;
-                    d[q] = bta[m] * d[q] - bta[m] * gam[m] * y2[q];
-                }
-#pragma unroll
-                for (int q = 0; q < CW / 8; ++q)
-                    *reinterpret_cast<uint4 *>(DA + sw128_chunk(C, i64, cb / 8 + q)) =
-                        pack8(d + 8 * q);
-            }
-        }
-        operands_ready();
-        if (tid == 0) {  // T1 = A^T dA (M = 64)
-            const uint32_t id = idesc_bf16(64, 64, 1, 1);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem + cT1, desc_mnmajor(ab, C, s), desc_mnmajor(dab, C, s), id, s > 0);
-            mma_commit(&mbar);
-        }
-        // meanwhile: k . Z
-        {
-            const ColSw kcol(QK + C * 128, D, r);
-            ldcw(tmem, cZ + cb, d);  // partial k . Z = -k . Zp
-#pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
-            warp_colsum(d, wsum, w4, cb, l);
-        }
-        __syncthreads();
-        if (tid < C) kz[tid] = (wsum[tid] + wsum[64 + tid]) + (wsum[128 + tid] + wsum[192 + tid]);
-        ok = cta_wait(&mbar, phase, p, 23);
-        phase ^= 1;
-        if (!ok) break;
-        ldcw(tmem, cT1 + cb, d);
-        if (i64 >= 0) {
-#pragma unroll
-            for (int q = 0; q < CW / 8; ++q)
-                *reinterpret_cast<uint4 *>(T1 + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
-        }
-        operands_ready();
-        if (tid == 0) {  // [dA; T1] A^T (M = 128): lanes 64-127 hold T1 A^T = -dL, next to K K^T
-            const uint32_t id = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem + cDL, desc_kmajor(dab, D, s), desc_kmajor(ab, C, s), id, s > 0);
-            mma_commit(&mbar);
-        }
-        ok = cta_wait(&mbar, phase, p, 24);
-        phase ^= 1;
+        ok = cta_wait(&mbar_z, it & 1, p, 22);  // -dL and Zp
         if (!ok) break;
         if (more) {  // A of the next unit (its last product is done)
             if (tid == 0) grads_fetch(p, sm, next, ci, kGrpA, 0, lbar);
             pend |= kGrpA;
         }
+        if (w4 >= 2) fine = thread_wait(&mbar, phase ^ 1, p.wait_limit);  // K K^T (its phase
+                                                                           // is still the last)
         if (w4 >= 2) {  // row i = r - 64: dL (strictly lower), Gam . K K^T; dLG = diag(b) dL . Gam
             const int i = r - C;
             float kk[CW];
@@ -891,23 +841,65 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             dbl2[wg * 64 + i] = dbl;
             warp_colsum(kk, wsum + 768, w4, cb, l);
         }
-        operands_ready();
+        {  // partial k . Z = -k . Zp (its first set of partials was consumed above)
+            const ColSw kcol(QK + C * 128, D, r);
+            ldcw(tmem, cZ + cb, d);
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
+            warp_colsum(d, wsum, w4, cb, l);
+        }
+        fine = thread_wait(&mbar_c, it & 1, p.wait_limit) && fine;  // X1, X2
+        {  // column readers of q and k are built where used (they cost 8 registers each)
+            const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
+            ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
+            warp_colsum(d, wsum + 256, w4, cb, l);
+            ldcw(tmem, cX2 + cb, d);  // partial k . X2
+#pragma unroll
+            for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
+            warp_colsum(d, wsum + 512, w4, cb, l);
+        }
+        fence_async_smem();  // the dPG and dLG tiles are read by the products below
+        tc_fence_before();
+        ok = __syncthreads_and(fine);
+        tc_fence_after();
+        if (!ok) {
+            if (tid == 0) record_timeout(p, 23);
+            break;
+        }
+        if (more) {  // S, dSn, U^T, dU^T, G and b, and the dO and v rows of the next unit
+                     // (every product reading them is complete: X2 was the last)
+            if (tid == 0) {
+                grads_fetch(p, sm, next, ci, kGrpImg, (it + 1) & 1, lbar);
+                grads_fetch(p, sm, next, chunk_at(p, next / H), kGrpDV, 0, lbar);
+            }
+            pend |= kGrpImg | kGrpDV;
+            ppar = (it + 1) & 1;
+        }
         if (tid == 2 * 32) {  // warp 2 has no part in the row sums and the scan below
+            const GradTiles t(smb);
             const uint32_t imk = idesc_bf16(128, 64, 1, 0), imm = idesc_bf16(128, 64, 1, 1);
 #pragma unroll
             for (int s = 0; s < 4; ++s)  // (dPG K)^T = K^T dPG^T
-                mma_bf16(tmem + cDQ, desc_mnmajor(kb, D, s), desc_kmajor(dpb, C, s), imk, s > 0);
+                mma_bf16(tmem + cDQ, desc_mnmajor(t.k, D, s), desc_kmajor(t.dpg, C, s), imk, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)  // (dPG^T Q)^T = Q^T dPG
-                mma_bf16(tmem + cDKA, desc_mnmajor(qkb, D, s), desc_mnmajor(dpb, C, s), imm, s > 0);
+                mma_bf16(tmem + cDKA, desc_mnmajor(t.qk, D, s), desc_mnmajor(t.dpg, C, s), imm, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)  // (diag(b) dLG K)^T
-                mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_kmajor(dlb, C, s), imk, s > 0);
+                mma_bf16(tmem + cDK, desc_mnmajor(t.k, D, s), desc_kmajor(t.dlg, C, s), imk, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)  // ((diag(b) dLG)^T K)^T
-                mma_bf16(tmem + cDK, desc_mnmajor(kb, D, s), desc_mnmajor(dlb, C, s), imm, 1);
+                mma_bf16(tmem + cDK, desc_mnmajor(t.k, D, s), desc_mnmajor(t.dlg, C, s), imm, 1);
             mma_commit(&mbar);
         }
+        if (tid < 3 * C) {
+            const int k = tid >> 6, i = tid & 63;
+            const float *w = wsum + k * 256 + i;
+            (k == 0 ? kz : k == 1 ? qx : kx)[i] = (w[0] + w[64]) + (w[128] + w[192]);
+        }
+        __syncthreads();
         // meanwhile: dbeta and dG (rows), then dg = reverse cumulative sum of dG.  The
         // row sums of P . dP + dL . L are the row partials plus b times the dL rows'
         // sums; the column sums come from the last set of warp partials.
@@ -954,7 +946,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             pend |= kGrpQK;
         }
         {  // dq = scale (diag(gam) X1 + dPG K); dk = diag(e) X2 + diag(b gam) Z + dPG^T Q'
-           // + dL terms; staged (thread r holds column r): dq in X3, dk in dA/T1
+           // + dL terms; staged (thread r holds column r): dq in TA, dk in DKS
             float a[CW];
             tmem_ld16(tmq(tmem, cX1 + cb), d);
             tmem_ld16(tmq(tmem, cDQ + cb), a);
@@ -962,7 +954,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
 #pragma unroll
             for (int q = 0; q < CW; ++q) d[q] = p.scale * (gam[cb + q] * d[q] + a[q]);
             if (p.l2norm) project_rows(d, ColSw(QK, D, r), qinv, qdot, wsum, w4, cb, l);
-            stage_col(X3, d, cb, r);
+            stage_col(TA, d, cb, r);
             tmem_ld16(tmq(tmem, cX2 + cb), d);
             tmem_ld16(tmq(tmem, cZ + cb), a);
             tmem_ld_wait();
@@ -976,7 +968,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             for (int q = 0; q < CW; ++q) d[q] += a[q];
             if (p.l2norm)
                 project_rows(d, ColSw(QK + C * 128, D, r), kinv, kdot, wsum + 256, w4, cb, l);
-            stage_col(DA, d, cb, r);
+            stage_col(DKS, d, cb, r);
         }
         fence_async_smem();
         __syncthreads();  // the unit's reads are done and the staged rows are visible
@@ -984,8 +976,8 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             if (tid == 0) grads_fetch(p, sm, next, chunk_at(p, next / H), kGrpQK, 0, lbar);
             pend |= kGrpQK;
         }
-        store_tile(&p.tm_dq, static_cast<bf16 *>(p.dq), X3, ci.tok0, ci.len, h, H, p.K);
-        store_tile(&p.tm_dk, static_cast<bf16 *>(p.dk), DA, ci.tok0, ci.len, h, H, p.K);
+        store_tile(&p.tm_dq, static_cast<bf16 *>(p.dq), TA, ci.tok0, ci.len, h, H, p.K);
+        store_tile(&p.tm_dk, static_cast<bf16 *>(p.dk), DKS, ci.tok0, ci.len, h, H, p.K);
         if (ci.len < C) __syncthreads();  // (the next unit rewrites the tiles)
     }
     if (!ok && tid == 0) groups_drain(lbar, pend, ppar);  // leave no copy in flight
@@ -1026,10 +1018,8 @@ cudaError_t launch_tc_bwd(const Params &p, const Problem &, cudaStream_t stream)
     }
     if (nch > 0) {
         if ((e = set_smem(tc_grads_kernel, kGradSmem))) return e;
-        int dev = 0, nsm = 0;  // one persistent CTA per SM (or per unit, if fewer)
-        if ((e = cudaGetDevice(&dev))) return e;
-        if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev))) return e;
-        const int grid = nch < nsm ? nch : nsm;
+        int grid = 0;  // one persistent CTA per SM (or per unit, if fewer)
+        if ((e = persistent_grid(nch, 1, grid))) return e;
         GDN_LAUNCH(kKTcGrads, stream, tc_grads_kernel<<<grid, NG, kGradSmem, stream>>>(p));
     }
     return cudaSuccess;

@@ -82,16 +82,17 @@ __device__ __forceinline__ void fix_rows(uint8_t *tile, int R, int row0, int len
     }
 }
 
-// Bounded wait for phase 0 of `bar` (a CTA's input copies), decided by the
+// Bounded wait for phase `parity` of `bar` (a CTA's input copies), decided by the
 // whole CTA (a barrier); the caller must have made the mbarrier's init visible
 // to every thread (a barrier after it) first.  On failure records `where` and
 // waits once more, bounded, so that no copy is left in flight when the CTA
 // gives up.
-__device__ __forceinline__ bool copies_arrived(uint64_t *bar, const Params &p, int where) {
-    const bool ok = __syncthreads_and(mbar_wait(bar, 0, p.wait_limit));
+__device__ __forceinline__ bool copies_arrived(uint64_t *bar, const Params &p, int where,
+                                               uint32_t parity = 0) {
+    const bool ok = __syncthreads_and(mbar_wait(bar, parity, p.wait_limit));
     if (!ok && threadIdx.x == 0) {
         record_timeout(p, where);
-        mbar_wait(bar, 0, kWaitLimit);
+        mbar_wait(bar, parity, kWaitLimit);
     }
     return ok;
 }
@@ -160,6 +161,16 @@ __device__ __forceinline__ int m64_row() {
 template <typename Kern>
 inline cudaError_t set_smem(Kern k, int bytes) {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// Grid of a persistent launch: `per_sm` CTAs on every SM of the current device, or
+// one per unit if there are fewer units.
+inline cudaError_t persistent_grid(int units, int per_sm, int &grid) {
+    int dev = 0, nsm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    grid = units < per_sm * nsm ? units : per_sm * nsm;
+    return e;
 }
 
 // The layer's optional q/k normalisation inside a kernel (jax-linear-attention
