@@ -193,13 +193,13 @@ __device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
             for (int s = 0; s < D / 16; ++s)
                 mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, local || s > 0);
             mma_commit(&mbar);
-            if (a.snapshots) {
-                bulk_store(static_cast<uint8_t *>(p.tdSn) + ch * kImg128, sb, (uint32_t)kImg128);
-                bulk_commit();
-                // the previous chunk's stores (dU^T, and the dS image this chunk's update
-                // rewrites) have read their sources
-                bulk_wait_read_n<1>();
-            }
+        }
+        if (v == 0 && a.snapshots) {
+            bulk_store(static_cast<uint8_t *>(p.tdSn) + ch * kImg128, sb, (uint32_t)kImg128);
+            bulk_commit();
+            // the previous chunk's stores (dU^T, and the dS image this chunk's update
+            // rewrites) have read their sources
+            bulk_wait_read_n<1>();
         }
         if (!cta_wait(&mbar, phase, p, a.where + 1)) break;
         phase ^= 1;
@@ -221,10 +221,10 @@ __device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
                 mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(wb, C, s), idy,
                          local || s > 0);
             mma_commit(&mbar);
-            if (a.snapshots) {
-                bulk_store(static_cast<uint8_t *>(p.tdUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
-                bulk_commit();
-            }
+        }
+        if (v == 0 && a.snapshots) {
+            bulk_store(static_cast<uint8_t *>(p.tdUT) + ch * kImgUT, smem_u32(dUs), (uint32_t)kImgUT);
+            bulk_commit();
         }
         if (!cta_wait(&mbar, phase, p, a.where + 2)) break;
         phase ^= 1;
@@ -391,14 +391,15 @@ constexpr int CW = 16;  // columns per warpgroup
 struct GradSmem {
     // q rows 0-63 and k rows 64-127 form one 128-row tile, dO and v another; then the
     // images S, dSn, U^T, dU^T, A; TA: the dU^T A operand tile, then dq's staged rows;
-    // DKS: dk's staged rows, whose second half first holds the Y = dU U^T operand tile
+    // DKS: dv's staged rows, then dk's; the dPG tile; the dLG tile, which first holds
+    // the Y = dU U^T operand tile
     static constexpr int kQK = 0, kDV = 32768, kSC = 65536, kDSN = 98304, kUT = 131072,
                          kDUT = 147456, kAB = 163840, kTA = 172032, kDKS = 188416,
-                         kY = kDKS + C * 128, kDPG = 204800, kDLG = 212992, kVec = 221184,
+                         kDPG = 204800, kDLG = 212992, kY = kDLG, kVec = 221184,
                          kVecFloats = 2432, kEnd = kVec + kVecFloats * 4;
 };
 constexpr int kGradSmem = GradSmem::kEnd + 1024;
-static_assert(GradSmem::kDPG == GradSmem::kDKS + 2 * C * 128, "dk's staged rows: 16 KB");
+static_assert(GradSmem::kDPG == GradSmem::kDKS + 2 * C * 128, "dv's and dk's staged rows: 16 KB");
 static_assert(GradSmem::kAB == GradSmem::kDUT + 2 * C * 128 && GradSmem::kAB % 1024 == 0,
               "the 8 KB before A (the second half of dU^T) are the unused rows of A^T Y");
 
@@ -609,7 +610,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
     uint8_t *sm = align1k(smem_raw);
     // MMA completions (one phase in flight on each): mbar_a Y and (A^T dU)^T; mbar
     // [Q;K] K^T and dP, then the last products; mbar_z -dL and Zp; mbar_c X1^T, X2^T
-    __shared__ uint64_t mbar, mbar_a, mbar_c, mbar_z, lbar[kGrpCount];
+    __shared__ uint64_t mbar, mbar_a, mbar_c, mbar_z, ibar, lbar[kGrpCount];
     __shared__ uint32_t tslot;
     __shared__ float s_hd;
     if (p.hdr->status) return;
@@ -635,6 +636,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         mbar_init(&mbar_a, 1);
         mbar_init(&mbar_c, 1);
         mbar_init(&mbar_z, 1);
+        mbar_init(&ibar, 1);
         fence_mbar_init();
     }
     if (tid < 32) {
@@ -659,18 +661,25 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         const bool more = next < nunits;
         const ChunkInfo ci = chunk_at(p, c);
         const float *G = vec + (it & 1) * 128, *bta = G + 64;
-        ok = groups_arrived(lbar, pend, ppar, p, 20);
+        // A full chunk with 128-wide heads and no normalisation needs no pass over its
+        // rows: its q and k rows are then waited for by the thread that issues [Q;K] K^T
+        // only, after the products that do not read them
+        const bool late_qk = ci.len == C && p.K == D && p.V == D && !p.l2norm;
+        const uint32_t first = late_qk ? (pend & ~uint32_t(kGrpQK)) : pend;
+        ok = groups_arrived(lbar, first, ppar, p, 20);
         if (!ok) break;
-        pend = 0;
+        pend &= ~first;
         if (tid < C) {
             gam[tid] = expf(G[tid]);
             e[tid] = expf(G[C - 1] - G[tid]);
         }
-        fix_rows(QK, D, 0, ci.len, p.K, NG);
-        fix_rows(QK, D, C, ci.len, p.K, NG);
-        fix_rows(DV, D, 0, ci.len, p.V, NG);
-        fix_rows(DV, D, C, ci.len, p.V, NG);
-        operands_ready();
+        if (!late_qk) {
+            fix_rows(QK, D, 0, ci.len, p.K, NG);
+            fix_rows(QK, D, C, ci.len, p.K, NG);
+            fix_rows(DV, D, 0, ci.len, p.V, NG);
+            fix_rows(DV, D, C, ci.len, p.V, NG);
+            operands_ready();
+        }
         if (p.l2norm) {  // q rows (threads 0-127) and k rows (128-255) divided by their norms
             l2norm_tile_rows(QK, D, 0, qinv, 0);
             l2norm_tile_rows(QK, D, C, kinv, 2 * C);
@@ -683,10 +692,10 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
         constexpr int cQK = 0, cX1 = 64, cX2 = 128, cDK = 192, cDP = 256, cAU = 320, cY = 384,
                       cDKA = 448, cZ = cAU, cDL = cY, cDQ = cDP;
         float d[CW];
+        bool qk_ok = true;
         if (tid == 0) {  // the products the SIMT work needs first
             const GradTiles t(smb);
-            const uint32_t i64mm = idesc_bf16(64, 64, 1, 1), i128 = idesc_bf16(128, 64, 0, 0),
-                           i128km = idesc_bf16(128, 64, 0, 1);
+            const uint32_t i64mm = idesc_bf16(64, 64, 1, 1), i128km = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
             for (int s = 0; s < 8; ++s)  // Y = dU U^T (M = 64, over v)
                 mma_bf16(tmem + cY, desc_mnmajor(t.dut, D, s), desc_mnmajor(t.ut, D, s), i64mm, s > 0);
@@ -694,17 +703,28 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             for (int s = 0; s < 4; ++s)  // (A^T dU)^T = dU^T A
                 mma_bf16(tmem + cAU, desc_kmajor(t.dut, D, s), desc_mnmajor(t.a, C, s), i128km, s > 0);
             mma_commit(&mbar_a);
+            mbar_arrive(&ibar);  // the products of the P . dP phase go in after these
+        } else if (tid == 32) {  // warp 1's leader: the products of the P . dP phase
+            const GradTiles t(smb);
+            const uint32_t i128 = idesc_bf16(128, 64, 0, 0), i128km = idesc_bf16(128, 64, 0, 1);
+            qk_ok = mbar_wait(&ibar, it & 1, p.wait_limit);
+            if (qk_ok) {
 #pragma unroll
-            for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
-                mma_bf16(tmem + cQK, desc_kmajor(t.qk, D, s), desc_kmajor(t.k, D, s), i128, s > 0);
+                for (int s = 0; s < 8; ++s)  // [dO; V] U^T: lanes 0-63 dP = dO U^T, next to P
+                    mma_bf16(tmem + cDP, desc_kmajor(t.dv, D, s), desc_mnmajor(t.ut, D, s), i128km,
+                             s > 0);
+                qk_ok = !(pend & kGrpQK) || mbar_wait(&lbar[3], ppar, p.wait_limit);
+            }
+            if (qk_ok) {
 #pragma unroll
-            for (int s = 0; s < 8; ++s)  // [dO; V] U^T: lanes 0-63 dP = dO U^T, next to P
-                mma_bf16(tmem + cDP, desc_kmajor(t.dv, D, s), desc_mnmajor(t.ut, D, s), i128km,
-                         s > 0);
+                for (int s = 0; s < 8; ++s)  // [Q;K] K^T: lanes 0-63 Q K^T, lanes 64-127 K K^T
+                    mma_bf16(tmem + cQK, desc_kmajor(t.qk, D, s), desc_kmajor(t.k, D, s), i128,
+                             s > 0);
+            }
             mma_commit(&mbar);
-        } else if (tid >= 32) {  // <S, dSn> (identically laid out images) by warps 1-15
+        } else if (tid >= 64) {  // <S, dSn> (identically laid out images) by warps 2-15
             float s = 0.f;
-            for (int t = tid - 32; t < D * D / 8; t += NG - 32) {
+            for (int t = tid - 64; t < D * D / 8; t += NG - 64) {
                 float a[8], b[8];
                 unpack8(*reinterpret_cast<const uint4 *>(SC + t * 16), a);
                 unpack8(*reinterpret_cast<const uint4 *>(DSN + t * 16), b);
@@ -712,17 +732,26 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 for (int q = 0; q < 8; ++q) s = fmaf(a[q], b[q], s);
             }
             for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            if (l == 0) tmp[(tid >> 5) - 1] = s;
-            bar_sync(1, NG - 32);
-            if (tid == 32) {
+            if (l == 0) tmp[(tid >> 5) - 2] = s;
+            bar_sync(1, NG - 64);
+            if (tid == 64) {
                 float a = 0.f;
-                for (int w = 0; w < NG / 32 - 1; ++w) a += tmp[w];
+                for (int w = 0; w < NG / 32 - 2; ++w) a += tmp[w];
                 s_hd = a;  // read after later barriers
             }
         }
         if (tid == 0) bulk_wait_read();  // the previous unit's dq and dk rows staged in TA, DKS are out
-        ok = cta_wait(&mbar_a, it & 1, p, 26);
-        if (!ok) break;
+        {
+            const bool ok_a = mbar_wait(&mbar_a, it & 1, p.wait_limit);
+            ok = __syncthreads_and(ok_a && qk_ok);  // (qk_ok: thread 32's wait for the q, k rows)
+            tc_fence_after();
+            if (!ok) {
+                if (!ok_a) record_timeout(p, 26);
+                if (!qk_ok) record_timeout(p, 20);
+                break;
+            }
+        }
+        pend &= ~uint32_t(kGrpQK);
         ldcw(tmem, cY + cb, d);  // Y as a 64 x 64 operand tile (rows of the M = 64 layout)
         if (i64 >= 0) {
 #pragma unroll
@@ -730,17 +759,16 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 *reinterpret_cast<uint4 *>(YT + sw128_chunk(C, i64, cb / 8 + q)) = pack8(d + 8 * q);
         }
         {  // (A^T dU)^T = dU^T A (thread r holds row v = r): as an operand tile in TA;
-           // dv = diag(b) A^T dU, stored from here; partial v . (A^T dU)
+           // dv = diag(b) A^T dU, staged in DKS (thread r holds column r); partial v . (A^T dU)
             ldcw(tmem, cAU + cb, d);
 #pragma unroll
             for (int q = 0; q < CW / 8; ++q)
                 *reinterpret_cast<uint4 *>(TA + sw128_chunk(D, r, cb / 8 + q)) = pack8(d + 8 * q);
-            if (r < p.V) {  // (each warp writes 64 contiguous bytes per token)
-                bf16 *dvp = static_cast<bf16 *>(p.dv) + ((int64_t)(ci.tok0 + cb) * H + h) * p.V + r;
-                const int64_t ts = (int64_t)H * p.V;
+            {
+                float y[CW];
 #pragma unroll
-                for (int q = 0; q < CW; ++q)
-                    if (cb + q < ci.len) dvp[q * ts] = __float2bfloat16_rn(bta[cb + q] * d[q]);
+                for (int q = 0; q < CW; ++q) y[q] = bta[cb + q] * d[q];
+                stage_col(DKS, y, cb, r);
             }
             {
                 const ColSw vcol(DV + C * 128, D, r);
@@ -749,7 +777,8 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             }
             warp_colsum(d, wsum, w4, cb, l);
         }
-        operands_ready();
+        operands_ready();  // (also publishes the staged dv rows to the tensor-map store)
+        store_tile(&p.tm_dv, static_cast<bf16 *>(p.dv), DKS, ci.tok0, ci.len, h, H, p.V);
         if (tid == 2 * 32) {  // warp 2 (rows 64-95) has no part in the P . dP phase below
             const GradTiles t(smb);
             const uint32_t i128mm = idesc_bf16(128, 64, 1, 1), i128mk = idesc_bf16(128, 64, 1, 0);
@@ -841,24 +870,28 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             dbl2[wg * 64 + i] = dbl;
             warp_colsum(kk, wsum + 768, w4, cb, l);
         }
-        {  // partial k . Z = -k . Zp (its first set of partials was consumed above)
-            const ColSw kcol(QK + C * 128, D, r);
-            ldcw(tmem, cZ + cb, d);
-#pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] *= -kcol.at(cb, q);
-            warp_colsum(d, wsum, w4, cb, l);
-        }
         fine = thread_wait(&mbar_c, it & 1, p.wait_limit) && fine;  // X1, X2
-        {  // column readers of q and k are built where used (they cost 8 registers each)
-            const ColSw qcol(QK, D, r), kcol(QK + C * 128, D, r);
-            ldcw(tmem, cX1 + cb, d);  // partial q' . X1 (thread kk)
+        {  // partial q' . X1 (thread kk); a column reader costs 8 registers: built where used
+            const ColSw qcol(QK, D, r);
+            ldcw(tmem, cX1 + cb, d);
 #pragma unroll
             for (int q = 0; q < CW; ++q) d[q] *= p.scale * qcol.at(cb, q);
             warp_colsum(d, wsum + 256, w4, cb, l);
-            ldcw(tmem, cX2 + cb, d);  // partial k . X2
+        }
+        {  // partial k . X2, and k . Z = -k . Zp (its set of partials was consumed above)
+            const ColSw kcol(QK + C * 128, D, r);
+            float z[CW];
+            tmem_ld16(tmq(tmem, cX2 + cb), d);
+            tmem_ld16(tmq(tmem, cZ + cb), z);
+            tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] *= kcol.at(cb, q);
+            for (int q = 0; q < CW; ++q) {
+                const float kv = kcol.at(cb, q);
+                d[q] *= kv;
+                z[q] *= -kv;
+            }
             warp_colsum(d, wsum + 512, w4, cb, l);
+            warp_colsum(z, wsum, w4, cb, l);
         }
         fence_async_smem();  // the dPG and dLG tiles are read by the products below
         tc_fence_before();
@@ -877,7 +910,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             pend |= kGrpImg | kGrpDV;
             ppar = (it + 1) & 1;
         }
-        if (tid == 2 * 32) {  // warp 2 has no part in the row sums and the scan below
+        if (tid == 7 * 32) {  // warp 7 has no part in the sums and the scan below
             const GradTiles t(smb);
             const uint32_t imk = idesc_bf16(128, 64, 1, 0), imm = idesc_bf16(128, 64, 1, 1);
 #pragma unroll
@@ -894,12 +927,12 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 mma_bf16(tmem + cDK, desc_mnmajor(t.k, D, s), desc_mnmajor(t.dlg, C, s), imm, 1);
             mma_commit(&mbar);
         }
-        if (tid < 3 * C) {
+        if (tid < 3 * C) {  // (warps 0-5)
             const int k = tid >> 6, i = tid & 63;
             const float *w = wsum + k * 256 + i;
             (k == 0 ? kz : k == 1 ? qx : kx)[i] = (w[0] + w[64]) + (w[128] + w[192]);
+            bar_sync(2, 3 * C);
         }
-        __syncthreads();
         // meanwhile: dbeta and dG (rows), then dg = reverse cumulative sum of dG.  The
         // row sums of P . dP + dL . L are the row partials plus b times the dL rows'
         // sums; the column sums come from the last set of warp partials.
@@ -912,8 +945,8 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             const float csum = (w[0] + w[64]) + (w[128] + w[192]);
             dG[i] = -e[i] * kx[i] + gam[i] * qx[i] + (rsum - csum) + bta[i] * gam[i] * kz[i];
             dB[i] += dbs + gam[i] * kz[i];
+            bar_sync(3, C);  // (warps 0-1)
         }
-        __syncthreads();
         if (tid < 32) {  // dg = reverse cumulative sum of dG (+ the terms of the last token)
             const float a = dG[2 * l], b = dG[2 * l + 1];
             float s = e[2 * l] * kx[2 * l] + e[2 * l + 1] * kx[2 * l + 1];
@@ -938,6 +971,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
                 p.dbeta[o] = dB[i0 + 1];
             }
         }
+        if (tid == 0) bulk_wait_read();  // the staged dv rows are out (dk's are staged next)
         ok = cta_wait(&mbar, phase, p, 25);
         phase ^= 1;
         if (!ok) break;
@@ -960,12 +994,14 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < CW; ++q) d[q] = e[cb + q] * d[q] - bta[cb + q] * gam[cb + q] * a[q];
-            ldcw(tmem, cDKA + cb, a);
+            {
+                float z[CW];
+                tmem_ld16(tmq(tmem, cDKA + cb), a);
+                tmem_ld16(tmq(tmem, cDK + cb), z);
+                tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] += p.scale * a[q];
-            ldcw(tmem, cDK + cb, a);
-#pragma unroll
-            for (int q = 0; q < CW; ++q) d[q] += a[q];
+                for (int q = 0; q < CW; ++q) d[q] += p.scale * a[q] + z[q];
+            }
             if (p.l2norm)
                 project_rows(d, ColSw(QK + C * 128, D, r), kinv, kdot, wsum + 256, w4, cb, l);
             stage_col(DKS, d, cb, r);

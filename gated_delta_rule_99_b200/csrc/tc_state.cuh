@@ -22,9 +22,13 @@ constexpr int kStateSmem = StateSmem::kEnd + 1024;
 
 // Bulk copies (thread 0) of chunk ch's W, Kd and Ut images (Ut unless the run
 // takes it as zero) and its gate row into buffer `buf`, completing on `bar`.
+// Thread kPrefetcher issues the chains' prefetch copies and snapshot stores, so that
+// thread 0, which issues the products, is not held up by them.
+constexpr int kPrefetcher = 64;
+
 __device__ __forceinline__ void state_prefetch(uint8_t *sm, int buf, size_t ch, const Params &p,
                                                bool with_ut, uint64_t *bar) {
-    if (threadIdx.x != 0) return;
+    if (threadIdx.x != kPrefetcher) return;
     mbar_arrive_expect_tx(bar, (with_ut ? 3u : 2u) * (uint32_t)kImg64 + C * 4u);
     bulk_load(smem_u32(sm + StateSmem::kW0 + buf * 16384),
               static_cast<const uint8_t *>(p.tW) + ch * kImg64, kImg64, bar);
@@ -120,10 +124,6 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         const int buf = (c - c0) & 1;
         const size_t ch = (size_t)c * H + h;
         uint8_t *Ss = sm + StateSmem::kS0 + buf * 32768, *Sn = sm + StateSmem::kS0 + (buf ^ 1) * 32768;
-        if (c + 1 < c1) {
-            state_prefetch(sm, buf ^ 1, ch + H, p, with_ut, &lbar[buf ^ 1]);
-            pend |= 2u >> buf;
-        }
         const bool lok = mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
         fence_async_smem();  // the state image written by the previous chunk's update
         tc_fence_before();
@@ -135,6 +135,11 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         }
         pend &= ~(1u << buf);
         lpar ^= 1u << buf;
+        // the other buffer's chunk was consumed by the previous chunk's products
+        if (c + 1 < c1) {
+            state_prefetch(sm, buf ^ 1, ch + H, p, with_ut, &lbar[buf ^ 1]);
+            pend |= 2u >> buf;
+        }
         const float gC =
             expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
         if (v == 0) {  // U^T = S (-W)^T + Ut^T I  (the W image is stored negated)
@@ -149,13 +154,13 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
                     mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(ib, C, s), idu, 1);
             }
             mma_commit(&mbar);
-            if (a.snapshots) {
-                bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128, sb, (uint32_t)kImg128);
-                bulk_commit();
-                // the previous chunk's stores (U^T, and the state image that this chunk's
-                // update rewrites) have read their sources
-                bulk_wait_read_n<1>();
-            }
+        }
+        if (v == kPrefetcher && a.snapshots) {
+            bulk_store(static_cast<uint8_t *>(p.tS) + ch * kImg128, smem_u32(Ss), (uint32_t)kImg128);
+            bulk_commit();
+            // the previous chunk's stores (U^T, and the state image that this chunk's
+            // update rewrites) have read their sources
+            bulk_wait_read_n<1>();
         }
         if (!cta_wait(&mbar, phase, p, a.where)) break;
         phase ^= 1;
@@ -176,10 +181,10 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
             mma_commit(&mbar);
-            if (a.snapshots) {
-                bulk_store(static_cast<uint8_t *>(p.tUT) + ch * kImgUT, ub, (uint32_t)kImgUT);
-                bulk_commit();
-            }
+        }
+        if (v == kPrefetcher && a.snapshots) {
+            bulk_store(static_cast<uint8_t *>(p.tUT) + ch * kImgUT, smem_u32(UTs), (uint32_t)kImgUT);
+            bulk_commit();
         }
         if (!cta_wait(&mbar, phase, p, a.where + 1)) break;
         phase ^= 1;
@@ -200,7 +205,7 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         __syncthreads();
         tc_fence_after();
     }
-    if (v == 0) {  // copies still in flight after an early exit
+    if (v == kPrefetcher) {  // copies still in flight after an early exit
         for (int b = 0; b < 2; ++b)
             if ((pend >> b) & 1u) mbar_wait(&lbar[b], (lpar >> b) & 1u, kWaitLimit);
         if (a.snapshots) bulk_wait_all();
@@ -229,15 +234,14 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
 // the chain has issued the chunk's first product (m1bar) and U^T P^T once it has
 // issued the second (m2bar), so they run in the tensor pipe's gaps while the
 // chain's own issuing thread is not held up; then the warpgroup reads the
-// accumulator, stages it as token rows and stores them.  The chain waits for
+// accumulator and stores the output columns it holds.  The chain waits for
 // sqbar (S Qg^T has read the state image) before rewriting the state image and
 // for obar (the chunk's output is complete) before rewriting the U^T image or
 // refilling the chunk's prefetch slot.  Every wait is bounded.
 struct OutChainSmem {
-    // the state image, U^T, the identity block, the output staging rows, then per
-    // prefetch slot the W, Kd, Ut and Qg images and the P tile; the slots' gate rows
-    static constexpr int kS = 0, kUT = kS + 32768, kI = kUT + 16384, kStage = kI + 8192,
-                         kBuf = kStage + 16384;
+    // the state image, U^T, the identity block, then per prefetch slot the W, Kd, Ut
+    // and Qg images and the P tile; the slots' gate rows
+    static constexpr int kS = 0, kUT = kS + 32768, kI = kUT + 16384, kBuf = kI + 8192;
     static constexpr int kW = 0, kKd = 16384, kUt = 32768, kQg = 49152, kP = 65536,
                          kBufBytes = 73728;
     static constexpr int kG0 = kBuf + 2 * kBufBytes, kEnd = kG0 + 2 * 256;
@@ -316,7 +320,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             S[kk] = (init && kk < p.K && v < p.V) ? init[kk * p.V + v] : 0.f;
         state_image(Ss, S, v);  // the state entering the first chunk
         uint32_t phase = 0, pend = 0, lpar = 0;
-        if (c0 < c1 && v == 0) {
+        if (c0 < c1 && v == kPrefetcher) {
             outchain_prefetch(sm, 0, (size_t)c0 * H + h, p, &lbar[0]);
             pend = 1;
         }
@@ -327,12 +331,8 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             const size_t ch = (size_t)c * H + h;
             uint8_t *b = sm + OutChainSmem::kBuf + buf * OutChainSmem::kBufBytes;
             // the previous chunk's output is complete: its U^T image (rewritten below) and
-            // its prefetch slot (refilled now) are free
+            // its prefetch slot (refilled below) are free
             bool ok = it == 0 || mbar_wait(&obar[(it - 1) & 1], ((it - 1) >> 1) & 1, p.wait_limit);
-            if (v == 0 && c + 1 < c1 && ok) {
-                outchain_prefetch(sm, buf ^ 1, ch + H, p, &lbar[buf ^ 1]);
-                pend |= 2u >> buf;
-            }
             const bool lok = ok && mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
             fence_async_smem();  // the state image written by the previous chunk's update
             tc_fence_before();
@@ -344,6 +344,10 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             }
             pend &= ~(1u << buf);
             lpar ^= 1u << buf;
+            if (v == kPrefetcher && c + 1 < c1) {  // (while thread 0 issues the products)
+                outchain_prefetch(sm, buf ^ 1, ch + H, p, &lbar[buf ^ 1]);
+                pend |= 2u >> buf;
+            }
             const float gC =
                 expf(reinterpret_cast<const float *>(sm + OutChainSmem::kG0 + buf * 256)[C - 1]);
             if (v == 0) {
@@ -385,26 +389,23 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             }
             if (!wg_wait(&mbar, phase, p, 1, 53)) break;
             phase ^= 1;
-            // S Qg^T has read the state image before it is rewritten
-            if (!wg_wait(&sqbar, it & 1, p, 1, 52)) break;
 #pragma unroll
-            for (int c32 = 0; c32 < D; c32 += 32) {  // S <- gam_n S + U^T Kd, and its image
+            for (int c32 = 0; c32 < D; c32 += 32) {  // S <- gam_n S + U^T Kd
                 float d[32];
                 tmem_ld16(tm(tmem, 64 + c32), d);
                 tmem_ld16(tm(tmem, 64 + c32 + 16), d + 16);
                 tmem_ld_wait();
 #pragma unroll
                 for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(Ss + sw128_chunk(D, v, c32 / 8 + q)) =
-                        pack8(S + c32 + 8 * q);
             }
+            // S Qg^T has read the state image before it is rewritten
+            if (!wg_wait(&sqbar, it & 1, p, 1, 52)) break;
+            state_image(Ss, S, v);
             tc_fence_before();
             bar_sync(1, NT);
             tc_fence_after();
         }
-        if (v == 0) {  // copies still in flight after an early exit
+        if (v == kPrefetcher) {  // copies still in flight after an early exit
             for (int b2 = 0; b2 < 2; ++b2)
                 if ((pend >> b2) & 1u) mbar_wait(&lbar[b2], (lpar >> b2) & 1u, kWaitLimit);
         }
@@ -417,7 +418,6 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
     } else {
         // ---------------------------------------------------------- warpgroup 1: the output
         const int r = tid - NT;  // row v = r of O^T (warp 4 + w reaches TMEM lane quadrant w)
-        bf16 *stage = reinterpret_cast<bf16 *>(sm + OutChainSmem::kStage);
         bf16 *o = static_cast<bf16 *>(p.o);
         for (int c = c0; c < c1; ++c) {
             const int it = c - c0, buf = it & 1;
@@ -448,23 +448,22 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             }
             if (!bar_and(2, NT, ok)) break;
             if (!wg_wait(&obar[buf], (it >> 1) & 1, p, 2, 54)) break;
+            // thread r holds row v = r of O^T, column v of the chunk's output rows: stored
+            // from registers (each warp writes 64 contiguous bytes of a token's row)
+            const ChunkInfo ci = chunk_in_seq(p, n, c0, c);
+            bf16 *ov = o + ((int64_t)ci.tok0 * H + h) * p.V + r;
+            const int64_t ts = (int64_t)H * p.V;
             for (int c16 = 0; c16 < C; c16 += 16) {
                 float d[16];
                 tmem_ld16(tmq(ob, c16), d);
                 tmem_ld_wait();
+                if (r < p.V) {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) stage[(c16 + q) * D + r] = __float2bfloat16_rn(d[q]);
+                    for (int q = 0; q < 16; ++q)
+                        if (c16 + q < ci.len) ov[(c16 + q) * ts] = __float2bfloat16_rn(d[q]);
+                }
             }
-            tc_fence_before();
-            bar_sync(2, NT);  // the staged rows are complete and buffer `buf` is read
-            const ChunkInfo ci = chunk_in_seq(p, n, c0, c);
-            for (int t = r; t < C * 16; t += NT) {
-                const int i = t >> 4, j = t & 15;
-                if (i < ci.len && j * 8 < p.V)
-                    *reinterpret_cast<uint4 *>(o + ((int64_t)(ci.tok0 + i) * H + h) * p.V + j * 8) =
-                        *reinterpret_cast<const uint4 *>(stage + i * D + j * 8);
-            }
-            bar_sync(2, NT);  // the stores have read the staging rows
+            tc_fence_before();  // (buffer `buf` is read: the next barrier orders its reuse)
         }
     }
     tc_fence_before();
