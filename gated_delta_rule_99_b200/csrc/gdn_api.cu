@@ -226,6 +226,7 @@ bool encode_row_maps(Params &p, bool bwd) {
     if (p.BT <= 0) return true;  // nothing is loaded
     return encode_rows(&p.tm_q, p.q, p.BT, p.H, p.K) && encode_rows(&p.tm_k, p.k, p.BT, p.H, p.K) &&
            encode_rows(&p.tm_v, p.v, p.BT, p.H, p.V) &&
+           (bwd || !p.o || encode_rows(&p.tm_o, p.o, p.BT, p.H, p.V)) &&
            (!bwd || (encode_rows(&p.tm_do, p.do_, p.BT, p.H, p.V) &&
                      encode_rows(&p.tm_dq, p.dq, p.BT, p.H, p.K) &&
                      encode_rows(&p.tm_dk, p.dk, p.BT, p.H, p.K) &&

@@ -79,7 +79,7 @@ struct Params {
     // tensor maps of the bf16 [tokens][H][d] inputs for the tensor-core path: a box is 64
     // tokens x 64 elements of one head, written to shared memory with the operand tiles'
     // 128-byte swizzle (encoded on the host for every call)
-    CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv;
+    CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, tm_o;
 };
 
 // Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).

@@ -43,7 +43,8 @@ __global__ void __launch_bounds__(NT, 1) tc_state_fwd_kernel(Params p) {
 // ============================================================ tc_state_fwd_out
 // The forward chain with the output formed in the same CTA (the default forward
 // of sequences that run without the piece scan or value slices).
-__global__ void __launch_bounds__(kOutChainThreads, 1) tc_state_fwd_out_kernel(Params p) {
+__global__ void __launch_bounds__(kOutChainThreads, 1)
+    tc_state_fwd_out_kernel(const __grid_constant__ Params p) {
     state_fwd_out_body(p, blockIdx.x);
 }
 

@@ -140,6 +140,20 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
     return u;
 }
 
+// Writes x[0, 2 NW) as NW packed bf16 pairs (the lower element in the low half) to
+// TMEM columns [0, NW) from taddr in this thread's lane: a row of a K-major A
+// operand of the products (NW a multiple of 16).  Warp-collective.
+template <int NW>
+__device__ __forceinline__ void tmem_store_bf16(uint32_t taddr, const float *x) {
+#pragma unroll
+    for (int c = 0; c < NW; c += 16) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pack_bf16(x[2 * (c + i)], x[2 * (c + i) + 1]);
+        tmem_st16(taddr + (uint32_t)c, w);
+    }
+}
+
 // TMEM address of (lane base of this warp, column col).
 __device__ __forceinline__ uint32_t tm(uint32_t tmem, int col) {
     return tmem + ((uint32_t)((threadIdx.x >> 5) * 32) << 16) + (uint32_t)col;

@@ -225,23 +225,26 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
 
 // ============================================================ chain with the output
 // The forward pass's chain with the output formed in the same CTA.  Each chunk's
-// state image S and U^T image are in shared memory anyway, so
+// state S and U^T are on the SM anyway, so
 //   O^T = S Qg^T + U^T P^T    (M = 128 values, N = 64 tokens, K = 128 + 64)
 // over tc_prep's Qg and P images gives the chunk's output without S or U^T
-// leaving the SM.  Threads 0-127 (warpgroup 0) run the chain as chain_fwd does
-// (thread v owns row v of S; the state image is rewritten during the update).
-// Threads 128-255 (warpgroup 1) form the output: their leader issues S Qg^T once
-// the chain has issued the chunk's first product (m1bar) and U^T P^T once it has
-// issued the second (m2bar), so they run in the tensor pipe's gaps while the
-// chain's own issuing thread is not held up; then the warpgroup reads the
-// accumulator and stores the output columns it holds.  The chain waits for
-// sqbar (S Qg^T has read the state image) before rewriting the state image and
-// for obar (the chunk's output is complete) before rewriting the U^T image or
-// refilling the chunk's prefetch slot.  Every wait is bounded.
+// leaving the SM.  The state and U^T operand images live in TMEM (bf16 pairs,
+// the A operand of every product that reads them), so the products read only
+// their B operands from shared memory.  Threads 0-127 (warpgroup 0) run the
+// chain (thread v owns row v of S; thread 0 issues its products).  Threads
+// 128-255 (warpgroup 1) form the output: their leader issues S Qg^T once the
+// chain has issued the chunk's first product (m1bar) and U^T P^T once it has
+// issued the second (m2bar), into one of two TMEM buffers; then the warpgroup
+// reads the accumulator, stages it as token rows and stores them by the tensor
+// engine.  The chain waits for sqbar (S Qg^T has read the state image) before
+// rewriting the state image and for obar (the chunk's output is complete) before
+// rewriting the U^T image or refilling the chunk's prefetch slot.  Every wait is
+// bounded.
 struct OutChainSmem {
-    // the state image, U^T, the identity block, then per prefetch slot the W, Kd, Ut
-    // and Qg images and the P tile; the slots' gate rows
-    static constexpr int kS = 0, kUT = kS + 32768, kI = kUT + 16384, kBuf = kI + 8192;
+    // the identity block, two staging tiles of output rows, then per prefetch slot the
+    // W, Kd, Ut and Qg images and the P tile; the slots' gate rows (the state and U^T
+    // images are in TMEM)
+    static constexpr int kI = 0, kStage = kI + 8192, kBuf = kStage + 2 * 16384;
     static constexpr int kW = 0, kKd = 16384, kUt = 32768, kQg = 49152, kP = 65536,
                          kBufBytes = 73728;
     static constexpr int kG0 = kBuf + 2 * kBufBytes, kEnd = kG0 + 2 * 256;
@@ -301,14 +304,16 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
         tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
-    // TMEM columns: 0-63 U^T, 64-191 the state update, 256 + 64 b output buffer b
-    uint8_t *Ss = sm + OutChainSmem::kS, *UTs = sm + OutChainSmem::kUT;
+    // TMEM columns: 0-63 U^T, 64-191 the state update, 192-255 the state image (bf16
+    // pairs: the A operand of U^T and S Qg^T), 256 + 64 b output buffer b, 384-415 the
+    // U^T image (the A operand of the update and U^T P^T)
+    constexpr uint32_t cSI = 192, cUI = 384;
     if (tid < NT) identity_tile(sm + OutChainSmem::kI);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = tslot, sb = smem_u32(Ss), utb = smem_u32(UTs);
+    const uint32_t tmem = tslot;
     const uint32_t id1 = idesc_bf16(128, 64, 0, 0);
     if (tid < NT) {
         // ---------------------------------------------------------- warpgroup 0: the chain
@@ -318,7 +323,8 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
 #pragma unroll
         for (int kk = 0; kk < D; ++kk)
             S[kk] = (init && kk < p.K && v < p.V) ? init[kk * p.V + v] : 0.f;
-        state_image(Ss, S, v);  // the state entering the first chunk
+        tmem_store_bf16<64>(tm(tmem, cSI), S);  // the state entering the first chunk
+        tmem_st_wait();
         uint32_t phase = 0, pend = 0, lpar = 0;
         if (c0 < c1 && v == kPrefetcher) {
             outchain_prefetch(sm, 0, (size_t)c0 * H + h, p, &lbar[0]);
@@ -334,8 +340,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             // its prefetch slot (refilled below) are free
             bool ok = it == 0 || mbar_wait(&obar[(it - 1) & 1], ((it - 1) >> 1) & 1, p.wait_limit);
             const bool lok = ok && mbar_wait(&lbar[buf], (lpar >> buf) & 1u, p.wait_limit);
-            fence_async_smem();  // the state image written by the previous chunk's update
-            tc_fence_before();
+            tc_fence_before();  // (the state image written by the previous chunk's update)
             const bool all = bar_and(1, NT, lok);
             tc_fence_after();
             if (!all) {
@@ -355,7 +360,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
                                ub = smem_u32(b + OutChainSmem::kUt);
 #pragma unroll
                 for (int s = 0; s < D / 16; ++s)  // U^T = S (-W)^T + Ut^T I
-                    mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
+                    mma_bf16_ta(tmem, tmem + cSI + 8 * s, desc_kmajor(wb, C, s), id1, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
                     mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(ib, C, s), idu, 1);
@@ -365,17 +370,14 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             if (!wg_wait(&mbar, phase, p, 1, 51)) break;
             phase ^= 1;
 #pragma unroll
-            for (int c32 = 0; c32 < C; c32 += 32) {  // U^T as an operand tile (row v)
+            for (int c32 = 0; c32 < C; c32 += 32) {  // U^T as an operand (row v)
                 float d[32];
                 tmem_ld16(tm(tmem, c32), d);
                 tmem_ld16(tm(tmem, c32 + 16), d + 16);
                 tmem_ld_wait();
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) =
-                        pack8(d + 8 * q);
+                tmem_store_bf16<16>(tm(tmem, cUI + c32 / 2), d);
             }
-            fence_async_smem();
+            tmem_st_wait();
             tc_fence_before();
             bar_sync(1, NT);
             tc_fence_after();
@@ -383,7 +385,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
                 const uint32_t kb = smem_u32(b + OutChainSmem::kKd);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)  // S <- gam_n S + U^T Kd
-                    mma_bf16(tmem + 64, desc_kmajor(utb, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
+                    mma_bf16_ta(tmem + 64, tmem + cUI + 8 * s, desc_mnmajor(kb, C, s), id2, s > 0);
                 mma_commit(&mbar);
                 mbar_arrive(&m2bar);  // the U^T image is ready for U^T P^T
             }
@@ -400,7 +402,8 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             }
             // S Qg^T has read the state image before it is rewritten
             if (!wg_wait(&sqbar, it & 1, p, 1, 52)) break;
-            state_image(Ss, S, v);
+            tmem_store_bf16<64>(tm(tmem, cSI), S);
+            tmem_st_wait();
             tc_fence_before();
             bar_sync(1, NT);
             tc_fence_after();
@@ -431,7 +434,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
                     const uint32_t qg = smem_u32(b + OutChainSmem::kQg);
 #pragma unroll
                     for (int s = 0; s < D / 16; ++s)
-                        mma_bf16(ob, desc_kmajor(sb, D, s), desc_kmajor(qg, C, s), id1, s > 0);
+                        mma_bf16_ta(ob, tmem + cSI + 8 * s, desc_kmajor(qg, C, s), id1, s > 0);
                     mma_commit(&sqbar);
                     ok = mbar_wait(&m2bar, it & 1, p.wait_limit);
                 }
@@ -440,31 +443,52 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
                     const uint32_t pb = smem_u32(b + OutChainSmem::kP);
 #pragma unroll
                     for (int s = 0; s < C / 16; ++s)
-                        mma_bf16(ob, desc_kmajor(utb, D, s), desc_kmajor(pb, C, s), id1, 1);
+                        mma_bf16_ta(ob, tmem + cUI + 8 * s, desc_kmajor(pb, C, s), id1, 1);
                     mma_commit(&obar[buf]);
                 } else {
                     record_timeout(p, 55);
                 }
             }
+            // staging tile `buf` held chunk it - 2's rows: their store has read it
+            if (r == 0 && it >= 2) bulk_wait_read_n<1>();
             if (!bar_and(2, NT, ok)) break;
             if (!wg_wait(&obar[buf], (it >> 1) & 1, p, 2, 54)) break;
-            // thread r holds row v = r of O^T, column v of the chunk's output rows: stored
-            // from registers (each warp writes 64 contiguous bytes of a token's row)
-            const ChunkInfo ci = chunk_in_seq(p, n, c0, c);
-            bf16 *ov = o + ((int64_t)ci.tok0 * H + h) * p.V + r;
-            const int64_t ts = (int64_t)H * p.V;
+            // thread r holds row v = r of O^T, column v of the chunk's output rows: staged
+            // as token rows, then stored by the tensor engine (a full chunk) or by 16-byte
+            // stores of the warpgroup (rows past the chunk's end are not written)
+            uint8_t *stg = sm + OutChainSmem::kStage + buf * 16384;
             for (int c16 = 0; c16 < C; c16 += 16) {
                 float d[16];
                 tmem_ld16(tmq(ob, c16), d);
                 tmem_ld_wait();
-                if (r < p.V) {
+                uint8_t *c0p = stg + (r >> 6) * C * 128 + (r & 7) * 2;
+                const int cp = (r & 63) >> 3;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        if (c16 + q < ci.len) ov[(c16 + q) * ts] = __float2bfloat16_rn(d[q]);
-                }
+                for (int q = 0; q < 16; ++q)  // row c16 + q, whose swizzle term is q % 8
+                    *reinterpret_cast<bf16 *>(c0p + (c16 + q) * 128 + ((cp ^ (q & 7)) << 4)) =
+                        __float2bfloat16_rn(d[q]);
             }
+            fence_async_smem();
             tc_fence_before();  // (buffer `buf` is read: the next barrier orders its reuse)
+            bar_sync(2, NT);
+            const ChunkInfo ci = chunk_in_seq(p, n, c0, c);
+            if (ci.len == C) {
+                if (r == 0) {
+                    tma_store_3d(&p.tm_o, 0, h, (int)ci.tok0, smem_u32(stg));
+                    if (p.V == D) tma_store_3d(&p.tm_o, 64, h, (int)ci.tok0, smem_u32(stg) + C * 128);
+                    bulk_commit();
+                }
+            } else {
+                for (int t = r; t < C * 16; t += NT) {
+                    const int i = t >> 4, j = t & 15;
+                    if (i < ci.len && j * 8 < p.V)
+                        *reinterpret_cast<uint4 *>(o + ((int64_t)(ci.tok0 + i) * H + h) * p.V + j * 8) =
+                            *reinterpret_cast<const uint4 *>(stg + sw128_chunk(C, i, j));
+                }
+                bar_sync(2, NT);  // the staging rows are read before the tile is rewritten
+            }
         }
+        if (r == 0) bulk_wait_all();  // (the stores read the staging tiles)
     }
     tc_fence_before();
     __syncthreads();

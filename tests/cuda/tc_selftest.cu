@@ -14,6 +14,7 @@ struct Args {
     float *D;
     int M, N, Kd, a_mn, b_mn, swap;
     int *err;
+    int a_tmem;  // A from TMEM (K-major, packed bf16 pairs) instead of shared memory
 };
 
 __device__ __forceinline__ uint64_t desc_mn_variant(uint32_t base, int R, int s, int swap) {
@@ -45,21 +46,44 @@ __global__ void __launch_bounds__(128, 1) mma_selftest(Args a) {
         fence_mbar_init();
     }
     if (tid < 32) {
-        tmem_alloc(&tslot, 256);
+        tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
+    constexpr uint32_t kAcol = 256;  // A's columns when it is taken from TMEM
+    if (a.a_tmem) {  // thread tid writes row m = tid of A into its lane, bf16 pairs
+        const int w = tid / 32;
+        for (int c = 0; c < a.Kd / 2; c += 16) {
+            uint32_t r[16];
+            for (int i = 0; i < 16; ++i) {
+                const int k = 2 * (c + i);
+                const __nv_bfloat16 lo = tid < a.M ? a.A[(size_t)tid * a.Kd + k] : __float2bfloat16(0.f);
+                const __nv_bfloat16 hi = tid < a.M ? a.A[(size_t)tid * a.Kd + k + 1] : __float2bfloat16(0.f);
+                r[i] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+            }
+            tmem_st16(tmem + ((uint32_t)(w * 32) << 16) + kAcol + (uint32_t)c, r);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
     if (tid == 0) {
         const uint32_t idesc = idesc_bf16(a.M, a.N, a.a_mn, a.b_mn);
         const uint32_t sa = smem_u32(As), sb = smem_u32(Bs);
         for (int s = 0; s < a.Kd / 16; ++s) {
-            const uint64_t da = a.a_mn ? desc_mn_variant(sa, RA, s, a.swap) : desc_kmajor(sa, RA, s);
             const uint64_t db =
                 a.b_mn ? desc_mn_variant(sb, a.Kd, s, a.swap) : desc_kmajor(sb, a.N, s);
-            mma_bf16(tmem, da, db, idesc, s > 0 ? 1u : 0u);
+            if (a.a_tmem) {
+                mma_bf16_ta(tmem, tmem + kAcol + 8u * s, db, idesc, s > 0 ? 1u : 0u);
+            } else {
+                const uint64_t da =
+                    a.a_mn ? desc_mn_variant(sa, RA, s, a.swap) : desc_kmajor(sa, RA, s);
+                mma_bf16(tmem, da, db, idesc, s > 0 ? 1u : 0u);
+            }
         }
         mma_commit(&mbar);
     }
@@ -75,15 +99,16 @@ __global__ void __launch_bounds__(128, 1) mma_selftest(Args a) {
     }
     tc_fence_before();
     __syncthreads();
-    if (tid < 32) tmem_dealloc(tmem, 256);
+    if (tid < 32) tmem_dealloc(tmem, 512);
 }
 
 extern "C" int tc_selftest_run(const void *A, const void *B, float *D, int M, int N, int Kd,
-                               int a_mn, int b_mn, int swap, int *err_dev) {
+                               int a_mn, int b_mn, int swap, int *err_dev, int a_tmem) {
     if (M != 64 && M != 128) return -1;
     if (N < 16 || N > 256 || N % 16 || Kd < 16 || Kd > 128 || Kd % 16) return -1;
+    if (a_tmem && (M != 128 || a_mn || Kd % 32)) return -1;
     Args a{(const __nv_bfloat16 *)A, (const __nv_bfloat16 *)B, D, M, N, Kd, a_mn, b_mn, swap,
-           err_dev};
+           err_dev, a_tmem};
     const int smem = 65536 * 2 + 1024;
     cudaFuncSetAttribute(mma_selftest, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     mma_selftest<<<1, 128, smem>>>(a);

@@ -25,16 +25,17 @@ def _lib():
                                "-I", os.path.dirname(hdr), "-o", SO, SRC])
     L = ctypes.CDLL(SO)
     L.tc_selftest_run.restype = ctypes.c_int
-    L.tc_selftest_run.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [ctypes.c_void_p]
+    L.tc_selftest_run.argtypes = ([ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [ctypes.c_void_p] +
+                                  [ctypes.c_int])
     return L
 
 
-def run(A, B, M, N, Kd, a_mn, b_mn, swap=0):
+def run(A, B, M, N, Kd, a_mn, b_mn, swap=0, a_tmem=0):
     L = _lib()
     D = torch.full((128, N), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = L.tc_selftest_run(A.data_ptr(), B.data_ptr(), D.data_ptr(), M, N, Kd, a_mn, b_mn, swap,
-                           err.data_ptr())
+                           err.data_ptr(), a_tmem)
     assert rc == 0, rc
     assert int(err.item()) == 0, "mbarrier wait timed out"
     return D.cpu()
@@ -58,6 +59,19 @@ def test_mma_m128(M, N, Kd, a_mn, b_mn):
     print("mma M=%d N=%d K=%d a_mn=%d b_mn=%d: err by lbo/sbo variant %s" % (M, N, Kd, a_mn, b_mn,
                                                                             results))
     assert results[0] < 1e-3, results
+
+
+@pytest.mark.parametrize("N,Kd,b_mn", [(64, 128, 0), (128, 64, 1), (64, 64, 0), (128, 128, 1)])
+def test_mma_a_from_tmem(N, Kd, b_mn):
+    """A (128 x K, K-major) taken from TMEM as packed bf16 pairs, B from shared memory."""
+    g = torch.Generator().manual_seed(900 + N + Kd + b_mn)
+    A = torch.randn(128, Kd, generator=g).to(torch.bfloat16)
+    B = torch.randn(N, Kd, generator=g).to(torch.bfloat16)
+    ref = A.float() @ B.float().T
+    D = run(A.cuda(), B.cuda(), 128, N, Kd, 0, b_mn, 0, a_tmem=1)
+    err = float((D - ref).abs().max() / ref.abs().max())
+    print("mma with A in TMEM, N=%d K=%d b_mn=%d: err %.2e" % (N, Kd, b_mn, err))
+    assert err < 1e-3, err
 
 
 def test_tmem_layout_m64():
