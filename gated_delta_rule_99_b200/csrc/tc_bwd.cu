@@ -122,14 +122,20 @@ __device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
         fence_mbar_init();
     }
     if (v < 32) {
-        tmem_alloc(&tslot, 256);
+        tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
-    state_image(sm + SbwdSmem::kdS0, S, v);  // dS leaving the last chunk
+    if (a.snapshots) state_image(sm + SbwdSmem::kdS0, S, v);  // dS leaving the last chunk
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
+    // TMEM columns: 0-63 dU^T, 64-191 the dS update, 256-319 the dS image and 320-351
+    // the dU^T image (bf16 pairs: the A operands of the products that read them; the
+    // shared-memory images are kept for the snapshots only)
+    constexpr uint32_t cSI = 256, cUI = 320;
+    tmem_store_bf16<64>(tm(tmem, cSI), S);
+    tmem_st_wait();
     const int c0 = a.c0, c1 = a.c1;
     const bool local = !a.zero_local;
     uint32_t phase = 0;
@@ -191,7 +197,7 @@ __device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
             // + dS Kd^T: M = 128 (v), N = 64 tokens, K = 128 keys
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(kb, C, s), id1, local || s > 0);
+                mma_bf16_ta(tmem, tmem + cSI + 8 * s, desc_kmajor(kb, C, s), id1, local || s > 0);
             mma_commit(&mbar);
         }
         if (v == 0 && a.snapshots) {
@@ -209,17 +215,22 @@ __device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
             tmem_ld16(tm(tmem, c32), d);
             tmem_ld16(tm(tmem, c32 + 16), d + 16);
             tmem_ld_wait();
+            tmem_store_bf16<16>(tm(tmem, cUI + c32 / 2), d);
+            if (a.snapshots) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(dUs + sw128_chunk(D, v, c32 / 8 + q)) =
+                        pack8(d + 8 * q);
+            }
         }
+        tmem_st_wait();
         operands_ready();
         if (v == 0) {  // + dU^T (-W): M = 128 (v), N = 128 keys, K = 64 tokens (W image negated)
-            const uint32_t ub = smem_u32(dUs), wb = smem_u32(b + SbwdSmem::kW);
+            const uint32_t wb = smem_u32(b + SbwdSmem::kW);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(wb, C, s), idy,
-                         local || s > 0);
+                mma_bf16_ta(tmem + 64, tmem + cUI + 8 * s, desc_mnmajor(wb, C, s), idy,
+                            local || s > 0);
             mma_commit(&mbar);
         }
         if (v == 0 && a.snapshots) {
@@ -236,11 +247,15 @@ __device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
+            tmem_store_bf16<16>(tm(tmem, cSI + c32 / 2), S + c32);  // the next chunk's dS image
+            if (a.snapshots) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)  // the next chunk's dS image
-                *reinterpret_cast<uint4 *>(dSn + sw128_chunk(D, v, c32 / 8 + q)) =
-                    pack8(S + c32 + 8 * q);
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(dSn + sw128_chunk(D, v, c32 / 8 + q)) =
+                        pack8(S + c32 + 8 * q);
+            }
         }
+        tmem_st_wait();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -260,7 +275,7 @@ __device__ __forceinline__ void chain_bwd(const Params &p, const ChainBwd &a) {
     }
     tc_fence_before();
     __syncthreads();
-    if (v < 32) tmem_dealloc(tmem, 256);
+    if (v < 32) tmem_dealloc(tmem, 512);
 }
 
 // Body of the reverse state pass for CTA `blk` (sequence blk / H, head blk % H):

@@ -45,6 +45,13 @@ __device__ __forceinline__ uint32_t qk_src(int off, int row0) {
     return (uint32_t)((off >> 13) * 16384 + row0 * 128 + (off & 8191));
 }
 
+// Byte offset, in the [Q; K] tile of 128 rows, of chunk j (0-15) of row i of a 64-row
+// tile image staged in rows [row0, row0 + 64): 64-column block j / 8 of the image
+// lies in the tile's block j / 8, so each block leaves by one contiguous copy.
+__device__ __forceinline__ uint32_t qk_stage(int row0, int j, int i) {
+    return (uint32_t)((j >> 3) * 2 * C * 128 + (row0 + i) * 128 + (((j & 7) ^ (i & 7)) << 4));
+}
+
 // Body of the prep step for CTA `ch` (chunk ch / H, head ch % H).
 __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     extern __shared__ uint8_t smem_raw[];
@@ -328,25 +335,32 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         ok = cta_wait(&mbar, phase, p, 2);
         phase ^= 1;
         if (ok) {
+            // W, stored negated (both chains subtract W products), is staged in the K rows'
+            // place (the product has read them) and leaves by two bulk copies
             const int i = m64_row();
-            uint8_t *Wimg = static_cast<uint8_t *>(p.tW) + (size_t)ch * kImg64;
             for (int c0 = 0; c0 < D; c0 += 32) {
                 float w[32];
                 tmem_ld16(tm(tmem, c0), w);
                 tmem_ld16(tm(tmem, c0 + 16), w + 16);
                 tmem_ld_wait();
-                if (i >= 0) {  // stored negated: both chains subtract W products
+                if (i >= 0) {
 #pragma unroll
                     for (int q = 0; q < 32; ++q) w[q] = -w[q];
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4 *>(Wimg + sw128_chunk(C, i, c0 / 8 + q)) =
-                            pack8(w + 8 * q);
+                        *reinterpret_cast<uint4 *>(QK + qk_stage(C, c0 / 8 + q, i)) = pack8(w + 8 * q);
                 }
             }
+            fence_async_smem();
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
+            if (tid == 0) {
+                uint8_t *Wimg = static_cast<uint8_t *>(p.tW) + (size_t)ch * kImg64;
+                bulk_store(Wimg, smem_u32(QK) + C * 128, (uint32_t)kImg64 / 2);
+                bulk_store(Wimg + kImg64 / 2, smem_u32(QK) + 3 * C * 128, (uint32_t)kImg64 / 2);
+                bulk_commit();
+            }
             // the V rows (loaded into the Q rows' place after the first product)
             ok = copies_arrived(&vbar, p, 34);
             v_pending = false;
@@ -365,9 +379,9 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     }
     if (v_pending && tid == 0) mbar_wait(&vbar, 0, kWaitLimit);  // leave no copy in flight
     if (ok) {  // Ut as a 64 x 128 tile image (rows = tokens): an operand of the chains'
-               // first product, whose 64-column blocks are the two halves of the values
+               // first product, whose 64-column blocks are the two halves of the values;
+               // staged in the V rows' place (the product has read them), two bulk copies
         const int i = m64_row();
-        uint8_t *Ut = static_cast<uint8_t *>(p.tUt) + (size_t)ch * kImg64;
         for (int c0 = 0; c0 < D; c0 += 32) {
             float u[32];
             tmem_ld16(tm(tmem, c0), u);
@@ -376,12 +390,20 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
             if (i >= 0) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(Ut + sw128_chunk(C, i, c0 / 8 + q)) = pack8(u + 8 * q);
+                    *reinterpret_cast<uint4 *>(QK + qk_stage(0, c0 / 8 + q, i)) = pack8(u + 8 * q);
             }
         }
+        fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
+    if (ok && tid == 0) {
+        uint8_t *Ut = static_cast<uint8_t *>(p.tUt) + (size_t)ch * kImg64;
+        bulk_store(Ut, smem_u32(QK), (uint32_t)kImg64 / 2);
+        bulk_store(Ut + kImg64 / 2, smem_u32(QK) + 2 * C * 128, (uint32_t)kImg64 / 2);
+        bulk_commit();
+    }
+    if (tid == 0) bulk_wait_read();  // (the staged rows are read before the CTA exits)
     if (tid < 32) tmem_dealloc(tmem, 128);
 }
 

@@ -99,16 +99,22 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         fence_mbar_init();
     }
     if (v < 32) {
-        tmem_alloc(&tslot, 256);
+        tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
     const bool with_ut = !a.zero_ut;
     identity_tile(sm + StateSmem::kI);
-    state_image(sm + StateSmem::kS0, S, v);  // the state entering the first chunk
+    if (a.snapshots) state_image(sm + StateSmem::kS0, S, v);  // the state entering the first chunk
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
+    // TMEM columns: 0-63 U^T, 64-191 the state update, 256-319 the state image and
+    // 320-351 the U^T image (bf16 pairs: the A operands of the products that read them;
+    // the shared-memory images are kept for the snapshots only)
+    constexpr uint32_t cSI = 256, cUI = 320;
+    tmem_store_bf16<64>(tm(tmem, cSI), S);
+    tmem_st_wait();
     const int c0 = a.c0, c1 = a.c1;
     uint32_t phase = 0;
     // per buffer b (bit b): a copy in flight, and the parity of its next completion
@@ -143,11 +149,11 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         const float gC =
             expf(reinterpret_cast<const float *>(sm + StateSmem::kG0 + buf * 256)[C - 1]);
         if (v == 0) {  // U^T = S (-W)^T + Ut^T I  (the W image is stored negated)
-            const uint32_t sb = smem_u32(Ss), wb = smem_u32(sm + StateSmem::kW0 + buf * 16384),
+            const uint32_t wb = smem_u32(sm + StateSmem::kW0 + buf * 16384),
                            ub = smem_u32(sm + StateSmem::kUt0 + buf * 16384);
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tmem, desc_kmajor(sb, D, s), desc_kmajor(wb, C, s), id1, s > 0);
+                mma_bf16_ta(tmem, tmem + cSI + 8 * s, desc_kmajor(wb, C, s), id1, s > 0);
             if (with_ut) {
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
@@ -165,21 +171,26 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
         if (!cta_wait(&mbar, phase, p, a.where)) break;
         phase ^= 1;
 #pragma unroll
-        for (int c32 = 0; c32 < C; c32 += 32) {  // U^T as an operand tile (row v)
+        for (int c32 = 0; c32 < C; c32 += 32) {  // U^T as an operand (row v)
             float d[32];
             tmem_ld16(tm(tmem, c32), d);
             tmem_ld16(tm(tmem, c32 + 16), d + 16);
             tmem_ld_wait();
+            tmem_store_bf16<16>(tm(tmem, cUI + c32 / 2), d);
+            if (a.snapshots) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) = pack8(d + 8 * q);
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(UTs + sw128_chunk(D, v, c32 / 8 + q)) =
+                        pack8(d + 8 * q);
+            }
         }
+        tmem_st_wait();
         operands_ready();
         if (v == 0) {
-            const uint32_t ub = smem_u32(UTs), kb = smem_u32(sm + StateSmem::kKd0 + buf * 16384);
+            const uint32_t kb = smem_u32(sm + StateSmem::kKd0 + buf * 16384);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tmem + 64, desc_kmajor(ub, D, s), desc_mnmajor(kb, C, s), id2, s > 0);
+                mma_bf16_ta(tmem + 64, tmem + cUI + 8 * s, desc_mnmajor(kb, C, s), id2, s > 0);
             mma_commit(&mbar);
         }
         if (v == kPrefetcher && a.snapshots) {
@@ -196,11 +207,15 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
+            tmem_store_bf16<16>(tm(tmem, cSI + c32 / 2), S + c32);
+            if (a.snapshots) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(Sn + sw128_chunk(D, v, c32 / 8 + q)) =
-                    pack8(S + c32 + 8 * q);
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(Sn + sw128_chunk(D, v, c32 / 8 + q)) =
+                        pack8(S + c32 + 8 * q);
+            }
         }
+        tmem_st_wait();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -220,7 +235,7 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
     }
     tc_fence_before();
     __syncthreads();
-    if (v < 32) tmem_dealloc(tmem, 256);
+    if (v < 32) tmem_dealloc(tmem, 512);
 }
 
 // ============================================================ chain with the output
