@@ -72,7 +72,9 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
     const int tid = threadIdx.x;
     const uint32_t qkb = smem_u32(QK), kb = qkb + C * 128;  // K rows: 64-127 of the tile
 
-    if (tid == 0) {  // Q and K rows by the tensor engine (V comes once Q is consumed)
+    // warp 3 sets up (the mbarriers, the Q and K copies, TMEM) while warps 0-1 load the
+    // gates, the first global reads of the CTA
+    if (tid == 3 * 32) {  // Q and K rows by the tensor engine (V comes once Q is consumed)
         mbar_init(&mbar, 1);
         mbar_init(&lbar, 1);
         mbar_init(&vbar, 1);
@@ -84,7 +86,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         load_rows_tma(QK, D, 0, &p.tm_q, ci.tok0, h, p.K, &lbar);
         load_rows_tma(QK, D, C, &p.tm_k, ci.tok0, h, p.K, &lbar);
     }
-    if (tid < 32) {
+    if (tid >= 3 * 32) {
         tmem_alloc(&tslot, 128);
         tmem_relinquish();
     }
@@ -404,7 +406,7 @@ __device__ __forceinline__ void prep_body(const Params &p, int ch, int want_A) {
         bulk_commit();
     }
     if (tid == 0) bulk_wait_read();  // (the staged rows are read before the CTA exits)
-    if (tid < 32) tmem_dealloc(tmem, 128);
+    if (tid >= 3 * 32) tmem_dealloc(tmem, 128);
 }
 
 }  // namespace tc

@@ -251,10 +251,10 @@ __device__ __forceinline__ void chain_fwd(const Params &p, const ChainFwd &a) {
 // chain has issued the chunk's first product (m1bar) and U^T P^T once it has
 // issued the second (m2bar), into one of two TMEM buffers; then the warpgroup
 // reads the accumulator, stages it as token rows and stores them by the tensor
-// engine.  The chain waits for sqbar (S Qg^T has read the state image) before
-// rewriting the state image and for obar (the chunk's output is complete) before
-// rewriting the U^T image or refilling the chunk's prefetch slot.  Every wait is
-// bounded.
+// engine.  The state image is double-buffered, so the chain writes the next
+// chunk's while S Qg^T may still read the current one; it waits for obar (the
+// previous chunk's output is complete) before rewriting the U^T image, the other
+// state image or the previous chunk's prefetch slot.  Every wait is bounded.
 struct OutChainSmem {
     // the identity block, two staging tiles of output rows, then per prefetch slot the
     // W, Kd, Ut and Qg images and the P tile; the slots' gate rows (the state and U^T
@@ -299,7 +299,7 @@ __device__ __forceinline__ bool wg_wait(uint64_t *bar, uint32_t parity, const Pa
 __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1k(smem_raw);
-    __shared__ uint64_t mbar, m1bar, m2bar, sqbar, lbar[2], obar[2];
+    __shared__ uint64_t mbar, m1bar, m2bar, lbar[2], obar[2];
     __shared__ uint32_t tslot;
     if (p.hdr->status) return;
     const int H = p.H, n = blk / H, h = blk % H, tid = threadIdx.x;
@@ -308,7 +308,6 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
         mbar_init(&mbar, 1);
         mbar_init(&m1bar, 1);
         mbar_init(&m2bar, 1);
-        mbar_init(&sqbar, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&lbar[b], 1);
             mbar_init(&obar[b], 1);
@@ -319,10 +318,12 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
         tmem_alloc(&tslot, 512);
         tmem_relinquish();
     }
-    // TMEM columns: 0-63 U^T, 64-191 the state update, 192-255 the state image (bf16
-    // pairs: the A operand of U^T and S Qg^T), 256 + 64 b output buffer b, 384-415 the
-    // U^T image (the A operand of the update and U^T P^T)
-    constexpr uint32_t cSI = 192, cUI = 384;
+    // TMEM columns: 0-63 U^T, 64-191 the state update, 256 + 64 b output buffer b, 384-415
+    // the U^T image (the A operand of the update and U^T P^T), and two state images (bf16
+    // pairs: the A operand of U^T and S Qg^T) at 192 and 448, the one of chunk it at
+    // sI(it): the update writes the next chunk's into the other
+    constexpr uint32_t cUI = 384;
+    auto sI = [](int it) -> uint32_t { return (it & 1) ? 448u : 192u; };
     if (tid < NT) identity_tile(sm + OutChainSmem::kI);
     fence_async_smem();
     tc_fence_before();
@@ -338,7 +339,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
 #pragma unroll
         for (int kk = 0; kk < D; ++kk)
             S[kk] = (init && kk < p.K && v < p.V) ? init[kk * p.V + v] : 0.f;
-        tmem_store_bf16<64>(tm(tmem, cSI), S);  // the state entering the first chunk
+        tmem_store_bf16<64>(tm(tmem, sI(0)), S);  // the state entering the first chunk
         tmem_st_wait();
         uint32_t phase = 0, pend = 0, lpar = 0;
         if (c0 < c1 && v == kPrefetcher) {
@@ -375,7 +376,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
                                ub = smem_u32(b + OutChainSmem::kUt);
 #pragma unroll
                 for (int s = 0; s < D / 16; ++s)  // U^T = S (-W)^T + Ut^T I
-                    mma_bf16_ta(tmem, tmem + cSI + 8 * s, desc_kmajor(wb, C, s), id1, s > 0);
+                    mma_bf16_ta(tmem, tmem + sI(it) + 8 * s, desc_kmajor(wb, C, s), id1, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
                     mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(ib, C, s), idu, 1);
@@ -415,9 +416,9 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
 #pragma unroll
                 for (int q = 0; q < 32; ++q) S[c32 + q] = fmaf(gC, S[c32 + q], d[q]);
             }
-            // S Qg^T has read the state image before it is rewritten
-            if (!wg_wait(&sqbar, it & 1, p, 1, 52)) break;
-            tmem_store_bf16<64>(tm(tmem, cSI), S);
+            // the next chunk's image: its buffer was last read by the previous chunk's
+            // S Qg^T, complete with that chunk's output (obar, waited for at this step's start)
+            tmem_store_bf16<64>(tm(tmem, sI(it + 1)), S);
             tmem_st_wait();
             tc_fence_before();
             bar_sync(1, NT);
@@ -449,8 +450,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
                     const uint32_t qg = smem_u32(b + OutChainSmem::kQg);
 #pragma unroll
                     for (int s = 0; s < D / 16; ++s)
-                        mma_bf16_ta(ob, tmem + cSI + 8 * s, desc_kmajor(qg, C, s), id1, s > 0);
-                    mma_commit(&sqbar);
+                        mma_bf16_ta(ob, tmem + sI(it) + 8 * s, desc_kmajor(qg, C, s), id1, s > 0);
                     ok = mbar_wait(&m2bar, it & 1, p.wait_limit);
                 }
                 if (ok) {
