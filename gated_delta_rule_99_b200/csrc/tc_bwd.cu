@@ -822,9 +822,12 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             dB[tid] = (w[0] + w[64]) + (w[128] + w[192]);
         }
         // meanwhile, each thread waiting for what it reads itself (no barrier waits on the
-        // issuing warp); the CTA decides on a failed wait at the barrier after them
+        // issuing warp); the CTA decides on a failed wait at the barrier after them.  The
+        // P . dP phase (rows on lanes 0-63) and the dL phase (lanes 64-127) run side by side
         bool fine = true;
         if (w4 < 2) fine = thread_wait(&mbar, phase, p.wait_limit);  // Q K^T and dP
+        else  // K K^T, and -dL
+            fine = thread_wait(&mbar, phase, p.wait_limit) && thread_wait(&mbar_z, it & 1, p.wait_limit);
         phase ^= 1;
         if (w4 < 2) {  // row i = r of P and dP: P . dP (row and column partials), dPG = dP . Gam
             float pq[CW];
@@ -847,21 +850,7 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             for (int q = 0; q < CW / 8; ++q)
                 *reinterpret_cast<uint4 *>(DPG + sw128_chunk(C, r, cb / 8 + q)) = pack8(d + 8 * q);
             warp_colsum(pq, wsum + 768, w4, cb, l);
-        }
-        ok = __syncthreads_and(fine);
-        if (!ok) {
-            if (tid == 0) record_timeout(p, 21);
-            break;
-        }
-        ok = cta_wait(&mbar_z, it & 1, p, 22);  // -dL and Zp
-        if (!ok) break;
-        if (more) {  // A of the next unit (its last product is done)
-            if (tid == 0) grads_fetch(p, sm, next, ci, kGrpA, 0, lbar);
-            pend |= kGrpA;
-        }
-        if (w4 >= 2) fine = thread_wait(&mbar, phase ^ 1, p.wait_limit);  // K K^T (its phase
-                                                                           // is still the last)
-        if (w4 >= 2) {  // row i = r - 64: dL (strictly lower), Gam . K K^T; dLG = diag(b) dL . Gam
+        } else {  // row i = r - 64: dL (strictly lower), Gam . K K^T; dLG = diag(b) dL . Gam
             const int i = r - C;
             float kk[CW];
             tmem_ld16(tmq(tmem, cQK + cb), kk);
@@ -885,7 +874,16 @@ __global__ void __launch_bounds__(NG, 1) tc_grads_kernel(const __grid_constant__
             dbl2[wg * 64 + i] = dbl;
             warp_colsum(kk, wsum + 768, w4, cb, l);
         }
-        fine = thread_wait(&mbar_c, it & 1, p.wait_limit) && fine;  // X1, X2
+        ok = __syncthreads_and(fine);
+        if (!ok) {
+            if (tid == 0) record_timeout(p, 21);
+            break;
+        }
+        if (more) {  // A of the next unit (its last product is done)
+            if (tid == 0) grads_fetch(p, sm, next, ci, kGrpA, 0, lbar);
+            pend |= kGrpA;
+        }
+        fine = thread_wait(&mbar_c, it & 1, p.wait_limit);  // X1, X2
         {  // partial q' . X1 (thread kk); a column reader costs 8 registers: built where used
             const ColSw qcol(QK, D, r);
             ldcw(tmem, cX1 + cb, d);

@@ -348,6 +348,7 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
         }
         const uint32_t idu = idesc_bf16(128, 64, 1, 0), id2 = idesc_bf16(128, 128, 0, 1),
                        ib = smem_u32(sm + OutChainSmem::kI);
+        bool ut_in = false;  // thread 0: the chunk's Ut^T I is already in the U^T accumulator
         for (int c = c0; c < c1; ++c) {
             const int it = c - c0, buf = it & 1;
             const size_t ch = (size_t)c * H + h;
@@ -371,15 +372,17 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
             }
             const float gC =
                 expf(reinterpret_cast<const float *>(sm + OutChainSmem::kG0 + buf * 256)[C - 1]);
-            if (v == 0) {
+            if (v == 0) {  // U^T = Ut^T I + S (-W)^T  (the W image is stored negated)
                 const uint32_t wb = smem_u32(b + OutChainSmem::kW),
                                ub = smem_u32(b + OutChainSmem::kUt);
+                if (!ut_in) {
 #pragma unroll
-                for (int s = 0; s < D / 16; ++s)  // U^T = S (-W)^T + Ut^T I
-                    mma_bf16_ta(tmem, tmem + sI(it) + 8 * s, desc_kmajor(wb, C, s), id1, s > 0);
+                    for (int s = 0; s < C / 16; ++s)
+                        mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(ib, C, s), idu, s > 0);
+                }
 #pragma unroll
-                for (int s = 0; s < C / 16; ++s)
-                    mma_bf16(tmem, desc_mnmajor(ub, C, s), desc_kmajor(ib, C, s), idu, 1);
+                for (int s = 0; s < D / 16; ++s)
+                    mma_bf16_ta(tmem, tmem + sI(it) + 8 * s, desc_kmajor(wb, C, s), id1, 1);
                 mma_commit(&mbar);
                 mbar_arrive(&m1bar);  // the state image and the slot are ready for S Qg^T
             }
@@ -404,6 +407,17 @@ __device__ __forceinline__ void state_fwd_out_body(const Params &p, int blk) {
                     mma_bf16_ta(tmem + 64, tmem + cUI + 8 * s, desc_mnmajor(kb, C, s), id2, s > 0);
                 mma_commit(&mbar);
                 mbar_arrive(&m2bar);  // the U^T image is ready for U^T P^T
+                // the next chunk's Ut^T I into the (read) U^T accumulator while the state
+                // is updated, if that chunk's copies have landed already (no wait here)
+                ut_in = c + 1 < c1 && mbar_test(&lbar[buf ^ 1], (lpar >> (buf ^ 1)) & 1u);
+                if (ut_in) {
+                    tc_fence_after();
+                    const uint32_t un = smem_u32(sm + OutChainSmem::kBuf +
+                                                 (buf ^ 1) * OutChainSmem::kBufBytes + OutChainSmem::kUt);
+#pragma unroll
+                    for (int s = 0; s < C / 16; ++s)
+                        mma_bf16(tmem, desc_mnmajor(un, C, s), desc_kmajor(ib, C, s), idu, s > 0);
+                }
             }
             if (!wg_wait(&mbar, phase, p, 1, 53)) break;
             phase ^= 1;
