@@ -601,10 +601,13 @@ def run_report(args, rank, world, local_rank):
     # a long single row forward + backward (a quarter of the long-context row, which is
     # a forward workload), with and without the piece scan of both chains
     lrow = dict(WORKLOADS[4], T=1 << 18, bwd=True, name="gdn_fwdbwd_bf16_B1_T262144_H8_d128")
+    # head dim 256 (fp32 CUDA-core kernels): the benchmark's token count per head, 8 heads
+    d256 = dict(WORKLOADS[2], B=1, H=8, K=256, V=256, name="gdn_fwdbwd_bf16_B1_T4096_H8_d256")
     runs = ([(i, dict(WORKLOADS[i]), False, False) for i in sorted(WORKLOADS)] +
             [(4, dict(WORKLOADS[4]), True, False), (2, dict(WORKLOADS[2]), False, True),
              (None, d64, False, False), (None, p64, False, False),
-             (None, lrow, False, False), (None, lrow, True, False)])
+             (None, lrow, False, False), (None, lrow, True, False),
+             (None, d256, False, False)])
     for idx, w, piece, l2 in runs:
         if idx is not None and not l2:
             inp = workload(idx, device="cuda" if idx == 4 else "cpu")
@@ -663,14 +666,18 @@ def run_report(args, rank, world, local_rank):
         fwd_b = (3 * el * K if K == V else el * (2 * K + V)) + 8 + el * V
         bwd_b = el * (2 * K + 2 * V) + 8 + el * (2 * K + V) + 8
         bytes_ = (fwd_b + (bwd_b if bwd else 0)) * th
-        t_bound = max(flops / (pk["tc"] * 1e12), bytes_ / (pk["hbm"] * 1e9))
+        # the fp32 path (fp32 inputs, or a head dim of 256) runs on the CUDA cores: its
+        # flops are bound by the fp32 FMA peak, the tensor-core path's by the bf16 MMA peak
+        cuda_core = w["dtype"] != "bf16" or K > 128 or V > 128
+        fpeak = alu_peak_tflops(pk["sm_mhz"]) if cuda_core else pk["tc"]
+        t_bound = max(flops / (fpeak * 1e12), bytes_ / (pk["hbm"] * 1e9))
         if rank == 0:
             print(json.dumps({
                 "workload": w["name"] + ("+piece_scan" if piece else "") + ("+qk_l2norm" if l2 else ""),
                 "pass": "fwd+bwd" if bwd else "fwd",
                 "tokens_per_s": B * T / (ms / 1e3), "ms_per_call": ms,
                 "roofline_frac": t_bound * 1e3 / ms, "roofline_us": t_bound * 1e6,
-                "path": "tensor-core" if w["dtype"] == "bf16" else "fp32",
+                "path": "cuda-core fp32" if cuda_core else "tensor-core",
                 "peaks": pk["src"]}), flush=True)
         del d, ws, o, hT, grads
         torch.cuda.empty_cache()

@@ -21,7 +21,9 @@ gdn_status describe(const gdn_desc *d, Problem *p) {
     if (!d) return GDN_ERR_INVALID_ARG;
     if (d->B < 1 || d->T < 0 || d->H < 1 || d->n_seqs < 0) return GDN_ERR_INVALID_ARG;
     if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return GDN_ERR_UNSUPPORTED;
-    if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN_ERR_UNSUPPORTED;
+    // head dims 64 and 128 (both paths) and 256 (the fp32 CUDA-core kernels, either dtype)
+    const auto dim_ok = [](int64_t x) { return x == 64 || x == 128 || x == 256; };
+    if (!dim_ok(d->dk) || !dim_ok(d->dv)) return GDN_ERR_UNSUPPORTED;
     if (d->n_seqs > 0 && d->B != 1) return GDN_ERR_INVALID_ARG;
     // range checks before any product is formed (no signed overflow on huge inputs)
     constexpr int64_t kLim = int64_t(1) << 31;
@@ -290,7 +292,7 @@ Layout make_layout(const Problem &pb, bool bwd) {
         }
         // one scratch slot per CTA of the chunk-parallel kernels (grid = min(NC*H, kSimtSlots))
         const size_t slots = nch < (size_t)kSimtSlots ? (nch > 0 ? nch : 1) : (size_t)kSimtSlots;
-        L.scratch = take(slots * kSimtScratchFloats * f);
+        L.scratch = take(slots * simt_scratch_floats(simt_tile_width((int)pb.K, (int)pb.V)) * f);
         if (pb.l2norm) {  // normalised copies of q and k, and their inverse norms
             const size_t rows = (size_t)pb.BT * pb.H, es = pb.dtype == GDN_BF16 ? 2 : 4;
             L.qn = take(rows * pb.K * es);

@@ -60,7 +60,7 @@ struct Params {
     int32_t *seq_first;            // N + 1 entries: first chunk of each sequence
     // fp32 per-(chunk, head) intermediates of the SIMT path
     float *W, *Ut, *A, *U, *Hs, *dUloc, *dU, *dHn;
-    float *scratch;                // kSimtSlots slots of kSimtScratchFloats
+    float *scratch;                // kSimtSlots slots of simt_scratch_floats(tile width)
     // bf16 tensor-core path intermediates, per (chunk, head): tile images
     // (128-byte-swizzled, as the MMAs read them) and plain rows
     void *tW, *tUt, *tKd;          // 64x128 W image, 64x128 Ut rows, 64x128 diag(e)K image
@@ -82,8 +82,12 @@ struct Params {
     CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv, tm_o;
 };
 
-// Per-CTA scratch floats of the SIMT chunk-parallel kernels (K, V <= 128).
-constexpr size_t kSimtScratchFloats = 64 * 128 * 14 + 64 * 64 * 10 + 64 * 8;
+// Row width (floats) of the SIMT path's 64-row chunk tiles: 128, or 256 when a head
+// dim is 256; and the per-CTA scratch floats of its chunk-parallel kernels.
+__host__ __device__ constexpr int simt_tile_width(int K, int V) { return (K > 128 || V > 128) ? 256 : 128; }
+__host__ __device__ constexpr size_t simt_scratch_floats(int D) {
+    return (size_t)64 * D * 14 + 64 * 64 * 10 + 64 * 8;
+}
 
 // Chunk c of the call: from the table build_chunks writes for packed documents,
 // or in closed form for dense rows (row c / n, chunk c % n of a row, n = ceil(T / 64)),

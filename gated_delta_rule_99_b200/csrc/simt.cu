@@ -125,15 +125,16 @@ __device__ void invert_unit_lower(float *A, const float *M) {
 }
 
 __device__ __forceinline__ float *slot(const Params &p) {
-    return p.scratch + (size_t)blockIdx.x * kSimtScratchFloats;
+    return p.scratch + (size_t)blockIdx.x * simt_scratch_floats(simt_tile_width(p.K, p.V));
 }
 
 // ---------------------------------------------------------------- prep: A, W, Ut
 __global__ void __launch_bounds__(kThreads) simt_prep_kernel(Params p) {
     if (p.hdr->status) return;
     const int K = p.K, V = p.V, H = p.H;
-    float *fk = slot(p), *fv = fk + C * 128, *bk = fv + C * 128, *bv = bk + C * 128;
-    float *M = bv + C * 128, *G = M + C * C, *bta = G + C;
+    const int TW = C * simt_tile_width(K, V);
+    float *fk = slot(p), *fv = fk + TW, *bk = fv + TW, *bv = bk + TW;
+    float *M = bv + TW, *G = M + C * C, *bta = G + C;
     for (int ch = blockIdx.x; ch < p.NC * H; ch += gridDim.x) {
         const int c = ch / H, h = ch % H;
         const ChunkInfo ci = chunk_at(p, c);
@@ -214,7 +215,8 @@ __global__ void __launch_bounds__(kThreads) simt_state_fwd_kernel(Params p) {
 __global__ void __launch_bounds__(kThreads) simt_out_kernel(Params p) {
     if (p.hdr->status) return;
     const int K = p.K, V = p.V, H = p.H;
-    float *fq = slot(p), *fk = fq + C * 128, *O = fk + C * 128, *P = O + C * 128, *G = P + C * C;
+    const int TW = C * simt_tile_width(K, V);
+    float *fq = slot(p), *fk = fq + TW, *O = fk + TW, *P = O + TW, *G = P + C * C;
     for (int ch = blockIdx.x; ch < p.NC * H; ch += gridDim.x) {
         const int c = ch / H, h = ch % H;
         const ChunkInfo ci = chunk_at(p, c);
@@ -242,7 +244,8 @@ __global__ void __launch_bounds__(kThreads) simt_out_kernel(Params p) {
 __global__ void __launch_bounds__(kThreads) simt_duloc_kernel(Params p) {
     if (p.hdr->status) return;
     const int K = p.K, V = p.V, H = p.H;
-    float *fq = slot(p), *fk = fq + C * 128, *fdo = fk + C * 128, *P = fdo + C * 128,
+    const int TW = C * simt_tile_width(K, V);
+    float *fq = slot(p), *fk = fq + TW, *fdo = fk + TW, *P = fdo + TW,
           *G = P + C * C;
     for (int ch = blockIdx.x; ch < p.NC * H; ch += gridDim.x) {
         const int c = ch / H, h = ch % H;
@@ -322,7 +325,8 @@ __global__ void __launch_bounds__(kThreads) simt_state_bwd_kernel(Params p) {
 __global__ void __launch_bounds__(kThreads) simt_grads_kernel(Params p) {
     if (p.hdr->status) return;
     const int K = p.K, V = p.V, H = p.H;
-    constexpr int T8 = C * 128, T4 = C * C;
+    const int T8 = C * simt_tile_width(K, V);
+    constexpr int T4 = C * C;
     float *fq = slot(p), *fk = fq + T8, *fv = fk + T8, *fdo = fv + T8, *X1 = fdo + T8,
           *X2 = X1 + T8, *X3 = X2 + T8, *Z = X3 + T8, *AtdU = Z + T8, *bv = AtdU + T8,
           *bgk = bv + T8, *dQ = bgk + T8, *dK = dQ + T8;

@@ -60,7 +60,7 @@ extern "C" {
 typedef enum gdn_status {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = 1, /* bad shape, null pointer, bad cu_seqlens */
-    GDN_ERR_UNSUPPORTED = 2, /* head dim not in {64, 128}, unknown dtype */
+    GDN_ERR_UNSUPPORTED = 2, /* head dim not in {64, 128, 256} ({64, 128} for decode), unknown dtype */
     GDN_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte (workspace: 256-byte) aligned */
     GDN_ERR_WORKSPACE = 4,   /* workspace missing or too small */
     GDN_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch, copy) */
@@ -76,8 +76,8 @@ typedef struct gdn_desc {
     int64_t B;      /* rows (must be 1 when n_seqs > 0) */
     int64_t T;      /* tokens per row; B * T < 2^31 */
     int64_t H;      /* heads */
-    int64_t dk;     /* key/query head dim: 64 or 128 */
-    int64_t dv;     /* value head dim: 64 or 128 */
+    int64_t dk;     /* key/query head dim: 64, 128 or 256 (256: CUDA-core kernels; not decode) */
+    int64_t dv;     /* value head dim: 64, 128 or 256 (256: CUDA-core kernels; not decode) */
     int64_t n_seqs; /* 0: B dense rows; > 0: packed documents given by cu_seqlens */
     int32_t dtype;  /* gdn_dtype */
     float scale;    /* output scale applied to q (1.0 for the plain recurrence) */

@@ -41,7 +41,8 @@ def test_status_strings():
 
 
 @pytest.mark.parametrize("bad,code", [
-    (dict(dk=96), 2), (dict(dv=32), 2), (dict(dtype=7), 2), (dict(B=0), 1), (dict(H=0), 1),
+    (dict(dk=96), 2), (dict(dv=32), 2), (dict(dk=512), 2), (dict(dv=192), 2), (dict(dtype=7), 2),
+    (dict(B=0), 1), (dict(H=0), 1),
     (dict(T=-1), 1), (dict(n_seqs=3, B=2), 1), (dict(B=1 << 20, T=1 << 12), 1)])
 def test_workspace_size_rejects_bad_descriptors(bad, code):
     args = dict(B=2, T=100, H=3, dk=64, dv=128, n_seqs=0, dtype=0, scale=1.0)
@@ -50,6 +51,18 @@ def test_workspace_size_rejects_bad_descriptors(bad, code):
     assert gdn.fwd_workspace_size(d) == 0 and gdn.bwd_workspace_size(d) == 0
     rc = _fwd(d, ws_bytes=1 << 40)
     assert rc == code
+
+
+def test_head_dim_256_takes_the_cuda_core_layout_for_both_dtypes():
+    """d = 256 runs on the fp32 CUDA-core kernels whatever the dtype: its workspace
+    is that path's (fp32 intermediates and scratch slots with 256-float rows), the
+    same for bf16 and fp32 inputs, and larger than at d = 128."""
+    for K, V in ((256, 256), (256, 128), (64, 256)):
+        w = [gdn.fwd_workspace_size(gdn.make_desc(2, 100, 3, K, V, dtype=dt)) for dt in (0, 1)]
+        b = [gdn.bwd_workspace_size(gdn.make_desc(2, 100, 3, K, V, dtype=dt)) for dt in (0, 1)]
+        assert w[0] == w[1] > 0 and b[0] == b[1] > w[0]
+    small = gdn.fwd_workspace_size(gdn.make_desc(2, 100, 3, 128, 128, dtype=1))
+    assert gdn.fwd_workspace_size(gdn.make_desc(2, 100, 3, 256, 256, dtype=1)) > small
 
 
 def test_flags_match_header_and_unknown_bits_are_rejected():
@@ -166,6 +179,7 @@ def test_decode_rejects_bad_arguments():
     ok = gdn.make_desc(4, 1, 2, 128, 128)
     st = FAKE
     assert L.gdn_decode(ctypes.byref(gdn.make_desc(4, 1, 2, 96, 128)), *p, st, FAKE, None) == 2
+    assert L.gdn_decode(ctypes.byref(gdn.make_desc(4, 1, 2, 256, 128)), *p, st, FAKE, None) == 2
     assert L.gdn_decode(ctypes.byref(gdn.make_desc(4, 0, 2, 128, 128)), *p, st, FAKE, None) == 1
     assert L.gdn_decode(ctypes.byref(gdn.make_desc(1, 1, 2, 128, 128, n_seqs=1)), *p, st, FAKE,
                         None) == 1
