@@ -125,8 +125,8 @@ typedef struct gdn_desc {
  * of the products inside the tensor cores; not bitwise equal to the default.
  * On a B200 it is not faster (a chain step is bound by the fixed latency of
  * its two dependent tensor-core products, which does not shrink with their
- * size), so it is off by default.  Applies to the bf16 forward (and the piece
- * scan); ignored elsewhere, and by gdn_bwd and gdn_decode. */
+ * size), so it is off by default.  Applies to the bf16 forward with head dims
+ * 64 or 128 (and the piece scan); ignored elsewhere, and by gdn_bwd and gdn_decode. */
 #define GDN_FLAG_VALUE_SLICES 4
 
 /* Library version (major * 10000 + minor * 100 + patch). */

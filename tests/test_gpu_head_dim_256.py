@@ -62,3 +62,17 @@ def test_head_dim_256_packed_documents():
 def test_head_dim_256_strong_decay_over_several_chunks():
     inp = make_inputs(B=1, T=300, H=1, K=256, V=256, dtype="fp32", seed=43, gate_scale=3.0)
     _check(inp, TOL["fp32"])
+
+
+def test_head_dim_256_ignores_the_tensor_core_options():
+    """The value-slices and piece-scan options apply to the tensor-core kernels
+    only: at head dim 256 the results are bitwise those of the default call."""
+    inp = make_inputs(B=1, T=1100, H=2, K=256, V=256, dtype="bf16", seed=44)
+    d = inp.to("cuda")
+    base = gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, h0=d.h0)
+    for kw in (dict(value_slices=True), dict(piece_scan=True)):
+        o, hT = gdn.gdn_fwd(d.q, d.k, d.v, d.g, d.beta, h0=d.h0, **kw)
+        assert torch.equal(o, base[0]) and torch.equal(hT, base[1]), kw
+    g0 = gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, h0=d.h0, dhT=d.dhT)
+    g1 = gdn.gdn_bwd(d.q, d.k, d.v, d.g, d.beta, d.do, h0=d.h0, dhT=d.dhT, piece_scan=True)
+    assert all(torch.equal(a, b) for a, b in zip(g0, g1))

@@ -42,7 +42,7 @@ def test_tensor_core_path_packed_ragged():
 
 
 @pytest.mark.parametrize("dtype,K,V", [("fp32", 64, 128), ("bf16", 64, 64), ("fp32", 128, 64),
-                                       ("bf16", 128, 64)])
+                                       ("bf16", 128, 64), ("bf16", 256, 256), ("fp32", 256, 128)])
 def test_other_head_dims_and_fp32(dtype, K, V):
     inp = make_inputs(B=2, T=150, H=2, K=K, V=V, dtype=dtype, seed=62, raw_qk=True)
     _check(inp, TOL[dtype])
