@@ -114,9 +114,9 @@ def test_orthogonal_keys_reduce_to_gated_linear_attention():
     np.testing.assert_allclose(o, 0.9 * ref, rtol=1e-12, atol=1e-14)
 
 
-def test_whole_sequence_matrix_form():
+@pytest.mark.parametrize("L,K,V", [(23, 6, 7), (70, 256, 128)])
+def test_whole_sequence_matrix_form(L, K, V):
     # h0 = 0: U = (I + strict_lower(diag(b) K K^T * Gam))^-1 diag(b) V ; O = lower(Q K^T * Gam) U
-    L, K, V = 23, 6, 7
     q, k, v, g, beta = rand_unit(L, K, V)
     o, _ = fwd1(q, k, v, g, beta, scale=0.8)
     G = np.cumsum(g)
@@ -213,6 +213,35 @@ def _loss_packed(x, cu, do, dhT, scale):
     o, hT = oracle.gdn_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=cu, h0=x["h0"],
                            scale=scale)
     return float(np.sum(o * do) + np.sum(hT * dhT))
+
+
+def test_backward_directional_derivatives_head_dim_256():
+    """At head dim 256 (two packed documents): for a random direction per input,
+    the central difference of the loss sum(o . do) + sum(hT . dhT) along it equals
+    the oracle's gradient dotted with it."""
+    rng = np.random.default_rng(12)
+    lens = [40, 31]
+    T, H, K, V = sum(lens), 1, 256, 256
+    cu = np.cumsum([0] + lens)
+    x = dict(q=rng.standard_normal((1, T, H, K)) / 16, k=rng.standard_normal((1, T, H, K)) / 16,
+             v=rng.standard_normal((1, T, H, V)), g=-rng.random((1, T, H)) * 0.5,
+             beta=rng.random((1, T, H)), h0=rng.standard_normal((2, H, K, V)) * 0.1)
+    do = rng.standard_normal((1, T, H, V))
+    dhT = rng.standard_normal((2, H, K, V)) * 0.1
+    s = 0.7
+    dq, dk, dv, dg, db, dh0 = oracle.gdn_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], do,
+                                             cu_seqlens=cu, h0=x["h0"], dhT=dhT, scale=s)
+    grads = dict(q=dq, k=dk, v=dv, g=dg, beta=db, h0=dh0)
+    eps = 1e-5
+    for name, gr in grads.items():
+        d = rng.standard_normal(x[name].shape)
+        xp = {kk: vv.copy() for kk, vv in x.items()}
+        xm = {kk: vv.copy() for kk, vv in x.items()}
+        xp[name] += eps * d
+        xm[name] -= eps * d
+        fd = (_loss_packed(xp, cu, do, dhT, s) - _loss_packed(xm, cu, do, dhT, s)) / (2 * eps)
+        an = float(np.sum(gr * d))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
 
 
 def test_backward_finite_differences_and_euler():
